@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the fused MoE FFN layer on B200.
+
+One step = one pass of the whole layer over one batch of the large workload
+(c4): a prefill forward of 4 x 8192 = 32768 tokens followed by a batched
+decode forward of 64 tokens on the same weights (d_model=2048, 60 routed
+experts + 1 shared of hidden 1024, top-4, INT4 group-32 weights, INT8
+activations, FP32 router).  Inputs are seeded synthetic draws resident in HBM.
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and a device
+synchronise, CUDA events on the launching stream, max over ranks.  Every rank
+runs an independent replica (the layer needs no exchange between GPUs), so
+`value` is the tokens of all ranks divided by the slowest rank's time.
+
+--impl reference times the CPU oracle (the plain C implementation in
+oracle/) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer prefill tokens/s & decode us/layer; % of INT8-TC / HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c4", help="prefill workload (c2, c3a, c3b, c4); c4 adds its 64-token decode batch")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU work budget of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas: a barrier and max/sum reductions only)
+# --------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(backend: str, world: int):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=180))
+    return dist if world > 1 else None
+
+
+def aggregate(elapsed_ms: float, units: float, dist, device=None):
+    """(max elapsed over ranks, sum of units over ranks)."""
+    if dist is None:
+        return elapsed_ms, units
+    import torch
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpus):
+        self.gpus = set(gpus)
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.f.read().splitlines():
+            c = [v.strip() for v in line.split(",")]
+            if len(c) < 9 or not c[0].isdigit() or int(c[0]) not in self.gpus:
+                continue
+            try:
+                sm.append(float(c[1]))
+                smax.append(float(c[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, c[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# workload
+# --------------------------------------------------------------------------
+def workload_config(name):
+    from moe_ffn_layer_fp32_b200 import synth
+    w = synth.WORKLOADS[name]
+    dec = synth.WORKLOADS["c4dec"] if name == "c4" else None
+    return w, dec
+
+
+def layer_counts(w, T):
+    """Algorithmic work of one forward of T tokens (2 ops per MAC; INT4 + FP32 scale = 0.625 B per weight)."""
+    rows_routed, rows_shared = T * w.k, T
+    gu_ops = 4 * w.d * (rows_routed * w.h + rows_shared * w.hs)
+    dn_ops = 2 * w.d * (rows_routed * w.h + rows_shared * w.hs)
+    return gu_ops, dn_ops
+
+
+def quantized_on_device(w, device):
+    """Seeded FP32 weights (synth) quantised on the GPU by the library's Eq. (6) kernel."""
+    import torch
+
+    from moe_ffn_layer_fp32_b200 import synth
+    from moe_ffn_layer_fp32_b200.layer import quantize_int4
+    lw = synth.workload_layer(w)
+    gu_w, gu_s, dn_w, dn_s = [], [], [], []
+    for g in range(w.E + 1):
+        p, s = quantize_int4(torch.from_numpy(lw.w_gate_up[g]).to(device))
+        gu_w.append(p.reshape(-1)); gu_s.append(s.reshape(-1))
+        p, s = quantize_int4(torch.from_numpy(lw.w_down[g]).to(device))
+        dn_w.append(p.reshape(-1)); dn_s.append(s.reshape(-1))
+    wr = torch.from_numpy(lw.w_router).to(device)
+    bias = None if lw.router_bias is None else torch.from_numpy(lw.router_bias).to(device)
+    return (wr, bias, torch.cat(gu_w), torch.cat(gu_s), torch.cat(dn_w), torch.cat(dn_s)), lw
+
+
+def weight_bytes(w, experts):
+    return sum((3 * w.d * (w.h if g < w.E else w.hs)) * 0.625 for g in experts)
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# --------------------------------------------------------------------------
+def oracle_rate(w, budget_s, lw=None):
+    """Tokens/s of the CPU oracle on a bounded sample of the workload's tokens."""
+    import numpy as np
+
+    import oracle
+    from moe_ffn_layer_fp32_b200 import synth
+    if lw is None:
+        lw = synth.workload_layer(w)
+    q = oracle.quantize_layer(lw)
+    cores = oracle.num_threads()
+    x = synth.workload_x(w, T=min(w.T, 4096))
+    n = max(2, cores)
+    t0 = time.perf_counter()
+    oracle.moe_tokens(q, x, np.arange(n))
+    dt = time.perf_counter() - t0
+    n2 = int(min(x.shape[0], max(n, budget_s / max(dt / n, 1e-9))))
+    t0 = time.perf_counter()
+    oracle.moe_tokens(q, x, np.arange(n2))
+    dt2 = time.perf_counter() - t0
+    return n2 / dt2, cores, n2, dt2
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w, dec = workload_config(args.workload)
+    budget = max(1.0, args.cpu_seconds / max(1, args.steps))
+    rates = []
+    cores = n = None
+    for i in range(args.warmup + args.steps):
+        r, cores, n, dt = oracle_rate(w, budget if i >= args.warmup else 1.0)
+        if i >= args.warmup:
+            rates.append(r)
+    value = statistics.median(rates)
+    sample = (f"{n} of the {w.T} prefill tokens of {w.name} per step ({w.desc}); "
+              "oracle tokens/s applies to prefill and decode tokens alike")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8xint4->int32, f32", "data": "synthetic (seeded N(0,1) x, N(0,0.02) weights)",
+            "config": {"workload": w.desc, "global_batch": w.T, "seq_len": 8192 if w.name == "c4" else w.T,
+                       "parallelism": "cpu oracle"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    from moe_ffn_layer_fp32_b200 import build, synth
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl", world)
+    if rank == 0:
+        build.build()
+    if dist is not None:
+        dist.barrier()
+    build.build()
+
+    w, dec = workload_config(args.workload)
+    tensors, lw = quantized_on_device(w, dev)
+    Tp = w.T
+    Td = dec.T if dec else 0
+    mk = dict(shared_hidden=w.hs, n_experts=w.E, top_k=w.k, gating=0, has_router_bias=lw.router_bias is not None,
+              device=local)
+    pre = MoELayer(w.d, w.h, max_tokens=Tp, **mk)
+    pre.load(*tensors)
+    decl = None
+    if dec:
+        decl = MoELayer(w.d, w.h, max_tokens=Td, **mk)
+        decl.load(*tensors)
+    xp_np = synth.workload_x(w)
+    xp = torch.from_numpy(xp_np.view(np.int16)).to(dev).view(torch.bfloat16)
+    yp = torch.empty((Tp, w.d), dtype=torch.float32, device=dev)
+    if dec:
+        xd_np = synth.workload_x(dec)
+        xd = torch.from_numpy(xd_np.view(np.int16)).to(dev).view(torch.bfloat16)
+        yd = torch.empty((Td, w.d), dtype=torch.float32, device=dev)
+        idx_d = torch.empty((Td, w.k), dtype=torch.int32, device=dev)
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        pre.forward(xp, yp)
+        if ev is not None:
+            ev[0].record(stream)
+        if dec:
+            flush.fill_(1.0)  # decode weights must come from HBM, not from the prefill's L2 residue
+            if ev is not None:
+                ev[1].record(stream)
+            decl.forward(xd, yd, topk_idx=idx_d)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    pre.profile(True)
+    if decl:
+        decl.profile(True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(range(world)) if rank == 0 else None
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    start.record(stream)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    elapsed = start.elapsed_time(end)
+    prefill_ms = statistics.median(starts[i].elapsed_time(evs[i][0]) for i in range(args.steps))
+    decode_ms = statistics.median(evs[i][1].elapsed_time(starts[i + 1] if i + 1 < args.steps else end)
+                                  for i in range(args.steps)) if dec else None
+    prof_p = pre.profile_read()
+    prof_d = decl.profile_read() if decl else {}
+    pre.profile(False)
+    if decl:
+        decl.profile(False)
+
+    tokens_per_step = Tp + Td
+    tmax, units = aggregate(elapsed, tokens_per_step * args.steps, dist, dev)
+    launches = sum(v[0] for v in prof_p.values()) + sum(v[0] for v in prof_d.values())
+
+    # dominant kernel: the prefill gate/up GEMM (INT8 x INT4 -> INT32, tensor-bound)
+    gu_ops, dn_ops = layer_counts(w, Tp)
+    n_gu, ms_gu = prof_p["gate_up"]
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        int8_peak = 2.0 * float(peaks["bf16_tflops_sustained"])
+        peak_note = "measured cuBLAS bf16 sustained x 2 (nominal int8/bf16 ratio)"
+    except (OSError, KeyError, ValueError):
+        int8_peak = 2.0 * 1400.0
+        peak_note = "fallback 1.4 PFLOP/s bf16 sustained x 2"
+    gu_avg_s = (ms_gu / max(n_gu, 1)) / 1e3
+    achieved = gu_ops / gu_avg_s / 1e12 if gu_avg_s > 0 else 0.0
+    traffic = None
+    roofline = {"kernel": "gate_up (prefill)", "bound": "tensor", "achieved": achieved, "peak": int8_peak,
+                "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": traffic, "op_dtype": "int8",
+                "peak_source": peak_note, "ops_per_launch": gu_ops, "avg_launch_ms": gu_avg_s * 1e3}
+
+    decode = None
+    if dec:
+        hbm = float(peaks.get("hbm_gbs", 6650.0))
+        idx = idx_d.cpu().numpy()
+        experts = sorted(set(idx.ravel().tolist()) | {w.E})
+        dbytes = weight_bytes(w, experts) + w.d * w.E * 4
+        decode = {"tokens": Td, "us_per_layer": decode_ms * 1e3, "distinct_experts": len(experts),
+                  "algorithmic_bytes": dbytes, "achieved_gbs": dbytes / (decode_ms / 1e3) / 1e9,
+                  "hbm_peak_gbs": hbm, "hbm_frac": dbytes / (decode_ms / 1e3) / 1e9 / hbm,
+                  "stages_ms": {k: v[1] / args.steps for k, v in prof_d.items() if v[0] or v[1]}}
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hx = torch.empty((Tp, w.d), dtype=torch.int16, pin_memory=True)
+        hx.numpy()[:] = xp_np.view(np.int16)
+        hy = torch.empty((Tp, w.d), dtype=torch.float32, pin_memory=True)
+        if dec:
+            hxd = torch.empty((Td, w.d), dtype=torch.int16, pin_memory=True)
+            hxd.numpy()[:] = xd_np.view(np.int16)
+            hyd = torch.empty((Td, w.d), dtype=torch.float32, pin_memory=True)
+        hxn, hyn = hx.numpy().view(np.uint16), hy.numpy()
+
+        def estep():
+            pre.forward_host(hxn, hyn)
+            if dec:
+                decl.forward_host(hxd.numpy().view(np.uint16), hyd.numpy())
+
+        for _ in range(max(1, args.warmup)):
+            estep()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            estep()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        et, eu = aggregate(e0.elapsed_time(e1), tokens_per_step * args.steps, dist, dev)
+        e2e = {"value": eu / (et / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": (Tp + Td) * w.d * 2, "d2h_bytes_per_step": (Tp + Td) * w.d * 4,
+               "api": "mmoe_forward_host (pinned host x and y)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, n, dt = oracle_rate(w, args.cpu_seconds, lw)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n} prefill tokens of {w.name} ({dt:.1f} s of CPU work)"}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    value = units / (tmax / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tmax / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8xint4->int32, f32 (router f32)",
+        "data": "synthetic (seeded N(0,1) BF16 x, N(0,0.02) weights quantised by Eq. (6))",
+        "config": {"workload": (w.desc + (f" + decode batch of {Td} tokens on the same weights" if dec else "")),
+                   "global_batch": tokens_per_step * world, "seq_len": 8192 if w.name == "c4" else Tp,
+                   "parallelism": f"replicas x{world} (no exchange)",
+                   "l2": "inputs larger than L2 (x 134 MB, y 268 MB, weights 240 MB); L2 flushed before each decode batch"},
+        "prefill": {"tokens": Tp, "ms": prefill_ms, "tokens_per_s": Tp / (prefill_ms / 1e3),
+                    "stages_ms": {k: v[1] / args.steps for k, v in prof_p.items() if v[0] or v[1]}},
+        "decode": decode,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

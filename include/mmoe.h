@@ -1,0 +1,223 @@
+/*
+ * mmoe.h -- C ABI of the fused MoE feed-forward layer for B200 (sm_100a).
+ *
+ * The layer is Eq. (*) of "MobileMoE: Scaling On-Device Mixture of Experts"
+ * (paper-archivist reading, section "MoE preliminaries and three design
+ * factors"):
+ *
+ *     y = sum_{i in Top-k} router_i(x) * FFN_i(x) + FFN^(s)(x)
+ *
+ * 60 fine-grained routed SwiGLU experts, top-4, one always-on shared expert
+ * ("Finding 3" and the final architecture paragraph), an FP32 router
+ * ("MoE training stability techniques"), symmetric group-32 INT4 weights with
+ * FP32 scales (Eq. (6), section "QAT") and INT8 activations quantised per
+ * token on the fly (same section).  The pages run the whole FFN as one fused
+ * operator call (section "custom MoE kernel", principle 2); mmoe_forward is
+ * that call.
+ *
+ * Conventions for every function below:
+ *   - Every function returns an mmoe_status; no exception or signal crosses
+ *     the ABI.  On failure, mmoe_last_error() returns a thread-local message
+ *     that stays valid until the next call on the same thread.
+ *   - "device" pointers are CUDA global-memory addresses on the handle's
+ *     device; "host" pointers are ordinary process memory (pinned memory
+ *     makes the copies asynchronous, pageable memory is accepted too).
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *     default stream.  Work is enqueued on it in order; no function except
+ *     mmoe_forward_host, mmoe_create and mmoe_destroy waits for the GPU.
+ *   - A handle is not thread-safe: one forward at a time per handle.
+ *   - Arguments are checked before anything is launched; a rejected call
+ *     leaves the handle and every buffer untouched.
+ */
+#ifndef MMOE_H
+#define MMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mmoe_handle mmoe_handle; /* opaque */
+
+typedef enum {
+    MMOE_OK = 0,
+    MMOE_ERR_INVALID_ARG = 1,   /* bad pointer, size, shape or enum value */
+    MMOE_ERR_NOT_LOADED = 2,    /* forward before mmoe_load_quantized_weights */
+    MMOE_ERR_OOM = 3,           /* a device or host allocation failed */
+    MMOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (message has the CUDA error) */
+    MMOE_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up; the context stays usable */
+    MMOE_ERR_UNIMPLEMENTED = 6  /* a valid request this build does not serve */
+} mmoe_status;
+
+/* Router gating.  Selection is always the top-k of the FP32 biased logits,
+ * the lower expert index first among equal logits; only the gate differs. */
+typedef enum {
+    /* p = softmax over all experts, gate_j = p[idx_j], no renormalisation
+     * (the gating the layer benchmark fixes) */
+    MMOE_GATE_SOFTMAX = 0,
+    /* p_e = sigmoid(l_e), gate_j = p[idx_j] / sum_j' p[idx_j'] ("sigmoid
+     * gating with per-token top-k normalisation", section "MoE training
+     * stability techniques") */
+    MMOE_GATE_SIGMOID_TOPK_NORM = 1
+} mmoe_gating;
+
+/* mmoe_config.flags */
+#define MMOE_FLAG_DETERMINISTIC 1u /* combine in a fixed order: y = FFN_s + g_0 FFN_0 + ... + g_{k-1} FFN_{k-1};
+                                      needs an extra [max_tokens*(k+1), d_model] FP32 workspace */
+
+typedef struct {
+    int32_t d_model;        /* multiple of 32, 64 <= d_model <= 8192 */
+    int32_t n_experts;      /* routed experts, 1..64 (60 in MobileMoE) */
+    int32_t top_k;          /* 1..min(n_experts, 8) (4 in MobileMoE); with n_experts = top_k every expert runs */
+    int32_t expert_hidden;  /* routed expert hidden size h, multiple of 32, 32..4096 */
+    int32_t shared_hidden;  /* shared expert hidden size, multiple of 32, 32..4096 */
+    int32_t group_size;     /* must be 32 (Eq. (6) group size) */
+    int32_t max_tokens;     /* largest T a forward may pass, 1..2^20; sizes the workspace */
+    int32_t gating;         /* mmoe_gating */
+    int32_t has_router_bias;/* 0 or 1: a per-expert FP32 bias added to the logits before gating */
+    uint32_t flags;         /* MMOE_FLAG_* */
+} mmoe_config;
+
+/* Quantised weights in the interchange layout (row-major, packed INT4 with
+ * the element of even K index in the low nibble, sign in two's complement,
+ * one FP32 scale per 32 consecutive K elements of a row, as Eq. (6)).
+ * Expert index n_experts is the shared expert; its blocks follow the routed
+ * ones at the same per-expert stride (so expert g starts at g times the
+ * routed expert's block size) and hold shared_hidden rows/columns.
+ *
+ *   w_router    FP32 [d_model, n_experts]
+ *   router_bias FP32 [n_experts], or NULL when has_router_bias = 0
+ *   w_gate_up   uint8 expert g at byte g*2h*d/2: [2*hid, d/2]; rows 0..hid-1 are
+ *               the gate projection, rows hid..2hid-1 the up projection
+ *   s_gate_up   FP32  expert g at g*2h*d/32:     [2*hid, d/32]
+ *   w_down      uint8 expert g at byte g*d*h/2:  [d, hid/2]
+ *   s_down      FP32  expert g at g*d*h/32:      [d, hid/32]
+ * (h = expert_hidden, hid = h for routed experts and shared_hidden for the
+ * shared one, d = d_model). */
+typedef struct {
+    const float* w_router;
+    const float* router_bias;
+    const uint8_t* w_gate_up;
+    const float* s_gate_up;
+    const uint8_t* w_down;
+    const float* s_down;
+    int32_t on_device; /* 1: all pointers are device pointers; 0: host pointers */
+} mmoe_weights;
+
+/* Creates a handle on CUDA device `device` and allocates its workspace (sized
+ * by max_tokens) and weight buffers.  The handle owns that memory until
+ * mmoe_destroy.  *out is set only on success.
+ * Errors: INVALID_ARG (cfg out of range, bad device), OOM, CUDA. */
+mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out);
+
+/* Copies the weights into the handle's buffers and re-tiles them into the
+ * kernels' layouts (stream-ordered, asynchronous).  The caller keeps
+ * ownership of `w` and may free or reuse it once the stream has reached this
+ * point.  May be called again to replace the weights.
+ * Errors: INVALID_ARG (NULL pointer, bias presence not matching the config), CUDA. */
+mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, void* stream);
+
+/* The layer, Eq. (*): y[T, d_model] (FP32, device) from x[T, d_model]
+ * (BF16 bit patterns, device).  Optional device outputs, each may be NULL:
+ *   topk_idx      int32 [T, top_k]  selected experts, by descending logit
+ *   topk_gate     FP32  [T, top_k]  their gates
+ *   expert_counts int32 [n_experts + 1] tokens per routed expert, then T for
+ *                 the shared expert (the expert-utilisation histogram)
+ * T = 0 is a no-op.  x and y must not overlap; y is fully overwritten.
+ * Errors: INVALID_ARG (T < 0, T > max_tokens, NULL x or y), NOT_LOADED,
+ * TIMEOUT (a bounded wait of an earlier call gave up), CUDA. */
+mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, float* y, void* stream,
+                         int32_t* topk_idx, float* topk_gate, int32_t* expert_counts);
+
+/* The same layer with HOST buffers: copies x (host, BF16 bits [T, d_model])
+ * to the handle's staging buffer, runs mmoe_forward, copies y back to the
+ * host buffer and waits for the stream.  The copies use one cudaMemcpyAsync
+ * each.  Errors: as mmoe_forward. */
+mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_bf16_host, int64_t T, float* y_host,
+                              void* stream);
+
+/* Waits for the handle's pending work, frees everything it owns and the
+ * handle itself.  NULL is accepted (no-op). */
+mmoe_status mmoe_destroy(mmoe_handle* h);
+
+/* Thread-local text of the last error on this thread ("" if none). */
+const char* mmoe_last_error(void);
+
+/* Eq. (6) (section "QAT") on the device: W[rows, K] FP32 (device) ->
+ * packed INT4 [rows, K/2] (device, interchange layout) and scales
+ * FP32 [rows, K/32] (device): s = 2 max|W_g| / 15 (IEEE division),
+ * q = clamp(round-half-even(W / s), -8, 7); an all-zero group gets s = 0.
+ * Errors: INVALID_ARG (NULL pointer, rows < 0, K not a multiple of 32), CUDA. */
+mmoe_status mmoe_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t* packed, float* scales,
+                               void* stream);
+
+/* ---- inspection of the last forward (tests and profiling) ----------------
+ * Copies an internal buffer of the handle, as left by the last mmoe_forward,
+ * into `dst` (device, `bytes` long; stream-ordered).  R = T*(top_k+1) rows:
+ * rows of the routed experts in expert order, each expert's rows in
+ * ascending (token, slot), then the T shared-expert rows in token order.
+ *   MMOE_STAGE_XQ       int8  [T, d_model]  activation codes
+ *   MMOE_STAGE_SX       FP32  [T]           activation scales
+ *   MMOE_STAGE_OFFSETS  int32 [n_experts+2] first row of each group, then R
+ *   MMOE_STAGE_ROW_SRC  int32 [R]           token of each row
+ *   MMOE_STAGE_SLOT_ROW int32 [T, top_k]    row of each (token, slot)
+ *   MMOE_STAGE_HQ       int8  [R, hmax]     SwiGLU output codes (hmax = max hidden)
+ *   MMOE_STAGE_SH       FP32  [R]           SwiGLU output scales
+ *   MMOE_STAGE_LOGITS   FP32  [T, n_experts] biased router logits
+ * Errors: INVALID_ARG (unknown stage, bytes larger than the stage), CUDA. */
+typedef enum {
+    MMOE_STAGE_XQ = 0,
+    MMOE_STAGE_SX = 1,
+    MMOE_STAGE_OFFSETS = 2,
+    MMOE_STAGE_ROW_SRC = 3,
+    MMOE_STAGE_SLOT_ROW = 4,
+    MMOE_STAGE_HQ = 5,
+    MMOE_STAGE_SH = 6,
+    MMOE_STAGE_LOGITS = 7
+} mmoe_stage;
+
+mmoe_status mmoe_debug_copy_stage(mmoe_handle* h, int32_t stage, void* dst, size_t bytes, void* stream);
+
+/* Re-runs the expert GEMMs of the last forward with their INT32 group
+ * partials written out (the exact per-group INT8 x INT4 sums the tensor
+ * cores accumulate), for rows [row0, row0 + nrows) of the permuted order:
+ *   which = 0: gate/up partials  int32 [nrows, 2*hmax, d_model/32] (gate rows, then up rows)
+ *   which = 1: down partials     int32 [nrows, d_model, hmax/32]
+ * `dst` is device memory.  Errors: INVALID_ARG, NOT_LOADED, CUDA. */
+mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int64_t nrows, int32_t* dst,
+                                void* stream);
+
+/* ---- per-stage timing ------------------------------------------------------
+ * While profiling is enabled, every forward records a CUDA event pair on its
+ * own stream around each stage's kernels.  mmoe_profile_read waits for those
+ * events and returns, per stage, the number of kernel launches and their
+ * summed device time in milliseconds, accumulated since the last enable.
+ * Stages (index into the arrays):
+ *   MMOE_PROF_ZERO_Y    clearing y before the atomic combine (a memset, not a kernel)
+ *   MMOE_PROF_ROUTER    activation quantiser + FP32 router + top-k
+ *   MMOE_PROF_PERMUTE   histogram, scan, stable scatter, row gather
+ *   MMOE_PROF_GATE_UP   grouped gate/up GEMM with SwiGLU
+ *   MMOE_PROF_REQUANT   per-row requantisation of the SwiGLU output
+ *   MMOE_PROF_DOWN      grouped down GEMM with the gate-weighted combine
+ *   MMOE_PROF_COMBINE   deterministic combine
+ * Errors: INVALID_ARG (n < 1, NULL arrays), CUDA. */
+enum {
+    MMOE_PROF_ZERO_Y = 0,
+    MMOE_PROF_ROUTER = 1,
+    MMOE_PROF_PERMUTE = 2,
+    MMOE_PROF_GATE_UP = 3,
+    MMOE_PROF_REQUANT = 4,
+    MMOE_PROF_DOWN = 5,
+    MMOE_PROF_COMBINE = 6,
+    MMOE_PROF_STAGES = 8
+};
+
+mmoe_status mmoe_profile_enable(mmoe_handle* h, int32_t enable);
+mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_ms, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MMOE_H */

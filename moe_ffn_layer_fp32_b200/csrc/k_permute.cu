@@ -1,0 +1,143 @@
+// K3: expert histogram, exclusive scan and stable token permutation.
+//
+// MobileMoE pages (paper-archivist reading, section "custom MoE kernel",
+// principle 1): tokens are reordered by their assigned expert id with a
+// counting sort, so that each expert's tokens are contiguous and every expert
+// processes its slice as one batched matmul.  Dispatch is dropless (section
+// "SFT" and the counting sort keep every token).
+//
+// Row order: routed rows grouped by expert, each expert's rows in ascending
+// (token, slot) order; then the T rows of the shared expert in token order.
+#include "mmoe_internal.cuh"
+
+namespace mmoe {
+namespace {
+
+constexpr int kThreads = 256;
+
+// per-chunk expert counts
+__global__ void __launch_bounds__(kThreads) count_kernel(Plan p)
+{
+    __shared__ int c[kMaxExperts];
+    for (int i = threadIdx.x; i < kMaxExperts; i += kThreads) c[i] = 0;
+    __syncthreads();
+    const int64_t S = p.Tk;
+    const int64_t s0 = (int64_t)blockIdx.x * kChunk;
+    for (int i = threadIdx.x; i < kChunk; i += kThreads) {
+        const int64_t s = s0 + i;
+        if (s < S) atomicAdd(&c[p.idx[s]], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kMaxExperts; i += kThreads) p.chunk_cnt[(int64_t)blockIdx.x * kMaxExperts + i] = c[i];
+}
+
+// totals, group offsets, per-chunk bases and the GEMM tile table (one block)
+__global__ void __launch_bounds__(kThreads) scan_kernel(Plan p)
+{
+    __shared__ int tot[kMaxExperts + 1];
+    __shared__ int off[kMaxExperts + 2];
+    __shared__ int tstart[kMaxExperts + 2];
+    const int E = p.E;
+    const int tid = threadIdx.x;
+    if (tid < E) {
+        int acc = 0;
+        for (int c = 0; c < p.nchunks; ++c) {
+            p.chunk_base[(int64_t)c * kMaxExperts + tid] = acc;  // running count before chunk c
+            acc += p.chunk_cnt[(int64_t)c * kMaxExperts + tid];
+        }
+        tot[tid] = acc;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int o = 0, ts = 0;
+        for (int e = 0; e < E; ++e) {
+            off[e] = o;
+            tstart[e] = ts;
+            o += tot[e];
+            ts += (tot[e] + kTileRows - 1) / kTileRows;
+        }
+        tot[E] = (int)p.T;
+        off[E] = o;             // = T*k
+        off[E + 1] = o + (int)p.T;
+        tstart[E] = ts;
+        ts += (int)((p.T + kTileRows - 1) / kTileRows);
+        tstart[E + 1] = ts;
+        *p.tile_count = ts;
+    }
+    __syncthreads();
+    if (tid < E) {
+        for (int c = 0; c < p.nchunks; ++c) p.chunk_base[(int64_t)c * kMaxExperts + tid] += off[tid];
+    }
+    for (int e = tid; e < E + 2; e += kThreads) p.offsets[e] = off[e];
+    for (int e = tid; e <= E; e += kThreads) p.counts[e] = tot[e];
+    // tile table: entry i -> (group, tile index within the group)
+    const int ntiles = tstart[E + 1];
+    for (int i = tid; i < ntiles; i += kThreads) {
+        int g = 0;
+        while (tstart[g + 1] <= i) ++g;
+        p.tiles[i] = (g << 24) | (i - tstart[g]);
+    }
+}
+
+// stable scatter: rank of every slot among same-expert slots of lower index
+__global__ void __launch_bounds__(kThreads) scatter_kernel(Plan p)
+{
+    __shared__ int base[kMaxExperts];
+    __shared__ int wcnt[kThreads / 32][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t S = p.Tk;
+    const int64_t c = blockIdx.x;
+    for (int i = tid; i < kMaxExperts; i += kThreads) base[i] = p.chunk_base[c * kMaxExperts + i];
+    for (int round = 0; round < kChunk / kThreads; ++round) {
+        for (int i = tid; i < (kThreads / 32) * kMaxExperts; i += kThreads) (&wcnt[0][0])[i] = 0;
+        __syncthreads();
+        const int64_t s = c * kChunk + round * kThreads + tid;
+        const bool valid = s < S;
+        const int e = valid ? p.idx[s] : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(same & ((1u << lane) - 1u));
+        if (valid && rank == 0) wcnt[warp][e] = __popc(same);
+        __syncthreads();
+        if (valid) {
+            int pre = 0;
+            for (int w = 0; w < warp; ++w) pre += wcnt[w][e];
+            const int r = base[e] + pre + rank;
+            p.row_src[r] = (int32_t)(s / p.k);
+            p.row_gate[r] = p.gate[s];
+            p.slot_row[s] = r;
+        }
+        __syncthreads();
+        if (tid < kMaxExperts) {
+            int sum = 0;
+            for (int w = 0; w < kThreads / 32; ++w) sum += wcnt[w][tid];
+            base[tid] += sum;
+        }
+        __syncthreads();
+    }
+}
+
+// gather the activation codes of every routed row from its token's row
+__global__ void __launch_bounds__(kThreads) gather_rows_kernel(Plan p)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    if (row >= p.Tk) return;
+    const int64_t t = p.row_src[row];
+    const uint4* src = reinterpret_cast<const uint4*>(p.xq + (p.Tk + t) * p.d);
+    uint4* dst = reinterpret_cast<uint4*>(p.xq + row * p.d);
+    for (int i = lane; i < p.d / 16; i += 32) dst[i] = src[i];
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const Plan& p, cudaStream_t s) {
+    if (p.T == 0) return cudaSuccess;
+    count_kernel<<<p.nchunks, kThreads, 0, s>>>(p);
+    scan_kernel<<<1, kThreads, 0, s>>>(p);
+    scatter_kernel<<<p.nchunks, kThreads, 0, s>>>(p);
+    const int64_t blocks = (p.Tk + kThreads / 32 - 1) / (kThreads / 32);
+    gather_rows_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace mmoe

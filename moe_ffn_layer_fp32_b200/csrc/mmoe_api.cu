@@ -1,0 +1,488 @@
+// C ABI of the fused MoE FFN layer (declared in include/mmoe.h): handle,
+// workspace, weight loading and the stream-ordered forward pass.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "mmoe.h"
+#include "mmoe_internal.cuh"
+
+using namespace mmoe;
+
+namespace {
+
+thread_local std::string g_err;
+
+mmoe_status fail(mmoe_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+mmoe_status fail(mmoe_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+mmoe_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(e == cudaErrorMemoryAllocation ? MMOE_ERR_OOM : MMOE_ERR_CUDA, "%s: %s (%s)", what,
+                cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+#define MMOE_CUDA(call, what)                          \
+    do {                                               \
+        cudaError_t e_ = (call);                       \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+// Makes the handle's device current for the scope and restores the caller's.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
+}  // namespace
+
+struct mmoe_handle {
+    mmoe_config cfg;
+    int device = 0;
+    int hmax = 0;
+    int64_t max_tokens = 0;
+    bool loaded = false;
+    int64_t last_T = -1;
+    // weights (interchange layout)
+    float* w_router = nullptr;
+    float* router_bias = nullptr;
+    uint8_t* w_gate_up = nullptr;
+    float* s_gate_up = nullptr;
+    uint8_t* w_down = nullptr;
+    float* s_down = nullptr;
+    size_t n_gu_bytes = 0, n_gu_scales = 0, n_d_bytes = 0, n_d_scales = 0;
+    // workspace
+    int8_t* xq = nullptr;
+    float* sx = nullptr;
+    float* logits = nullptr;
+    int32_t* idx = nullptr;
+    float* gate = nullptr;
+    int32_t* chunk_cnt = nullptr;
+    int32_t* chunk_base = nullptr;
+    int32_t* offsets = nullptr;
+    int32_t* counts = nullptr;
+    int32_t* tiles = nullptr;
+    int32_t* tile_count = nullptr;
+    int32_t* row_src = nullptr;
+    float* row_gate = nullptr;
+    int32_t* slot_row = nullptr;
+    float* act = nullptr;
+    int8_t* hq = nullptr;
+    float* sh = nullptr;
+    float* obuf = nullptr;
+    uint16_t* x_stage = nullptr;
+    float* y_stage = nullptr;
+    // per-stage timing (mmoe_profile_*)
+    struct ProfRec {
+        int stage, launches;
+        cudaEvent_t a, b;
+    };
+    bool prof_on = false;
+    std::vector<ProfRec> prof;
+    std::vector<cudaEvent_t> ev_pool;
+    int32_t prof_launches[MMOE_PROF_STAGES] = {};
+    double prof_ms[MMOE_PROF_STAGES] = {};
+};
+
+namespace {
+
+template <class T>
+cudaError_t dalloc(T** p, size_t count) {
+    *p = nullptr;
+    if (count == 0) count = 1;
+    return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
+}
+
+void free_all(mmoe_handle* h) {
+    void* ptrs[] = {h->w_router, h->router_bias, h->w_gate_up, h->s_gate_up, h->w_down, h->s_down,
+                    h->xq, h->sx, h->logits, h->idx, h->gate, h->chunk_cnt, h->chunk_base, h->offsets,
+                    h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
+                    h->sh, h->obuf, h->x_stage, h->y_stage};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+}
+
+mmoe_status check_config(const mmoe_config* c) {
+    if (!c) return fail(MMOE_ERR_INVALID_ARG, "config is NULL");
+    if (c->d_model < 64 || c->d_model > 8192 || c->d_model % kGroup)
+        return fail(MMOE_ERR_INVALID_ARG, "d_model=%d: must be a multiple of 32 in [64, 8192]", c->d_model);
+    if (c->n_experts < 1 || c->n_experts > kMaxExperts)
+        return fail(MMOE_ERR_INVALID_ARG, "n_experts=%d: must be in [1, %d]", c->n_experts, kMaxExperts);
+    if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > kMaxTopK)
+        return fail(MMOE_ERR_INVALID_ARG, "top_k=%d: must be in [1, min(n_experts, %d)]", c->top_k, kMaxTopK);
+    if (c->expert_hidden < 32 || c->expert_hidden > 4096 || c->expert_hidden % kGroup)
+        return fail(MMOE_ERR_INVALID_ARG, "expert_hidden=%d: must be a multiple of 32 in [32, 4096]",
+                    c->expert_hidden);
+    if (c->shared_hidden < 32 || c->shared_hidden > 4096 || c->shared_hidden % kGroup)
+        return fail(MMOE_ERR_INVALID_ARG, "shared_hidden=%d: must be a multiple of 32 in [32, 4096]",
+                    c->shared_hidden);
+    if (c->group_size != kGroup) return fail(MMOE_ERR_INVALID_ARG, "group_size=%d: must be 32", c->group_size);
+    if (c->max_tokens < 1 || c->max_tokens > (1 << 20))
+        return fail(MMOE_ERR_INVALID_ARG, "max_tokens=%d: must be in [1, 2^20]", c->max_tokens);
+    if (c->gating != MMOE_GATE_SOFTMAX && c->gating != MMOE_GATE_SIGMOID_TOPK_NORM)
+        return fail(MMOE_ERR_INVALID_ARG, "gating=%d: unknown", c->gating);
+    if (c->has_router_bias != 0 && c->has_router_bias != 1)
+        return fail(MMOE_ERR_INVALID_ARG, "has_router_bias=%d: must be 0 or 1", c->has_router_bias);
+    if (c->flags & ~MMOE_FLAG_DETERMINISTIC) return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
+    return MMOE_OK;
+}
+
+Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
+    const mmoe_config& c = h->cfg;
+    Plan p{};
+    p.d = c.d_model;
+    p.h = c.expert_hidden;
+    p.hs = c.shared_hidden;
+    p.hmax = h->hmax;
+    p.E = c.n_experts;
+    p.k = c.top_k;
+    p.gating = c.gating;
+    p.T = T;
+    p.Tk = T * c.top_k;
+    p.R = T * (c.top_k + 1);
+    p.deterministic = (c.flags & MMOE_FLAG_DETERMINISTIC) != 0;
+    p.w_router = h->w_router;
+    p.router_bias = c.has_router_bias ? h->router_bias : nullptr;
+    p.w_gate_up = h->w_gate_up;
+    p.s_gate_up = h->s_gate_up;
+    p.w_down = h->w_down;
+    p.s_down = h->s_down;
+    p.x = x;
+    p.y = y;
+    p.xq = h->xq;
+    p.sx = h->sx;
+    p.logits = h->logits;
+    p.idx = h->idx;
+    p.gate = h->gate;
+    p.chunk_cnt = h->chunk_cnt;
+    p.chunk_base = h->chunk_base;
+    p.offsets = h->offsets;
+    p.counts = h->counts;
+    p.tiles = h->tiles;
+    p.tile_count = h->tile_count;
+    p.row_src = h->row_src;
+    p.row_gate = h->row_gate;
+    p.slot_row = h->slot_row;
+    p.act = h->act;
+    p.hq = h->hq;
+    p.sh = h->sh;
+    p.obuf = h->obuf;
+    p.max_tiles = max_tiles_for(T, c.top_k, c.n_experts);
+    p.nchunks = (int)((p.Tk + kChunk - 1) / kChunk);
+    return p;
+}
+
+cudaEvent_t take_event(mmoe_handle* h) {
+    if (!h->ev_pool.empty()) {
+        cudaEvent_t e = h->ev_pool.back();
+        h->ev_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Runs one stage's launches, bracketed by an event pair when profiling is on.
+template <class F>
+cudaError_t run_stage(mmoe_handle* h, int stage, int launches, cudaStream_t s, F&& f) {
+    if (!h->prof_on) return f();
+    cudaEvent_t a = take_event(h), b = take_event(h);
+    if (!a || !b) return cudaErrorMemoryAllocation;
+    cudaError_t e = cudaEventRecord(a, s);
+    if (e == cudaSuccess) e = f();
+    if (e == cudaSuccess) e = cudaEventRecord(b, s);
+    if (e != cudaSuccess) {
+        h->ev_pool.push_back(a);
+        h->ev_pool.push_back(b);
+        return e;
+    }
+    h->prof.push_back({stage, launches, a, b});
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mmoe_last_error(void) { return g_err.c_str(); }
+
+mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
+    if (!out) return fail(MMOE_ERR_INVALID_ARG, "out is NULL");
+    mmoe_status st = check_config(cfg);
+    if (st != MMOE_OK) return st;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+        return fail(MMOE_ERR_INVALID_ARG, "device %d: not a CUDA device (found %d)", device, ndev);
+    DeviceGuard dg(device);
+    if (!dg.ok) return fail(MMOE_ERR_CUDA, "cudaSetDevice(%d) failed", device);
+
+    mmoe_handle* h = new (std::nothrow) mmoe_handle();
+    if (!h) return fail(MMOE_ERR_OOM, "host allocation of the handle failed");
+    h->cfg = *cfg;
+    h->device = device;
+    h->hmax = cfg->expert_hidden > cfg->shared_hidden ? cfg->expert_hidden : cfg->shared_hidden;
+    h->max_tokens = cfg->max_tokens;
+
+    const int64_t d = cfg->d_model, hh = cfg->expert_hidden, hs = cfg->shared_hidden, E = cfg->n_experts;
+    const int64_t k = cfg->top_k, Tm = cfg->max_tokens, R = Tm * (k + 1);
+    h->n_gu_bytes = (size_t)(E * 2 * hh + 2 * hs) * (d / 2);
+    h->n_gu_scales = (size_t)(E * 2 * hh + 2 * hs) * (d / kGroup);
+    h->n_d_bytes = (size_t)(E * hh + hs) * d / 2;
+    h->n_d_scales = (size_t)(E * hh + hs) * d / kGroup;
+    const int64_t nchunks = (Tm * k + kChunk - 1) / kChunk;
+
+    cudaError_t e = cudaSuccess;
+#define ALLOC(ptr, n) \
+    if (e == cudaSuccess) e = dalloc(&h->ptr, (size_t)(n))
+    ALLOC(w_router, d * E);
+    ALLOC(router_bias, E);
+    ALLOC(w_gate_up, h->n_gu_bytes);
+    ALLOC(s_gate_up, h->n_gu_scales);
+    ALLOC(w_down, h->n_d_bytes);
+    ALLOC(s_down, h->n_d_scales);
+    ALLOC(xq, R * d);
+    ALLOC(sx, Tm);
+    ALLOC(logits, Tm * E);
+    ALLOC(idx, Tm * k);
+    ALLOC(gate, Tm * k);
+    ALLOC(chunk_cnt, nchunks * kMaxExperts);
+    ALLOC(chunk_base, nchunks * kMaxExperts);
+    ALLOC(offsets, E + 2);
+    ALLOC(counts, E + 1);
+    ALLOC(tiles, max_tiles_for(Tm, (int)k, (int)E));
+    ALLOC(tile_count, 1);
+    ALLOC(row_src, R);
+    ALLOC(row_gate, R);
+    ALLOC(slot_row, Tm * k);
+    ALLOC(act, R * h->hmax);
+    ALLOC(hq, R * h->hmax);
+    ALLOC(sh, R);
+    if (cfg->flags & MMOE_FLAG_DETERMINISTIC) ALLOC(obuf, R * d);
+#undef ALLOC
+    if (e != cudaSuccess) {
+        free_all(h);
+        delete h;
+        return cuda_fail(e, "workspace allocation");
+    }
+    *out = h;
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, void* stream) {
+    if (!h || !w) return fail(MMOE_ERR_INVALID_ARG, "handle or weights is NULL");
+    if (!w->w_router || !w->w_gate_up || !w->s_gate_up || !w->w_down || !w->s_down)
+        return fail(MMOE_ERR_INVALID_ARG, "a weight pointer is NULL");
+    if (h->cfg.has_router_bias && !w->router_bias)
+        return fail(MMOE_ERR_INVALID_ARG, "the config has a router bias but router_bias is NULL");
+    if (w->on_device != 0 && w->on_device != 1) return fail(MMOE_ERR_INVALID_ARG, "on_device must be 0 or 1");
+    DeviceGuard dg(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const cudaMemcpyKind kind = w->on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    const size_t d = h->cfg.d_model, E = h->cfg.n_experts;
+    MMOE_CUDA(cudaMemcpyAsync(h->w_router, w->w_router, d * E * sizeof(float), kind, s), "copy w_router");
+    if (h->cfg.has_router_bias)
+        MMOE_CUDA(cudaMemcpyAsync(h->router_bias, w->router_bias, E * sizeof(float), kind, s), "copy router_bias");
+    MMOE_CUDA(cudaMemcpyAsync(h->w_gate_up, w->w_gate_up, h->n_gu_bytes, kind, s), "copy w_gate_up");
+    MMOE_CUDA(cudaMemcpyAsync(h->s_gate_up, w->s_gate_up, h->n_gu_scales * sizeof(float), kind, s), "copy s_gate_up");
+    MMOE_CUDA(cudaMemcpyAsync(h->w_down, w->w_down, h->n_d_bytes, kind, s), "copy w_down");
+    MMOE_CUDA(cudaMemcpyAsync(h->s_down, w->s_down, h->n_d_scales * sizeof(float), kind, s), "copy s_down");
+    h->loaded = true;
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y, void* stream,
+                         int32_t* topk_idx, float* topk_gate, int32_t* expert_counts) {
+    if (!h) return fail(MMOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || T > h->max_tokens)
+        return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be in [0, max_tokens=%lld]", (long long)T,
+                    (long long)h->max_tokens);
+    if (!h->loaded) return fail(MMOE_ERR_NOT_LOADED, "forward before mmoe_load_quantized_weights");
+    if (T == 0) return MMOE_OK;
+    if (!x || !y) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
+    DeviceGuard dg(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Plan p = make_plan(h, x, T, y);
+    if (!p.deterministic)
+        MMOE_CUDA(run_stage(h, MMOE_PROF_ZERO_Y, 0, s,
+                            [&] { return cudaMemsetAsync(y, 0, (size_t)T * p.d * sizeof(float), s); }),
+                  "zero y");
+    MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_quant(p, s); }),
+              "router/quantiser launch");
+    MMOE_CUDA(run_stage(h, MMOE_PROF_PERMUTE, 4, s, [&] { return launch_permute(p, s); }), "permute launch");
+    MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return launch_gate_up(p, s, nullptr, 0, 0); }),
+              "gate/up launch");
+    MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
+    MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return launch_down(p, s, nullptr, 0, 0); }), "down launch");
+    if (p.deterministic)
+        MMOE_CUDA(run_stage(h, MMOE_PROF_COMBINE, 1, s, [&] { return launch_combine(p, s); }), "combine launch");
+    if (topk_idx)
+        MMOE_CUDA(cudaMemcpyAsync(topk_idx, h->idx, (size_t)p.Tk * sizeof(int32_t), cudaMemcpyDeviceToDevice, s),
+                  "copy topk_idx");
+    if (topk_gate)
+        MMOE_CUDA(cudaMemcpyAsync(topk_gate, h->gate, (size_t)p.Tk * sizeof(float), cudaMemcpyDeviceToDevice, s),
+                  "copy topk_gate");
+    if (expert_counts)
+        MMOE_CUDA(cudaMemcpyAsync(expert_counts, h->counts, (size_t)(p.E + 1) * sizeof(int32_t),
+                                  cudaMemcpyDeviceToDevice, s),
+                  "copy expert_counts");
+    h->last_T = T;
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T, float* y_host, void* stream) {
+    if (!h) return fail(MMOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0 || T > h->max_tokens)
+        return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be in [0, max_tokens=%lld]", (long long)T,
+                    (long long)h->max_tokens);
+    if (!h->loaded) return fail(MMOE_ERR_NOT_LOADED, "forward before mmoe_load_quantized_weights");
+    if (T == 0) return MMOE_OK;
+    if (!x_host || !y_host) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
+    DeviceGuard dg(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t d = h->cfg.d_model;
+    if (!h->x_stage) {
+        MMOE_CUDA(dalloc(&h->x_stage, (size_t)h->max_tokens * d), "staging allocation");
+        MMOE_CUDA(dalloc(&h->y_stage, (size_t)h->max_tokens * d), "staging allocation");
+    }
+    MMOE_CUDA(cudaMemcpyAsync(h->x_stage, x_host, (size_t)T * d * sizeof(uint16_t), cudaMemcpyHostToDevice, s),
+              "copy x to the device");
+    mmoe_status st = mmoe_forward(h, h->x_stage, T, h->y_stage, stream, nullptr, nullptr, nullptr);
+    if (st != MMOE_OK) return st;
+    MMOE_CUDA(cudaMemcpyAsync(y_host, h->y_stage, (size_t)T * d * sizeof(float), cudaMemcpyDeviceToHost, s),
+              "copy y to the host");
+    MMOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_destroy(mmoe_handle* h) {
+    if (!h) return MMOE_OK;
+    DeviceGuard dg(h->device);
+    cudaError_t e = cudaDeviceSynchronize();
+    for (auto& r : h->prof) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (cudaEvent_t ev : h->ev_pool) cudaEventDestroy(ev);
+    free_all(h);
+    delete h;
+    if (e != cudaSuccess) return cuda_fail(e, "synchronize before destroy");
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t* packed, float* scales,
+                               void* stream) {
+    if (rows < 0 || K <= 0 || K % kGroup)
+        return fail(MMOE_ERR_INVALID_ARG, "rows=%lld K=%lld: rows >= 0 and K a positive multiple of 32",
+                    (long long)rows, (long long)K);
+    if (rows == 0) return MMOE_OK;
+    if (!w || !packed || !scales) return fail(MMOE_ERR_INVALID_ARG, "a pointer is NULL");
+    if ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(packed)) & 15)
+        return fail(MMOE_ERR_INVALID_ARG, "w and packed must be 16-byte aligned");
+    MMOE_CUDA(launch_quantize_int4(w, rows, K, packed, scales, reinterpret_cast<cudaStream_t>(stream)),
+              "quantize launch");
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_debug_copy_stage(mmoe_handle* h, int32_t stage, void* dst, size_t bytes, void* stream) {
+    if (!h || !dst) return fail(MMOE_ERR_INVALID_ARG, "handle or dst is NULL");
+    if (h->last_T < 0) return fail(MMOE_ERR_INVALID_ARG, "no forward has run on this handle");
+    const int64_t T = h->last_T, k = h->cfg.top_k, E = h->cfg.n_experts, d = h->cfg.d_model;
+    const int64_t R = T * (k + 1);
+    const void* src = nullptr;
+    size_t have = 0;
+    switch (stage) {
+        case MMOE_STAGE_XQ: src = h->xq + T * k * d; have = (size_t)(T * d); break;
+        case MMOE_STAGE_SX: src = h->sx; have = (size_t)T * 4; break;
+        case MMOE_STAGE_OFFSETS: src = h->offsets; have = (size_t)(E + 2) * 4; break;
+        case MMOE_STAGE_ROW_SRC: src = h->row_src; have = (size_t)R * 4; break;
+        case MMOE_STAGE_SLOT_ROW: src = h->slot_row; have = (size_t)(T * k) * 4; break;
+        case MMOE_STAGE_HQ: src = h->hq; have = (size_t)(R * h->hmax); break;
+        case MMOE_STAGE_SH: src = h->sh; have = (size_t)R * 4; break;
+        case MMOE_STAGE_LOGITS: src = h->logits; have = (size_t)(T * E) * 4; break;
+        default: return fail(MMOE_ERR_INVALID_ARG, "stage %d: unknown", stage);
+    }
+    if (bytes > have) return fail(MMOE_ERR_INVALID_ARG, "stage %d holds %zu bytes, asked for %zu", stage, have, bytes);
+    DeviceGuard dg(h->device);
+    MMOE_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, reinterpret_cast<cudaStream_t>(stream)),
+              "copy stage");
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int64_t nrows, int32_t* dst,
+                                void* stream) {
+    if (!h || !dst) return fail(MMOE_ERR_INVALID_ARG, "handle or dst is NULL");
+    if (!h->loaded) return fail(MMOE_ERR_NOT_LOADED, "no weights loaded");
+    if (h->last_T <= 0) return fail(MMOE_ERR_INVALID_ARG, "no forward with T > 0 has run on this handle");
+    const int64_t R = h->last_T * (h->cfg.top_k + 1);
+    if (which != 0 && which != 1) return fail(MMOE_ERR_INVALID_ARG, "which=%d: must be 0 or 1", which);
+    if (row0 < 0 || nrows < 0 || row0 + nrows > R)
+        return fail(MMOE_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, %lld)", (long long)row0,
+                    (long long)(row0 + nrows), (long long)R);
+    DeviceGuard dg(h->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Plan p = make_plan(h, nullptr, h->last_T, nullptr);
+    if (which == 0) MMOE_CUDA(launch_gate_up(p, s, dst, row0, nrows), "gate/up dump launch");
+    else MMOE_CUDA(launch_down(p, s, dst, row0, nrows), "down dump launch");
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_profile_enable(mmoe_handle* h, int32_t enable) {
+    if (!h) return fail(MMOE_ERR_INVALID_ARG, "handle is NULL");
+    DeviceGuard dg(h->device);
+    if (enable) {
+        for (auto& r : h->prof) {
+            h->ev_pool.push_back(r.a);
+            h->ev_pool.push_back(r.b);
+        }
+        h->prof.clear();
+        for (int i = 0; i < MMOE_PROF_STAGES; ++i) {
+            h->prof_launches[i] = 0;
+            h->prof_ms[i] = 0.0;
+        }
+    }
+    h->prof_on = enable != 0;
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_ms, int32_t n) {
+    if (!h || !launches || !total_ms || n < 1) return fail(MMOE_ERR_INVALID_ARG, "bad arguments");
+    DeviceGuard dg(h->device);
+    for (auto& r : h->prof) {
+        MMOE_CUDA(cudaEventSynchronize(r.b), "profile event wait");
+        float ms = 0.0f;
+        MMOE_CUDA(cudaEventElapsedTime(&ms, r.a, r.b), "profile elapsed time");
+        h->prof_launches[r.stage] += r.launches;
+        h->prof_ms[r.stage] += ms;
+        h->ev_pool.push_back(r.a);
+        h->ev_pool.push_back(r.b);
+    }
+    h->prof.clear();
+    for (int i = 0; i < n; ++i) {
+        launches[i] = i < MMOE_PROF_STAGES ? h->prof_launches[i] : 0;
+        total_ms[i] = i < MMOE_PROF_STAGES ? h->prof_ms[i] : 0.0;
+    }
+    return MMOE_OK;
+}
+
+}  // extern "C"

@@ -97,6 +97,7 @@ int oracle_quantize_int4(const float* W, int64_t rows, int64_t K, uint8_t* packe
 {
     if (K % ORACLE_GROUP) return -1;
     int64_t ng = K / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         const float* w = W + r * K;
         uint8_t* p = packed + r * (K / 2);
@@ -209,14 +210,20 @@ static void router_token(const oracle_layer* L, const float* xf, float* logits, 
 int oracle_router(const oracle_layer* L, const uint16_t* x, int64_t T, float* logits, float* probs,
                   int32_t* idx, float* gate)
 {
-    float* xf = (float*)malloc((size_t)L->d * sizeof(float));
-    if (!xf) return -1;
-    for (int64_t t = 0; t < T; ++t) {
-        for (int64_t i = 0; i < L->d; ++i) xf[i] = bf16_to_f32(x[t * L->d + i]);
-        router_token(L, xf, logits + t * L->E, probs + t * L->E, idx + t * L->k, gate + t * L->k);
+    int err = 0;
+#pragma omp parallel reduction(| : err)
+    {
+        float* xf = (float*)malloc((size_t)L->d * sizeof(float));
+        if (!xf) err |= 1;
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            if (!xf) continue;
+            for (int64_t i = 0; i < L->d; ++i) xf[i] = bf16_to_f32(x[t * L->d + i]);
+            router_token(L, xf, logits + t * L->E, probs + t * L->E, idx + t * L->k, gate + t * L->k);
+        }
+        free(xf);
     }
-    free(xf);
-    return 0;
+    return err ? -1 : 0;
 }
 
 /* Byte / element offsets of expert g's blocks (expert E is the shared one and

@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle.
+
+Bit-exact: Eq. (6) codes and scales, activation codes and scales, routing
+(outside the 1e-5 router-margin band), counts, offsets, the permutation and
+every INT32 group partial.  Within tolerance: gates (relative error at most
+twice the largest logit difference plus 1e-6), SwiGLU
+codes (equal or one apart near a rounding boundary) and y
+(max|dy| <= 2e-3 max|y_ref|)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_ffn_layer_fp32_b200 import _lib, synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def workload(name):
+    if name not in _CACHE:
+        w = synth.WORKLOADS[name]
+        q = oracle.quantize_layer(synth.workload_layer(w))
+        _CACHE[name] = (w, q)
+    return _CACHE[name]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    gu.ensure_built()
+
+
+# ---------------------------------------------------------------------------
+def test_quantizer_matches_oracle_bit_exact():
+    from moe_ffn_layer_fp32_b200.layer import quantize_int4
+    rng = np.random.default_rng(0)
+    W = (rng.standard_normal((513, 512)) * 0.02).astype(np.float32)
+    W[7] = 0.0
+    W[8, :32] = np.float32(7.5) * np.float32(2.0 ** -6)
+    W[9, 5] = 1e-30
+    W[10] = rng.standard_normal(512).astype(np.float32) * 1e4
+    for name in ("eq6_int4_cases.txt",):
+        from tests.conftest import read_cases
+        for i, c in enumerate(read_cases(name)):
+            W[20 + i, :32] = c["w"].astype(np.float32)
+    p_gpu, s_gpu = quantize_int4(torch.from_numpy(W).cuda())
+    p_ref, s_ref = oracle.quantize_int4(W)
+    assert np.array_equal(p_gpu.cpu().numpy(), p_ref)
+    assert np.array_equal(s_gpu.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None):
+    T = x.shape[0]
+    L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic)
+    out = gu.run_gpu(L, q, x)
+    y, D = oracle.moe_layer(q, x, dumps=True)
+    rep = {}
+    assert np.array_equal(out["xq"], D["xq"]) and np.array_equal(out["sx"].view(np.uint32), D["sx"].view(np.uint32))
+    assert np.max(np.abs(out["logits"] - D["logits"])) <= 1e-5 * max(1.0, np.abs(D["logits"]).max())
+    gu.check_routing_and_permutation(q, out, D["idx"], D["gate"], D["probs"], rep, D["logits"])
+    gu.check_hq(q, out, D, rep)
+    gu.check_y(out["y"], y, rep)
+    if partial_rows is not None:
+        gu.check_partials(L, q, out, partial_rows)
+    L.close()
+    return rep, out
+
+
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_c0_all_stages(deterministic):
+    w, q = workload("c0")
+    x = synth.workload_x(w)
+    R = w.T * (q.k + 1)
+    rep, out = _full_check(q, x, deterministic, partial_rows=range(0, R, 3))
+    print("c0", rep)
+
+
+def test_deterministic_mode_is_reproducible():
+    w, q = workload("c0")
+    x = synth.workload_x(w)
+    L = gu.make_gpu_layer(q, w.T, deterministic=True)
+    a = gu.run_gpu(L, q, x, stages=False)["y"]
+    b = gu.run_gpu(L, q, x, stages=False)["y"]
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+@pytest.mark.parametrize("T", [1, 2, 7, 31, 33, 63, 65, 129, 300])
+def test_ragged_token_counts(T):
+    w, q = workload("c0")
+    x = synth.draw_x(T, w.d, seed=100 + T)
+    rep, out = _full_check(q, x, max_tokens=512)
+    assert out["counts"][q.E] == T
+
+
+def test_T0_is_a_noop():
+    w, q = workload("c0")
+    L = gu.make_gpu_layer(q, 8)
+    y = torch.full((1, w.d), 7.0, device="cuda")
+    L.forward(torch.zeros((0, w.d), dtype=torch.bfloat16, device="cuda"), y[:0])
+    torch.cuda.synchronize()
+    assert torch.all(y == 7.0)
+
+
+def test_skewed_routing_empty_and_hot_experts():
+    # a bias that sends every token to experts 5, 9, 33, 58: 56 experts get no rows
+    w = synth.WORKLOADS["c0"]
+    lw = synth.draw_layer(w.d, w.h, seed=40, bias_coef=None)
+    lw.router_bias = np.full(60, -30.0, np.float32)
+    lw.router_bias[[5, 9, 33, 58]] = 0.0
+    q = oracle.quantize_layer(lw)
+    x = synth.draw_x(200, w.d, seed=41)
+    rep, out = _full_check(q, x, partial_rows=[0, 199, 200, 799, 800, 999])
+    assert sorted(np.nonzero(out["counts"][:60])[0].tolist()) == [5, 9, 33, 58]
+
+
+def test_sigmoid_topk_normalised_gating():
+    w = synth.WORKLOADS["c0"]
+    q = oracle.quantize_layer(synth.workload_layer(w), gating=1)
+    x = synth.workload_x(w)
+    rep, out = _full_check(q, x)
+    assert np.allclose(out["gate"].sum(axis=1), 1.0, atol=1e-6)
+
+
+def test_shared_expert_wider_than_routed():
+    # MobileMoE's shared expert is 4x a routed expert (final-architecture paragraph)
+    lw = synth.draw_layer(256, 64, seed=42, shared_hidden=256)
+    q = oracle.quantize_layer(lw)
+    x = synth.draw_x(70, 256, seed=43)
+    rep, out = _full_check(q, x, partial_rows=[0, 100, 279, 280, 349])
+
+
+def test_forward_host_matches_device():
+    w, q = workload("c0")
+    x = synth.workload_x(w)
+    L = gu.make_gpu_layer(q, w.T, deterministic=True)
+    a = gu.run_gpu(L, q, x, stages=False)["y"]
+    b = L.forward_host(x)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_errors_on_device():
+    w, q = workload("c0")
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    L = MoELayer(q.d, q.h, max_tokens=8)
+    x = torch.zeros((4, w.d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(_lib.MMoEError) as ei:
+        L.forward(x)
+    assert ei.value.status == 2  # NOT_LOADED
+    L.load(q.w_router, q.router_bias, q.w_gate_up, q.s_gate_up, q.w_down, q.s_down)
+    with pytest.raises(_lib.MMoEError) as ei:
+        L.forward(torch.zeros((9, w.d), dtype=torch.bfloat16, device="cuda"))
+    assert ei.value.status == 1
+    L.forward(x)
+    with pytest.raises(_lib.MMoEError):
+        L.stage(_lib.STAGE_SX, (9,), torch.float32)
+    with pytest.raises(_lib.MMoEError):
+        L.partials(0, 0, 100)
+
+
+# --- the benchmark workloads ------------------------------------------------
+def test_c1_decode_layers():
+    w = synth.WORKLOADS["c1"]
+    for layer in (0, 23):
+        q = oracle.quantize_layer(synth.workload_layer(w, layer))
+        for T in (1, 8):
+            x = synth.workload_x(w, step=layer, T=T)
+            rep, _ = _full_check(q, x, max_tokens=64)
+            print("c1 layer", layer, "T", T, rep)
+
+
+def test_c2_prefill():
+    w, q = workload("c2")
+    x = synth.workload_x(w)
+    rep, out = _full_check(q, x, partial_rows=[0, 1, 4095, 8191, 8192, 10239])
+    print("c2", rep)
+
+
+def _sampled_check(name, n_sample=192, T=None):
+    w, q = workload(name)
+    T = w.T if T is None else T
+    x = synth.workload_x(w, T=T)
+    L = gu.make_gpu_layer(q, T)
+    out = gu.run_gpu(L, q, x)
+    rep = {}
+    logits, probs, idx, gate = oracle.router(q, x)
+    assert np.max(np.abs(out["logits"] - logits)) <= 1e-5 * max(1.0, np.abs(logits).max())
+    gu.check_routing_and_permutation(q, out, idx, gate, probs, rep, logits)
+    xq, sx = oracle.quantize_act(x)
+    assert np.array_equal(out["xq"], xq) and np.array_equal(out["sx"], sx)
+    rng = np.random.default_rng(7)
+    toks = np.unique(np.concatenate([rng.choice(T, size=min(n_sample, T), replace=False), [0, T - 1]]))
+    yref = oracle.moe_tokens(q, x, toks)
+    gu.check_y(out["y"], yref, rep, rows=toks)
+    R = T * (q.k + 1)
+    gu.check_partials(L, q, out, [0, R // 3, T * q.k - 1, T * q.k, R - 1])
+    L.close()
+    return rep, out
+
+
+@pytest.mark.parametrize("name", ["c3a", "c3b"])
+def test_c3_skewed_prefill(name):
+    rep, out = _sampled_check(name)
+    print(name, rep, "counts", out["counts"].tolist())
+    if name == "c3a":
+        assert (out["counts"][:60] == 0).sum() > 0, "the literal 1.5 bias leaves experts without tokens"
+
+
+def test_c4_prefill_sampled():
+    rep, out = _sampled_check("c4")
+    print("c4", rep)
+
+
+def test_c4_decode_batch64():
+    w, q = workload("c4dec")
+    x = synth.workload_x(w)
+    rep, out = _full_check(q, x, partial_rows=[0, 63, 255, 256, 319])
+    print("c4dec", rep)
