@@ -217,6 +217,41 @@ enum {
 mmoe_status mmoe_profile_enable(mmoe_handle* h, int32_t enable);
 mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_ms, int32_t n);
 
+/* ---- forward without any allocation --------------------------------------
+ * The paper has no counterpart to this entry point; it serves callers that
+ * must not allocate device memory on their own: a host framework that owns
+ * all of the GPU's memory through its own pool and hands an operator only the
+ * buffers it passes, or a serving loop that may not block on (or fail in)
+ * cudaMalloc once it runs.  mmoe_create allocates its workspace and weight
+ * copies, so those callers cannot use a handle.
+ *
+ * This call runs the same layer as mmoe_forward on weights the caller keeps
+ * on the device in the interchange layout (mmoe_weights, on_device = 1,
+ * read in place: nothing is copied or re-tiled), with x and y as in
+ * mmoe_forward.  All intermediate data lives in one array that the library
+ * declares at file scope in device memory, MMOE_STATIC_SCRATCH_BYTES long;
+ * every GPU that loads the library holds that array until the process exits.
+ *   - Size limit: the scratch a call needs grows with T, d_model, the hidden
+ *     sizes and top_k (about T*(top_k+1)*(d_model + 5*max_hidden) bytes, plus
+ *     T*(top_k+1)*d_model*4 more with MMOE_FLAG_DETERMINISTIC); a call that
+ *     needs more than the array holds is rejected with MMOE_ERR_INVALID_ARG
+ *     before anything is launched.  cfg->max_tokens is not used.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - Sharing: every call on a device uses the same array and leaves its
+ *     contents behind.  Each kernel writes every scratch word it later reads,
+ *     so nothing needs clearing between calls, but calls whose work overlaps
+ *     on the GPU (different streams, or different host threads) race on the
+ *     array and corrupt each other's results: order them on one stream.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ * Errors: INVALID_ARG (bad config, NULL or host weight pointers, T < 0, the
+ * scratch limit), CUDA. */
+#define MMOE_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weights* w, const uint16_t* x_bf16,
+                                        int64_t T, float* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,9 @@ STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAG
 # every symbol include/mmoe.h declares
 EXPORTS = ("mmoe_create", "mmoe_load_quantized_weights", "mmoe_forward", "mmoe_forward_host", "mmoe_destroy",
            "mmoe_last_error", "mmoe_quantize_int4", "mmoe_debug_copy_stage", "mmoe_debug_partials",
-           "mmoe_profile_enable", "mmoe_profile_read")
+           "mmoe_profile_enable", "mmoe_profile_read", "mmoe_forward_static_scratch")
+
+STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 PROF_STAGES = ("zero_y", "router", "permute", "gate_up", "requant", "down", "combine", "unused")
 
@@ -72,6 +74,7 @@ def lib() -> C.CDLL:
     L.mmoe_debug_partials.argtypes = [vp, i32, i64, i64, vp, vp]
     L.mmoe_profile_enable.argtypes = [vp, i32]
     L.mmoe_profile_read.argtypes = [vp, vp, vp, i32]
+    L.mmoe_forward_static_scratch.argtypes = [C.POINTER(Config), C.POINTER(Weights), vp, i64, vp, vp]
     for name in EXPORTS:
         if name != "mmoe_last_error":
             getattr(L, name).restype = st

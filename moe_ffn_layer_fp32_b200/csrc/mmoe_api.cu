@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -219,6 +220,61 @@ cudaError_t run_stage(mmoe_handle* h, int stage, int launches, cudaStream_t s, F
     }
     h->prof.push_back({stage, launches, a, b});
     return cudaSuccess;
+}
+
+// Scratch of mmoe_forward_static_scratch: one array per device, alive for the
+// whole process.  Host code must not use its name as a device address; it
+// reaches the kernels only through the address cudaGetSymbolAddress returns.
+static __device__ __align__(256) unsigned char g_static_scratch[MMOE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device (looked up once per device).
+mmoe_status static_scratch_address(int dev, unsigned char** out) {
+    if (dev < 0 || dev >= kMaxDevices) return fail(MMOE_ERR_INVALID_ARG, "device %d: unsupported index", dev);
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void* a = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&a, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+        g_static_addr[dev] = a;
+    }
+    *out = static_cast<unsigned char*>(g_static_addr[dev]);
+    return MMOE_OK;
+}
+
+// Lays the forward's intermediate buffers out in [base, base + cap); returns
+// the bytes needed (more than cap means the call does not fit).
+size_t carve_static_plan(Plan& p, unsigned char* base, size_t cap) {
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> void* {
+        off = (off + 255) & ~size_t(255);
+        void* q = off + bytes <= cap ? static_cast<void*>(base + off) : nullptr;
+        off += bytes;
+        return q;
+    };
+    const size_t R = (size_t)p.R, T = (size_t)p.T, d = (size_t)p.d, k = (size_t)p.k, E = (size_t)p.E;
+    p.xq = static_cast<int8_t*>(take(R * d));
+    p.sx = static_cast<float*>(take(T * 4));
+    p.logits = static_cast<float*>(take(T * E * 4));
+    p.idx = static_cast<int32_t*>(take(T * k * 4));
+    p.gate = static_cast<float*>(take(T * k * 4));
+    p.chunk_cnt = static_cast<int32_t*>(take((size_t)p.nchunks * kMaxExperts * 4));
+    p.chunk_base = static_cast<int32_t*>(take((size_t)p.nchunks * kMaxExperts * 4));
+    p.offsets = static_cast<int32_t*>(take((E + 2) * 4));
+    p.counts = static_cast<int32_t*>(take((E + 1) * 4));
+    p.tiles = static_cast<int32_t*>(take((size_t)p.max_tiles * 4));
+    p.tile_count = static_cast<int32_t*>(take(4));
+    p.row_src = static_cast<int32_t*>(take(R * 4));
+    p.row_gate = static_cast<float*>(take(R * 4));
+    p.slot_row = static_cast<int32_t*>(take(T * k * 4));
+    p.act = static_cast<float*>(take(R * (size_t)p.hmax * 4));
+    p.hq = static_cast<int8_t*>(take(R * (size_t)p.hmax));
+    p.sh = static_cast<float*>(take(R * 4));
+    p.obuf = p.deterministic ? static_cast<float*>(take(R * d * 4)) : nullptr;
+    return off;
 }
 
 }  // namespace
@@ -482,6 +538,68 @@ mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_m
         launches[i] = i < MMOE_PROF_STAGES ? h->prof_launches[i] : 0;
         total_ms[i] = i < MMOE_PROF_STAGES ? h->prof_ms[i] : 0.0;
     }
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weights* w, const uint16_t* x,
+                                        int64_t T, float* y, void* stream) {
+    mmoe_status st = check_config(cfg);
+    if (st != MMOE_OK) return st;
+    if (!w || !w->w_router || !w->w_gate_up || !w->s_gate_up || !w->w_down || !w->s_down)
+        return fail(MMOE_ERR_INVALID_ARG, "weights or a weight pointer is NULL");
+    if (w->on_device != 1) return fail(MMOE_ERR_INVALID_ARG, "weights must be device pointers (on_device = 1)");
+    if (cfg->has_router_bias && !w->router_bias)
+        return fail(MMOE_ERR_INVALID_ARG, "the config has a router bias but router_bias is NULL");
+    if (T < 0) return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be >= 0", (long long)T);
+    if (T == 0) return MMOE_OK;
+    if (!x || !y) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
+
+    Plan p{};
+    p.d = cfg->d_model;
+    p.h = cfg->expert_hidden;
+    p.hs = cfg->shared_hidden;
+    p.hmax = p.h > p.hs ? p.h : p.hs;
+    p.E = cfg->n_experts;
+    p.k = cfg->top_k;
+    p.gating = cfg->gating;
+    p.T = T;
+    p.Tk = T * p.k;
+    p.R = T * (p.k + 1);
+    p.deterministic = (cfg->flags & MMOE_FLAG_DETERMINISTIC) != 0;
+    p.w_router = w->w_router;
+    p.router_bias = cfg->has_router_bias ? w->router_bias : nullptr;
+    p.w_gate_up = w->w_gate_up;
+    p.s_gate_up = w->s_gate_up;
+    p.w_down = w->w_down;
+    p.s_down = w->s_down;
+    p.x = x;
+    p.y = y;
+    p.max_tiles = max_tiles_for(T, p.k, p.E);
+    p.nchunks = (int)((p.Tk + kChunk - 1) / kChunk);
+
+    // size check first (no device needed), then the one-time address lookup
+    Plan probe = p;
+    const size_t need = carve_static_plan(probe, nullptr, 0);
+    if (need > MMOE_STATIC_SCRATCH_BYTES)
+        return fail(MMOE_ERR_INVALID_ARG,
+                    "T=%lld needs %zu bytes of scratch; the static scratch array holds %u bytes "
+                    "(use fewer tokens per call)",
+                    (long long)T, need, (unsigned)MMOE_STATIC_SCRATCH_BYTES);
+    int dev = 0;
+    MMOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    unsigned char* base = nullptr;
+    st = static_scratch_address(dev, &base);
+    if (st != MMOE_OK) return st;
+    carve_static_plan(p, base, MMOE_STATIC_SCRATCH_BYTES);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!p.deterministic) MMOE_CUDA(cudaMemsetAsync(y, 0, (size_t)T * p.d * sizeof(float), s), "zero y");
+    MMOE_CUDA(launch_router_quant(p, s), "router/quantiser launch");
+    MMOE_CUDA(launch_permute(p, s), "permute launch");
+    MMOE_CUDA(launch_gate_up(p, s, nullptr, 0, 0), "gate/up launch");
+    MMOE_CUDA(launch_requant(p, s), "requant launch");
+    MMOE_CUDA(launch_down(p, s, nullptr, 0, 0), "down launch");
+    if (p.deterministic) MMOE_CUDA(launch_combine(p, s), "combine launch");
     return MMOE_OK;
 }
 

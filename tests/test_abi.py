@@ -76,3 +76,18 @@ def test_create_without_a_device_is_an_error_not_a_crash(L):
     h = C.c_void_p()
     assert L.mmoe_create(C.byref(valid_cfg()), 0, C.byref(h)) == 1
     assert b"device" in L.mmoe_last_error()
+
+
+def test_static_scratch_forward_validates_before_any_device_work(L):
+    cfg = valid_cfg(d_model=2048, expert_hidden=1024, shared_hidden=1024)
+    fake = C.c_void_p(0x1000)
+    w = _lib.Weights(fake, None, fake, fake, fake, fake, 1)
+    # too many tokens for the static array: rejected before touching a device
+    st = L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, 100000, fake, None)
+    assert st == 1 and b"static scratch" in L.mmoe_last_error()
+    # host weights are refused (nothing is copied)
+    wh = _lib.Weights(fake, None, fake, fake, fake, fake, 0)
+    assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(wh), fake, 1, fake, None) == 1
+    assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, -1, fake, None) == 1
+    assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, 0, fake, None) == 0
+    assert L.mmoe_forward_static_scratch(None, C.byref(w), fake, 1, fake, None) == 1
