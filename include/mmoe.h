@@ -66,6 +66,9 @@ typedef enum {
 /* mmoe_config.flags */
 #define MMOE_FLAG_DETERMINISTIC 1u /* combine in a fixed order: y = FFN_s + g_0 FFN_0 + ... + g_{k-1} FFN_{k-1};
                                       needs an extra [max_tokens*(k+1), d_model] FP32 workspace */
+#define MMOE_FLAG_CUDA_CORES 2u    /* run the expert GEMMs on CUDA cores (dp4a) even where the tensor-core
+                                      kernels apply (those need d_model and both hidden sizes to be
+                                      multiples of 128); same results, slower */
 
 typedef struct {
     int32_t d_model;        /* multiple of 32, 64 <= d_model <= 8192 */

@@ -18,6 +18,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NOT_LOADED", 3: "OOM", 4: "CUDA",
 GATE_SOFTMAX = 0
 GATE_SIGMOID_TOPK_NORM = 1
 FLAG_DETERMINISTIC = 1
+FLAG_CUDA_CORES = 2
 
 STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAGE_SH, STAGE_LOGITS = range(8)
 

@@ -1,0 +1,593 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, kind::i8).
+//
+// MobileMoE pages (paper-archivist reading): every expert runs its contiguous
+// token slice as one batched matmul, gate and up projections in one GEMM per
+// expert, then SwiGLU, the down projection and the weighted scatter back to
+// token order (section "custom MoE kernel"); weights are symmetric group-32
+// INT4 with FP32 scales (Eq. (6)), activations INT8 (section "QAT").
+//
+// One CTA computes a 128 x 128 tile: 128 weight rows (M) x 128 token rows
+// (N), over the whole K range.
+//   gate/up: the 128 weight rows are 64 gate rows and the 64 up rows of the
+//            same 64 hidden features, so one MMA per K group yields both
+//            halves of SwiGLU; K = d_model.
+//   down:    128 output features; K = hidden size of the group's expert.
+// Pipeline (one CTA per SM, 12 warps):
+//   warp 0      producer: 1-D bulk copy of the packed INT4 weight tile
+//               (pre-tiled at load time, 8 KB per 128-K stage) and a 2-D TMA
+//               load (128B swizzle) of the 128 x 128 INT8 activation tile;
+//   warp 1      allocates TMEM; one elected lane issues tcgen05.mma
+//               (M=128, N=128, K=32, INT8 x INT8 -> INT32), one instruction
+//               per 32-element K group, each into a fresh TMEM buffer
+//               (4 buffers of 128 columns), and commits to mbarriers;
+//   warps 2-3   unpack INT4 -> INT8 into the canonical K-major SW128 layout;
+//   warps 4-11  promotion: read each group's INT32 partials from TMEM and
+//               accumulate acc = fma(float(P_j), s_j, acc) in registers
+//               (2 warpgroups x 64 token columns, one weight row per thread),
+//               then the epilogue.
+// The exact INT32 group partial is needed because every 32-element group of K
+// has its own FP32 weight scale; the promotion order (j ascending, fused
+// multiply-add) is the oracle's, so the FP32 result is identical to it.
+// Every mbarrier wait is bounded by wall time; a wait that gives up raises
+// the handle's error flag and the CTA drains and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "mmoe_internal.cuh"
+
+namespace mmoe {
+namespace tc {
+
+constexpr int BM = 128;                    // weight rows per tile
+constexpr int BN = kTcTileRows;            // token rows per tile (128)
+constexpr int BK = 128;                    // K elements (bytes of INT8) per stage
+constexpr int kStages = 4;
+constexpr int kBufs = 4;                   // TMEM accumulator buffers, 128 columns each
+constexpr int kThreads = 384;
+constexpr int kPromoThreads = 256;
+constexpr int kUnpackThreads = 64;
+constexpr int kAPackedBytes = BM * BK / 2; // 8 KB
+constexpr int kAI8Bytes = BM * BK;         // 16 KB
+constexpr int kBBytes = BN * BK;           // 16 KB
+constexpr int kStageBytes = kAI8Bytes + kBBytes + kAPackedBytes;
+constexpr int kXchBytes = 64 * BN * 4;     // up-projection values handed to the gate threads
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+enum Epi { kEpiSwiGLU = 0, kEpiCombine = 1 };
+
+struct Smem {
+    // stage buffers are carved from the 1024-aligned base: [A_i8 | B | A_packed] x kStages
+    uint64_t full[kStages];
+    uint64_t unpacked[kStages];
+    uint64_t empty[kStages];
+    uint64_t accf[kBufs];
+    uint64_t acce[kBufs];
+    uint32_t tmem_base;
+    int abort;
+    float colf[BN];      // per token column: activation scale (gate/up) or SwiGLU scale (down)
+    float colg[BN];      // per token column: gate of the row (down)
+    int colrow[BN];      // per token column: token id (down)
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(su32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase of the given parity; gives up after kTimeoutNs or once
+// another thread of the CTA has given up.  Returns false on giving up.
+// On giving up it records `where` in the device flag (read by every later CTA,
+// which then exits at once) and in the host-visible flag.
+struct ErrFlags {
+    int* dev;
+    int* host;
+};
+
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem* sm, ErrFlags err, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*reinterpret_cast<volatile int*>(&sm->abort)) return false;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            atomicExch(&sm->abort, 1);
+            if (err.dev) *reinterpret_cast<volatile int*>(err.dev) = where;
+            if (err.host) *reinterpret_cast<volatile int*>(err.host) = where;
+            __threadfence_system();
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     su32(dst)),
+                 "l"(src), "r"(bytes), "r"(su32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major operand in the 128-byte swizzle layout: 8-row core groups 1024 B apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+    const uint64_t a = (su32(p) >> 4) & 0x3fff;
+    return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// kind::i8: signed A and B, S32 accumulator, both K-major, M = 128, N = BN.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(0)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// exact int32 -> float for |v| < 2^22: integer add into the mantissa of 1.5 * 2^23
+__device__ __forceinline__ float exact_i2f(int32_t v) { return __int_as_float(v + 0x4B400000) - 12582912.0f; }
+
+// 8 packed nibbles stored as [v0 v4 v1 v5 v2 v6 v3 v7] -> signed bytes (v0..v3), (v4..v7)
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t l = w & 0x0f0f0f0fu, h = (w >> 4) & 0x0f0f0f0fu;
+    lo = l | ((l & 0x08080808u) * 0x1eu);
+    hi = h | ((h & 0x08080808u) * 0x1eu);
+}
+
+struct TcArgs {
+    const uint8_t* wtiles;  // pre-tiled packed weights of the expert kind (gate/up or down)
+    const float* stiles;    // pre-tiled group scales
+    int64_t w_expert_stride_tiles;  // tiles (of kAPackedBytes) per routed expert
+    int mblocks_routed;     // weight-row blocks of a routed expert (gate/up: h/64, down: d/128)
+    int mblocks_shared;
+    int ks_routed;          // K stages of a routed expert (gate/up: d/128, down: h/128)
+    int ks_shared;
+    int32_t* dump;          // optional INT32 partial dump
+    int64_t drow0, dnrows;
+};
+
+// Bounded wait used while draining after an abort: ignores the abort flag,
+// gives up only on time.
+__device__ __noinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kTimeoutNs) return;
+}
+
+// --------------------------------------------------------------- the kernel
+template <int kEpi, bool kDump>
+__global__ void __launch_bounds__(kThreads, 1)
+expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = base;
+    float* xch = reinterpret_cast<float*>(base + kStages * kStageBytes);
+    Smem* sm = reinterpret_cast<Smem*>(base + kStages * kStageBytes + kXchBytes);
+
+    // ---- tile -> (group, rows, weight block); nothing to do after an earlier wait gave up
+    if ((int)blockIdx.y >= *p.tile_count) return;
+    if (p.err && *reinterpret_cast<volatile int*>(p.err)) return;
+    const ErrFlags ef{p.err, p.err_host};
+    const int code = p.tiles[blockIdx.y];
+    const int g = code >> 24;
+    const int ti = code & 0xffffff;
+    const bool shared_grp = g == p.E;
+    const int mblocks = shared_grp ? a.mblocks_shared : a.mblocks_routed;
+    const int mb = blockIdx.x;
+    if (mb >= mblocks) return;
+    const int nks = shared_grp ? a.ks_shared : a.ks_routed;
+    const int ng = nks * (BK / kGroup);
+    const int cnt = p.offsets[g + 1] - p.offsets[g];
+    const int64_t row0 = (int64_t)p.offsets[g] + (int64_t)ti * BN;
+    const int nr = min(BN, cnt - ti * BN);
+    const int64_t tile0 = (int64_t)g * a.w_expert_stride_tiles + (int64_t)mb * nks;  // first weight tile
+    const uint8_t* wsrc = a.wtiles + tile0 * kAPackedBytes;
+    const float* ssrc = a.stiles + tile0 * (BK / kGroup) * BM;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm->full[s], 1);
+            mbar_init(&sm->unpacked[s], kUnpackThreads);
+            mbar_init(&sm->empty[s], 1);
+        }
+        for (int b = 0; b < kBufs; ++b) {
+            mbar_init(&sm->accf[b], 1);
+            mbar_init(&sm->acce[b], kPromoThreads);
+        }
+        sm->abort = 0;
+        fence_barrier_init();
+    }
+    // per-column data of the token tile
+    for (int c = tid; c < BN; c += kThreads) {
+        const int64_t r = row0 + (c < nr ? c : 0);
+        if (kEpi == kEpiSwiGLU) {
+            sm->colf[c] = p.sx[p.row_src[r]];
+        } else {
+            sm->colf[c] = p.sh[r];
+            sm->colg[c] = p.row_gate[r];
+            sm->colrow[c] = p.row_src[r];
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&sm->tmem_base)),
+                     "r"(kBufs * 128)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_before_sync();
+    }
+    __syncthreads();
+    tc_after_sync();
+    const uint32_t tmem = sm->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int ks = 0; ks < nks; ++ks) {
+                const int s = ks % kStages;
+                if (ks >= kStages && !mbar_wait(&sm->empty[s], ((ks / kStages) - 1) & 1, sm, ef, 1)) break;
+                uint8_t* st = stages + s * kStageBytes;
+                mbar_expect_tx(&sm->full[s], kAPackedBytes + kBBytes);
+                bulk_load(st + kAI8Bytes + kBBytes, wsrc + (int64_t)ks * kAPackedBytes, kAPackedBytes, &sm->full[s]);
+                tma_load_2d(st + kAI8Bytes, &bmap, ks * BK, (int)row0, &sm->full[s]);
+                issued = ks + 1;
+            }
+            // every issued copy has landed before the CTA may exit
+            for (int ks = issued > kStages ? issued - kStages : 0; ks < issued; ++ks)
+                mbar_wait_drain(&sm->full[ks % kStages], (ks / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            bool ok = true;
+            int last_j = -1;
+            for (int ks = 0; ks < nks && ok; ++ks) {
+                const int s = ks % kStages;
+                if (!mbar_wait(&sm->unpacked[s], (ks / kStages) & 1, sm, ef, 2)) { ok = false; break; }
+                tc_after_sync();
+                uint8_t* st = stages + s * kStageBytes;
+                const uint64_t ad = smem_desc_sw128(st);
+                const uint64_t bd = smem_desc_sw128(st + kAI8Bytes);
+                for (int jj = 0; jj < BK / kGroup; ++jj) {
+                    const int j = ks * (BK / kGroup) + jj;
+                    const int b = j % kBufs;
+                    if (j >= kBufs && !mbar_wait(&sm->acce[b], ((j / kBufs) - 1) & 1, sm, ef, 3)) { ok = false; break; }
+                    tc_after_sync();
+                    mma_i8(tmem + b * 128, ad + (uint64_t)(jj * 2), bd + (uint64_t)(jj * 2));
+                    mma_commit(&sm->accf[b]);
+                    last_j = j;
+                }
+                mma_commit(&sm->empty[s]);
+            }
+            // every MMA issued has completed before TMEM is released
+            if (last_j >= 0) mbar_wait_drain(&sm->accf[last_j % kBufs], (last_j / kBufs) & 1);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ INT4 -> INT8 unpack
+        const int t = tid - 64;
+        for (int ks = 0; ks < nks; ++ks) {
+            const int s = ks % kStages;
+            if (!mbar_wait(&sm->full[s], (ks / kStages) & 1, sm, ef, 4)) break;
+            uint8_t* st = stages + s * kStageBytes;
+            const uint8_t* src = st + kAI8Bytes + kBBytes;
+#pragma unroll
+            for (int i = 0; i < (BM * BK / 2 / 16) / kUnpackThreads; ++i) {
+                const int q = i * kUnpackThreads + t;   // 16-byte chunk of packed data (one K group of one row)
+                const int row = q >> 2, c = q & 3;
+                const uint4 w = *reinterpret_cast<const uint4*>(src + row * 64 + c * 16);
+                uint4 o0, o1;
+                unpack_word(w.x, o0.x, o0.y);
+                unpack_word(w.y, o0.z, o0.w);
+                unpack_word(w.z, o1.x, o1.y);
+                unpack_word(w.w, o1.z, o1.w);
+                uint8_t* rowp = st + row * 128;
+                *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = o0;
+                *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = o1;
+            }
+            fence_proxy_async();
+            mbar_arrive(&sm->unpacked[s]);
+        }
+    } else {
+        // ------------------------------------------------------------ promotion + epilogue
+        const int pw = warp - 4;            // 0..7
+        const int wg = pw >> 2;             // token-column half
+        const int quarter = warp & 3;       // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;  // weight row of this thread (0..127)
+        const int col0 = wg * 64;
+        float acc[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)col0;
+        float s_next = ng > 0 ? __ldg(ssrc + row) : 0.0f;
+        for (int j = 0; j < ng; ++j) {
+            const int b = j % kBufs;
+            const float s = s_next;
+            if (j + 1 < ng) s_next = __ldg(ssrc + (int64_t)(j + 1) * BM + row);
+            if (!mbar_wait(&sm->accf[b], (j / kBufs) & 1, sm, ef, 5)) break;
+            tc_after_sync();
+            int32_t v0[32], v1[32];
+            tmem_ld32(tl + b * 128, v0);
+            tmem_ld32(tl + b * 128 + 32, v1);
+            tmem_wait_ld();
+            tc_before_sync();
+            mbar_arrive(&sm->acce[b]);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                acc[c] = fmaf(exact_i2f(v0[c]), s, acc[c]);
+                acc[32 + c] = fmaf(exact_i2f(v1[c]), s, acc[32 + c]);
+            }
+            if (kDump) {
+                // INT32 partials of rows [drow0, drow0 + dnrows) for the inspection entry point
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const int cc = col0 + c;
+                    const int64_t grow = row0 + cc;
+                    if (cc >= nr || grow < a.drow0 || grow >= a.drow0 + a.dnrows) continue;
+                    const int32_t v = c < 32 ? v0[c & 31] : v1[c & 31];
+                    if (kEpi == kEpiSwiGLU) {
+                        const int f = mb * 64 + (row & 63);
+                        const int n = row < 64 ? f : p.hmax + f;
+                        a.dump[((grow - a.drow0) * 2 * p.hmax + n) * (p.d / kGroup) + j] = v;
+                    } else {
+                        const int m = mb * BM + row;
+                        a.dump[((grow - a.drow0) * p.d + m) * (p.hmax / kGroup) + j] = v;
+                    }
+                }
+            }
+        }
+        const bool aborted = *reinterpret_cast<volatile int*>(&sm->abort) != 0;
+        if (kEpi == kEpiSwiGLU) {
+            // rows 0..63: gate of feature mb*64 + row; rows 64..127: up of the same feature
+            const int named = 1 + wg;
+            if (row >= 64) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) xch[(col0 + c) * 64 + (row - 64)] = acc[c];
+            }
+            asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");
+            if (row < 64 && !aborted && !kDump) {
+                const int f = mb * 64 + row;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const int cc = col0 + c;
+                    if (cc >= nr) continue;
+                    const float sx = sm->colf[cc];
+                    const float gv = __fmul_rn(acc[c], sx);
+                    const float uv = __fmul_rn(xch[cc * 64 + row], sx);
+                    const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+                    p.act[(row0 + cc) * p.hmax + f] = __fmul_rn(silu, uv);
+                }
+            }
+        } else if (!aborted && !kDump) {
+            const int m = mb * BM + row;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const int cc = col0 + c;
+                if (cc >= nr) continue;
+                const float o = __fmul_rn(acc[c], sm->colf[cc]);
+                if (p.deterministic) {
+                    p.obuf[(row0 + cc) * p.d + m] = o;
+                } else {
+                    atomicAdd(p.y + (int64_t)sm->colrow[cc] * p.d + m, __fmul_rn(sm->colg[cc], o));
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kBufs * 128) : "memory");
+    }
+}
+
+// --------------------------------------------------------------- weight re-tiling (load time)
+// gate/up tile (g, fb, ks): 128 rows x 64 bytes; rows 0..63 gate rows fb*64.., rows 64..127 the up rows of the
+// same features; bytes [ks*64, ks*64+64) of each interchange row with every 32-bit word's nibbles reordered
+// to [v0 v4 v1 v5 v2 v6 v3 v7].  Scales (g, fb, j): 128 floats, one per tile row.
+__device__ __forceinline__ uint32_t interleave_nibbles(uint32_t w) {
+    uint32_t o = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o |= ((w >> (4 * i)) & 15u) << (8 * i);
+        o |= ((w >> (4 * (i + 4))) & 15u) << (8 * i + 4);
+    }
+    return o;
+}
+
+// one thread per 16-byte chunk of a tile row
+__global__ void retile_weights_kernel(const uint8_t* __restrict__ src, const float* __restrict__ ssrc,
+                                      uint8_t* __restrict__ dst, float* __restrict__ sdst, int E, int K_routed,
+                                      int K_shared, int rows_routed, int rows_shared, int gate_up, int h, int hs,
+                                      int64_t total_chunks)
+{
+    const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (q >= total_chunks) return;
+    // q -> (expert, tile, row, chunk)
+    const int64_t per_routed = (int64_t)rows_routed / BM * (K_routed / BK) * BM * 4;  // chunks of a routed expert
+    int g;
+    int64_t r;
+    if (q < per_routed * E) { g = (int)(q / per_routed); r = q % per_routed; }
+    else { g = E; r = q - per_routed * E; }
+    const int K = g < E ? K_routed : K_shared;
+    const int nks = K / BK;
+    const int chunk = (int)(r % 4);
+    const int trow = (int)((r / 4) % BM);
+    const int64_t tile = r / (4 * BM);  // mb * nks + ks
+    const int ks = (int)(tile % nks);
+    const int mb = (int)(tile / nks);
+    const int hid = g < E ? h : hs;
+    int64_t srow;  // row inside the expert's interchange block
+    if (gate_up) srow = trow < 64 ? (int64_t)mb * 64 + trow : (int64_t)hid + mb * 64 + (trow - 64);
+    else srow = (int64_t)mb * BM + trow;
+    // interchange block of expert g starts at g * (routed block size)
+    const int64_t src_rows_routed = gate_up ? 2 * (int64_t)h : (int64_t)rows_routed;
+    const int64_t src_row_bytes = K / 2;
+    const int64_t src_expert_bytes = src_rows_routed * ((int64_t)K_routed / 2);
+    const uint8_t* s = src + (int64_t)g * src_expert_bytes + srow * src_row_bytes + (int64_t)ks * 64 + chunk * 16;
+    const uint4 w = *reinterpret_cast<const uint4*>(s);
+    const uint4 o = make_uint4(interleave_nibbles(w.x), interleave_nibbles(w.y), interleave_nibbles(w.z),
+                               interleave_nibbles(w.w));
+    const int64_t dst_tiles_routed = (int64_t)rows_routed / BM * (K_routed / BK);
+    const int64_t dtile = (int64_t)g * dst_tiles_routed + tile;
+    reinterpret_cast<uint4*>(dst + dtile * kAPackedBytes + trow * 64)[chunk] = o;
+    // scale of group (ks*4 + chunk) of this row
+    const int64_t src_expert_scales = src_rows_routed * ((int64_t)K_routed / kGroup);
+    const float sc = ssrc[(int64_t)g * src_expert_scales + srow * (K / kGroup) + ks * 4 + chunk];
+    sdst[(dtile * 4 + chunk) * BM + trow] = sc;
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------ host side
+bool tc_supported(int d, int h, int hs) { return d % 128 == 0 && h % 128 == 0 && hs % 128 == 0; }
+
+size_t tc_smem_bytes() { return 1024 + tc::kStages * tc::kStageBytes + tc::kXchBytes + sizeof(tc::Smem); }
+
+cudaError_t launch_retile(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn, uint8_t* gu_t,
+                          float* sgu_t, uint8_t* dn_t, float* sdn_t, int d, int h, int hs, int E, cudaStream_t s) {
+    // gate/up: rows of a tile are 128 (64 features x 2); "rows" counted as 2*hid
+    const int64_t gu_chunks = ((int64_t)E * (2 * h / tc::BM) + (2 * hs / tc::BM)) * (d / tc::BK) * tc::BM * 4;
+    tc::retile_weights_kernel<<<(unsigned)((gu_chunks + 255) / 256), 256, 0, s>>>(gu, sgu, gu_t, sgu_t, E, d, d, 2 * h,
+                                                                                   2 * hs, 1, h, hs, gu_chunks);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t dn_chunks = ((int64_t)E * (h / tc::BK) + (hs / tc::BK)) * (d / tc::BM) * tc::BM * 4;
+    tc::retile_weights_kernel<<<(unsigned)((dn_chunks + 255) / 256), 256, 0, s>>>(dn, sdn, dn_t, sdn_t, E, h, hs, d, d,
+                                                                                   0, h, hs, dn_chunks);
+    return cudaGetLastError();
+}
+
+size_t tensor_map_bytes() { return sizeof(CUtensorMap); }
+
+cudaError_t make_tensor_map(void* map_, void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_stride) {
+    CUtensorMap* map = static_cast<CUtensorMap*>(map_);
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {inner_bytes, rows};
+    const cuuint64_t strides[1] = {row_stride};
+    const cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)tc::BN};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int kEpi, bool kDump>
+static cudaError_t launch_tc(const Plan& p, cudaStream_t s, const CUtensorMap* map, const tc::TcArgs& a, int gx) {
+    auto kern = tc::expert_gemm_tc_kernel<kEpi, kDump>;
+    const size_t smem = tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)gx, (unsigned)p.max_tiles);
+    kern<<<grid, tc::kThreads, smem, s>>>(*map, p, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate_up_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
+    if (p.T == 0) return cudaSuccess;
+    tc::TcArgs a{};
+    a.wtiles = p.w_gate_up_t;
+    a.stiles = p.s_gate_up_t;
+    a.mblocks_routed = p.h / 64;
+    a.mblocks_shared = p.hs / 64;
+    a.ks_routed = a.ks_shared = p.d / tc::BK;
+    a.w_expert_stride_tiles = (int64_t)a.mblocks_routed * a.ks_routed;
+    a.dump = dump;
+    a.drow0 = row0;
+    a.dnrows = nrows;
+    const int gx = p.hmax / 64;
+    const CUtensorMap* map = static_cast<const CUtensorMap*>(p.tmap_xq);
+    return dump ? launch_tc<tc::kEpiSwiGLU, true>(p, s, map, a, gx)
+                : launch_tc<tc::kEpiSwiGLU, false>(p, s, map, a, gx);
+}
+
+cudaError_t launch_down_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
+    if (p.T == 0) return cudaSuccess;
+    tc::TcArgs a{};
+    a.wtiles = p.w_down_t;
+    a.stiles = p.s_down_t;
+    a.mblocks_routed = a.mblocks_shared = p.d / tc::BM;
+    a.ks_routed = p.h / tc::BK;
+    a.ks_shared = p.hs / tc::BK;
+    a.w_expert_stride_tiles = (int64_t)a.mblocks_routed * a.ks_routed;
+    a.dump = dump;
+    a.drow0 = row0;
+    a.dnrows = nrows;
+    const int gx = p.d / tc::BM;
+    const CUtensorMap* map = static_cast<const CUtensorMap*>(p.tmap_hq);
+    return dump ? launch_tc<tc::kEpiCombine, true>(p, s, map, a, gx)
+                : launch_tc<tc::kEpiCombine, false>(p, s, map, a, gx);
+}
+
+}  // namespace mmoe

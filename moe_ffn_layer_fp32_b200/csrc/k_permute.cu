@@ -54,13 +54,13 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(Plan p)
             off[e] = o;
             tstart[e] = ts;
             o += tot[e];
-            ts += (tot[e] + kTileRows - 1) / kTileRows;
+            ts += (tot[e] + p.tile_rows - 1) / p.tile_rows;
         }
         tot[E] = (int)p.T;
         off[E] = o;             // = T*k
         off[E + 1] = o + (int)p.T;
         tstart[E] = ts;
-        ts += (int)((p.T + kTileRows - 1) / kTileRows);
+        ts += (int)((p.T + p.tile_rows - 1) / p.tile_rows);
         tstart[E + 1] = ts;
         *p.tile_count = ts;
     }

@@ -93,6 +93,17 @@ struct mmoe_handle {
     float* obuf = nullptr;
     uint16_t* x_stage = nullptr;
     float* y_stage = nullptr;
+    // tensor-core path: pre-tiled weights, tensor maps of xq / hq, error flag
+    bool use_tc = false;
+    uint8_t* w_gate_up_t = nullptr;
+    float* s_gate_up_t = nullptr;
+    uint8_t* w_down_t = nullptr;
+    float* s_down_t = nullptr;
+    alignas(64) unsigned char tmap_xq[128] = {};
+    alignas(64) unsigned char tmap_hq[128] = {};
+    int* err_host = nullptr;   // mapped pinned host memory; kernels write its device alias
+    int* err_host_dev = nullptr;
+    int* err_dev = nullptr;    // device memory copy read by every CTA
     // per-stage timing (mmoe_profile_*)
     struct ProfRec {
         int stage, launches;
@@ -118,9 +129,11 @@ void free_all(mmoe_handle* h) {
     void* ptrs[] = {h->w_router, h->router_bias, h->w_gate_up, h->s_gate_up, h->w_down, h->s_down,
                     h->xq, h->sx, h->logits, h->idx, h->gate, h->chunk_cnt, h->chunk_base, h->offsets,
                     h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
-                    h->sh, h->obuf, h->x_stage, h->y_stage};
+                    h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
+                    h->s_down_t, h->err_dev};
     for (void* p : ptrs)
         if (p) cudaFree(p);
+    if (h->err_host) cudaFreeHost(h->err_host);
 }
 
 mmoe_status check_config(const mmoe_config* c) {
@@ -144,7 +157,8 @@ mmoe_status check_config(const mmoe_config* c) {
         return fail(MMOE_ERR_INVALID_ARG, "gating=%d: unknown", c->gating);
     if (c->has_router_bias != 0 && c->has_router_bias != 1)
         return fail(MMOE_ERR_INVALID_ARG, "has_router_bias=%d: must be 0 or 1", c->has_router_bias);
-    if (c->flags & ~MMOE_FLAG_DETERMINISTIC) return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
+    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES))
+        return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
     return MMOE_OK;
 }
 
@@ -188,9 +202,38 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.hq = h->hq;
     p.sh = h->sh;
     p.obuf = h->obuf;
-    p.max_tiles = max_tiles_for(T, c.top_k, c.n_experts);
+    p.use_tc = h->use_tc;
+    p.tile_rows = p.use_tc ? kTcTileRows : kTileRows;
+    p.max_tiles = max_tiles_for(T, c.top_k, c.n_experts, p.tile_rows);
     p.nchunks = (int)((p.Tk + kChunk - 1) / kChunk);
+    p.w_gate_up_t = h->w_gate_up_t;
+    p.s_gate_up_t = h->s_gate_up_t;
+    p.w_down_t = h->w_down_t;
+    p.s_down_t = h->s_down_t;
+    p.tmap_xq = h->tmap_xq;
+    p.tmap_hq = h->tmap_hq;
+    p.err = h->err_dev;
+    p.err_host = h->err_host_dev;
     return p;
+}
+
+cudaError_t run_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t r0, int64_t nr) {
+    return p.use_tc ? launch_gate_up_tc(p, s, dump, r0, nr) : launch_gate_up(p, s, dump, r0, nr);
+}
+
+cudaError_t run_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t r0, int64_t nr) {
+    return p.use_tc ? launch_down_tc(p, s, dump, r0, nr) : launch_down(p, s, dump, r0, nr);
+}
+
+// A bounded device-side wait of an earlier call gave up: report it once and
+// clear both copies of the flag (the device copy in stream order).
+mmoe_status check_device_flag(mmoe_handle* h, cudaStream_t s) {
+    if (!h->err_host) return MMOE_OK;
+    const int v = *reinterpret_cast<volatile int*>(h->err_host);
+    if (v == 0) return MMOE_OK;
+    *reinterpret_cast<volatile int*>(h->err_host) = 0;
+    cudaMemsetAsync(h->err_dev, 0, sizeof(int), s);
+    return fail(MMOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (site %d); its results were not written", v);
 }
 
 cudaEvent_t take_event(mmoe_handle* h) {
@@ -335,6 +378,22 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(hq, R * h->hmax);
     ALLOC(sh, R);
     if (cfg->flags & MMOE_FLAG_DETERMINISTIC) ALLOC(obuf, R * d);
+    h->use_tc = !(cfg->flags & MMOE_FLAG_CUDA_CORES) && tc_supported((int)d, (int)hh, (int)hs);
+    if (h->use_tc) {
+        ALLOC(w_gate_up_t, h->n_gu_bytes);
+        ALLOC(s_gate_up_t, h->n_gu_scales);
+        ALLOC(w_down_t, h->n_d_bytes);
+        ALLOC(s_down_t, h->n_d_scales);
+        ALLOC(err_dev, 1);
+        if (e == cudaSuccess) e = cudaMemset(h->err_dev, 0, sizeof(int));
+        if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&h->err_host), sizeof(int), cudaHostAllocMapped);
+        if (e == cudaSuccess) {
+            *h->err_host = 0;
+            e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->err_host_dev), h->err_host, 0);
+        }
+        if (e == cudaSuccess) e = make_tensor_map(h->tmap_xq, h->xq, (uint64_t)d, (uint64_t)R, (uint64_t)d);
+        if (e == cudaSuccess) e = make_tensor_map(h->tmap_hq, h->hq, (uint64_t)h->hmax, (uint64_t)R, (uint64_t)h->hmax);
+    }
 #undef ALLOC
     if (e != cudaSuccess) {
         free_all(h);
@@ -363,6 +422,11 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
     MMOE_CUDA(cudaMemcpyAsync(h->s_gate_up, w->s_gate_up, h->n_gu_scales * sizeof(float), kind, s), "copy s_gate_up");
     MMOE_CUDA(cudaMemcpyAsync(h->w_down, w->w_down, h->n_d_bytes, kind, s), "copy w_down");
     MMOE_CUDA(cudaMemcpyAsync(h->s_down, w->s_down, h->n_d_scales * sizeof(float), kind, s), "copy s_down");
+    if (h->use_tc)
+        MMOE_CUDA(launch_retile(h->w_gate_up, h->s_gate_up, h->w_down, h->s_down, h->w_gate_up_t, h->s_gate_up_t,
+                                h->w_down_t, h->s_down_t, h->cfg.d_model, h->cfg.expert_hidden, h->cfg.shared_hidden,
+                                h->cfg.n_experts, s),
+                  "weight re-tiling launch");
     h->loaded = true;
     return MMOE_OK;
 }
@@ -378,6 +442,8 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     if (!x || !y) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
     DeviceGuard dg(h->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    mmoe_status fst = check_device_flag(h, s);
+    if (fst != MMOE_OK) return fst;
     const Plan p = make_plan(h, x, T, y);
     if (!p.deterministic)
         MMOE_CUDA(run_stage(h, MMOE_PROF_ZERO_Y, 0, s,
@@ -386,10 +452,10 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_quant(p, s); }),
               "router/quantiser launch");
     MMOE_CUDA(run_stage(h, MMOE_PROF_PERMUTE, 4, s, [&] { return launch_permute(p, s); }), "permute launch");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return launch_gate_up(p, s, nullptr, 0, 0); }),
+    MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return run_gate_up(p, s, nullptr, 0, 0); }),
               "gate/up launch");
     MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return launch_down(p, s, nullptr, 0, 0); }), "down launch");
+    MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return run_down(p, s, nullptr, 0, 0); }), "down launch");
     if (p.deterministic)
         MMOE_CUDA(run_stage(h, MMOE_PROF_COMBINE, 1, s, [&] { return launch_combine(p, s); }), "combine launch");
     if (topk_idx)
@@ -435,6 +501,7 @@ mmoe_status mmoe_destroy(mmoe_handle* h) {
     if (!h) return MMOE_OK;
     DeviceGuard dg(h->device);
     cudaError_t e = cudaDeviceSynchronize();
+    const int flag = h->err_host ? *reinterpret_cast<volatile int*>(h->err_host) : 0;
     for (auto& r : h->prof) {
         cudaEventDestroy(r.a);
         cudaEventDestroy(r.b);
@@ -443,6 +510,7 @@ mmoe_status mmoe_destroy(mmoe_handle* h) {
     free_all(h);
     delete h;
     if (e != cudaSuccess) return cuda_fail(e, "synchronize before destroy");
+    if (flag) return fail(MMOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (site %d)", flag);
     return MMOE_OK;
 }
 
@@ -498,8 +566,8 @@ mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int
     DeviceGuard dg(h->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Plan p = make_plan(h, nullptr, h->last_T, nullptr);
-    if (which == 0) MMOE_CUDA(launch_gate_up(p, s, dst, row0, nrows), "gate/up dump launch");
-    else MMOE_CUDA(launch_down(p, s, dst, row0, nrows), "down dump launch");
+    if (which == 0) MMOE_CUDA(run_gate_up(p, s, dst, row0, nrows), "gate/up dump launch");
+    else MMOE_CUDA(run_down(p, s, dst, row0, nrows), "down dump launch");
     return MMOE_OK;
 }
 
@@ -574,7 +642,9 @@ mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weigh
     p.s_down = w->s_down;
     p.x = x;
     p.y = y;
-    p.max_tiles = max_tiles_for(T, p.k, p.E);
+    p.use_tc = false;
+    p.tile_rows = kTileRows;
+    p.max_tiles = max_tiles_for(T, p.k, p.E, p.tile_rows);
     p.nchunks = (int)((p.Tk + kChunk - 1) / kChunk);
 
     // size check first (no device needed), then the one-time address lookup

@@ -13,7 +13,8 @@ constexpr int kGroup = 32;          // Eq. (6) group size along K
 constexpr int kMaxExperts = 64;     // routed experts supported by the router kernel
 constexpr int kMaxTopK = 8;
 constexpr int kChunk = 1024;        // routing slots per permutation block
-constexpr int kTileRows = 32;       // rows (token slots) per expert-GEMM tile
+constexpr int kTileRows = 32;       // rows (token slots) per CUDA-core expert-GEMM tile
+constexpr int kTcTileRows = 128;    // rows per tensor-core expert-GEMM tile
 
 // Everything a forward pass needs, as plain device pointers.
 struct Plan {
@@ -51,11 +52,22 @@ struct Plan {
     float* obuf;            // [R, d] expert outputs (deterministic combine only)
     int64_t max_tiles;
     int nchunks;
+    int tile_rows;          // kTileRows (CUDA-core GEMMs) or kTcTileRows (tensor-core GEMMs)
+    // tensor-core path
+    bool use_tc;
+    const uint8_t* w_gate_up_t;   // pre-tiled weights (tensor-core layout)
+    const float* s_gate_up_t;
+    const uint8_t* w_down_t;
+    const float* s_down_t;
+    const void* tmap_xq;          // host pointers to CUtensorMap of xq and hq (128B-swizzled 128 x 128 boxes)
+    const void* tmap_hq;
+    int* err;                     // device flag: a bounded wait gave up (later CTAs exit at once)
+    int* err_host;                // device alias of the host-mapped copy of that flag
 };
 
-// Upper bound on the number of kTileRows-row tiles over all groups.
-inline int64_t max_tiles_for(int64_t T, int k, int E) {
-    return (T * k + kTileRows - 1) / kTileRows + E + (T + kTileRows - 1) / kTileRows + 1;
+// Upper bound on the number of tile_rows-row tiles over all groups.
+inline int64_t max_tiles_for(int64_t T, int k, int E, int tile_rows = kTileRows) {
+    return (T * k + tile_rows - 1) / tile_rows + E + (T + tile_rows - 1) / tile_rows + 1;
 }
 
 // launchers (each returns the launch error, if any)
@@ -65,6 +77,14 @@ cudaError_t launch_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t
 cudaError_t launch_requant(const Plan& p, cudaStream_t s);
 cudaError_t launch_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_combine(const Plan& p, cudaStream_t s);
+// tensor-core path (k_expert_tc.cu)
+bool tc_supported(int d, int h, int hs);
+cudaError_t launch_gate_up_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
+cudaError_t launch_down_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
+cudaError_t launch_retile(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn, uint8_t* gu_t,
+                          float* sgu_t, uint8_t* dn_t, float* sdn_t, int d, int h, int hs, int E, cudaStream_t s);
+size_t tensor_map_bytes();
+cudaError_t make_tensor_map(void* map, void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_stride);
 cudaError_t launch_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t* packed, float* scales,
                                  cudaStream_t s);
 

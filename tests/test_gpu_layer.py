@@ -53,9 +53,9 @@ def test_quantizer_matches_oracle_bit_exact():
     assert np.array_equal(s_gpu.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
-def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None):
+def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False):
     T = x.shape[0]
-    L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic)
+    L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic, cuda_cores=cuda_cores)
     out = gu.run_gpu(L, q, x)
     y, D = oracle.moe_layer(q, x, dumps=True)
     rep = {}
@@ -70,13 +70,14 @@ def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None):
     return rep, out
 
 
-@pytest.mark.parametrize("deterministic", [False, True])
-def test_c0_all_stages(deterministic):
+@pytest.mark.parametrize("cuda_cores", [False, True], ids=["tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("deterministic", [False, True], ids=["atomic", "fixed_order"])
+def test_c0_all_stages(deterministic, cuda_cores):
     w, q = workload("c0")
     x = synth.workload_x(w)
     R = w.T * (q.k + 1)
-    rep, out = _full_check(q, x, deterministic, partial_rows=range(0, R, 3))
-    print("c0", rep)
+    rep, out = _full_check(q, x, deterministic, partial_rows=range(0, R, 3), cuda_cores=cuda_cores)
+    print("c0", "cuda cores" if cuda_cores else "tensor cores", rep)
 
 
 def test_deterministic_mode_is_reproducible():
@@ -88,12 +89,18 @@ def test_deterministic_mode_is_reproducible():
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
 
 
-@pytest.mark.parametrize("T", [1, 2, 7, 31, 33, 63, 65, 129, 300])
+@pytest.mark.parametrize("T", [1, 2, 7, 31, 33, 63, 65, 127, 129, 300])
 def test_ragged_token_counts(T):
     w, q = workload("c0")
     x = synth.draw_x(T, w.d, seed=100 + T)
-    rep, out = _full_check(q, x, max_tokens=512)
+    rep, out = _full_check(q, x, max_tokens=512, partial_rows=[0, T * q.k - 1, T * q.k, T * (q.k + 1) - 1])
     assert out["counts"][q.E] == T
+
+
+def test_c2_prefill_cuda_cores():
+    w, q = workload("c2")
+    x = synth.workload_x(w, T=512)
+    rep, out = _full_check(q, x, cuda_cores=True, partial_rows=[0, 2047, 2048, 2559])
 
 
 def test_T0_is_a_noop():
