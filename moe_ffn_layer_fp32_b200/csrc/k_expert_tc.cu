@@ -6,30 +6,36 @@
 // token order (section "custom MoE kernel"); weights are symmetric group-32
 // INT4 with FP32 scales (Eq. (6)), activations INT8 (section "QAT").
 //
-// One CTA computes a 128 x 128 tile: 128 weight rows (M) x 128 token rows
-// (N), over the whole K range.
+// A persistent kernel (one CTA per SM) walks over 128 x 128 output tiles:
+// 128 weight rows (M) x 128 token rows (N), each over the whole K range.
 //   gate/up: the 128 weight rows are 64 gate rows and the 64 up rows of the
 //            same 64 hidden features, so one MMA per K group yields both
 //            halves of SwiGLU; K = d_model.
 //   down:    128 output features; K = hidden size of the group's expert.
-// Pipeline (one CTA per SM, 12 warps):
+// Roles (20 warps):
 //   warp 0      producer: 1-D bulk copy of the packed INT4 weight tile
 //               (pre-tiled at load time, 8 KB per 128-K stage) and a 2-D TMA
-//               load (128B swizzle) of the 128 x 128 INT8 activation tile;
-//   warp 1      allocates TMEM; one elected lane issues tcgen05.mma
-//               (M=128, N=128, K=32, INT8 x INT8 -> INT32), one instruction
-//               per 32-element K group, each into a fresh TMEM buffer
-//               (4 buffers of 128 columns), and commits to mbarriers;
+//               load (128B swizzle) of the 128 x 128 INT8 activation tile,
+//               running ahead across tile boundaries;
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=128,
+//               K=32, INT8 x INT8 -> INT32), one instruction per 32-element
+//               K group into one of 4 TMEM buffers of 128 columns, handed
+//               over to the promotion warps two groups (a pair of buffers) at
+//               a time;
 //   warps 2-3   unpack INT4 -> INT8 into the canonical K-major SW128 layout;
-//   warps 4-11  promotion: read each group's INT32 partials from TMEM and
+//   warps 4-19  promotion: read each group's INT32 partials from TMEM and
 //               accumulate acc = fma(float(P_j), s_j, acc) in registers
-//               (2 warpgroups x 64 token columns, one weight row per thread),
-//               then the epilogue.
+//               (4 warpgroups x 32 token columns, one weight row per thread),
+//               then the tile's epilogue, which overlaps the MMAs of the next
+//               tile.  After reading a buffer they refill it with the bit
+//               pattern of 1.5 * 2^23; the next MMA accumulates onto it, so
+//               the INT32 result P arrives as the float 1.5 * 2^23 + P
+//               (exact for |P| < 2^22) and one exact subtraction converts it.
 // The exact INT32 group partial is needed because every 32-element group of K
 // has its own FP32 weight scale; the promotion order (j ascending, fused
 // multiply-add) is the oracle's, so the FP32 result is identical to it.
-// Every mbarrier wait is bounded by wall time; a wait that gives up raises
-// the handle's error flag and the CTA drains and exits.
+// Every mbarrier wait is bounded; a wait that gives up raises the handle's
+// error flag and the CTA drains and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -41,32 +47,49 @@ namespace tc {
 constexpr int BM = 128;                    // weight rows per tile
 constexpr int BN = kTcTileRows;            // token rows per tile (128)
 constexpr int BK = 128;                    // K elements (bytes of INT8) per stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kBufs = 4;                   // TMEM accumulator buffers, 128 columns each
-constexpr int kThreads = 384;
-constexpr int kPromoThreads = 256;
+constexpr int kPairs = kBufs / 2;          // buffers are handed over two at a time
+constexpr int kPromoWarpgroups = 4;        // each covers 32 token columns of all 128 weight rows
+constexpr int kPromoThreads = kPromoWarpgroups * 128;
+constexpr int kThreads = 128 + kPromoThreads;   // producer, MMA, 2 unpack warps, promotion warps
+constexpr int kCols = BN / kPromoWarpgroups;    // token columns per promotion thread
+
 constexpr int kUnpackThreads = 64;
 constexpr int kAPackedBytes = BM * BK / 2; // 8 KB
 constexpr int kAI8Bytes = BM * BK;         // 16 KB
 constexpr int kBBytes = BN * BK;           // 16 KB
 constexpr int kStageBytes = kAI8Bytes + kBBytes + kAPackedBytes;
-constexpr int kXchBytes = 64 * BN * 4;     // up-projection values handed to the gate threads
-constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kXchBytes = BM * BN * 4;     // finished FP32 tile handed to the epilogue, [column][row]
+constexpr long long kTimeoutClk = 4000000000ll;  // about 2 s of SM clock
 
 enum Epi { kEpiSwiGLU = 0, kEpiCombine = 1 };
+
+constexpr int kTInfo = 4;                  // tile-info ring entries
+constexpr int kTInfoConsumers = 1 + 2 + kPromoWarpgroups * 4;  // MMA lane, unpack warps, promotion warps
+
+// What every role needs to know about one tile, gathered by the producer warp
+// ahead of time (tile decode, per-column data, the first two group scales).
+struct TileInfo {
+    int row0, nr, mb, nks, tile0, end;
+    float colf[BN];      // per token column: activation scale (gate/up) or SwiGLU scale (down)
+    float colg[BN];      // per token column: gate of the row (down)
+    int colrow[BN];      // per token column: token id (down)
+    float s01[2][BM];    // scales of groups 0 and 1, per weight row
+};
 
 struct Smem {
     // stage buffers are carved from the 1024-aligned base: [A_i8 | B | A_packed] x kStages
     uint64_t full[kStages];
     uint64_t unpacked[kStages];
     uint64_t empty[kStages];
-    uint64_t accf[kBufs];
-    uint64_t acce[kBufs];
+    uint64_t accf[kPairs];   // a pair of buffers holds two finished groups
+    uint64_t acce[kPairs];   // a pair of buffers has been read and preset again
+    uint64_t tfull[kTInfo];  // tile info written
+    uint64_t tempty[kTInfo]; // tile info no longer needed
     uint32_t tmem_base;
     int abort;
-    float colf[BN];      // per token column: activation scale (gate/up) or SwiGLU scale (down)
-    float colg[BN];      // per token column: gate of the row (down)
-    int colrow[BN];      // per token column: token id (down)
+    TileInfo ti[kTInfo];
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -102,23 +125,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase of the given parity; gives up after kTimeoutNs or once
-// another thread of the CTA has given up.  Returns false on giving up.
-// On giving up it records `where` in the device flag (read by every later CTA,
-// which then exits at once) and in the host-visible flag.
+__device__ __forceinline__ long long clk() {
+    long long t;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+    return t;
+}
+
+// Waits for the phase of the given parity; gives up after kTimeoutClk SM
+// clocks or once another thread of the CTA has given up.  On giving up it
+// records `where` in the device flag (read by every later CTA, which then
+// exits at once) and in the host-visible flag.  Returns false on giving up.
 struct ErrFlags {
     int* dev;
     int* host;
 };
 
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem* sm, ErrFlags err, int where) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, Smem* sm, ErrFlags err, int where) {
+    const long long t0 = clk();
     for (;;) {
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*reinterpret_cast<volatile int*>(&sm->abort)) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
+        if (clk() - t0 > kTimeoutClk) {
             atomicExch(&sm->abort, 1);
             if (err.dev) *reinterpret_cast<volatile int*>(err.dev) = where;
             if (err.host) *reinterpret_cast<volatile int*>(err.host) = where;
@@ -126,6 +154,11 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem* sm,
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem* sm, ErrFlags err, int where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, sm, err, where);
 }
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -157,12 +190,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
 // kind::i8: signed A and B, S32 accumulator, both K-major, M = 128, N = BN.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
+// D += A * B (the accumulator holds the preset 1.5 * 2^23 bit pattern)
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(0)
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(1)
         : "memory");
 }
 
@@ -182,7 +216,38 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, int32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, int32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive columns of this warp's lanes <- v
+__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;
 
 // exact int32 -> float for |v| < 2^22: integer add into the mantissa of 1.5 * 2^23
 __device__ __forceinline__ float exact_i2f(int32_t v) { return __int_as_float(v + 0x4B400000) - 12582912.0f; }
@@ -202,6 +267,7 @@ struct TcArgs {
     int mblocks_shared;
     int ks_routed;          // K stages of a routed expert (gate/up: d/128, down: h/128)
     int ks_shared;
+    int fblocks;            // weight-row blocks per token tile in the launch (the larger of the two)
     int32_t* dump;          // optional INT32 partial dump
     int64_t drow0, dnrows;
 };
@@ -209,12 +275,46 @@ struct TcArgs {
 // Bounded wait used while draining after an abort: ignores the abort flag,
 // gives up only on time.
 __device__ __noinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer();
+    const long long t0 = clk();
     while (!mbar_try_wait(bar, parity))
-        if (globaltimer() - t0 > kTimeoutNs) return;
+        if (clk() - t0 > kTimeoutClk) return;
 }
 
 // --------------------------------------------------------------- the kernel
+struct Tile {
+    int g, mb, nks, nr;
+    int row0;           // first row of the token tile
+    bool valid;
+    int tile0;          // first weight tile (index into the pre-tiled arrays)
+};
+
+// Tile L of the launch: weight-row block L % fblocks of token tile L / fblocks.
+__device__ __forceinline__ Tile decode_tile(const Plan& p, const TcArgs& a, int L) {
+    Tile t;
+    const int fb = L % a.fblocks;
+    const int ti = L / a.fblocks;
+    const int code = p.tiles[ti];
+    t.g = code >> 24;
+    const int tin = code & 0xffffff;
+    const bool shared_grp = t.g == p.E;
+    const int mblocks = shared_grp ? a.mblocks_shared : a.mblocks_routed;
+    t.valid = fb < mblocks;
+    t.mb = fb;
+    t.nks = shared_grp ? a.ks_shared : a.ks_routed;
+    const int cnt = p.offsets[t.g + 1] - p.offsets[t.g];
+    t.row0 = p.offsets[t.g] + tin * BN;
+    t.nr = min(BN, cnt - tin * BN);
+    t.tile0 = t.g * (int)a.w_expert_stride_tiles + fb * t.nks;
+    return t;
+}
+
+// One lane waits, the warp follows.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem* sm, ErrFlags ef, int where) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, sm, ef, where);
+    return __shfl_sync(0xffffffffu, ok, 0);
+}
+
 template <int kEpi, bool kDump>
 __global__ void __launch_bounds__(kThreads, 1)
 expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a)
@@ -225,26 +325,11 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
     float* xch = reinterpret_cast<float*>(base + kStages * kStageBytes);
     Smem* sm = reinterpret_cast<Smem*>(base + kStages * kStageBytes + kXchBytes);
 
-    // ---- tile -> (group, rows, weight block); nothing to do after an earlier wait gave up
-    if ((int)blockIdx.y >= *p.tile_count) return;
+    // nothing to do after an earlier wait gave up
     if (p.err && *reinterpret_cast<volatile int*>(p.err)) return;
+    const int total = (*p.tile_count) * a.fblocks;
+    if ((int)blockIdx.x >= total) return;
     const ErrFlags ef{p.err, p.err_host};
-    const int code = p.tiles[blockIdx.y];
-    const int g = code >> 24;
-    const int ti = code & 0xffffff;
-    const bool shared_grp = g == p.E;
-    const int mblocks = shared_grp ? a.mblocks_shared : a.mblocks_routed;
-    const int mb = blockIdx.x;
-    if (mb >= mblocks) return;
-    const int nks = shared_grp ? a.ks_shared : a.ks_routed;
-    const int ng = nks * (BK / kGroup);
-    const int cnt = p.offsets[g + 1] - p.offsets[g];
-    const int64_t row0 = (int64_t)p.offsets[g] + (int64_t)ti * BN;
-    const int nr = min(BN, cnt - ti * BN);
-    const int64_t tile0 = (int64_t)g * a.w_expert_stride_tiles + (int64_t)mb * nks;  // first weight tile
-    const uint8_t* wsrc = a.wtiles + tile0 * kAPackedBytes;
-    const float* ssrc = a.stiles + tile0 * (BK / kGroup) * BM;
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -253,23 +338,16 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
             mbar_init(&sm->unpacked[s], kUnpackThreads);
             mbar_init(&sm->empty[s], 1);
         }
-        for (int b = 0; b < kBufs; ++b) {
+        for (int b = 0; b < kPairs; ++b) {
             mbar_init(&sm->accf[b], 1);
-            mbar_init(&sm->acce[b], kPromoThreads);
+            mbar_init(&sm->acce[b], kPromoThreads / 32);
+        }
+        for (int b = 0; b < kTInfo; ++b) {
+            mbar_init(&sm->tfull[b], 32);
+            mbar_init(&sm->tempty[b], kTInfoConsumers);
         }
         sm->abort = 0;
         fence_barrier_init();
-    }
-    // per-column data of the token tile
-    for (int c = tid; c < BN; c += kThreads) {
-        const int64_t r = row0 + (c < nr ? c : 0);
-        if (kEpi == kEpiSwiGLU) {
-            sm->colf[c] = p.sx[p.row_src[r]];
-        } else {
-            sm->colf[c] = p.sh[r];
-            sm->colg[c] = p.row_gate[r];
-            sm->colrow[c] = p.row_src[r];
-        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&sm->tmem_base)),
@@ -283,156 +361,263 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
     const uint32_t tmem = sm->tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int ks = 0; ks < nks; ++ks) {
-                const int s = ks % kStages;
-                if (ks >= kStages && !mbar_wait(&sm->empty[s], ((ks / kStages) - 1) & 1, sm, ef, 1)) break;
-                uint8_t* st = stages + s * kStageBytes;
-                mbar_expect_tx(&sm->full[s], kAPackedBytes + kBBytes);
-                bulk_load(st + kAI8Bytes + kBBytes, wsrc + (int64_t)ks * kAPackedBytes, kAPackedBytes, &sm->full[s]);
-                tma_load_2d(st + kAI8Bytes, &bmap, ks * BK, (int)row0, &sm->full[s]);
-                issued = ks + 1;
+        // ------------------------------------------------------------ producer (whole warp)
+        int sc = 0, tcount = 0;
+        bool ok = true;
+        for (int L = blockIdx.x; ok; L += gridDim.x) {
+            Tile t{};
+            const bool last = L >= total;  // past the last tile: publish the end marker and stop
+            if (!last) {
+                if (lane == 0) t = decode_tile(p, a, L);
+                t.valid = __shfl_sync(0xffffffffu, t.valid, 0);
+                if (!t.valid) continue;
+                t.mb = __shfl_sync(0xffffffffu, t.mb, 0);
+                t.nks = __shfl_sync(0xffffffffu, t.nks, 0);
+                t.nr = __shfl_sync(0xffffffffu, t.nr, 0);
+                t.row0 = __shfl_sync(0xffffffffu, t.row0, 0);
+                t.tile0 = __shfl_sync(0xffffffffu, t.tile0, 0);
             }
-            // every issued copy has landed before the CTA may exit
-            for (int ks = issued > kStages ? issued - kStages : 0; ks < issued; ++ks)
-                mbar_wait_drain(&sm->full[ks % kStages], (ks / kStages) & 1);
+            // publish the tile's information (or the end marker)
+            const int b = tcount % kTInfo;
+            if (tcount >= kTInfo && !warp_wait(&sm->tempty[b], ((tcount / kTInfo) - 1) & 1, sm, ef, 6)) { ok = false; break; }
+            TileInfo& ti = sm->ti[b];
+            if (lane == 0) {
+                ti.end = last ? 1 : 0;
+                ti.row0 = t.row0; ti.nr = t.nr; ti.mb = t.mb; ti.nks = t.nks; ti.tile0 = t.tile0;
+            }
+            if (!last) {
+                for (int c = lane; c < BN; c += 32) {
+                    const int r = t.row0 + (c < t.nr ? c : 0);
+                    if (kEpi == kEpiSwiGLU) {
+                        ti.colf[c] = p.sx[p.row_src[r]];
+                    } else {
+                        ti.colf[c] = p.sh[r];
+                        ti.colg[c] = p.row_gate[r];
+                        ti.colrow[c] = p.row_src[r];
+                    }
+                }
+                const float* sp = a.stiles + (size_t)t.tile0 * (BK / kGroup) * BM;
+                for (int r = lane; r < 2 * BM; r += 32) ti.s01[r / BM][r % BM] = __ldg(sp + r);
+            }
+            mbar_arrive(&sm->tfull[b]);
+            ++tcount;
+            if (last) break;
+            // the tile's stages
+            if (lane == 0) {
+                for (int ks = 0; ks < t.nks; ++ks, ++sc) {
+                    const int s = sc % kStages;
+                    if (sc >= kStages && !mbar_wait(&sm->empty[s], ((sc / kStages) - 1) & 1, sm, ef, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = stages + s * kStageBytes;
+                    mbar_expect_tx(&sm->full[s], kAPackedBytes + kBBytes);
+                    bulk_load(st + kAI8Bytes + kBBytes, a.wtiles + ((int64_t)t.tile0 + ks) * kAPackedBytes, kAPackedBytes,
+                              &sm->full[s]);
+                    tma_load_2d(st + kAI8Bytes, &bmap, ks * BK, t.row0, &sm->full[s]);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
         }
+        // every issued copy has landed before the CTA may exit
+        if (lane == 0)
+            for (int i = sc > kStages ? sc - kStages : 0; i < sc; ++i)
+                mbar_wait_drain(&sm->full[i % kStages], (i / kStages) & 1);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            int sc = 0, pc = 0, tcount = 0;
             bool ok = true;
-            int last_j = -1;
-            for (int ks = 0; ks < nks && ok; ++ks) {
-                const int s = ks % kStages;
-                if (!mbar_wait(&sm->unpacked[s], (ks / kStages) & 1, sm, ef, 2)) { ok = false; break; }
-                tc_after_sync();
-                uint8_t* st = stages + s * kStageBytes;
-                const uint64_t ad = smem_desc_sw128(st);
-                const uint64_t bd = smem_desc_sw128(st + kAI8Bytes);
-                for (int jj = 0; jj < BK / kGroup; ++jj) {
-                    const int j = ks * (BK / kGroup) + jj;
-                    const int b = j % kBufs;
-                    if (j >= kBufs && !mbar_wait(&sm->acce[b], ((j / kBufs) - 1) & 1, sm, ef, 3)) { ok = false; break; }
+            while (ok) {
+                const int tb = tcount % kTInfo;
+                if (!mbar_wait(&sm->tfull[tb], (tcount / kTInfo) & 1, sm, ef, 7)) break;
+                const int nks = sm->ti[tb].nks, end = sm->ti[tb].end;
+                mbar_arrive(&sm->tempty[tb]);
+                ++tcount;
+                if (end) break;
+                for (int ks = 0; ks < nks && ok; ++ks, ++sc) {
+                    const int s = sc % kStages;
+                    if (!mbar_wait(&sm->unpacked[s], (sc / kStages) & 1, sm, ef, 2)) { ok = false; break; }
                     tc_after_sync();
-                    mma_i8(tmem + b * 128, ad + (uint64_t)(jj * 2), bd + (uint64_t)(jj * 2));
-                    mma_commit(&sm->accf[b]);
-                    last_j = j;
+                    uint8_t* st = stages + s * kStageBytes;
+                    const uint64_t ad = smem_desc_sw128(st);
+                    const uint64_t bd = smem_desc_sw128(st + kAI8Bytes);
+#pragma unroll
+                    for (int pp = 0; pp < (BK / kGroup) / 2; ++pp, ++pc) {
+                        const int b = pc & 1;
+                        if (!mbar_wait(&sm->acce[b], (pc >> 1) & 1, sm, ef, 3)) { ok = false; break; }
+                        tc_after_sync();
+#pragma unroll
+                        for (int gg = 0; gg < 2; ++gg) {
+                            const int jj = pp * 2 + gg;
+                            mma_i8(tmem + (2 * b + gg) * 128, ad + (uint64_t)(jj * 2), bd + (uint64_t)(jj * 2));
+                        }
+                        mma_commit(&sm->accf[b]);
+                    }
+                    mma_commit(&sm->empty[s]);
                 }
-                mma_commit(&sm->empty[s]);
             }
             // every MMA issued has completed before TMEM is released
-            if (last_j >= 0) mbar_wait_drain(&sm->accf[last_j % kBufs], (last_j / kBufs) & 1);
+            if (pc > 0) mbar_wait_drain(&sm->accf[(pc - 1) & 1], ((pc - 1) >> 1) & 1);
         }
     } else if (warp < 4) {
         // ------------------------------------------------------------ INT4 -> INT8 unpack
         const int t = tid - 64;
-        for (int ks = 0; ks < nks; ++ks) {
-            const int s = ks % kStages;
-            if (!mbar_wait(&sm->full[s], (ks / kStages) & 1, sm, ef, 4)) break;
-            uint8_t* st = stages + s * kStageBytes;
-            const uint8_t* src = st + kAI8Bytes + kBBytes;
-#pragma unroll
-            for (int i = 0; i < (BM * BK / 2 / 16) / kUnpackThreads; ++i) {
-                const int q = i * kUnpackThreads + t;   // 16-byte chunk of packed data (one K group of one row)
-                const int row = q >> 2, c = q & 3;
-                const uint4 w = *reinterpret_cast<const uint4*>(src + row * 64 + c * 16);
-                uint4 o0, o1;
-                unpack_word(w.x, o0.x, o0.y);
-                unpack_word(w.y, o0.z, o0.w);
-                unpack_word(w.z, o1.x, o1.y);
-                unpack_word(w.w, o1.z, o1.w);
-                uint8_t* rowp = st + row * 128;
-                *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = o0;
-                *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = o1;
+        int sc = 0, tcount = 0;
+        bool ok = true;
+        while (ok) {
+            const int tb = tcount % kTInfo;
+            if (!warp_wait(&sm->tfull[tb], (tcount / kTInfo) & 1, sm, ef, 8)) break;
+            const int nks = sm->ti[tb].nks, end = sm->ti[tb].end;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->tempty[tb]);
+            ++tcount;
+            if (end) break;
+            for (int ks = 0; ks < nks; ++ks, ++sc) {
+                const int s = sc % kStages;
+                if (!mbar_wait(&sm->full[s], (sc / kStages) & 1, sm, ef, 4)) { ok = false; break; }
+                uint8_t* st = stages + s * kStageBytes;
+                const uint8_t* src = st + kAI8Bytes + kBBytes;
+#pragma unroll 2
+                for (int i = 0; i < (BM * BK / 2 / 16) / kUnpackThreads; ++i) {
+                    const int q = i * kUnpackThreads + t;   // 16-byte chunk of packed data (one K group of one row)
+                    const int row = q >> 2, c = q & 3;
+                    const uint4 w = *reinterpret_cast<const uint4*>(src + row * 64 + c * 16);
+                    uint4 o0, o1;
+                    unpack_word(w.x, o0.x, o0.y);
+                    unpack_word(w.y, o0.z, o0.w);
+                    unpack_word(w.z, o1.x, o1.y);
+                    unpack_word(w.w, o1.z, o1.w);
+                    uint8_t* rowp = st + row * 128;
+                    *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = o0;
+                    *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = o1;
+                }
+                fence_proxy_async();
+                mbar_arrive(&sm->unpacked[s]);
             }
-            fence_proxy_async();
-            mbar_arrive(&sm->unpacked[s]);
         }
     } else {
         // ------------------------------------------------------------ promotion + epilogue
-        const int pw = warp - 4;            // 0..7
-        const int wg = pw >> 2;             // token-column half
+        const int pw = warp - 4;            // 0..15
+        const int wg = pw >> 2;             // token-column quarter
         const int quarter = warp & 3;       // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;  // weight row of this thread (0..127)
-        const int col0 = wg * 64;
-        float acc[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+        const int col0 = wg * kCols;
         const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)col0;
-        float s_next = ng > 0 ? __ldg(ssrc + row) : 0.0f;
-        for (int j = 0; j < ng; ++j) {
-            const int b = j % kBufs;
-            const float s = s_next;
-            if (j + 1 < ng) s_next = __ldg(ssrc + (int64_t)(j + 1) * BM + row);
-            if (!mbar_wait(&sm->accf[b], (j / kBufs) & 1, sm, ef, 5)) break;
-            tc_after_sync();
-            int32_t v0[32], v1[32];
-            tmem_ld32(tl + b * 128, v0);
-            tmem_ld32(tl + b * 128 + 32, v1);
-            tmem_wait_ld();
-            tc_before_sync();
-            mbar_arrive(&sm->acce[b]);
+        // preset every buffer; this is completion 0 of both acce barriers
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                acc[c] = fmaf(exact_i2f(v0[c]), s, acc[c]);
-                acc[32 + c] = fmaf(exact_i2f(v1[c]), s, acc[32 + c]);
+        for (int b = 0; b < kBufs; ++b) {
+            tmem_st16_const(tl + b * 128, kMagicBits);
+            tmem_st16_const(tl + b * 128 + 16, kMagicBits);
+        }
+        tmem_wait_st();
+        tc_before_sync();
+        __syncwarp();
+        if (lane == 0)
+            for (int b = 0; b < kPairs; ++b) mbar_arrive(&sm->acce[b]);
+        int pc = 0, tcount = 0;
+        bool ok = true;
+        while (ok) {
+            const int tb = tcount % kTInfo;
+            if (!warp_wait(&sm->tfull[tb], (tcount / kTInfo) & 1, sm, ef, 9)) break;
+            const TileInfo& ti = sm->ti[tb];
+            if (ti.end) break;
+            const int nks = ti.nks, nr = ti.nr, mb = ti.mb, row0 = ti.row0;
+            const float* sp = a.stiles + (size_t)ti.tile0 * (BK / kGroup) * BM + row;
+            float acc[kCols];
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) acc[c] = 0.0f;
+            const int ng = nks * (BK / kGroup);
+            float s0 = ti.s01[0][row], s1 = ti.s01[1][row];
+            for (int j = 0; j < ng; j += 2, ++pc) {
+                const int b = pc & 1;
+                const float sa = s0, sb = s1;
+                if (j + 2 < ng) {
+                    s0 = __ldg(sp + (j + 2) * BM);
+                    s1 = __ldg(sp + (j + 3) * BM);
+                }
+                if (!warp_wait(&sm->accf[b], (pc >> 1) & 1, sm, ef, 5)) { ok = false; break; }
+                tc_after_sync();
+#pragma unroll 1
+                for (int gg = 0; gg < 2; ++gg) {
+                    const float sc = gg ? sb : sa;
+                    const uint32_t ta = tl + (2 * b + gg) * 128;
+                    int32_t v[16], w[16];
+                    tmem_ld16(ta, v);
+                    tmem_wait_ld();
+                    tmem_st16_const(ta, kMagicBits);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) acc[c] = fmaf(__int_as_float(v[c]) - kMagic, sc, acc[c]);
+                    tmem_ld16(ta + 16, w);
+                    tmem_wait_ld();
+                    tmem_st16_const(ta + 16, kMagicBits);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) acc[16 + c] = fmaf(__int_as_float(w[c]) - kMagic, sc, acc[16 + c]);
+                    if (kDump) {
+                        // INT32 partials of rows [drow0, drow0 + dnrows) for the inspection entry point
+                        const int jg = j + gg;
+#pragma unroll
+                        for (int c = 0; c < kCols; ++c) {
+                            const int cc = col0 + c;
+                            const int64_t grow = (int64_t)row0 + cc;
+                            if (cc >= nr || grow < a.drow0 || grow >= a.drow0 + a.dnrows) continue;
+                            const int32_t pv = (int32_t)((c < 16 ? v[c & 15] : w[c & 15]) - (int32_t)kMagicBits);
+                            if (kEpi == kEpiSwiGLU) {
+                                const int f = mb * 64 + (row & 63);
+                                const int n = row < 64 ? f : p.hmax + f;
+                                a.dump[((grow - a.drow0) * 2 * p.hmax + n) * (p.d / kGroup) + jg] = pv;
+                            } else {
+                                const int m = mb * BM + row;
+                                a.dump[((grow - a.drow0) * p.d + m) * (p.hmax / kGroup) + jg] = pv;
+                            }
+                        }
+                    }
+                }
+                tmem_wait_st();
+                tc_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->acce[b]);
             }
-            if (kDump) {
-                // INT32 partials of rows [drow0, drow0 + dnrows) for the inspection entry point
+            if (!ok || *reinterpret_cast<volatile int*>(&sm->abort)) break;
+            // epilogue: park the tile in shared memory ([column][row]), then each warpgroup finishes its columns
+            const int named = 1 + wg;
+            asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");  // previous tile's readers are done
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int cc = col0 + c;
-                    const int64_t grow = row0 + cc;
-                    if (cc >= nr || grow < a.drow0 || grow >= a.drow0 + a.dnrows) continue;
-                    const int32_t v = c < 32 ? v0[c & 31] : v1[c & 31];
-                    if (kEpi == kEpiSwiGLU) {
-                        const int f = mb * 64 + (row & 63);
-                        const int n = row < 64 ? f : p.hmax + f;
-                        a.dump[((grow - a.drow0) * 2 * p.hmax + n) * (p.d / kGroup) + j] = v;
-                    } else {
-                        const int m = mb * BM + row;
-                        a.dump[((grow - a.drow0) * p.d + m) * (p.hmax / kGroup) + j] = v;
+            for (int c = 0; c < kCols; ++c) xch[(col0 + c) * BM + row] = acc[c];
+            asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");
+            if (!kDump) {
+                if (kEpi == kEpiSwiGLU) {
+                    // rows 0..63 hold the gate of feature mb*64 + row, rows 64..127 the up of the same feature;
+                    // thread (row) finishes feature row & 63 for half of the warpgroup's columns
+                    const int fl = row & 63;
+                    const int f = mb * 64 + fl;
+                    const int cbeg = col0 + (row >> 6) * (kCols / 2);
+#pragma unroll 1
+                    for (int cc = cbeg; cc < cbeg + kCols / 2; ++cc) {
+                        if (cc >= nr) break;
+                        const float sx = ti.colf[cc];
+                        const float gv = __fmul_rn(xch[cc * BM + fl], sx);
+                        const float uv = __fmul_rn(xch[cc * BM + 64 + fl], sx);
+                        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+                        p.act[((int64_t)row0 + cc) * p.hmax + f] = __fmul_rn(silu, uv);
+                    }
+                } else {
+                    const int m = mb * BM + row;
+#pragma unroll 1
+                    for (int cc = col0; cc < col0 + kCols; ++cc) {
+                        if (cc >= nr) break;
+                        const float o = __fmul_rn(xch[cc * BM + row], ti.colf[cc]);
+                        if (p.deterministic) {
+                            p.obuf[((int64_t)row0 + cc) * p.d + m] = o;
+                        } else {
+                            atomicAdd(p.y + (int64_t)ti.colrow[cc] * p.d + m, __fmul_rn(ti.colg[cc], o));
+                        }
                     }
                 }
             }
-        }
-        const bool aborted = *reinterpret_cast<volatile int*>(&sm->abort) != 0;
-        if (kEpi == kEpiSwiGLU) {
-            // rows 0..63: gate of feature mb*64 + row; rows 64..127: up of the same feature
-            const int named = 1 + wg;
-            if (row >= 64) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) xch[(col0 + c) * 64 + (row - 64)] = acc[c];
-            }
-            asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");
-            if (row < 64 && !aborted && !kDump) {
-                const int f = mb * 64 + row;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int cc = col0 + c;
-                    if (cc >= nr) continue;
-                    const float sx = sm->colf[cc];
-                    const float gv = __fmul_rn(acc[c], sx);
-                    const float uv = __fmul_rn(xch[cc * 64 + row], sx);
-                    const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
-                    p.act[(row0 + cc) * p.hmax + f] = __fmul_rn(silu, uv);
-                }
-            }
-        } else if (!aborted && !kDump) {
-            const int m = mb * BM + row;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const int cc = col0 + c;
-                if (cc >= nr) continue;
-                const float o = __fmul_rn(acc[c], sm->colf[cc]);
-                if (p.deterministic) {
-                    p.obuf[(row0 + cc) * p.d + m] = o;
-                } else {
-                    atomicAdd(p.y + (int64_t)sm->colrow[cc] * p.d + m, __fmul_rn(sm->colg[cc], o));
-                }
-            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->tempty[tb]);
+            ++tcount;
         }
     }
 
@@ -505,6 +690,7 @@ __global__ void retile_weights_kernel(const uint8_t* __restrict__ src, const flo
 bool tc_supported(int d, int h, int hs) { return d % 128 == 0 && h % 128 == 0 && hs % 128 == 0; }
 
 size_t tc_smem_bytes() { return 1024 + tc::kStages * tc::kStageBytes + tc::kXchBytes + sizeof(tc::Smem); }
+static_assert(1024 + tc::kStages * tc::kStageBytes + tc::kXchBytes + sizeof(tc::Smem) <= 232448, "shared memory");
 
 cudaError_t launch_retile(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn, uint8_t* gu_t,
                           float* sgu_t, uint8_t* dn_t, float* sdn_t, int d, int h, int hs, int E, cudaStream_t s) {
@@ -543,13 +729,26 @@ cudaError_t make_tensor_map(void* map_, void* base, uint64_t inner_bytes, uint64
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+static int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
+}
+
 template <int kEpi, bool kDump>
-static cudaError_t launch_tc(const Plan& p, cudaStream_t s, const CUtensorMap* map, const tc::TcArgs& a, int gx) {
+static cudaError_t launch_tc(const Plan& p, cudaStream_t s, const CUtensorMap* map, tc::TcArgs a, int fblocks) {
     auto kern = tc::expert_gemm_tc_kernel<kEpi, kDump>;
     const size_t smem = tc_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)gx, (unsigned)p.max_tiles);
+    a.fblocks = fblocks;
+    // persistent: one CTA per SM (never more CTAs than the largest possible tile count)
+    const int64_t upper = p.max_tiles * (int64_t)fblocks;
+    const unsigned grid = (unsigned)(upper < sm_count() ? upper : sm_count());
     kern<<<grid, tc::kThreads, smem, s>>>(*map, p, a);
     return cudaGetLastError();
 }
