@@ -42,6 +42,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="c4", help="prefill workload (c2, c3a, c3b, c4); c4 adds its 64-token decode batch")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-sweep", action="store_true", help="skip the 24-layer decode sweep (T=1 and T=8)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU work budget of the oracle sample")
     return ap.parse_args(argv)
 
@@ -139,13 +140,13 @@ def layer_counts(w, T):
     return gu_ops, dn_ops
 
 
-def quantized_on_device(w, device):
+def quantized_on_device(w, device, layer=0):
     """Seeded FP32 weights (synth) quantised on the GPU by the library's Eq. (6) kernel."""
     import torch
 
     from moe_ffn_layer_fp32_b200 import synth
     from moe_ffn_layer_fp32_b200.layer import quantize_int4
-    lw = synth.workload_layer(w)
+    lw = synth.workload_layer(w, layer)
     gu_w, gu_s, dn_w, dn_s = [], [], [], []
     for g in range(w.E + 1):
         p, s = quantize_int4(torch.from_numpy(lw.w_gate_up[g]).to(device))
@@ -159,6 +160,73 @@ def quantized_on_device(w, device):
 
 def weight_bytes(w, experts):
     return sum((3 * w.d * (w.h if g < w.E else w.hs)) * 0.625 for g in experts)
+
+
+def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8)):
+    """The decode workload: 24 distinct layers (d_model=1024, h=512; 1.44 GB of INT4 weights and scales, far
+    beyond L2) run back to back, layer l+1 reading layer l's y cast to BF16, captured once as a CUDA graph.
+    Step s feeds a fresh seeded x (seed 10^6 + s) to layer 0.  Returns us/layer and GB/s per token count."""
+    import numpy as np
+    import torch
+
+    from moe_ffn_layer_fp32_b200 import synth
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    w = synth.WORKLOADS["c1"]
+    layers = []
+    for l in range(w.layers):
+        tensors, lw = quantized_on_device(w, dev, l)
+        L = MoELayer(w.d, w.h, shared_hidden=w.hs, n_experts=w.E, top_k=w.k, max_tokens=max(token_counts),
+                     device=dev.index)
+        L.load(*tensors)
+        layers.append(L)
+        del tensors
+    torch.cuda.synchronize(dev)
+    out = {"workload": w.desc + " (chained: layer l+1 reads layer l's y as BF16)", "graph": "CUDA graph of 24 layers"}
+    for T in token_counts:
+        xs = [torch.empty((T, w.d), dtype=torch.bfloat16, device=dev) for _ in range(w.layers)]
+        ys = [torch.empty((T, w.d), dtype=torch.float32, device=dev) for _ in range(w.layers)]
+        idx = [torch.empty((T, w.k), dtype=torch.int32, device=dev) for _ in range(w.layers)]
+        x0 = [torch.from_numpy(synth.workload_x(w, step=s, T=T).view(np.int16)).to(dev).view(torch.bfloat16)
+              for s in range(warmup + steps)]
+
+        def sweep():
+            for l, L in enumerate(layers):
+                L.forward(xs[l], ys[l], topk_idx=idx[l])
+                if l + 1 < len(layers):
+                    xs[l + 1].copy_(ys[l])
+
+        xs[0].copy_(x0[0])
+        sweep()  # first call outside capture: lazy setup in the library and in torch
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            sweep()
+        stream = torch.cuda.current_stream(dev)
+        for s in range(warmup):
+            xs[0].copy_(x0[s])
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(steps):
+            xs[0].copy_(x0[warmup + s])
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        us_layer = e0.elapsed_time(e1) * 1e3 / (steps * w.layers)
+        # algorithmic bytes of the last step: the distinct experts each layer selected, the shared one, W_r
+        nbytes = 0.0
+        for l in range(w.layers):
+            ex = sorted(set(idx[l].cpu().numpy().ravel().tolist()) | {w.E})
+            nbytes += weight_bytes(w, ex) + w.d * w.E * 4
+        nbytes /= w.layers
+        gbs = nbytes / (us_layer * 1e-6) / 1e9
+        out[f"T{T}"] = {"us_per_layer": us_layer, "bytes_per_layer": nbytes, "achieved_gbs": gbs,
+                        "hbm_frac": gbs / hbm_gbs, "launches_per_layer": 3}
+        del g
+    for L in layers:
+        L.close()
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -368,6 +436,10 @@ def run_ours(args):
                "h2d_bytes_per_step": (Tp + Td) * w.d * 2, "d2h_bytes_per_step": (Tp + Td) * w.d * 4,
                "api": "mmoe_forward_host (pinned host x and y)"}
 
+    sweep = None
+    if not args.no_decode_sweep:
+        sweep = decode_sweep(dev, args.steps, args.warmup, float(peaks.get("hbm_gbs", 6650.0)))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, n, dt = oracle_rate(w, args.cpu_seconds, lw)
@@ -392,6 +464,7 @@ def run_ours(args):
         "prefill": {"tokens": Tp, "ms": prefill_ms, "tokens_per_s": Tp / (prefill_ms / 1e3),
                     "stages_ms": {k: v[1] / args.steps for k, v in prof_p.items() if v[0] or v[1]}},
         "decode": decode,
+        "decode_sweep": sweep,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,

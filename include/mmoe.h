@@ -69,6 +69,9 @@ typedef enum {
 #define MMOE_FLAG_CUDA_CORES 2u    /* run the expert GEMMs on CUDA cores (dp4a) even where the tensor-core
                                       kernels apply (those need d_model and both hidden sizes to be
                                       multiples of 128); same results, slower */
+#define MMOE_FLAG_NO_DECODE 4u     /* never take the decode path: by default a forward with few tokens
+                                      (T <= 64 where d_model and both hidden sizes are multiples of 64)
+                                      runs the weight-streaming decode kernels; same results */
 
 typedef struct {
     int32_t d_model;        /* multiple of 32, 64 <= d_model <= 8192 */

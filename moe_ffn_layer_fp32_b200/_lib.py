@@ -19,6 +19,7 @@ GATE_SOFTMAX = 0
 GATE_SIGMOID_TOPK_NORM = 1
 FLAG_DETERMINISTIC = 1
 FLAG_CUDA_CORES = 2
+FLAG_NO_DECODE = 4
 
 STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAGE_SH, STAGE_LOGITS = range(8)
 

@@ -1,0 +1,702 @@
+// K7: the decode path (T <= 64 tokens), the same mathematics as K1-K6 with
+// the work laid out for streaming weights rather than for reusing them.
+//
+// MobileMoE pages (paper-archivist reading): decode is bound by memory
+// bandwidth (section "on-device inference", the roofline discussion), so every
+// byte of a selected expert is read once and nothing of an unselected one is
+// read.  Eq. (*) and Eq. (6) fix what is computed: the INT32 partial of each
+// 32-element group, scaled by its FP32 weight scale and summed over groups in
+// ascending order, then the per-token activation scale, SwiGLU, the per-row
+// requantisation, the down projection and the gate-weighted combine.
+//
+// Three launches:
+//  1. router_decode_kernel: clusters of `cs` CTAs split the K range of the FP32
+//     router for 16 tokens; partial logits and partial absmax meet in
+//     distributed shared memory, each CTA quantises its slice of x, the owner
+//     CTA of a token runs softmax / top-k.  The last CTA of the launch builds
+//     the expert permutation (counts, offsets, stable scatter).
+//  2. expert_decode_kernel<gate/up>: one warp per 16 weight rows (8 gate + 8
+//     up rows of one output column block) of one selected group.  The warp
+//     streams its rows with bulk copies into a private ring, unpacks INT4 to
+//     INT8 in registers and multiplies with mma.sync m16n8k32 (weights as the
+//     16-row A operand, up to 8 tokens as B).  The accumulator starts at
+//     the bit pattern of 1.5 * 2^19, so the float with the result's bits
+//     minus 1.5 * 2^19 is the group partial exactly (weights enter as 16 x
+//     their code).  SwiGLU in registers, the row absmax by atomicMax.
+//  3. expert_decode_kernel<down>: requantises its group's rows from that
+//     absmax in the prologue, then the same streaming GEMV; the epilogue adds
+//     gate * o into y (or stores o for the fixed-order combine).
+#include <algorithm>
+
+#include "mmoe_internal.cuh"
+#include "sm100_async.cuh"
+
+namespace mmoe {
+namespace dec {
+namespace {
+
+using async::bulk_load;
+using async::clk;
+using async::fence_barrier_init;
+using async::mbar_expect_tx;
+using async::mbar_init;
+using async::mbar_try_wait;
+using async::su32;
+
+// decode weight layout: per group, per block of 16 weight rows, per pair of
+// K groups: 32 lanes x 16 bytes of packed codes, then 8 x 16 bytes of scales
+constexpr int kJP = 640;
+constexpr int kStageJP = 4;                     // K-group pairs per bulk copy
+constexpr int kStageBytes = kStageJP * kJP;     // 2560
+constexpr int kRing = 4;                        // bulk copies in flight per warp
+constexpr int kMaxWarps = 8;
+constexpr int kMaxChunks = 8;                   // 8 tokens per B operand, T <= 64
+constexpr int kHeadBytes = 512;                 // mbarriers (256) + row scales (64 floats)
+constexpr int kMaxT = kMaxChunks * 8;
+constexpr uint32_t kAccBias = 0x49400000u;      // bits of 786432.0f = 1.5 * 2^19 (ulp 1/16)
+constexpr float kAccBiasF = 786432.0f;
+constexpr long long kTimeoutClk = 4000000000ll; // about 2 s of SM clock
+constexpr int kSmemLimit = 232448;
+
+constexpr int kRThreads = 256;
+constexpr int kRTok = 16;                       // tokens per router cluster
+constexpr int kRHeadBytes = (kRTok * 64 + 2 * kRTok + 4) * 4;  // partial logits, absmax, s_x, flag
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// the address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ float ld_peer(const float* p, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(su32(p)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+
+// D = A * B + C on the tensor cores (m16n8k32, INT8 x INT8 -> INT32), C = kAccBias
+__device__ __forceinline__ void mma_bias(int32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    const int32_t c = (int32_t)kAccBias;
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %11, %12, %13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c), "r"(c), "r"(c), "r"(c));
+}
+
+// (a0, a1) = fma((P0, P1), s, (a0, a1)) with P the partials held in v0, v1
+// (float(bits) - 1.5 * 2^19 is exact); paired FP32 instructions, each half an
+// ordinary IEEE operation.
+__device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32_t v1, float s) {
+    asm("{\n\t.reg .b64 t, acc, sc, mg;\n\t"
+        "mov.b64 t, {%2, %3};\n\t"
+        "mov.b64 acc, {%0, %1};\n\t"
+        "mov.b64 mg, {%5, %5};\n\t"
+        "mov.b64 sc, {%4, %4};\n\t"
+        "sub.rn.f32x2 t, t, mg;\n\t"
+        "fma.rn.f32x2 acc, t, sc, acc;\n\t"
+        "mov.b64 {%0, %1}, acc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(v0), "r"(v1), "f"(s), "f"(kAccBiasF));
+}
+
+__device__ __forceinline__ int32_t partial_of(int32_t v) { return (v - (int32_t)kAccBias) >> 4; }
+
+__device__ __forceinline__ void set_error(const Plan& p, int where) {
+    if (p.err) *reinterpret_cast<volatile int*>(p.err) = where;
+    if (p.err_host) *reinterpret_cast<volatile int*>(p.err_host) = where;
+    __threadfence_system();
+}
+
+// bounded wait for the phase of `parity`; false after about 2 s
+__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clk();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (clk() - t0 > kTimeoutClk) return false;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_codes(float a, float b, float c, float d, float s) {
+    return (uint32_t)(quant_i8(a, s) & 0xff) | ((uint32_t)(quant_i8(b, s) & 0xff) << 8) |
+           ((uint32_t)(quant_i8(c, s) & 0xff) << 16) | ((uint32_t)(quant_i8(d, s) & 0xff) << 24);
+}
+
+// ------------------------------------------------------------------ router
+// The permutation of the routing slots, by one block of kRThreads threads:
+// per-expert counts, offsets, the list of groups with rows, and a stable
+// scatter (rows of an expert in ascending slot order).
+__device__ void permute_block(const Plan& p) {
+    __shared__ int cnt[kMaxExperts];
+    __shared__ int base[kMaxExperts];
+    __shared__ int wcnt[kRThreads / 32][kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = p.E, k = p.k;
+    const int S = (int)p.Tk;
+    for (int i = tid; i < kMaxExperts; i += kRThreads) cnt[i] = 0;
+    __syncthreads();
+    for (int s = tid; s < S; s += kRThreads) atomicAdd(&cnt[__ldcg(p.idx + s)], 1);
+    __syncthreads();
+    if (tid == 0) {
+        int o = 0, n = 0;
+        p.dec_groups[n++] = E;
+        for (int e = 0; e < E; ++e) {
+            base[e] = o;
+            p.offsets[e] = o;
+            p.counts[e] = cnt[e];
+            o += cnt[e];
+            if (cnt[e]) p.dec_groups[n++] = e;
+        }
+        p.offsets[E] = o;
+        p.offsets[E + 1] = o + (int)p.T;
+        p.counts[E] = (int)p.T;
+        *p.dec_ngroups = n;
+    }
+    __syncthreads();
+    for (int s0 = 0; s0 < S; s0 += kRThreads) {
+        for (int i = tid; i < (kRThreads / 32) * kMaxExperts; i += kRThreads) (&wcnt[0][0])[i] = 0;
+        __syncthreads();
+        const int s = s0 + tid;
+        const bool valid = s < S;
+        const int e = valid ? __ldcg(p.idx + s) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(same & ((1u << lane) - 1u));
+        if (valid && rank == 0) wcnt[warp][e] = __popc(same);
+        __syncthreads();
+        if (valid) {
+            int pre = 0;
+            for (int w = 0; w < warp; ++w) pre += wcnt[w][e];
+            const int r = base[e] + pre + rank;
+            p.row_src[r] = s / k;
+            p.row_gate[r] = __ldcg(p.gate + s);
+            p.slot_row[s] = r;
+        }
+        __syncthreads();
+        if (tid < E) {
+            int sum = 0;
+            for (int w = 0; w < kRThreads / 32; ++w) sum += wcnt[w][tid];
+            base[tid] += sum;
+        }
+        __syncthreads();
+    }
+    for (int i = tid; i < (int)p.R; i += kRThreads) p.amax_h[i] = 0u;
+    if (tid == 0) *p.dec_ticket = 0;
+}
+
+// grid (cs, ceil(T / 16)), clusters of (cs, 1, 1): cluster y handles tokens
+// [16 y, 16 y + 16), CTA `rank` the K rows [rank ks, (rank + 1) ks).
+__global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int d = p.d, E = p.E;
+    const int ks = d / cs;
+    float* part = reinterpret_cast<float*>(smem);             // [kRTok][64] partial logits
+    float* pmax = part + kRTok * 64;                          // [kRTok] partial absmax
+    float* sxs = pmax + kRTok;                                // [kRTok] s_x
+    int* flag = reinterpret_cast<int*>(sxs + kRTok);
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kRHeadBytes);  // [kRTok][ks]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rank = (int)cluster_rank();
+    const int64_t t0 = (int64_t)blockIdx.y * kRTok;
+    const int nt = (int)((p.T - t0) < kRTok ? (p.T - t0) : kRTok);
+    const int k0 = rank * ks;
+
+    const int nv = ks / 8;
+    for (int i = tid; i < kRTok * nv; i += kRThreads) {
+        const int t = i / nv, v = i % nv;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (t < nt) val = *reinterpret_cast<const uint4*>(p.x + (t0 + t) * d + k0 + v * 8);
+        reinterpret_cast<uint4*>(xs)[i] = val;
+    }
+    __syncthreads();
+    {
+        // expert lane e, tokens tq, tq + 4, tq + 8, tq + 12; FP32 sum over k ascending
+        const int e = tid & 63, tq = tid >> 6;
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (e < E) {
+            const float* w = p.w_router + (int64_t)k0 * E + e;
+            for (int kk = 0; kk < ks; kk += 8) {
+                float wv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) wv[u] = __ldg(w + (int64_t)(kk + u) * E);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xs + (tq + 4 * q) * ks + kk);
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        acc[q] = fmaf(__uint_as_float(xw[u] << 16), wv[2 * u], acc[q]);
+                        acc[q] = fmaf(__uint_as_float(xw[u] & 0xffff0000u), wv[2 * u + 1], acc[q]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) part[(tq + 4 * q) * 64 + e] = acc[q];
+    }
+    for (int t = warp; t < kRTok; t += kRThreads / 32) {
+        float m = 0.0f;
+        for (int i = lane; i < ks; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * ks + i])));
+        m = warp_max(m);
+        if (lane == 0) pmax[t] = m;
+    }
+    cluster_sync();
+    if (tid < kRTok) {
+        float m = 0.0f;
+        for (int c = 0; c < cs; ++c) m = fmaxf(m, ld_peer(&pmax[tid], (uint32_t)c));
+        sxs[tid] = __fdiv_rn(m, 127.0f);
+    }
+    __syncthreads();
+    // K1 on this CTA's slice: codes of the shared-expert rows (rows Tk + t of xq)
+    for (int i = tid; i < nt * (ks / 4); i += kRThreads) {
+        const int t = i / (ks / 4), v = i % (ks / 4);
+        const uint16_t* xr = xs + t * ks + v * 4;
+        const float s = sxs[t];
+        *reinterpret_cast<uint32_t*>(p.xq + (p.Tk + t0 + t) * d + k0 + v * 4) =
+            pack_codes(bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), s);
+    }
+    // logits (slices added in rank order), gating and top-k of the tokens this CTA owns
+    for (int t = rank + warp * cs; t < nt; t += (kRThreads / 32) * cs) {
+        float l0 = -INFINITY, l1 = -INFINITY;
+        if (lane < E) {
+            float s = 0.0f;
+            for (int c = 0; c < cs; ++c) s = __fadd_rn(s, ld_peer(&part[t * 64 + lane], (uint32_t)c));
+            if (p.router_bias) s = __fadd_rn(s, p.router_bias[lane]);
+            l0 = s;
+        }
+        if (lane + 32 < E) {
+            float s = 0.0f;
+            for (int c = 0; c < cs; ++c) s = __fadd_rn(s, ld_peer(&part[t * 64 + lane + 32], (uint32_t)c));
+            if (p.router_bias) s = __fadd_rn(s, p.router_bias[lane + 32]);
+            l1 = s;
+        }
+        const int64_t tg = t0 + t;
+        gate_topk_warp(p, tg, l0, l1, lane);
+        if (lane == 0) {
+            p.sx[tg] = sxs[t];
+            p.row_src[p.Tk + tg] = (int32_t)tg;
+            p.row_gate[p.Tk + tg] = 1.0f;
+        }
+    }
+    __threadfence();  // every writer of idx / gate orders its stores before the ticket below
+    cluster_sync();   // no CTA leaves while a peer may still read its shared memory
+    if (tid == 0) {
+        const int total = (int)(gridDim.x * gridDim.y);
+        flag[0] = atomicAdd(p.dec_ticket, 1) == total - 1;
+    }
+    __syncthreads();
+    if (!flag[0]) return;
+    __threadfence();
+    permute_block(p);
+}
+
+// ------------------------------------------------------------------ experts
+// grid: (groups that can have rows) x nbpg blocks; block: W warps, warp w
+// handles weight-row block blk * W + w of group dec_groups[blockIdx.x / nbpg].
+// Shared memory: mbarriers | row scales | W rings of kRing stages | codes of the
+// group's rows [8 * chunks][K + 32] (B-fragment order inside each 32-group).
+template <bool GU, bool DUMP>
+__global__ void __launch_bounds__(kMaxWarps * 32)
+expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnrows)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int W = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    float* shs = reinterpret_cast<float*>(smem + 256);
+    uint8_t* ring = smem + kHeadBytes;
+    uint8_t* codes = ring + W * kRing * kStageBytes;
+
+    if (GU && !DUMP && !p.deterministic && p.y) {
+        // y is accumulated by the down launch: clear it here, spread over every CTA
+        const int64_t n4 = p.T * p.d / 4;
+        const int64_t per = (n4 + gridDim.x - 1) / gridDim.x;
+        const int64_t a = (int64_t)blockIdx.x * per, b = a + per < n4 ? a + per : n4;
+        float4* y4 = reinterpret_cast<float4*>(p.y);
+        for (int64_t i = a + tid; i < b; i += blockDim.x) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+
+    const int gi = blockIdx.x / nbpg, blk = blockIdx.x % nbpg;
+    if (gi >= *p.dec_ngroups) return;
+    const int g = p.dec_groups[gi];
+    const int hid = g == p.E ? p.hs : p.h;
+    const int K = GU ? p.d : hid;
+    const int nrb = GU ? hid / 8 : p.d / 16;
+    const int rb0 = blk * W;
+    if (rb0 >= nrb) return;
+    const int nrows = p.counts[g];
+    const int64_t row0 = p.offsets[g];
+    const int nch = (nrows + 7) >> 3;
+    const int NJ = K / 64, nst = (NJ + kStageJP - 1) / kStageJP;
+    const int cs = K + 32;
+    const int rb = rb0 + warp;
+    const bool wact = rb < nrb;
+    uint64_t* wb = bars + warp * kRing;
+    uint8_t* wr = ring + warp * kRing * kStageBytes;
+    const uint8_t* src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
+                             : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
+                         (int64_t)rb * NJ * kJP;
+    auto issue = [&](int st) {
+        const int jp = NJ - st * kStageJP;
+        const uint32_t bytes = (uint32_t)((jp < kStageJP ? jp : kStageJP) * kJP);
+        uint64_t* bar = &wb[st % kRing];
+        mbar_expect_tx(bar, bytes);
+        bulk_load(wr + (st % kRing) * kStageBytes, src + (int64_t)st * kStageBytes, bytes, bar);
+    };
+    if (lane == 0) {
+        for (int s = 0; s < kRing; ++s) mbar_init(&wb[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (wact && lane == 0)
+        for (int s = 0; s < kRing && s < nst; ++s) issue(s);
+
+    // codes of the group's rows, zero rows up to a multiple of 8
+    const int ngr = K / 32;
+    if (GU) {
+        for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
+            const int i = it / ngr, j = it % ngr;
+            uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+            if (i < nrows) {
+                const int64_t t = p.row_src[row0 + i];
+                const uint4* s4 = reinterpret_cast<const uint4*>(p.xq + (p.Tk + t) * p.d + j * 32);
+                u0 = s4[0];
+                u1 = s4[1];
+            }
+            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
+            dst[0] = make_uint4(u0.x, u1.x, u0.y, u1.y);
+            dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
+        }
+    } else {
+        for (int i = tid; i < nch * 8; i += blockDim.x)
+            shs[i] = i < nrows ? __fdiv_rn(__uint_as_float(p.amax_h[row0 + i]), 127.0f) : 0.0f;
+        __syncthreads();
+        const bool keep = blk == 0 && !DUMP;  // one CTA per group records h_q and s_h
+        for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
+            const int i = it / ngr, j = it % ngr;
+            uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (i < nrows) {
+                const float s = shs[i];
+                const float4* a4 = reinterpret_cast<const float4*>(p.act + (row0 + i) * p.hmax + j * 32);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 a = a4[v];
+                    wv[v] = pack_codes(a.x, a.y, a.z, a.w, s);
+                }
+                if (keep) {
+                    uint4* q4 = reinterpret_cast<uint4*>(p.hq + (row0 + i) * p.hmax + j * 32);
+                    q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
+            dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
+            dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+        }
+        if (keep)
+            for (int i = tid; i < nrows; i += blockDim.x) p.sh[row0 + i] = shs[i];
+    }
+    __syncthreads();
+    if (!wact) return;
+
+    float alo[kMaxChunks][2], ahi[kMaxChunks][2];
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) alo[c][0] = alo[c][1] = ahi[c][0] = ahi[c][1] = 0.0f;
+    const int ng = p.d / kGroup, ngh = p.hmax / kGroup;
+    for (int st = 0; st < nst; ++st) {
+        if (!wait_bounded(&wb[st % kRing], (uint32_t)((st / kRing) & 1))) {
+            if (lane == 0) set_error(p, 7);
+            // let the copies in flight land before the CTA's shared memory goes away
+            const int issued = st + kRing < nst ? st + kRing : nst;
+            for (int s = st; s < issued; ++s) wait_bounded(&wb[s % kRing], (uint32_t)((s / kRing) & 1));
+            return;
+        }
+        const uint8_t* sb = wr + (st % kRing) * kStageBytes;
+        const int njs = NJ - st * kStageJP < kStageJP ? NJ - st * kStageJP : kStageJP;
+        for (int q = 0; q < njs; ++q) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(sb + q * kJP + lane * 16);
+            const float4 sv = *reinterpret_cast<const float4*>(sb + q * kJP + 512 + gid * 16);
+            const int jp = st * kStageJP + q;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const uint32_t w0 = jj ? wv.z : wv.x, w1 = jj ? wv.w : wv.y;
+                const float slo = jj ? sv.z : sv.x, shi = jj ? sv.w : sv.y;
+                const uint32_t a0 = (w0 << 4) & 0xF0F0F0F0u, a1 = w0 & 0xF0F0F0F0u;
+                const uint32_t a2 = (w1 << 4) & 0xF0F0F0F0u, a3 = w1 & 0xF0F0F0F0u;
+                const int j = 2 * jp + jj;
+                const uint8_t* bp = codes + (size_t)gid * cs + j * 32 + t4 * 8;
+#pragma unroll
+                for (int c = 0; c < kMaxChunks; ++c) {
+                    if (c < nch) {
+                        const uint2 b = *reinterpret_cast<const uint2*>(bp + (size_t)c * 8 * cs);
+                        int32_t dd[4];
+                        mma_bias(dd, a0, a1, a2, a3, b.x, b.y);
+                        if (DUMP) {
+#pragma unroll
+                            for (int q2 = 0; q2 < 2; ++q2) {
+                                const int i = c * 8 + 2 * t4 + q2;
+                                const int64_t r = row0 + i;
+                                if (i < nrows && r >= drow0 && r < drow0 + dnrows) {
+                                    if (GU) {
+                                        int32_t* base = dump + (r - drow0) * 2 * p.hmax * ng;
+                                        const int n = rb * 8 + gid;
+                                        base[(int64_t)n * ng + j] = partial_of(dd[q2]);
+                                        base[(int64_t)(p.hmax + n) * ng + j] = partial_of(dd[2 + q2]);
+                                    } else {
+                                        const int m = rb * 16 + gid;
+                                        dump[((r - drow0) * p.d + m) * ngh + j] = partial_of(dd[q2]);
+                                        dump[((r - drow0) * p.d + m + 8) * ngh + j] = partial_of(dd[2 + q2]);
+                                    }
+                                }
+                            }
+                        }
+                        promote2(alo[c][0], alo[c][1], dd[0], dd[1], slo);
+                        promote2(ahi[c][0], ahi[c][1], dd[2], dd[3], shi);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && st + kRing < nst) issue(st + kRing);
+    }
+    if (DUMP) return;
+
+    if (GU) {
+        const int n = rb * 8 + gid;
+#pragma unroll
+        for (int c = 0; c < kMaxChunks; ++c) {
+            if (c < nch) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int i = c * 8 + 2 * t4 + q;
+                    const bool valid = i < nrows;
+                    const int64_t r = row0 + i;
+                    float a = 0.0f;
+                    if (valid) {
+                        const float sxr = p.sx[p.row_src[r]];
+                        const float gv = __fmul_rn(alo[c][q], sxr), uv = __fmul_rn(ahi[c][q], sxr);
+                        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+                        a = __fmul_rn(silu, uv);
+                        p.act[r * p.hmax + n] = a;
+                    }
+                    float m = fabsf(a);
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                    if (valid && gid == 0) atomicMax(p.amax_h + r, __float_as_uint(m));
+                }
+            }
+        }
+    } else {
+        const int m0 = rb * 16 + gid;
+#pragma unroll
+        for (int c = 0; c < kMaxChunks; ++c) {
+            if (c < nch) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int i = c * 8 + 2 * t4 + q;
+                    if (i >= nrows) continue;
+                    const int64_t r = row0 + i;
+                    const float s = shs[i];
+                    const float olo = __fmul_rn(alo[c][q], s), ohi = __fmul_rn(ahi[c][q], s);
+                    if (p.deterministic) {
+                        p.obuf[r * p.d + m0] = olo;
+                        p.obuf[r * p.d + m0 + 8] = ohi;
+                    } else {
+                        const float gt = p.row_gate[r];
+                        float* yr = p.y + (int64_t)p.row_src[r] * p.d;
+                        atomicAdd(yr + m0, __fmul_rn(gt, olo));
+                        atomicAdd(yr + m0 + 8, __fmul_rn(gt, ohi));
+                    }
+                }
+            }
+        }
+    }
+}
+
+// INT4 interchange layout -> decode layout (see the top of this file).  For
+// gate/up, row block rb holds gate rows 8 rb .. 8 rb + 7 (the A rows 0-7) and
+// the matching up rows (A rows 8-15); for down, output rows 16 rb .. 16 rb + 15.
+// Lane (gid, t4) of K-group pair jp gets, for each of the two groups, the
+// words of A-fragment columns 4 t4 .. 4 t4 + 3 and 16 + 4 t4 .. 16 + 4 t4 + 3:
+// byte b = (code of row gid + 8) << 4 | (code of row gid).
+__global__ void retile_decode_kernel(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
+                                     uint8_t* gu_d, uint8_t* dn_d, int d, int h, int hs, int E)
+{
+    const int g = blockIdx.y;
+    const bool down = blockIdx.z == 1;
+    const int hid = g == E ? hs : h;
+    const int K = down ? hid : d;
+    const int nrb = down ? d / 16 : hid / 8;
+    const int NJ = K / 64;
+    const uint8_t* w = down ? dn + (int64_t)g * d * (h / 2) : gu + (int64_t)g * 2 * h * (d / 2);
+    const float* s = down ? sdn + (int64_t)g * d * (h / kGroup) : sgu + (int64_t)g * 2 * h * (d / kGroup);
+    uint8_t* dst = down ? dn_d + (int64_t)g * ((int64_t)d * h * 5 / 8) : gu_d + (int64_t)g * ((int64_t)h * d * 5 / 4);
+    const int rowb = K / 2, rows_s = K / kGroup;
+    const int64_t units = (int64_t)nrb * NJ * 32;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
+        const int lane = (int)(u & 31);
+        const int64_t q = u >> 5;
+        const int jp = (int)(q % NJ), rb = (int)(q / NJ);
+        const int gid = lane >> 2, t4 = lane & 3;
+        const int rlo = down ? rb * 16 + gid : rb * 8 + gid;
+        const int rhi = down ? rlo + 8 : hid + rb * 8 + gid;
+        uint32_t wv[4];
+        for (int jj = 0; jj < 2; ++jj)
+            for (int wd = 0; wd < 2; ++wd) {
+                uint32_t word = 0;
+                for (int b = 0; b < 4; ++b) {
+                    const int kk = (2 * jp + jj) * 32 + wd * 16 + 4 * t4 + b;
+                    const uint32_t nlo = (w[(int64_t)rlo * rowb + kk / 2] >> (4 * (kk & 1))) & 0xFu;
+                    const uint32_t nhi = (w[(int64_t)rhi * rowb + kk / 2] >> (4 * (kk & 1))) & 0xFu;
+                    word |= ((nhi << 4) | nlo) << (8 * b);
+                }
+                wv[jj * 2 + wd] = word;
+            }
+        uint8_t* o = dst + ((int64_t)rb * NJ + jp) * kJP;
+        *reinterpret_cast<uint4*>(o + lane * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        if (t4 == 0) {
+            const int j0 = 2 * jp, j1 = j0 + 1;
+            *reinterpret_cast<float4*>(o + 512 + gid * 16) =
+                make_float4(s[(int64_t)rlo * rows_s + j0], s[(int64_t)rhi * rows_s + j0],
+                            s[(int64_t)rlo * rows_s + j1], s[(int64_t)rhi * rows_s + j1]);
+        }
+    }
+}
+
+int sm_count() {
+    static int n[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!n[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        n[dev] = v > 0 ? v : 148;
+    }
+    return n[dev];
+}
+
+size_t expert_smem(int W, int64_t T, int K) {
+    return (size_t)kHeadBytes + (size_t)W * kRing * kStageBytes + (size_t)((T + 7) / 8) * 8 * (K + 32);
+}
+
+// warps per CTA: as many as keep at least two CTAs per SM busy
+int pick_warps(int64_t items) {
+    int W = kMaxWarps;
+    while (W > 1 && (items + W - 1) / W < 2 * sm_count()) W >>= 1;
+    return W;
+}
+
+template <bool GU>
+cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t r0, int64_t nr) {
+    if (p.T == 0) return cudaSuccess;
+    const int gmax = (int)(p.Tk < p.E ? p.Tk : p.E) + 1;
+    const int max_nrb = GU ? p.hmax / 8 : p.d / 16;
+    const int W = pick_warps((int64_t)gmax * max_nrb);
+    const int nbpg = (max_nrb + W - 1) / W;
+    const size_t smem = expert_smem(W, p.T, GU ? p.d : p.hmax);
+    auto kern = dump ? expert_decode_kernel<GU, true> : expert_decode_kernel<GU, false>;
+    // raise the shared-memory opt-in only when it grows (keeps the call out of stream captures)
+    static int granted[2][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int* have = (dev >= 0 && dev < 64) ? &granted[dump ? 1 : 0][dev] : nullptr;
+    if (!have || *have < (int)smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (have) *have = (int)smem;
+    }
+    kern<<<(unsigned)(gmax * nbpg), W * 32, smem, s>>>(p, nbpg, dump, r0, nr);
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace dec
+
+bool dec_supported(int d, int h, int hs) { return d % 64 == 0 && h % 64 == 0 && hs % 64 == 0; }
+
+int dec_max_tokens(int d, int hmax) {
+    const int K = d > hmax ? d : hmax;
+    int T = dec::kMaxT;
+    while (T > 0 && dec::expert_smem(dec::kMaxWarps, T, K) > (size_t)dec::kSmemLimit) T -= 8;
+    return T;
+}
+
+// CTAs per router cluster: 16 (non-portable size) where the device runs it,
+// else 8, else 4; each CTA's K slice must be a multiple of 8 elements.
+int dec_router_cluster(int d) {
+    const size_t smem = dec::kRHeadBytes + (size_t)dec::kRTok * (d / 4) * 2;
+    if (cudaFuncSetAttribute(dec::router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return 0;
+    for (int cs = 16; cs >= 4; cs >>= 1) {
+        if (d % (8 * cs)) continue;
+        if (cs > 8 &&
+            cudaFuncSetAttribute(dec::router_decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            continue;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cs, 1, 1);
+        cfg.blockDim = dim3(dec::kRThreads, 1, 1);
+        cfg.dynamicSmemBytes = dec::kRHeadBytes + (size_t)dec::kRTok * (d / cs) * 2;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = cs;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, dec::router_decode_kernel, &cfg) == cudaSuccess && n > 0) return cs;
+        cudaGetLastError();
+    }
+    return 0;
+}
+
+cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s) {
+    if (p.T == 0) return cudaSuccess;
+    const size_t smem = dec::kRHeadBytes + (size_t)dec::kRTok * (p.d / cluster) * 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cluster, (unsigned)((p.T + dec::kRTok - 1) / dec::kRTok), 1);
+    cfg.blockDim = dim3(dec::kRThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)cluster;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, dec::router_decode_kernel, p, cluster);
+}
+
+cudaError_t launch_gate_up_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
+    return dec::launch_expert<true>(p, s, dump, row0, nrows);
+}
+
+cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
+    return dec::launch_expert<false>(p, s, dump, row0, nrows);
+}
+
+cudaError_t launch_retile_dec(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
+                              uint8_t* gu_d, uint8_t* dn_d, int d, int h, int hs, int E, cudaStream_t s) {
+    dim3 grid(64, (unsigned)(E + 1), 2);
+    dec::retile_decode_kernel<<<grid, 256, 0, s>>>(gu, sgu, dn, sdn, gu_d, dn_d, d, h, hs, E);
+    return cudaGetLastError();
+}
+
+}  // namespace mmoe

@@ -40,6 +40,7 @@
 #include <cudaTypedefs.h>
 
 #include "mmoe_internal.cuh"
+#include "sm100_async.cuh"
 
 namespace mmoe {
 namespace tc {
@@ -93,43 +94,14 @@ struct Smem {
 };
 
 // ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(su32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ long long clk() {
-    long long t;
-    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
-    return t;
-}
+using async::su32;
+using async::mbar_init;
+using async::mbar_expect_tx;
+using async::mbar_arrive;
+using async::mbar_try_wait;
+using async::clk;
+using async::bulk_load;
+using async::fence_barrier_init;
 
 // Waits for the phase of the given parity; gives up after kTimeoutClk SM
 // clocks or once another thread of the CTA has given up.  On giving up it
@@ -161,13 +133,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Smem* 
     return mbar_wait_slow(bar, parity, sm, err, where);
 }
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     su32(dst)),
-                 "l"(src), "r"(bytes), "r"(su32(bar))
-                 : "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
@@ -177,7 +142,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 }
 
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 __device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -248,6 +212,22 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
 constexpr float kMagic = 12582912.0f;
+
+// Two columns at once with paired FP32 instructions (each half is an ordinary IEEE
+// operation, so the results equal the scalar ones):
+// (a0, a1) = fma((float(v0) - 1.5 * 2^23, float(v1) - 1.5 * 2^23), s, (a0, a1))
+__device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32_t v1, float s) {
+    asm("{\n\t.reg .b64 t, acc, sc, mg;\n\t"
+        "mov.b64 t, {%2, %3};\n\t"
+        "mov.b64 acc, {%0, %1};\n\t"
+        "mov.b64 mg, {%5, %5};\n\t"
+        "mov.b64 sc, {%4, %4};\n\t"
+        "sub.rn.f32x2 t, t, mg;\n\t"
+        "fma.rn.f32x2 acc, t, sc, acc;\n\t"
+        "mov.b64 {%0, %1}, acc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(v0), "r"(v1), "f"(s), "f"(12582912.0f));
+}
 
 // exact int32 -> float for |v| < 2^22: integer add into the mantissa of 1.5 * 2^23
 __device__ __forceinline__ float exact_i2f(int32_t v) { return __int_as_float(v + 0x4B400000) - 12582912.0f; }
@@ -547,12 +527,12 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                     tmem_wait_ld();
                     tmem_st16_const(ta, kMagicBits);
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) acc[c] = fmaf(__int_as_float(v[c]) - kMagic, sc, acc[c]);
+                    for (int c = 0; c < 16; c += 2) promote2(acc[c], acc[c + 1], v[c], v[c + 1], sc);
                     tmem_ld16(ta + 16, w);
                     tmem_wait_ld();
                     tmem_st16_const(ta + 16, kMagicBits);
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) acc[16 + c] = fmaf(__int_as_float(w[c]) - kMagic, sc, acc[16 + c]);
+                    for (int c = 0; c < 16; c += 2) promote2(acc[16 + c], acc[17 + c], w[c], w[c + 1], sc);
                     if (kDump) {
                         // INT32 partials of rows [drow0, drow0 + dnrows) for the inspection entry point
                         const int jg = j + gg;

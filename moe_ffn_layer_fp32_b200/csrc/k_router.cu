@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(kThreads)
 router_quant_kernel(Plan p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    const int d = p.d, E = p.E, k = p.k;
+    const int d = p.d, E = p.E;
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem);              // [TB][d]
     float* part = reinterpret_cast<float*>(xs + (size_t)TB * d);   // [4][TB][64]
     float* lg = part + 4 * TB * 64;                                // [TB][64]
@@ -107,57 +107,9 @@ router_quant_kernel(Plan p)
     // gating and top-k: one warp per token, lanes hold experts lane and lane + 32
     for (int tt = warp; tt < nt; tt += kThreads / 32) {
         const int64_t t = t0 + tt;
-        const bool v0 = lane < E, v1 = lane + 32 < E;
-        const float l0 = v0 ? lg[tt * 64 + lane] : -INFINITY;
-        const float l1 = v1 ? lg[tt * 64 + lane + 32] : -INFINITY;
-        if (p.logits) {
-            if (v0) p.logits[t * E + lane] = l0;
-            if (v1) p.logits[t * E + lane + 32] = l1;
-        }
-        float p0, p1;
-        if (p.gating == MMOE_GATE_SOFTMAX) {
-            const float mx = warp_max(fmaxf(l0, l1));
-            const float e0 = v0 ? expf(__fsub_rn(l0, mx)) : 0.0f;
-            const float e1 = v1 ? expf(__fsub_rn(l1, mx)) : 0.0f;
-            const float sum = warp_sum(__fadd_rn(e0, e1));
-            p0 = __fdiv_rn(e0, sum);
-            p1 = __fdiv_rn(e1, sum);
-        } else {
-            p0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l0)));
-            p1 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l1)));
-        }
-        bool taken0 = !v0, taken1 = !v1;
-        int sel[kMaxTopK];
-        float gsel[kMaxTopK];
-        float gsum = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            // this lane's best untaken candidate, then a warp arg-max on (logit desc, index asc)
-            float bv = -INFINITY;
-            int bi = 1 << 30;
-            if (!taken0) { bv = l0; bi = lane; }
-            if (!taken1 && (l1 > bv || bi == (1 << 30))) { bv = l1; bi = lane + 32; }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-            }
-            sel[j] = bi;
-            if (bi == lane) taken0 = true;
-            if (bi == lane + 32) taken1 = true;
-            const float pv = __shfl_sync(0xffffffffu, (bi < 32) ? p0 : p1, bi & 31);
-            gsel[j] = pv;
-            gsum = __fadd_rn(gsum, pv);
-        }
-        if (lane < k) {
-            int my = 0;
-            float g = 0.0f;
-            for (int j = 0; j < k; ++j)
-                if (j == lane) { my = sel[j]; g = gsel[j]; }
-            if (p.gating != MMOE_GATE_SOFTMAX) g = __fdiv_rn(g, gsum);
-            p.idx[t * k + lane] = my;
-            p.gate[t * k + lane] = g;
-        }
+        const float l0 = lane < E ? lg[tt * 64 + lane] : -INFINITY;
+        const float l1 = lane + 32 < E ? lg[tt * 64 + lane + 32] : -INFINITY;
+        gate_topk_warp(p, t, l0, l1, lane);
     }
 }
 

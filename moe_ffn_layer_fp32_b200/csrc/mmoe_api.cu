@@ -104,6 +104,17 @@ struct mmoe_handle {
     int* err_host = nullptr;   // mapped pinned host memory; kernels write its device alias
     int* err_host_dev = nullptr;
     int* err_dev = nullptr;    // device memory copy read by every CTA
+    // decode path: weights in the decode layout, row absmax, group list, router ticket
+    bool use_dec = false;
+    bool last_dec = false;
+    int dec_max_T = 0;
+    int dec_cluster = 0;
+    uint8_t* w_gate_up_d = nullptr;
+    uint8_t* w_down_d = nullptr;
+    uint32_t* amax_h = nullptr;
+    int32_t* dec_groups = nullptr;
+    int32_t* dec_ngroups = nullptr;
+    int32_t* dec_ticket = nullptr;
     // per-stage timing (mmoe_profile_*)
     struct ProfRec {
         int stage, launches;
@@ -130,7 +141,8 @@ void free_all(mmoe_handle* h) {
                     h->xq, h->sx, h->logits, h->idx, h->gate, h->chunk_cnt, h->chunk_base, h->offsets,
                     h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
                     h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
-                    h->s_down_t, h->err_dev};
+                    h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->amax_h, h->dec_groups,
+                    h->dec_ngroups, h->dec_ticket};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);
@@ -157,7 +169,7 @@ mmoe_status check_config(const mmoe_config* c) {
         return fail(MMOE_ERR_INVALID_ARG, "gating=%d: unknown", c->gating);
     if (c->has_router_bias != 0 && c->has_router_bias != 1)
         return fail(MMOE_ERR_INVALID_ARG, "has_router_bias=%d: must be 0 or 1", c->has_router_bias);
-    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES))
+    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE))
         return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
     return MMOE_OK;
 }
@@ -214,6 +226,12 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.tmap_hq = h->tmap_hq;
     p.err = h->err_dev;
     p.err_host = h->err_host_dev;
+    p.w_gate_up_d = h->w_gate_up_d;
+    p.w_down_d = h->w_down_d;
+    p.amax_h = h->amax_h;
+    p.dec_groups = h->dec_groups;
+    p.dec_ngroups = h->dec_ngroups;
+    p.dec_ticket = h->dec_ticket;
     return p;
 }
 
@@ -379,11 +397,23 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(sh, R);
     if (cfg->flags & MMOE_FLAG_DETERMINISTIC) ALLOC(obuf, R * d);
     h->use_tc = !(cfg->flags & MMOE_FLAG_CUDA_CORES) && tc_supported((int)d, (int)hh, (int)hs);
-    if (h->use_tc) {
-        ALLOC(w_gate_up_t, h->n_gu_bytes);
-        ALLOC(s_gate_up_t, h->n_gu_scales);
-        ALLOC(w_down_t, h->n_d_bytes);
-        ALLOC(s_down_t, h->n_d_scales);
+    h->use_dec = !(cfg->flags & (MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE)) && dec_supported((int)d, (int)hh, (int)hs);
+    if (h->use_dec) {
+        h->dec_max_T = dec_max_tokens((int)d, h->hmax);
+        h->dec_cluster = dec_router_cluster((int)d);
+        if (h->dec_max_T <= 0 || h->dec_cluster == 0) h->use_dec = false;
+    }
+    if (h->use_dec) {
+        const int64_t Rd = (Tm < h->dec_max_T ? Tm : h->dec_max_T) * (k + 1);
+        ALLOC(w_gate_up_d, h->n_gu_bytes + h->n_gu_scales * 4);
+        ALLOC(w_down_d, h->n_d_bytes + h->n_d_scales * 4);
+        ALLOC(amax_h, Rd);
+        ALLOC(dec_groups, E + 1);
+        ALLOC(dec_ngroups, 1);
+        ALLOC(dec_ticket, 1);
+        if (e == cudaSuccess) e = cudaMemset(h->dec_ticket, 0, sizeof(int32_t));
+    }
+    if (h->use_tc || h->use_dec) {
         ALLOC(err_dev, 1);
         if (e == cudaSuccess) e = cudaMemset(h->err_dev, 0, sizeof(int));
         if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&h->err_host), sizeof(int), cudaHostAllocMapped);
@@ -391,6 +421,12 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
             *h->err_host = 0;
             e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->err_host_dev), h->err_host, 0);
         }
+    }
+    if (h->use_tc) {
+        ALLOC(w_gate_up_t, h->n_gu_bytes);
+        ALLOC(s_gate_up_t, h->n_gu_scales);
+        ALLOC(w_down_t, h->n_d_bytes);
+        ALLOC(s_down_t, h->n_d_scales);
         if (e == cudaSuccess) e = make_tensor_map(h->tmap_xq, h->xq, (uint64_t)d, (uint64_t)R, (uint64_t)d);
         if (e == cudaSuccess) e = make_tensor_map(h->tmap_hq, h->hq, (uint64_t)h->hmax, (uint64_t)R, (uint64_t)h->hmax);
     }
@@ -427,6 +463,10 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
                                 h->w_down_t, h->s_down_t, h->cfg.d_model, h->cfg.expert_hidden, h->cfg.shared_hidden,
                                 h->cfg.n_experts, s),
                   "weight re-tiling launch");
+    if (h->use_dec)
+        MMOE_CUDA(launch_retile_dec(h->w_gate_up, h->s_gate_up, h->w_down, h->s_down, h->w_gate_up_d, h->w_down_d,
+                                    h->cfg.d_model, h->cfg.expert_hidden, h->cfg.shared_hidden, h->cfg.n_experts, s),
+                  "decode-layout re-tiling launch");
     h->loaded = true;
     return MMOE_OK;
 }
@@ -445,17 +485,29 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     mmoe_status fst = check_device_flag(h, s);
     if (fst != MMOE_OK) return fst;
     const Plan p = make_plan(h, x, T, y);
-    if (!p.deterministic)
+    const bool dec = h->use_dec && T <= h->dec_max_T;
+    if (dec) {
+        // decode path: router + permutation, gate/up (also clears y), down
+        MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_dec(p, h->dec_cluster, s); }),
+                  "decode router launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return launch_gate_up_dec(p, s, nullptr, 0, 0); }),
+                  "decode gate/up launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return launch_down_dec(p, s, nullptr, 0, 0); }),
+                  "decode down launch");
+    }
+    if (!dec && !p.deterministic)
         MMOE_CUDA(run_stage(h, MMOE_PROF_ZERO_Y, 0, s,
                             [&] { return cudaMemsetAsync(y, 0, (size_t)T * p.d * sizeof(float), s); }),
                   "zero y");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_quant(p, s); }),
-              "router/quantiser launch");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_PERMUTE, 4, s, [&] { return launch_permute(p, s); }), "permute launch");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return run_gate_up(p, s, nullptr, 0, 0); }),
-              "gate/up launch");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
-    MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return run_down(p, s, nullptr, 0, 0); }), "down launch");
+    if (!dec) {
+        MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_quant(p, s); }),
+                  "router/quantiser launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_PERMUTE, 4, s, [&] { return launch_permute(p, s); }), "permute launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return run_gate_up(p, s, nullptr, 0, 0); }),
+                  "gate/up launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return run_down(p, s, nullptr, 0, 0); }), "down launch");
+    }
     if (p.deterministic)
         MMOE_CUDA(run_stage(h, MMOE_PROF_COMBINE, 1, s, [&] { return launch_combine(p, s); }), "combine launch");
     if (topk_idx)
@@ -469,6 +521,7 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
                                   cudaMemcpyDeviceToDevice, s),
                   "copy expert_counts");
     h->last_T = T;
+    h->last_dec = dec;
     return MMOE_OK;
 }
 
@@ -566,8 +619,13 @@ mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int
     DeviceGuard dg(h->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Plan p = make_plan(h, nullptr, h->last_T, nullptr);
-    if (which == 0) MMOE_CUDA(run_gate_up(p, s, dst, row0, nrows), "gate/up dump launch");
-    else MMOE_CUDA(run_down(p, s, dst, row0, nrows), "down dump launch");
+    if (h->last_dec) {
+        if (which == 0) MMOE_CUDA(launch_gate_up_dec(p, s, dst, row0, nrows), "gate/up dump launch");
+        else MMOE_CUDA(launch_down_dec(p, s, dst, row0, nrows), "down dump launch");
+    } else {
+        if (which == 0) MMOE_CUDA(run_gate_up(p, s, dst, row0, nrows), "gate/up dump launch");
+        else MMOE_CUDA(run_down(p, s, dst, row0, nrows), "down dump launch");
+    }
     return MMOE_OK;
 }
 

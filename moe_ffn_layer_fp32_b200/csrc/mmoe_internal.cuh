@@ -63,6 +63,13 @@ struct Plan {
     const void* tmap_hq;
     int* err;                     // device flag: a bounded wait gave up (later CTAs exit at once)
     int* err_host;                // device alias of the host-mapped copy of that flag
+    // decode path (k_decode.cu)
+    const uint8_t* w_gate_up_d;   // weights + scales in the decode layout
+    const uint8_t* w_down_d;
+    uint32_t* amax_h;             // [R] bits of max |SwiGLU output| of each row (non-negative floats order as integers)
+    int32_t* dec_groups;          // [E + 1] groups with at least one row: the shared one first, then routed ascending
+    int32_t* dec_ngroups;         // [1]
+    int32_t* dec_ticket;          // [1] router CTAs finished; 0 between launches
 };
 
 // Upper bound on the number of tile_rows-row tiles over all groups.
@@ -83,6 +90,15 @@ cudaError_t launch_gate_up_tc(const Plan& p, cudaStream_t s, int32_t* dump, int6
 cudaError_t launch_down_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_retile(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn, uint8_t* gu_t,
                           float* sgu_t, uint8_t* dn_t, float* sdn_t, int d, int h, int hs, int E, cudaStream_t s);
+// decode path (k_decode.cu): T <= dec_max_tokens, expert GEMVs on mma.sync
+bool dec_supported(int d, int h, int hs);
+int dec_max_tokens(int d, int hmax);
+int dec_router_cluster(int d);
+cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s);
+cudaError_t launch_gate_up_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
+cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
+cudaError_t launch_retile_dec(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
+                              uint8_t* gu_d, uint8_t* dn_d, int d, int h, int hs, int E, cudaStream_t s);
 size_t tensor_map_bytes();
 cudaError_t make_tensor_map(void* map, void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_stride);
 cudaError_t launch_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t* packed, float* scales,
@@ -109,6 +125,63 @@ __device__ __forceinline__ int quant_i8(float v, float s) {
     if (!(s > 0.0f)) return 0;
     int q = __float2int_rn(__fdiv_rn(v, s));
     return max(-127, min(127, q));
+}
+
+// Gating and top-k of token t by one warp.  Lane l holds the logits of
+// experts l and l + 32 (-inf where the expert does not exist).  Softmax over
+// all experts (or per-expert sigmoid), then k rounds of a warp arg-max on
+// (logit descending, index ascending); writes logits (if kept), idx and gate.
+__device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane) {
+    const int E = p.E, k = p.k;
+    const bool v0 = lane < E, v1 = lane + 32 < E;
+    if (p.logits) {
+        if (v0) p.logits[t * E + lane] = l0;
+        if (v1) p.logits[t * E + lane + 32] = l1;
+    }
+    float p0, p1;
+    if (p.gating == MMOE_GATE_SOFTMAX) {
+        const float mx = warp_max(fmaxf(l0, l1));
+        const float e0 = v0 ? expf(__fsub_rn(l0, mx)) : 0.0f;
+        const float e1 = v1 ? expf(__fsub_rn(l1, mx)) : 0.0f;
+        const float sum = warp_sum(__fadd_rn(e0, e1));
+        p0 = __fdiv_rn(e0, sum);
+        p1 = __fdiv_rn(e1, sum);
+    } else {
+        p0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l0)));
+        p1 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l1)));
+    }
+    bool taken0 = !v0, taken1 = !v1;
+    int sel[kMaxTopK];
+    float gsel[kMaxTopK];
+    float gsum = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        // this lane's best untaken candidate, then a warp arg-max on (logit desc, index asc)
+        float bv = -INFINITY;
+        int bi = 1 << 30;
+        if (!taken0) { bv = l0; bi = lane; }
+        if (!taken1 && (l1 > bv || bi == (1 << 30))) { bv = l1; bi = lane + 32; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        sel[j] = bi;
+        if (bi == lane) taken0 = true;
+        if (bi == lane + 32) taken1 = true;
+        const float pv = __shfl_sync(0xffffffffu, (bi < 32) ? p0 : p1, bi & 31);
+        gsel[j] = pv;
+        gsum = __fadd_rn(gsum, pv);
+    }
+    if (lane < k) {
+        int my = 0;
+        float g = 0.0f;
+        for (int j = 0; j < k; ++j)
+            if (j == lane) { my = sel[j]; g = gsel[j]; }
+        if (p.gating != MMOE_GATE_SOFTMAX) g = __fdiv_rn(g, gsum);
+        p.idx[t * k + lane] = my;
+        p.gate[t * k + lane] = g;
+    }
 }
 
 }  // namespace mmoe

@@ -53,9 +53,10 @@ def test_quantizer_matches_oracle_bit_exact():
     assert np.array_equal(s_gpu.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
-def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False):
+def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False, decode=True):
     T = x.shape[0]
-    L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic, cuda_cores=cuda_cores)
+    L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic, cuda_cores=cuda_cores,
+                          decode=decode)
     out = gu.run_gpu(L, q, x)
     y, D = oracle.moe_layer(q, x, dumps=True)
     rep = {}
@@ -70,14 +71,16 @@ def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, c
     return rep, out
 
 
-@pytest.mark.parametrize("cuda_cores", [False, True], ids=["tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("path", ["decode", "tensor_cores", "cuda_cores"])
 @pytest.mark.parametrize("deterministic", [False, True], ids=["atomic", "fixed_order"])
-def test_c0_all_stages(deterministic, cuda_cores):
+def test_c0_all_stages(deterministic, path):
+    # T = 64 takes the decode kernels by default; the other two force the prefill kernels
     w, q = workload("c0")
     x = synth.workload_x(w)
     R = w.T * (q.k + 1)
-    rep, out = _full_check(q, x, deterministic, partial_rows=range(0, R, 3), cuda_cores=cuda_cores)
-    print("c0", "cuda cores" if cuda_cores else "tensor cores", rep)
+    rep, out = _full_check(q, x, deterministic, partial_rows=range(0, R, 3), cuda_cores=path == "cuda_cores",
+                           decode=path == "decode")
+    print("c0", path, rep)
 
 
 def test_deterministic_mode_is_reproducible():
@@ -89,12 +92,33 @@ def test_deterministic_mode_is_reproducible():
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
 
 
-@pytest.mark.parametrize("T", [1, 2, 7, 31, 33, 63, 65, 127, 129, 300])
-def test_ragged_token_counts(T):
+@pytest.mark.parametrize("T,decode", [(T, True) for T in (1, 2, 7, 31, 33, 63, 64, 65, 127, 129, 300)]
+                         + [(T, False) for T in (1, 7, 33, 64)])
+def test_ragged_token_counts(T, decode):
     w, q = workload("c0")
     x = synth.draw_x(T, w.d, seed=100 + T)
-    rep, out = _full_check(q, x, max_tokens=512, partial_rows=[0, T * q.k - 1, T * q.k, T * (q.k + 1) - 1])
+    rep, out = _full_check(q, x, max_tokens=512, partial_rows=[0, T * q.k - 1, T * q.k, T * (q.k + 1) - 1],
+                           decode=decode)
     assert out["counts"][q.E] == T
+
+
+def test_decode_hot_groups_of_64_rows():
+    # every token to experts 5, 9, 33, 58: four routed groups of 64 rows each (8 token blocks of the decode GEMV)
+    w = synth.WORKLOADS["c0"]
+    lw = synth.draw_layer(w.d, w.h, seed=44, bias_coef=None)
+    lw.router_bias = np.full(60, -30.0, np.float32)
+    lw.router_bias[[5, 9, 33, 58]] = 0.0
+    q = oracle.quantize_layer(lw)
+    x = synth.draw_x(64, w.d, seed=45)
+    rep, out = _full_check(q, x, partial_rows=[0, 63, 64, 255, 256, 319])
+    assert out["counts"][[5, 9, 33, 58]].tolist() == [64] * 4
+
+
+def test_decode_shared_expert_wider_than_routed():
+    lw = synth.draw_layer(256, 64, seed=46, shared_hidden=256)
+    q = oracle.quantize_layer(lw)
+    x = synth.draw_x(40, 256, seed=47)
+    rep, out = _full_check(q, x, partial_rows=[0, 77, 159, 160, 199])
 
 
 def test_c2_prefill_cuda_cores():
