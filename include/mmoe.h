@@ -131,9 +131,13 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
  *   topk_gate     FP32  [T, top_k]  their gates
  *   expert_counts int32 [n_experts + 1] tokens per routed expert, then T for
  *                 the shared expert (the expert-utilisation histogram)
- * T = 0 is a no-op.  x and y must not overlap; y is fully overwritten.
- * Errors: INVALID_ARG (T < 0, T > max_tokens, NULL x or y), NOT_LOADED,
- * TIMEOUT (a bounded wait of an earlier call gave up), CUDA. */
+ * T = 0 is a no-op.  x and y must be 16-byte aligned and must not overlap;
+ * y is fully overwritten.
+ * Paths: T <= 64 runs the decode kernels (weight streaming) unless the config
+ * sets MMOE_FLAG_NO_DECODE or the shapes do not allow them; larger T runs the
+ * prefill kernels (grouped tensor-core GEMMs).  Both give the same results.
+ * Errors: INVALID_ARG (T < 0, T > max_tokens, NULL or misaligned x or y),
+ * NOT_LOADED, TIMEOUT (a bounded wait of an earlier call gave up), CUDA. */
 mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, float* y, void* stream,
                          int32_t* topk_idx, float* topk_gate, int32_t* expert_counts);
 

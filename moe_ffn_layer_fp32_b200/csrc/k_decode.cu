@@ -10,11 +10,11 @@
 // requantisation, the down projection and the gate-weighted combine.
 //
 // Three launches:
-//  1. router_decode_kernel: clusters of `cs` CTAs split the K range of the FP32
-//     router for 16 tokens; partial logits and partial absmax meet in
+//  1. router_decode_kernel: one cluster of `cs` CTAs splits the K range of the
+//     FP32 router for all tokens; partial logits and partial absmax meet in
 //     distributed shared memory, each CTA quantises its slice of x, the owner
-//     CTA of a token runs softmax / top-k.  The last CTA of the launch builds
-//     the expert permutation (counts, offsets, stable scatter).
+//     CTA of a token runs softmax / top-k, and rank 0 builds the expert
+//     permutation (counts, offsets, stable scatter).
 //  2. expert_decode_kernel<gate/up>: one warp per 16 weight rows (8 gate + 8
 //     up rows of one output column block) of one selected group.  The warp
 //     streams its rows with bulk copies into a private ring, unpacks INT4 to
@@ -48,9 +48,10 @@ using async::su32;
 constexpr int kJP = 640;
 constexpr int kStageJP = 4;                     // K-group pairs per bulk copy
 constexpr int kStageBytes = kStageJP * kJP;     // 2560
-constexpr int kRing = 4;                        // bulk copies in flight per warp
+constexpr int kRing = 3;                        // bulk copies in flight per warp
 constexpr int kMaxWarps = 8;
-constexpr int kMaxChunks = 8;                   // 8 tokens per B operand, T <= 64
+constexpr int kMaxChunks = 8;                   // T <= 64 = 8 B operands of 8 tokens
+constexpr int kPassRows = 16;                   // rows of a group per pass (2 B operands)
 constexpr int kHeadBytes = 512;                 // mbarriers (256) + row scales (64 floats)
 constexpr int kMaxT = kMaxChunks * 8;
 constexpr uint32_t kAccBias = 0x49400000u;      // bits of 786432.0f = 1.5 * 2^19 (ulp 1/16)
@@ -59,8 +60,13 @@ constexpr long long kTimeoutClk = 4000000000ll; // about 2 s of SM clock
 constexpr int kSmemLimit = 232448;
 
 constexpr int kRThreads = 256;
-constexpr int kRTok = 16;                       // tokens per router cluster
-constexpr int kRHeadBytes = (kRTok * 64 + 2 * kRTok + 4) * 4;  // partial logits, absmax, s_x, flag
+constexpr int kRTok = 64;                       // tokens of the decode path (one router cluster)
+constexpr int kRHeadBytes = (kRTok * 64 + 2 * kRTok) * 4 + 16;  // partial logits, absmax, s_x, mbarrier
+
+// router shared memory: head | x slice [kRTok][ks] BF16 | W_r slice [ks][E] FP32
+__host__ __device__ constexpr size_t router_smem(int d, int cs, int E) {
+    return (size_t)kRHeadBytes + (size_t)kRTok * (d / cs) * 2 + (size_t)(d / cs) * E * 4;
+}
 
 // ------------------------------------------------------------------ helpers
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -73,13 +79,30 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// the address of the same shared variable in CTA `rank` of the cluster
+// the same shared variable in CTA `rank` of the cluster (read after a cluster barrier)
 __device__ __forceinline__ float ld_peer(const float* p, uint32_t rank) {
     uint32_t a;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(su32(p)), "r"(rank));
     float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a));
     return v;
+}
+
+// v[c] = the variable in CTA c, c < cs <= 16: all loads issued before any is used
+__device__ __forceinline__ void ld_peers(float (&v)[16], const float* p, int cs) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) v[c] = c < cs ? ld_peer(p, (uint32_t)c) : 0.0f;
+}
+
+// sum over the cluster in rank order
+__device__ __forceinline__ float cluster_sum(const float* p, int cs) {
+    float v[16];
+    ld_peers(v, p, cs);
+    float s = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+        if (c < cs) s = __fadd_rn(s, v[c]);
+    return s;
 }
 
 // D = A * B + C on the tensor cores (m16n8k32, INT8 x INT8 -> INT32), C = kAccBias
@@ -107,6 +130,11 @@ __device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32
         : "+f"(a0), "+f"(a1)
         : "r"(v0), "r"(v1), "f"(s), "f"(kAccBiasF));
 }
+
+// programmatic dependent launch: let the next launch of the stream start its
+// prologue / wait until the previous launch has completed and its writes are visible
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ int32_t partial_of(int32_t v) { return (v - (int32_t)kAccBias) >> 4; }
 
@@ -190,11 +218,15 @@ __device__ void permute_block(const Plan& p) {
         __syncthreads();
     }
     for (int i = tid; i < (int)p.R; i += kRThreads) p.amax_h[i] = 0u;
-    if (tid == 0) *p.dec_ticket = 0;
 }
 
-// grid (cs, ceil(T / 16)), clusters of (cs, 1, 1): cluster y handles tokens
-// [16 y, 16 y + 16), CTA `rank` the K rows [rank ks, (rank + 1) ks).
+// One cluster of `cs` CTAs handles all T <= 64 tokens; CTA `rank` the K rows
+// [rank ks, (rank + 1) ks) of W_r and x.  After the first cluster barrier
+// every CTA knows the activation scales (max over the cluster) and quantises
+// its slice; the owner CTA of token t (t mod cs) adds the partial logits in
+// rank order and runs gating and top-k; after the second barrier rank 0
+// builds the permutation (the barrier's release / acquire orders the owners'
+// writes of idx and gate before it).
 __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs)
 {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -203,34 +235,45 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
     float* part = reinterpret_cast<float*>(smem);             // [kRTok][64] partial logits
     float* pmax = part + kRTok * 64;                          // [kRTok] partial absmax
     float* sxs = pmax + kRTok;                                // [kRTok] s_x
-    int* flag = reinterpret_cast<int*>(sxs + kRTok);
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + kRHeadBytes - 16);
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kRHeadBytes);  // [kRTok][ks]
+    float* ws = reinterpret_cast<float*>(xs + kRTok * ks);            // [ks][E]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rank = (int)cluster_rank();
-    const int64_t t0 = (int64_t)blockIdx.y * kRTok;
-    const int nt = (int)((p.T - t0) < kRTok ? (p.T - t0) : kRTok);
+    const int nt = (int)p.T;
     const int k0 = rank * ks;
+    pdl_trigger();
 
-    const int nv = ks / 8;
-    for (int i = tid; i < kRTok * nv; i += kRThreads) {
-        const int t = i / nv, v = i % nv;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (t < nt) val = *reinterpret_cast<const uint4*>(p.x + (t0 + t) * d + k0 + v * 8);
-        reinterpret_cast<uint4*>(xs)[i] = val;
+    // W_r rows and x slices of this CTA: bulk copies (ks * E * 4 and ks * 2 bytes, multiples of 16)
+    if (tid == 0) {
+        mbar_init(wbar, 1);
+        fence_barrier_init();
+        const uint32_t wbytes = (uint32_t)ks * E * 4, xbytes = (uint32_t)ks * 2;
+        mbar_expect_tx(wbar, wbytes + xbytes * nt);
+        bulk_load(ws, p.w_router + (int64_t)k0 * E, wbytes, wbar);
+        for (int t = 0; t < nt; ++t) bulk_load(xs + t * ks, p.x + (int64_t)t * d + k0, xbytes, wbar);
     }
+    // rows of absent tokens are zero (disjoint from the copies)
+    for (int i = nt * (ks / 8) + tid; i < kRTok * (ks / 8); i += kRThreads)
+        reinterpret_cast<uint4*>(xs)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
+    const bool have = wait_bounded(wbar, 0);
+    if (!have && tid == 0) set_error(p, 8);
     {
-        // expert lane e, tokens tq, tq + 4, tq + 8, tq + 12; FP32 sum over k ascending
+        // expert lane e, tokens tq + 4 q; FP32 sum over k ascending
         const int e = tid & 63, tq = tid >> 6;
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (e < E) {
-            const float* w = p.w_router + (int64_t)k0 * E + e;
+        float acc[kRTok / 4];
+#pragma unroll
+        for (int q = 0; q < kRTok / 4; ++q) acc[q] = 0.0f;
+        if (e < E && have && tq < nt) {
+            const float* w = ws + e;
             for (int kk = 0; kk < ks; kk += 8) {
                 float wv[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) wv[u] = __ldg(w + (int64_t)(kk + u) * E);
+                for (int u = 0; u < 8; ++u) wv[u] = w[(kk + u) * E];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < kRTok / 4; ++q) {
+                    if (tq + 4 * q >= nt) continue;
                     const uint4 xv = *reinterpret_cast<const uint4*>(xs + (tq + 4 * q) * ks + kk);
                     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
@@ -242,187 +285,92 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
             }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) part[(tq + 4 * q) * 64 + e] = acc[q];
+        for (int q = 0; q < kRTok / 4; ++q) part[(tq + 4 * q) * 64 + e] = acc[q];
     }
-    for (int t = warp; t < kRTok; t += kRThreads / 32) {
+    for (int t = warp; t < nt; t += kRThreads / 32) {
         float m = 0.0f;
         for (int i = lane; i < ks; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * ks + i])));
         m = warp_max(m);
         if (lane == 0) pmax[t] = m;
     }
     cluster_sync();
-    if (tid < kRTok) {
+    for (int t = tid; t < nt; t += kRThreads) {
+        float v[16];
+        ld_peers(v, &pmax[t], cs);
         float m = 0.0f;
-        for (int c = 0; c < cs; ++c) m = fmaxf(m, ld_peer(&pmax[tid], (uint32_t)c));
-        sxs[tid] = __fdiv_rn(m, 127.0f);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) m = fmaxf(m, v[c]);
+        sxs[t] = __fdiv_rn(m, 127.0f);
     }
     __syncthreads();
     // K1 on this CTA's slice: codes of the shared-expert rows (rows Tk + t of xq)
     for (int i = tid; i < nt * (ks / 4); i += kRThreads) {
         const int t = i / (ks / 4), v = i % (ks / 4);
         const uint16_t* xr = xs + t * ks + v * 4;
-        const float s = sxs[t];
-        *reinterpret_cast<uint32_t*>(p.xq + (p.Tk + t0 + t) * d + k0 + v * 4) =
-            pack_codes(bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), s);
+        *reinterpret_cast<uint32_t*>(p.xq + (p.Tk + t) * d + k0 + v * 4) =
+            pack_codes(bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), sxs[t]);
     }
     // logits (slices added in rank order), gating and top-k of the tokens this CTA owns
     for (int t = rank + warp * cs; t < nt; t += (kRThreads / 32) * cs) {
+        const float s0 = cluster_sum(&part[t * 64 + lane], cs);
+        const float s1 = cluster_sum(&part[t * 64 + lane + 32], cs);
         float l0 = -INFINITY, l1 = -INFINITY;
-        if (lane < E) {
-            float s = 0.0f;
-            for (int c = 0; c < cs; ++c) s = __fadd_rn(s, ld_peer(&part[t * 64 + lane], (uint32_t)c));
-            if (p.router_bias) s = __fadd_rn(s, p.router_bias[lane]);
-            l0 = s;
-        }
-        if (lane + 32 < E) {
-            float s = 0.0f;
-            for (int c = 0; c < cs; ++c) s = __fadd_rn(s, ld_peer(&part[t * 64 + lane + 32], (uint32_t)c));
-            if (p.router_bias) s = __fadd_rn(s, p.router_bias[lane + 32]);
-            l1 = s;
-        }
-        const int64_t tg = t0 + t;
-        gate_topk_warp(p, tg, l0, l1, lane);
+        if (lane < E) l0 = p.router_bias ? __fadd_rn(s0, p.router_bias[lane]) : s0;
+        if (lane + 32 < E) l1 = p.router_bias ? __fadd_rn(s1, p.router_bias[lane + 32]) : s1;
+        gate_topk_warp(p, t, l0, l1, lane);
         if (lane == 0) {
-            p.sx[tg] = sxs[t];
-            p.row_src[p.Tk + tg] = (int32_t)tg;
-            p.row_gate[p.Tk + tg] = 1.0f;
+            p.sx[t] = sxs[t];
+            p.row_src[p.Tk + t] = t;
+            p.row_gate[p.Tk + t] = 1.0f;
         }
     }
-    __threadfence();  // every writer of idx / gate orders its stores before the ticket below
-    cluster_sync();   // no CTA leaves while a peer may still read its shared memory
-    if (tid == 0) {
-        const int total = (int)(gridDim.x * gridDim.y);
-        flag[0] = atomicAdd(p.dec_ticket, 1) == total - 1;
-    }
-    __syncthreads();
-    if (!flag[0]) return;
-    __threadfence();
-    permute_block(p);
+    cluster_sync();  // idx / gate of every token written; no CTA leaves while a peer may read its smem
+    if (rank == 0) permute_block(p);
 }
 
 // ------------------------------------------------------------------ experts
-// grid: (groups that can have rows) x nbpg blocks; block: W warps, warp w
-// handles weight-row block blk * W + w of group dec_groups[blockIdx.x / nbpg].
-// Shared memory: mbarriers | row scales | W rings of kRing stages | codes of the
-// group's rows [8 * chunks][K + 32] (B-fragment order inside each 32-group).
-template <bool GU, bool DUMP>
-__global__ void __launch_bounds__(kMaxWarps * 32)
-expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnrows)
-{
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int W = blockDim.x >> 5;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    float* shs = reinterpret_cast<float*>(smem + 256);
-    uint8_t* ring = smem + kHeadBytes;
-    uint8_t* codes = ring + W * kRing * kStageBytes;
-
-    if (GU && !DUMP && !p.deterministic && p.y) {
-        // y is accumulated by the down launch: clear it here, spread over every CTA
-        const int64_t n4 = p.T * p.d / 4;
-        const int64_t per = (n4 + gridDim.x - 1) / gridDim.x;
-        const int64_t a = (int64_t)blockIdx.x * per, b = a + per < n4 ? a + per : n4;
-        float4* y4 = reinterpret_cast<float4*>(p.y);
-        for (int64_t i = a + tid; i < b; i += blockDim.x) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
-
-    const int gi = blockIdx.x / nbpg, blk = blockIdx.x % nbpg;
-    if (gi >= *p.dec_ngroups) return;
-    const int g = p.dec_groups[gi];
-    const int hid = g == p.E ? p.hs : p.h;
-    const int K = GU ? p.d : hid;
-    const int nrb = GU ? hid / 8 : p.d / 16;
-    const int rb0 = blk * W;
-    if (rb0 >= nrb) return;
-    const int nrows = p.counts[g];
-    const int64_t row0 = p.offsets[g];
-    const int nch = (nrows + 7) >> 3;
-    const int NJ = K / 64, nst = (NJ + kStageJP - 1) / kStageJP;
-    const int cs = K + 32;
-    const int rb = rb0 + warp;
-    const bool wact = rb < nrb;
-    uint64_t* wb = bars + warp * kRing;
-    uint8_t* wr = ring + warp * kRing * kStageBytes;
-    const uint8_t* src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
-                             : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
-                         (int64_t)rb * NJ * kJP;
-    auto issue = [&](int st) {
+// One warp's weight stream for one pass: stage st (0 .. nst-1) of the pass is
+// global stage sc0 + st of the warp's ring, so slot and phase carry over
+// between passes.
+struct WarpStream {
+    const uint8_t* src;   // the warp's 16-row block in the decode layout
+    uint8_t* ring;
+    uint64_t* bars;
+    int NJ, nst, sc0;
+    __device__ __forceinline__ void issue(int st) const {
         const int jp = NJ - st * kStageJP;
         const uint32_t bytes = (uint32_t)((jp < kStageJP ? jp : kStageJP) * kJP);
-        uint64_t* bar = &wb[st % kRing];
-        mbar_expect_tx(bar, bytes);
-        bulk_load(wr + (st % kRing) * kStageBytes, src + (int64_t)st * kStageBytes, bytes, bar);
-    };
-    if (lane == 0) {
-        for (int s = 0; s < kRing; ++s) mbar_init(&wb[s], 1);
-        fence_barrier_init();
+        const int slot = (sc0 + st) % kRing;
+        mbar_expect_tx(&bars[slot], bytes);
+        bulk_load(ring + slot * kStageBytes, src + (int64_t)st * kStageBytes, bytes, &bars[slot]);
     }
-    __syncwarp();
-    if (wact && lane == 0)
-        for (int s = 0; s < kRing && s < nst; ++s) issue(s);
+};
 
-    // codes of the group's rows, zero rows up to a multiple of 8
-    const int ngr = K / 32;
-    if (GU) {
-        for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
-            const int i = it / ngr, j = it % ngr;
-            uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
-            if (i < nrows) {
-                const int64_t t = p.row_src[row0 + i];
-                const uint4* s4 = reinterpret_cast<const uint4*>(p.xq + (p.Tk + t) * p.d + j * 32);
-                u0 = s4[0];
-                u1 = s4[1];
-            }
-            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
-            dst[0] = make_uint4(u0.x, u1.x, u0.y, u1.y);
-            dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
-        }
-    } else {
-        for (int i = tid; i < nch * 8; i += blockDim.x)
-            shs[i] = i < nrows ? __fdiv_rn(__uint_as_float(p.amax_h[row0 + i]), 127.0f) : 0.0f;
-        __syncthreads();
-        const bool keep = blk == 0 && !DUMP;  // one CTA per group records h_q and s_h
-        for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
-            const int i = it / ngr, j = it % ngr;
-            uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (i < nrows) {
-                const float s = shs[i];
-                const float4* a4 = reinterpret_cast<const float4*>(p.act + (row0 + i) * p.hmax + j * 32);
+// The GEMV of one warp over one pass of up to 8 * NCH rows, then its
+// epilogue.  Returns false if a bounded wait gave up (nothing is written).
+template <bool GU, bool DUMP, int NCH>
+__device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs,
+                                          const float* shs, int lane, int rb, int64_t rrow0, int prows,
+                                          int32_t* dump, int64_t drow0, int64_t dnrows)
+{
+    const int gid = lane >> 2, t4 = lane & 3;
+    float alo[NCH][2], ahi[NCH][2];
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 a = a4[v];
-                    wv[v] = pack_codes(a.x, a.y, a.z, a.w, s);
-                }
-                if (keep) {
-                    uint4* q4 = reinterpret_cast<uint4*>(p.hq + (row0 + i) * p.hmax + j * 32);
-                    q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                }
-            }
-            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
-            dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
-            dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
-        }
-        if (keep)
-            for (int i = tid; i < nrows; i += blockDim.x) p.sh[row0 + i] = shs[i];
-    }
-    __syncthreads();
-    if (!wact) return;
-
-    float alo[kMaxChunks][2], ahi[kMaxChunks][2];
-#pragma unroll
-    for (int c = 0; c < kMaxChunks; ++c) alo[c][0] = alo[c][1] = ahi[c][0] = ahi[c][1] = 0.0f;
+    for (int c = 0; c < NCH; ++c) alo[c][0] = alo[c][1] = ahi[c][0] = ahi[c][1] = 0.0f;
     const int ng = p.d / kGroup, ngh = p.hmax / kGroup;
-    for (int st = 0; st < nst; ++st) {
-        if (!wait_bounded(&wb[st % kRing], (uint32_t)((st / kRing) & 1))) {
+    const uint8_t* bbase = codes + (size_t)gid * cs + t4 * 8;
+    for (int st = 0; st < S.nst; ++st) {
+        const int sc = S.sc0 + st;
+        if (!wait_bounded(&S.bars[sc % kRing], (uint32_t)((sc / kRing) & 1))) {
             if (lane == 0) set_error(p, 7);
             // let the copies in flight land before the CTA's shared memory goes away
-            const int issued = st + kRing < nst ? st + kRing : nst;
-            for (int s = st; s < issued; ++s) wait_bounded(&wb[s % kRing], (uint32_t)((s / kRing) & 1));
-            return;
+            const int issued = st + kRing < S.nst ? st + kRing : S.nst;
+            for (int s = st; s < issued; ++s)
+                wait_bounded(&S.bars[(S.sc0 + s) % kRing], (uint32_t)(((S.sc0 + s) / kRing) & 1));
+            return false;
         }
-        const uint8_t* sb = wr + (st % kRing) * kStageBytes;
-        const int njs = NJ - st * kStageJP < kStageJP ? NJ - st * kStageJP : kStageJP;
+        const uint8_t* sb = S.ring + (sc % kRing) * kStageBytes;
+        const int njs = S.NJ - st * kStageJP < kStageJP ? S.NJ - st * kStageJP : kStageJP;
         for (int q = 0; q < njs; ++q) {
             const uint4 wv = *reinterpret_cast<const uint4*>(sb + q * kJP + lane * 16);
             const float4 sv = *reinterpret_cast<const float4*>(sb + q * kJP + 512 + gid * 16);
@@ -434,93 +382,216 @@ expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnr
                 const uint32_t a0 = (w0 << 4) & 0xF0F0F0F0u, a1 = w0 & 0xF0F0F0F0u;
                 const uint32_t a2 = (w1 << 4) & 0xF0F0F0F0u, a3 = w1 & 0xF0F0F0F0u;
                 const int j = 2 * jp + jj;
-                const uint8_t* bp = codes + (size_t)gid * cs + j * 32 + t4 * 8;
 #pragma unroll
-                for (int c = 0; c < kMaxChunks; ++c) {
-                    if (c < nch) {
-                        const uint2 b = *reinterpret_cast<const uint2*>(bp + (size_t)c * 8 * cs);
-                        int32_t dd[4];
-                        mma_bias(dd, a0, a1, a2, a3, b.x, b.y);
-                        if (DUMP) {
+                for (int c = 0; c < NCH; ++c) {
+                    const uint2 b = *reinterpret_cast<const uint2*>(bbase + (size_t)c * 8 * cs + j * 32);
+                    int32_t dd[4];
+                    mma_bias(dd, a0, a1, a2, a3, b.x, b.y);
+                    if (DUMP) {
 #pragma unroll
-                            for (int q2 = 0; q2 < 2; ++q2) {
-                                const int i = c * 8 + 2 * t4 + q2;
-                                const int64_t r = row0 + i;
-                                if (i < nrows && r >= drow0 && r < drow0 + dnrows) {
-                                    if (GU) {
-                                        int32_t* base = dump + (r - drow0) * 2 * p.hmax * ng;
-                                        const int n = rb * 8 + gid;
-                                        base[(int64_t)n * ng + j] = partial_of(dd[q2]);
-                                        base[(int64_t)(p.hmax + n) * ng + j] = partial_of(dd[2 + q2]);
-                                    } else {
-                                        const int m = rb * 16 + gid;
-                                        dump[((r - drow0) * p.d + m) * ngh + j] = partial_of(dd[q2]);
-                                        dump[((r - drow0) * p.d + m + 8) * ngh + j] = partial_of(dd[2 + q2]);
-                                    }
+                        for (int q2 = 0; q2 < 2; ++q2) {
+                            const int i = c * 8 + 2 * t4 + q2;
+                            const int64_t r = rrow0 + i;
+                            if (i < prows && r >= drow0 && r < drow0 + dnrows) {
+                                if (GU) {
+                                    int32_t* base = dump + (r - drow0) * 2 * p.hmax * ng;
+                                    const int n = rb * 8 + gid;
+                                    base[(int64_t)n * ng + j] = partial_of(dd[q2]);
+                                    base[(int64_t)(p.hmax + n) * ng + j] = partial_of(dd[2 + q2]);
+                                } else {
+                                    const int m = rb * 16 + gid;
+                                    dump[((r - drow0) * p.d + m) * ngh + j] = partial_of(dd[q2]);
+                                    dump[((r - drow0) * p.d + m + 8) * ngh + j] = partial_of(dd[2 + q2]);
                                 }
                             }
                         }
-                        promote2(alo[c][0], alo[c][1], dd[0], dd[1], slo);
-                        promote2(ahi[c][0], ahi[c][1], dd[2], dd[3], shi);
                     }
+                    promote2(alo[c][0], alo[c][1], dd[0], dd[1], slo);
+                    promote2(ahi[c][0], ahi[c][1], dd[2], dd[3], shi);
                 }
             }
         }
         __syncwarp();
-        if (lane == 0 && st + kRing < nst) issue(st + kRing);
+        if (lane == 0 && st + kRing < S.nst) S.issue(st + kRing);
     }
-    if (DUMP) return;
+    if (DUMP) return true;
 
     if (GU) {
         const int n = rb * 8 + gid;
 #pragma unroll
-        for (int c = 0; c < kMaxChunks; ++c) {
-            if (c < nch) {
+        for (int c = 0; c < NCH; ++c) {
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int i = c * 8 + 2 * t4 + q;
-                    const bool valid = i < nrows;
-                    const int64_t r = row0 + i;
-                    float a = 0.0f;
-                    if (valid) {
-                        const float sxr = p.sx[p.row_src[r]];
-                        const float gv = __fmul_rn(alo[c][q], sxr), uv = __fmul_rn(ahi[c][q], sxr);
-                        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
-                        a = __fmul_rn(silu, uv);
-                        p.act[r * p.hmax + n] = a;
-                    }
-                    float m = fabsf(a);
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-                    if (valid && gid == 0) atomicMax(p.amax_h + r, __float_as_uint(m));
+            for (int q = 0; q < 2; ++q) {
+                const int i = c * 8 + 2 * t4 + q;
+                const bool valid = i < prows;
+                const int64_t r = rrow0 + i;
+                float a = 0.0f;
+                if (valid) {
+                    const float sxr = p.sx[p.row_src[r]];
+                    const float gv = __fmul_rn(alo[c][q], sxr), uv = __fmul_rn(ahi[c][q], sxr);
+                    const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+                    a = __fmul_rn(silu, uv);
+                    p.act[r * p.hmax + n] = a;
                 }
+                float m = fabsf(a);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                if (valid && gid == 0) atomicMax(p.amax_h + r, __float_as_uint(m));
             }
         }
     } else {
         const int m0 = rb * 16 + gid;
 #pragma unroll
-        for (int c = 0; c < kMaxChunks; ++c) {
-            if (c < nch) {
+        for (int c = 0; c < NCH; ++c) {
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int i = c * 8 + 2 * t4 + q;
-                    if (i >= nrows) continue;
-                    const int64_t r = row0 + i;
-                    const float s = shs[i];
-                    const float olo = __fmul_rn(alo[c][q], s), ohi = __fmul_rn(ahi[c][q], s);
-                    if (p.deterministic) {
-                        p.obuf[r * p.d + m0] = olo;
-                        p.obuf[r * p.d + m0 + 8] = ohi;
-                    } else {
-                        const float gt = p.row_gate[r];
-                        float* yr = p.y + (int64_t)p.row_src[r] * p.d;
-                        atomicAdd(yr + m0, __fmul_rn(gt, olo));
-                        atomicAdd(yr + m0 + 8, __fmul_rn(gt, ohi));
-                    }
+            for (int q = 0; q < 2; ++q) {
+                const int i = c * 8 + 2 * t4 + q;
+                if (i >= prows) continue;
+                const int64_t r = rrow0 + i;
+                const float s = shs[i];
+                const float olo = __fmul_rn(alo[c][q], s), ohi = __fmul_rn(ahi[c][q], s);
+                if (p.deterministic) {
+                    p.obuf[r * p.d + m0] = olo;
+                    p.obuf[r * p.d + m0 + 8] = ohi;
+                } else {
+                    const float gt = p.row_gate[r];
+                    float* yr = p.y + (int64_t)p.row_src[r] * p.d;
+                    atomicAdd(yr + m0, __fmul_rn(gt, olo));
+                    atomicAdd(yr + m0 + 8, __fmul_rn(gt, ohi));
                 }
             }
         }
+    }
+    return true;
+}
+
+// grid: (groups that can have rows) x nbpg blocks; block: W warps, warp w
+// handles weight-row block blk * W + w of group dec_groups[blockIdx.x / nbpg].
+// The group's rows go in passes of up to kPassRows; each pass stages their
+// codes (B-fragment order inside each 32-group) and streams the weights again
+// (from L2 after the first pass).  Shared memory: mbarriers | row scales |
+// W rings of kRing stages | codes [kPassRows][K + 32].
+template <bool GU, bool DUMP>
+__global__ void __launch_bounds__(kMaxWarps * 32)
+expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnrows)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int W = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    float* shs = reinterpret_cast<float*>(smem + 256);
+    uint8_t* ring = smem + kHeadBytes;
+    uint8_t* codes = ring + W * kRing * kStageBytes;
+
+    pdl_trigger();
+    if (GU && !DUMP && !p.deterministic && p.y) {
+        // y is accumulated by the down launch: clear it here, spread over every CTA (the
+        // router launch before this one does not touch y, so no wait is needed)
+        const int64_t n4 = p.T * p.d / 4;
+        const int64_t per = (n4 + gridDim.x - 1) / gridDim.x;
+        const int64_t a = (int64_t)blockIdx.x * per, b = a + per < n4 ? a + per : n4;
+        float4* y4 = reinterpret_cast<float4*>(p.y);
+        for (int64_t i = a + tid; i < b; i += blockDim.x) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+
+    // group slot 0 is always the shared expert (rows Tk .. Tk + T - 1), known before the
+    // previous launch has finished; every other slot waits for the routing
+    const int gi = blockIdx.x / nbpg, blk = blockIdx.x % nbpg;
+    const bool shared = gi == 0;
+    if (!shared) {
+        pdl_wait();
+        if (gi >= *p.dec_ngroups) return;
+    }
+    const int g = shared ? p.E : p.dec_groups[gi];
+    const int hid = g == p.E ? p.hs : p.h;
+    const int K = GU ? p.d : hid;
+    const int nrb = GU ? hid / 8 : p.d / 16;
+    const int rb0 = blk * W;
+    if (rb0 >= nrb) return;
+    const int nrows = shared ? (int)p.T : p.counts[g];
+    const int64_t row0 = shared ? p.Tk : p.offsets[g];
+    const int NJ = K / 64;
+    const int cs = K + 32;
+    const int ngr = K / 32;
+    const int rb = rb0 + warp;
+    const bool wact = rb < nrb;
+    WarpStream S;
+    S.src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
+                : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
+            (int64_t)rb * NJ * kJP;
+    S.ring = ring + warp * kRing * kStageBytes;
+    S.bars = bars + warp * kRing;
+    S.NJ = NJ;
+    S.nst = (NJ + kStageJP - 1) / kStageJP;
+    S.sc0 = 0;
+    if (lane == 0) {
+        for (int s = 0; s < kRing; ++s) mbar_init(&S.bars[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    const bool keep = blk == 0 && !DUMP;  // one CTA per group records h_q and s_h
+    bool alive = wact;                    // false once this warp's bounded wait gave up
+    const int npass = (nrows + kPassRows - 1) / kPassRows;
+    for (int pass = 0; pass < npass; ++pass, S.sc0 += S.nst) {
+        const int prow0 = pass * kPassRows;
+        const int prows = nrows - prow0 < kPassRows ? nrows - prow0 : kPassRows;
+        const int nch = (prows + 7) >> 3;
+        const int64_t rrow0 = row0 + prow0;
+        if (pass > 0) __syncthreads();  // every warp is done with the previous pass's codes
+        if (alive && lane == 0)
+            for (int s = 0; s < kRing && s < S.nst; ++s) S.issue(s);
+        if (pass == 0 && shared) pdl_wait();  // weights are in flight; now the previous launch's outputs
+
+        // codes of this pass's rows, zero rows up to a multiple of 8
+        if (GU) {
+            for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
+                const int i = it / ngr, j = it % ngr;
+                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+                if (i < prows) {
+                    const int64_t t = p.row_src[rrow0 + i];
+                    const uint4* s4 = reinterpret_cast<const uint4*>(p.xq + (p.Tk + t) * p.d + j * 32);
+                    u0 = s4[0];
+                    u1 = s4[1];
+                }
+                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
+                dst[0] = make_uint4(u0.x, u1.x, u0.y, u1.y);
+                dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
+            }
+        } else {
+            for (int i = tid; i < nch * 8; i += blockDim.x)
+                shs[i] = i < prows ? __fdiv_rn(__uint_as_float(p.amax_h[rrow0 + i]), 127.0f) : 0.0f;
+            __syncthreads();
+            for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
+                const int i = it / ngr, j = it % ngr;
+                uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                if (i < prows) {
+                    const float s = shs[i];
+                    const float4* a4 = reinterpret_cast<const float4*>(p.act + (rrow0 + i) * p.hmax + j * 32);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const float4 a = a4[v];
+                        wv[v] = pack_codes(a.x, a.y, a.z, a.w, s);
+                    }
+                    if (keep) {
+                        uint4* q4 = reinterpret_cast<uint4*>(p.hq + (rrow0 + i) * p.hmax + j * 32);
+                        q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                    }
+                }
+                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
+                dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
+                dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+            }
+            if (keep)
+                for (int i = tid; i < prows; i += blockDim.x) p.sh[rrow0 + i] = shs[i];
+        }
+        __syncthreads();
+        if (alive)  // a warp that gave up keeps taking the CTA barriers but issues and computes nothing
+            alive = nch == 1 ? warp_pass<GU, DUMP, 1>(p, S, codes, cs, shs, lane, rb, rrow0, prows, dump, drow0,
+                                                      dnrows)
+                             : warp_pass<GU, DUMP, 2>(p, S, codes, cs, shs, lane, rb, rrow0, prows, dump, drow0,
+                                                      dnrows);
     }
 }
 
@@ -574,6 +645,22 @@ __global__ void retile_decode_kernel(const uint8_t* gu, const float* sgu, const 
     }
 }
 
+// Raises a kernel's dynamic shared-memory opt-in to at least `bytes`, never
+// lowering it (handles of different sizes share the kernels) and calling the
+// runtime only when it grows (keeps the call out of stream captures).
+// `granted` holds the current opt-in per device.
+int g_router_smem[64] = {};
+
+cudaError_t raise_smem(const void* kern, int (&granted)[64], size_t bytes) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (granted[dev] >= (int)bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) granted[dev] = (int)bytes;
+    return e;
+}
+
 int sm_count() {
     static int n[64] = {};
     int dev = 0;
@@ -588,7 +675,8 @@ int sm_count() {
 }
 
 size_t expert_smem(int W, int64_t T, int K) {
-    return (size_t)kHeadBytes + (size_t)W * kRing * kStageBytes + (size_t)((T + 7) / 8) * 8 * (K + 32);
+    const int64_t rows = T < kPassRows ? T : kPassRows;
+    return (size_t)kHeadBytes + (size_t)W * kRing * kStageBytes + (size_t)((rows + 7) / 8) * 8 * (K + 32);
 }
 
 // warps per CTA: as many as keep at least two CTAs per SM busy
@@ -607,18 +695,20 @@ cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t 
     const int nbpg = (max_nrb + W - 1) / W;
     const size_t smem = expert_smem(W, p.T, GU ? p.d : p.hmax);
     auto kern = dump ? expert_decode_kernel<GU, true> : expert_decode_kernel<GU, false>;
-    // raise the shared-memory opt-in only when it grows (keeps the call out of stream captures)
     static int granted[2][64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    int* have = (dev >= 0 && dev < 64) ? &granted[dump ? 1 : 0][dev] : nullptr;
-    if (!have || *have < (int)smem) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (have) *have = (int)smem;
-    }
-    kern<<<(unsigned)(gmax * nbpg), W * 32, smem, s>>>(p, nbpg, dump, r0, nr);
-    return cudaGetLastError();
+    cudaError_t e = raise_smem((const void*)kern, granted[dump ? 1 : 0], smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(gmax * nbpg), 1, 1);
+    cfg.blockDim = dim3((unsigned)(W * 32), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p, nbpg, dump, r0, nr);
 }
 
 }  // namespace
@@ -634,14 +724,16 @@ int dec_max_tokens(int d, int hmax) {
 }
 
 // CTAs per router cluster: 16 (non-portable size) where the device runs it,
-// else 8, else 4; each CTA's K slice must be a multiple of 8 elements.
-int dec_router_cluster(int d) {
-    const size_t smem = dec::kRHeadBytes + (size_t)dec::kRTok * (d / 4) * 2;
-    if (cudaFuncSetAttribute(dec::router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return 0;
+// else 8, else 4; each CTA's K slice must be a multiple of 8 elements and its
+// x and W_r slices must fit in shared memory.  0: no size works.
+int dec_router_cluster(int d, int E) {
     for (int cs = 16; cs >= 4; cs >>= 1) {
-        if (d % (8 * cs)) continue;
+        const size_t smem = dec::router_smem(d, cs, E);
+        if (d % (8 * cs) || smem > (size_t)dec::kSmemLimit) continue;
+        if (dec::raise_smem((const void*)dec::router_decode_kernel, dec::g_router_smem, smem) != cudaSuccess) {
+            cudaGetLastError();
+            continue;
+        }
         if (cs > 8 &&
             cudaFuncSetAttribute(dec::router_decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess) {
@@ -651,7 +743,7 @@ int dec_router_cluster(int d) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(cs, 1, 1);
         cfg.blockDim = dim3(dec::kRThreads, 1, 1);
-        cfg.dynamicSmemBytes = dec::kRHeadBytes + (size_t)dec::kRTok * (d / cs) * 2;
+        cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = cs;
@@ -668,9 +760,11 @@ int dec_router_cluster(int d) {
 
 cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    const size_t smem = dec::kRHeadBytes + (size_t)dec::kRTok * (p.d / cluster) * 2;
+    const size_t smem = dec::router_smem(p.d, cluster, p.E);
+    cudaError_t e = dec::raise_smem((const void*)dec::router_decode_kernel, dec::g_router_smem, smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)cluster, (unsigned)((p.T + dec::kRTok - 1) / dec::kRTok), 1);
+    cfg.gridDim = dim3((unsigned)cluster, 1, 1);
     cfg.blockDim = dim3(dec::kRThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;

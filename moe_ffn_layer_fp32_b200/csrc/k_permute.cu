@@ -40,10 +40,18 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(Plan p)
     const int E = p.E;
     const int tid = threadIdx.x;
     if (tid < E) {
+        // running count of expert tid before each chunk; counts read 16 at a time (read-only path)
         int acc = 0;
-        for (int c = 0; c < p.nchunks; ++c) {
-            p.chunk_base[(int64_t)c * kMaxExperts + tid] = acc;  // running count before chunk c
-            acc += p.chunk_cnt[(int64_t)c * kMaxExperts + tid];
+        for (int c0 = 0; c0 < p.nchunks; c0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                v[u] = c0 + u < p.nchunks ? __ldg(p.chunk_cnt + (int64_t)(c0 + u) * kMaxExperts + tid) : 0;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                if (c0 + u < p.nchunks) p.chunk_base[(int64_t)(c0 + u) * kMaxExperts + tid] = acc;
+                acc += v[u];
+            }
         }
         tot[tid] = acc;
     }
@@ -65,17 +73,18 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(Plan p)
         *p.tile_count = ts;
     }
     __syncthreads();
-    if (tid < E) {
-        for (int c = 0; c < p.nchunks; ++c) p.chunk_base[(int64_t)c * kMaxExperts + tid] += off[tid];
-    }
     for (int e = tid; e < E + 2; e += kThreads) p.offsets[e] = off[e];
     for (int e = tid; e <= E; e += kThreads) p.counts[e] = tot[e];
     // tile table: entry i -> (group, tile index within the group)
     const int ntiles = tstart[E + 1];
     for (int i = tid; i < ntiles; i += kThreads) {
-        int g = 0;
-        while (tstart[g + 1] <= i) ++g;
-        p.tiles[i] = (g << 24) | (i - tstart[g]);
+        int lo = 0, hi = E;  // the last g with tstart[g] <= i
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tstart[mid] <= i) lo = mid;
+            else hi = mid - 1;
+        }
+        p.tiles[i] = (lo << 24) | (i - tstart[lo]);
     }
 }
 
@@ -87,7 +96,8 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(Plan p)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t S = p.Tk;
     const int64_t c = blockIdx.x;
-    for (int i = tid; i < kMaxExperts; i += kThreads) base[i] = p.chunk_base[c * kMaxExperts + i];
+    for (int i = tid; i < kMaxExperts; i += kThreads)
+        base[i] = i < p.E ? p.chunk_base[c * kMaxExperts + i] + p.offsets[i] : 0;
     for (int round = 0; round < kChunk / kThreads; ++round) {
         for (int i = tid; i < (kThreads / 32) * kMaxExperts; i += kThreads) (&wcnt[0][0])[i] = 0;
         __syncthreads();

@@ -128,10 +128,239 @@ cudaError_t launch_tb(const Plan& p, cudaStream_t s) {
 
 cudaError_t launch_router_quant(const Plan& p, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
+    if (p.w_router_split) return launch_router_mma(p, s);
     // token tile: as many rows as fit in about 160 KB of shared memory
     if ((size_t)32 * p.d * 2 <= 160 * 1024) return launch_tb<32>(p, s);
     if ((size_t)16 * p.d * 2 <= 160 * 1024) return launch_tb<16>(p, s);
     return launch_tb<8>(p, s);
+}
+
+}  // namespace mmoe
+
+// ---------------------------------------------------------------------------
+// K1 + K2 for prefill on the tensor cores.
+//
+// W_r (FP32) is held as three BF16 pieces w = hi + mid + lo, exact for every
+// normal FP32 value (each piece carries 8 significant bits of the remainder
+// left by the pieces before it, with round-to-nearest), so with BF16 x every
+// product x * piece is exact in FP32 and the logit is an FP32 sum of the
+// exact products x_k * w_k, accumulated by the tensor cores.
+//
+// Split layout: K chunks of 64; per chunk three pieces of [64 experts][72]
+// BF16 (64 K values + 8 of padding, which keeps the fragment loads free of
+// shared-memory bank conflicts); experts >= E are zero.
+namespace mmoe {
+namespace rmma {
+
+constexpr int kTok = 128;                 // tokens per CTA (8 warps x 16)
+constexpr int kThreads = 256;
+constexpr int kKC = 64;                   // K per chunk
+constexpr int kRow = 72;                  // padded BF16 row of a chunk
+constexpr int kXChunkBytes = kTok * kRow * 2;          // 18432
+constexpr int kWPieceBytes = 64 * kRow * 2;            // 9216
+constexpr int kWChunkBytes = 3 * kWPieceBytes;         // 27648
+constexpr int kStages = 2;
+constexpr int kLgRow = 65;                // padded logits row
+constexpr size_t kSmem = (size_t)kStages * (kXChunkBytes + kWChunkBytes);  // logits alias the stages
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// D = A * B (C = 0), m16n8k16, BF16 inputs, FP32 result
+__device__ __forceinline__ void mma_bf16_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// D += A * B, m16n8k16, BF16 inputs, FP32 accumulators
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float bf16_abs(uint32_t bits16) { return fabsf(__uint_as_float(bits16 << 16)); }
+
+// round-to-nearest-even FP32 -> BF16 bits (finite inputs)
+__device__ __forceinline__ uint32_t bf16_rn_bits(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
+}
+
+// stage K chunk c of x (rows t0 .. t0 + 127, zero beyond T) and of the split weights
+__device__ __forceinline__ void load_chunk(const Plan& p, int64_t t0, int nt, int c, uint8_t* xs, uint8_t* ws,
+                                           int tid) {
+    const int d = p.d;
+    for (int i = tid; i < kTok * (kKC / 8); i += kThreads) {
+        const int r = i >> 3, v = i & 7;
+        uint8_t* dst = xs + r * (kRow * 2) + v * 16;
+        if (r < nt) cp_async16(dst, p.x + (t0 + r) * d + c * kKC + v * 8);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.w_router_split) + (size_t)c * kWChunkBytes;
+    for (int i = tid; i < kWChunkBytes / 16; i += kThreads) cp_async16(ws + i * 16, src + i * 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int d = p.d, E = p.E;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
+    const int64_t t0 = (int64_t)blockIdx.x * kTok;
+    const int nt = (int)((p.T - t0) < kTok ? (p.T - t0) : kTok);
+    auto xs = [&](int c) { return smem + (c % kStages) * (kXChunkBytes + kWChunkBytes); };
+    auto ws = [&](int c) { return smem + (c % kStages) * (kXChunkBytes + kWChunkBytes) + kXChunkBytes; };
+    const int nchunks = d / kKC;
+    float acc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+    float amax_lo = 0.0f, amax_hi = 0.0f;  // |x| max of rows g and g + 8 of this warp, over this lane's elements
+
+    load_chunk(p, t0, nt, 0, xs(0), ws(0), tid);
+    cp_async_commit();
+    for (int c = 0; c < nchunks; ++c) {
+        if (c + 1 < nchunks) load_chunk(p, t0, nt, c + 1, xs(c + 1), ws(c + 1), tid);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const uint16_t* xa = reinterpret_cast<const uint16_t*>(xs(c)) + (warp * 16 + g) * kRow + 2 * t4;
+        const uint16_t* wb = reinterpret_cast<const uint16_t*>(ws(c)) + g * kRow + 2 * t4;
+#pragma unroll
+        for (int kk = 0; kk < kKC; kk += 16) {
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xa + kk);
+            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(xa + 8 * kRow + kk);
+            const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xa + kk + 8);
+            const uint32_t a3 = *reinterpret_cast<const uint32_t*>(xa + 8 * kRow + kk + 8);
+            amax_lo = fmaxf(amax_lo, fmaxf(fmaxf(bf16_abs(a0 & 0xffffu), bf16_abs(a0 >> 16)),
+                                           fmaxf(bf16_abs(a2 & 0xffffu), bf16_abs(a2 >> 16))));
+            amax_hi = fmaxf(amax_hi, fmaxf(fmaxf(bf16_abs(a1 & 0xffffu), bf16_abs(a1 >> 16)),
+                                           fmaxf(bf16_abs(a3 & 0xffffu), bf16_abs(a3 >> 16))));
+            // the 16-wide K step's partial (lo, mid, hi pieces) on the tensor cores, then one
+            // round-to-nearest FP32 addition into the running logit: the tensor cores only
+            // ever sum 48 exact products, so their internal rounding stays far below FP32's
+            // over the whole K range
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const uint16_t* wr = wb + n * 8 * kRow + kk;
+                float part[4];
+                mma_bf16_first(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes),
+                               *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes + 8));
+                mma_bf16(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes / 2),
+                         *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes / 2 + 8));
+                mma_bf16(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr),
+                         *reinterpret_cast<const uint32_t*>(wr + 8));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[n][i] = __fadd_rn(acc[n][i], part[i]);
+            }
+        }
+        __syncthreads();  // the stage is refilled by the next iteration
+    }
+    cp_async_wait<0>();
+
+    // logits into shared memory (aliasing the stages): D fragment rows g / g + 8, columns 2 t4, 2 t4 + 1
+    float* lg = reinterpret_cast<float*>(smem);
+    float* sxs = lg + kTok * kLgRow;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+        const int col = n * 8 + 2 * t4;
+        lg[(warp * 16 + g) * kLgRow + col] = acc[n][0];
+        lg[(warp * 16 + g) * kLgRow + col + 1] = acc[n][1];
+        lg[(warp * 16 + g + 8) * kLgRow + col] = acc[n][2];
+        lg[(warp * 16 + g + 8) * kLgRow + col + 1] = acc[n][3];
+    }
+    amax_lo = fmaxf(amax_lo, __shfl_xor_sync(0xffffffffu, amax_lo, 1));
+    amax_lo = fmaxf(amax_lo, __shfl_xor_sync(0xffffffffu, amax_lo, 2));
+    amax_hi = fmaxf(amax_hi, __shfl_xor_sync(0xffffffffu, amax_hi, 1));
+    amax_hi = fmaxf(amax_hi, __shfl_xor_sync(0xffffffffu, amax_hi, 2));
+    if (t4 == 0) {
+        sxs[warp * 16 + g] = __fdiv_rn(amax_lo, 127.0f);
+        sxs[warp * 16 + g + 8] = __fdiv_rn(amax_hi, 127.0f);
+    }
+    __syncthreads();
+
+    // gating and top-k, one warp per token; then the codes of the token's row (rows Tk + t of xq)
+    for (int tt = warp; tt < nt; tt += kThreads / 32) {
+        const int64_t t = t0 + tt;
+        float l0 = -INFINITY, l1 = -INFINITY;
+        if (lane < E) l0 = p.router_bias ? __fadd_rn(lg[tt * kLgRow + lane], p.router_bias[lane]) : lg[tt * kLgRow + lane];
+        if (lane + 32 < E)
+            l1 = p.router_bias ? __fadd_rn(lg[tt * kLgRow + lane + 32], p.router_bias[lane + 32])
+                               : lg[tt * kLgRow + lane + 32];
+        gate_topk_warp(p, t, l0, l1, lane);
+        const float s = sxs[tt];
+        const uint4* xr = reinterpret_cast<const uint4*>(p.x + t * d);
+        uint2* q = reinterpret_cast<uint2*>(p.xq + (p.Tk + t) * d);
+        for (int i = lane; i < d / 8; i += 32) {
+            const uint4 v = xr[i];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[2] = {0u, 0u};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t bits = (w[u >> 1] >> (16 * (u & 1))) & 0xffffu;
+                o[u >> 2] |= (uint32_t)(quant_i8(bf16_to_f32(bits), s) & 0xff) << (8 * (u & 3));
+            }
+            q[i] = make_uint2(o[0], o[1]);
+        }
+        if (lane == 0) {
+            p.sx[t] = s;
+            p.row_src[p.Tk + t] = (int32_t)t;
+            p.row_gate[p.Tk + t] = 1.0f;
+        }
+    }
+}
+
+// W_r [d, E] FP32 -> the split layout above (one thread per (chunk, expert row, k))
+__global__ void split_router_kernel(const float* w, int d, int E, uint16_t* out) {
+    const int64_t n = (int64_t)(d / kKC) * 64 * kKC;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int kk = (int)(i % kKC), e = (int)((i / kKC) % 64), c = (int)(i / (64 * kKC));
+        const float v = e < E ? w[(int64_t)(c * kKC + kk) * E + e] : 0.0f;
+        const uint32_t hi = bf16_rn_bits(v);
+        const float r1 = __fsub_rn(v, __uint_as_float(hi << 16));
+        const uint32_t mid = bf16_rn_bits(r1);
+        const float r2 = __fsub_rn(r1, __uint_as_float(mid << 16));
+        const uint32_t lo = bf16_rn_bits(r2);
+        uint16_t* base = out + (size_t)c * (kWChunkBytes / 2) + e * kRow + kk;
+        base[0] = (uint16_t)hi;
+        base[kWPieceBytes / 2] = (uint16_t)mid;
+        base[2 * (kWPieceBytes / 2)] = (uint16_t)lo;
+    }
+    // padding columns stay as the caller cleared them
+}
+
+}  // namespace rmma
+
+bool router_mma_supported(int d, int E) { return d % rmma::kKC == 0 && E <= 64; }
+
+size_t router_split_bytes(int d) { return (size_t)(d / rmma::kKC) * rmma::kWChunkBytes; }
+
+cudaError_t launch_split_router(const float* w, int d, int E, uint16_t* out, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(out, 0, router_split_bytes(d), s);
+    if (e != cudaSuccess) return e;
+    rmma::split_router_kernel<<<256, 256, 0, s>>>(w, d, E, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_mma(const Plan& p, cudaStream_t s) {
+    if (p.T == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(rmma::router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)rmma::kSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (p.T + rmma::kTok - 1) / rmma::kTok;
+    rmma::router_mma_kernel<<<(unsigned)blocks, rmma::kThreads, rmma::kSmem, s>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace mmoe

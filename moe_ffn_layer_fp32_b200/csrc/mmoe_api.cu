@@ -67,6 +67,7 @@ struct mmoe_handle {
     // weights (interchange layout)
     float* w_router = nullptr;
     float* router_bias = nullptr;
+    uint16_t* w_router_split = nullptr;  // tensor-core router pieces (when d_model % 64 == 0)
     uint8_t* w_gate_up = nullptr;
     float* s_gate_up = nullptr;
     uint8_t* w_down = nullptr;
@@ -104,7 +105,7 @@ struct mmoe_handle {
     int* err_host = nullptr;   // mapped pinned host memory; kernels write its device alias
     int* err_host_dev = nullptr;
     int* err_dev = nullptr;    // device memory copy read by every CTA
-    // decode path: weights in the decode layout, row absmax, group list, router ticket
+    // decode path: weights in the decode layout, row absmax, group list
     bool use_dec = false;
     bool last_dec = false;
     int dec_max_T = 0;
@@ -114,7 +115,6 @@ struct mmoe_handle {
     uint32_t* amax_h = nullptr;
     int32_t* dec_groups = nullptr;
     int32_t* dec_ngroups = nullptr;
-    int32_t* dec_ticket = nullptr;
     // per-stage timing (mmoe_profile_*)
     struct ProfRec {
         int stage, launches;
@@ -137,12 +137,12 @@ cudaError_t dalloc(T** p, size_t count) {
 }
 
 void free_all(mmoe_handle* h) {
-    void* ptrs[] = {h->w_router, h->router_bias, h->w_gate_up, h->s_gate_up, h->w_down, h->s_down,
+    void* ptrs[] = {h->w_router, h->router_bias, h->w_router_split, h->w_gate_up, h->s_gate_up, h->w_down, h->s_down,
                     h->xq, h->sx, h->logits, h->idx, h->gate, h->chunk_cnt, h->chunk_base, h->offsets,
                     h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
                     h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
                     h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->amax_h, h->dec_groups,
-                    h->dec_ngroups, h->dec_ticket};
+                    h->dec_ngroups};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);
@@ -190,6 +190,7 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.deterministic = (c.flags & MMOE_FLAG_DETERMINISTIC) != 0;
     p.w_router = h->w_router;
     p.router_bias = c.has_router_bias ? h->router_bias : nullptr;
+    p.w_router_split = h->w_router_split;
     p.w_gate_up = h->w_gate_up;
     p.s_gate_up = h->s_gate_up;
     p.w_down = h->w_down;
@@ -231,7 +232,6 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.amax_h = h->amax_h;
     p.dec_groups = h->dec_groups;
     p.dec_ngroups = h->dec_ngroups;
-    p.dec_ticket = h->dec_ticket;
     return p;
 }
 
@@ -374,6 +374,7 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     if (e == cudaSuccess) e = dalloc(&h->ptr, (size_t)(n))
     ALLOC(w_router, d * E);
     ALLOC(router_bias, E);
+    if (router_mma_supported((int)d, (int)E)) ALLOC(w_router_split, router_split_bytes((int)d) / 2);
     ALLOC(w_gate_up, h->n_gu_bytes);
     ALLOC(s_gate_up, h->n_gu_scales);
     ALLOC(w_down, h->n_d_bytes);
@@ -400,7 +401,7 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     h->use_dec = !(cfg->flags & (MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE)) && dec_supported((int)d, (int)hh, (int)hs);
     if (h->use_dec) {
         h->dec_max_T = dec_max_tokens((int)d, h->hmax);
-        h->dec_cluster = dec_router_cluster((int)d);
+        h->dec_cluster = dec_router_cluster((int)d, (int)E);
         if (h->dec_max_T <= 0 || h->dec_cluster == 0) h->use_dec = false;
     }
     if (h->use_dec) {
@@ -410,8 +411,6 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
         ALLOC(amax_h, Rd);
         ALLOC(dec_groups, E + 1);
         ALLOC(dec_ngroups, 1);
-        ALLOC(dec_ticket, 1);
-        if (e == cudaSuccess) e = cudaMemset(h->dec_ticket, 0, sizeof(int32_t));
     }
     if (h->use_tc || h->use_dec) {
         ALLOC(err_dev, 1);
@@ -454,6 +453,8 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
     MMOE_CUDA(cudaMemcpyAsync(h->w_router, w->w_router, d * E * sizeof(float), kind, s), "copy w_router");
     if (h->cfg.has_router_bias)
         MMOE_CUDA(cudaMemcpyAsync(h->router_bias, w->router_bias, E * sizeof(float), kind, s), "copy router_bias");
+    if (h->w_router_split)
+        MMOE_CUDA(launch_split_router(h->w_router, (int)d, (int)E, h->w_router_split, s), "router split launch");
     MMOE_CUDA(cudaMemcpyAsync(h->w_gate_up, w->w_gate_up, h->n_gu_bytes, kind, s), "copy w_gate_up");
     MMOE_CUDA(cudaMemcpyAsync(h->s_gate_up, w->s_gate_up, h->n_gu_scales * sizeof(float), kind, s), "copy s_gate_up");
     MMOE_CUDA(cudaMemcpyAsync(h->w_down, w->w_down, h->n_d_bytes, kind, s), "copy w_down");
@@ -480,6 +481,8 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     if (!h->loaded) return fail(MMOE_ERR_NOT_LOADED, "forward before mmoe_load_quantized_weights");
     if (T == 0) return MMOE_OK;
     if (!x || !y) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
+        return fail(MMOE_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
     DeviceGuard dg(h->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     mmoe_status fst = check_device_flag(h, s);

@@ -25,6 +25,7 @@ struct Plan {
     // weights (interchange layout)
     const float* w_router;
     const float* router_bias;
+    const uint16_t* w_router_split;  // W_r as three BF16 pieces (tensor-core router), or null
     const uint8_t* w_gate_up;
     const float* s_gate_up;
     const uint8_t* w_down;
@@ -69,7 +70,6 @@ struct Plan {
     uint32_t* amax_h;             // [R] bits of max |SwiGLU output| of each row (non-negative floats order as integers)
     int32_t* dec_groups;          // [E + 1] groups with at least one row: the shared one first, then routed ascending
     int32_t* dec_ngroups;         // [1]
-    int32_t* dec_ticket;          // [1] router CTAs finished; 0 between launches
 };
 
 // Upper bound on the number of tile_rows-row tiles over all groups.
@@ -79,6 +79,10 @@ inline int64_t max_tiles_for(int64_t T, int k, int E, int tile_rows = kTileRows)
 
 // launchers (each returns the launch error, if any)
 cudaError_t launch_router_quant(const Plan& p, cudaStream_t s);
+bool router_mma_supported(int d, int E);
+size_t router_split_bytes(int d);
+cudaError_t launch_split_router(const float* w, int d, int E, uint16_t* out, cudaStream_t s);
+cudaError_t launch_router_mma(const Plan& p, cudaStream_t s);
 cudaError_t launch_permute(const Plan& p, cudaStream_t s);
 cudaError_t launch_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_requant(const Plan& p, cudaStream_t s);
@@ -93,7 +97,7 @@ cudaError_t launch_retile(const uint8_t* gu, const float* sgu, const uint8_t* dn
 // decode path (k_decode.cu): T <= dec_max_tokens, expert GEMVs on mma.sync
 bool dec_supported(int d, int h, int hs);
 int dec_max_tokens(int d, int hmax);
-int dec_router_cluster(int d);
+int dec_router_cluster(int d, int E);
 cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s);
 cudaError_t launch_gate_up_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
