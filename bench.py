@@ -30,6 +30,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer prefill tokens/s & decode us/layer; % of INT8-TC / HBM roofline"
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# prefill gate/up GEMM, from one ncu capture of this bench command on B200
+# (`--metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:expert_gemm_tc`);
+# valid only while that kernel is unchanged.
+GATE_UP_TRAFFIC_BYTES = {"c4": 498230272 + 622415616}
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -89,7 +95,7 @@ class ClockSampler:
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                       "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
 
@@ -119,7 +125,8 @@ class ClockSampler:
                     reasons.add(n)
         os.unlink(self.f.name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "from the first warm-up step to the end of the last GPU measurement"}
 
 
 # --------------------------------------------------------------------------
@@ -142,20 +149,8 @@ def layer_counts(w, T):
 
 def quantized_on_device(w, device, layer=0):
     """Seeded FP32 weights (synth) quantised on the GPU by the library's Eq. (6) kernel."""
-    import torch
-
-    from moe_ffn_layer_fp32_b200 import synth
-    from moe_ffn_layer_fp32_b200.layer import quantize_int4
-    lw = synth.workload_layer(w, layer)
-    gu_w, gu_s, dn_w, dn_s = [], [], [], []
-    for g in range(w.E + 1):
-        p, s = quantize_int4(torch.from_numpy(lw.w_gate_up[g]).to(device))
-        gu_w.append(p.reshape(-1)); gu_s.append(s.reshape(-1))
-        p, s = quantize_int4(torch.from_numpy(lw.w_down[g]).to(device))
-        dn_w.append(p.reshape(-1)); dn_s.append(s.reshape(-1))
-    wr = torch.from_numpy(lw.w_router).to(device)
-    bias = None if lw.router_bias is None else torch.from_numpy(lw.router_bias).to(device)
-    return (wr, bias, torch.cat(gu_w), torch.cat(gu_s), torch.cat(dn_w), torch.cat(dn_s)), lw
+    from moe_ffn_layer_fp32_b200.run_case import quantized_weights
+    return quantized_weights(w, device, layer)
 
 
 def weight_bytes(w, experts):
@@ -335,6 +330,7 @@ def run_ours(args):
                 ev[1].record(stream)
             decl.forward(xd, yd, topk_idx=idx_d)
 
+    clocks = ClockSampler(range(world)) if rank == 0 else None
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -346,7 +342,6 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks = ClockSampler(range(world)) if rank == 0 else None
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -358,7 +353,6 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
-    clk = clocks.stop() if clocks else None
     elapsed = start.elapsed_time(end)
     prefill_ms = statistics.median(starts[i].elapsed_time(evs[i][0]) for i in range(args.steps))
     decode_ms = statistics.median(evs[i][1].elapsed_time(starts[i + 1] if i + 1 < args.steps else end)
@@ -386,9 +380,10 @@ def run_ours(args):
         peak_note = "fallback 1.4 PFLOP/s bf16 sustained x 2"
     gu_avg_s = (ms_gu / max(n_gu, 1)) / 1e3
     achieved = gu_ops / gu_avg_s / 1e12 if gu_avg_s > 0 else 0.0
-    traffic = None
+    traffic = GATE_UP_TRAFFIC_BYTES.get(w.name)
     roofline = {"kernel": "gate_up (prefill)", "bound": "tensor", "achieved": achieved, "peak": int8_peak,
-                "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": traffic, "op_dtype": "int8",
+                "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": traffic, "traffic_unit": "bytes per launch (ncu)",
+                "op_dtype": "int8",
                 "peak_source": peak_note, "ops_per_launch": gu_ops, "avg_launch_ms": gu_avg_s * 1e3}
 
     decode = None
@@ -440,6 +435,7 @@ def run_ours(args):
     if not args.no_decode_sweep:
         sweep = decode_sweep(dev, args.steps, args.warmup, float(peaks.get("hbm_gbs", 6650.0)))
 
+    clk = clocks.stop() if clocks else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, n, dt = oracle_rate(w, args.cpu_seconds, lw)

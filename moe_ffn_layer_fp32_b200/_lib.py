@@ -20,6 +20,7 @@ GATE_SIGMOID_TOPK_NORM = 1
 FLAG_DETERMINISTIC = 1
 FLAG_CUDA_CORES = 2
 FLAG_NO_DECODE = 4
+FLAG_ATOMIC_COMBINE = 8
 
 STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAGE_SH, STAGE_LOGITS = range(8)
 

@@ -371,7 +371,9 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
         }
         const uint8_t* sb = S.ring + (sc % kRing) * kStageBytes;
         const int njs = S.NJ - st * kStageJP < kStageJP ? S.NJ - st * kStageJP : kStageJP;
-        for (int q = 0; q < njs; ++q) {
+#pragma unroll
+        for (int q = 0; q < kStageJP; ++q) {
+            if (q >= njs) break;
             const uint4 wv = *reinterpret_cast<const uint4*>(sb + q * kJP + lane * 16);
             const float4 sv = *reinterpret_cast<const float4*>(sb + q * kJP + 512 + gid * 16);
             const int jp = st * kStageJP + q;

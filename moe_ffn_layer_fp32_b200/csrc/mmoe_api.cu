@@ -169,7 +169,7 @@ mmoe_status check_config(const mmoe_config* c) {
         return fail(MMOE_ERR_INVALID_ARG, "gating=%d: unknown", c->gating);
     if (c->has_router_bias != 0 && c->has_router_bias != 1)
         return fail(MMOE_ERR_INVALID_ARG, "has_router_bias=%d: must be 0 or 1", c->has_router_bias);
-    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE))
+    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE | MMOE_FLAG_ATOMIC_COMBINE))
         return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
     return MMOE_OK;
 }
@@ -396,7 +396,6 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(act, R * h->hmax);
     ALLOC(hq, R * h->hmax);
     ALLOC(sh, R);
-    if (cfg->flags & MMOE_FLAG_DETERMINISTIC) ALLOC(obuf, R * d);
     h->use_tc = !(cfg->flags & MMOE_FLAG_CUDA_CORES) && tc_supported((int)d, (int)hh, (int)hs);
     h->use_dec = !(cfg->flags & (MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE)) && dec_supported((int)d, (int)hh, (int)hs);
     if (h->use_dec) {
@@ -411,6 +410,13 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
         ALLOC(amax_h, Rd);
         ALLOC(dec_groups, E + 1);
         ALLOC(dec_ngroups, 1);
+    }
+    if (e == cudaSuccess) {
+        // the fixed-order combine needs the per-row outputs: always in deterministic mode, and by
+        // default whenever a forward can take the prefill path (more tokens than the decode path takes)
+        const bool det = (cfg->flags & MMOE_FLAG_DETERMINISTIC) != 0;
+        const bool prefill_possible = !h->use_dec || Tm > h->dec_max_T;
+        if (det || (prefill_possible && !(cfg->flags & MMOE_FLAG_ATOMIC_COMBINE))) ALLOC(obuf, R * d);
     }
     if (h->use_tc || h->use_dec) {
         ALLOC(err_dev, 1);
@@ -487,8 +493,11 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     mmoe_status fst = check_device_flag(h, s);
     if (fst != MMOE_OK) return fst;
-    const Plan p = make_plan(h, x, T, y);
     const bool dec = h->use_dec && T <= h->dec_max_T;
+    Plan p = make_plan(h, x, T, y);
+    // fixed-order combine: always in deterministic mode; on the prefill path unless atomics were asked for
+    p.deterministic = (h->cfg.flags & MMOE_FLAG_DETERMINISTIC) ||
+                      (!dec && !(h->cfg.flags & MMOE_FLAG_ATOMIC_COMBINE));
     if (dec) {
         // decode path: router + permutation, gate/up (also clears y), down
         MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_dec(p, h->dec_cluster, s); }),

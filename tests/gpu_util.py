@@ -22,11 +22,11 @@ def x_to_device(x_np: np.ndarray) -> torch.Tensor:
 
 
 def make_gpu_layer(q: oracle.QuantizedLayer, max_tokens: int, deterministic: bool = False, cuda_cores: bool = False,
-                   decode: bool = True):
+                   decode: bool = True, atomic_combine: bool = False):
     from moe_ffn_layer_fp32_b200.layer import MoELayer
     L = MoELayer(q.d, q.h, shared_hidden=q.hs, n_experts=q.E, top_k=q.k, max_tokens=max_tokens,
                  gating=q.gating, has_router_bias=q.router_bias is not None, deterministic=deterministic,
-                 cuda_cores=cuda_cores, decode=decode)
+                 cuda_cores=cuda_cores, decode=decode, atomic_combine=atomic_combine)
     L.load(q.w_router, q.router_bias, q.w_gate_up, q.s_gate_up, q.w_down, q.s_down)
     return L
 

@@ -53,10 +53,11 @@ def test_quantizer_matches_oracle_bit_exact():
     assert np.array_equal(s_gpu.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
-def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False, decode=True):
+def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False, decode=True,
+                atomic_combine=False):
     T = x.shape[0]
     L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic, cuda_cores=cuda_cores,
-                          decode=decode)
+                          decode=decode, atomic_combine=atomic_combine)
     out = gu.run_gpu(L, q, x)
     y, D = oracle.moe_layer(q, x, dumps=True)
     rep = {}
@@ -72,14 +73,16 @@ def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, c
 
 
 @pytest.mark.parametrize("path", ["decode", "tensor_cores", "cuda_cores"])
-@pytest.mark.parametrize("deterministic", [False, True], ids=["atomic", "fixed_order"])
-def test_c0_all_stages(deterministic, path):
-    # T = 64 takes the decode kernels by default; the other two force the prefill kernels
+@pytest.mark.parametrize("combine", ["atomic", "fixed_order"])
+def test_c0_all_stages(combine, path):
+    # T = 64 takes the decode kernels by default; the other two force the prefill kernels.
+    # atomic: the decode path's default, forced on the prefill path; fixed_order: forced on the decode path
     w, q = workload("c0")
     x = synth.workload_x(w)
     R = w.T * (q.k + 1)
-    rep, out = _full_check(q, x, deterministic, partial_rows=range(0, R, 3), cuda_cores=path == "cuda_cores",
-                           decode=path == "decode")
+    rep, out = _full_check(q, x, combine == "fixed_order", partial_rows=range(0, R, 3),
+                           cuda_cores=path == "cuda_cores", decode=path == "decode",
+                           atomic_combine=combine == "atomic")
     print("c0", path, rep)
 
 
@@ -125,6 +128,12 @@ def test_c2_prefill_cuda_cores():
     w, q = workload("c2")
     x = synth.workload_x(w, T=512)
     rep, out = _full_check(q, x, cuda_cores=True, partial_rows=[0, 2047, 2048, 2559])
+
+
+def test_c2_prefill_atomic_combine():
+    w, q = workload("c2")
+    x = synth.workload_x(w, T=1024)
+    rep, out = _full_check(q, x, atomic_combine=True, partial_rows=[0, 4095, 4096, 5119])
 
 
 def test_T0_is_a_noop():
