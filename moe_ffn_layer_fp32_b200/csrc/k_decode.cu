@@ -63,9 +63,9 @@ constexpr int kRThreads = 256;
 constexpr int kRTok = 64;                       // tokens of the decode path (one router cluster)
 constexpr int kRHeadBytes = (kRTok * 64 + 2 * kRTok) * 4 + 16;  // partial logits, absmax, s_x, mbarrier
 
-// router shared memory: head | x slice [kRTok][ks] BF16 | W_r slice [ks][E] FP32
-__host__ __device__ constexpr size_t router_smem(int d, int cs, int E) {
-    return (size_t)kRHeadBytes + (size_t)kRTok * (d / cs) * 2 + (size_t)(d / cs) * E * 4;
+// router shared memory: head | x slice [kRTok][ks + 8] BF16 | W_r pieces of the slice (ks / 64 chunks)
+__host__ __device__ constexpr size_t router_smem(int d, int cs) {
+    return (size_t)kRHeadBytes + (size_t)kRTok * (d / cs + 8) * 2 + (size_t)(d / cs / kRouterKChunk) * kRouterChunkBytes;
 }
 
 // ------------------------------------------------------------------ helpers
@@ -161,6 +161,17 @@ __device__ __forceinline__ uint32_t pack_codes(float a, float b, float c, float 
 }
 
 // ------------------------------------------------------------------ router
+__device__ __forceinline__ void prefetch_l2(const void* ptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
+constexpr int64_t kDownPrefetchLimit = 32ll << 20;
+
+// Asks L2 for `bytes` bytes at `ptr` in 32 KB pieces (bytes a multiple of 16); one thread.
+__device__ void prefetch_range(const uint8_t* ptr, int64_t bytes) {
+    for (int64_t o = 0; o < bytes; o += 32768) prefetch_l2(ptr + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768));
+}
+
 // The permutation of the routing slots, by one block of kRThreads threads:
 // per-expert counts, offsets, the list of groups with rows, and a stable
 // scatter (rows of an expert in ascending slot order).
@@ -175,20 +186,41 @@ __device__ void permute_block(const Plan& p) {
     __syncthreads();
     for (int s = tid; s < S; s += kRThreads) atomicAdd(&cnt[__ldcg(p.idx + s)], 1);
     __syncthreads();
-    if (tid == 0) {
-        int o = 0, n = 0;
-        p.dec_groups[n++] = E;
-        for (int e = 0; e < E; ++e) {
-            base[e] = o;
-            p.offsets[e] = o;
-            p.counts[e] = cnt[e];
-            o += cnt[e];
-            if (cnt[e]) p.dec_groups[n++] = e;
+    if (warp == 0) {
+        // exclusive scan of the counts (experts lane and lane + 32) and the list of groups with
+        // rows: the shared one first, then the routed ones in ascending order
+        const int c0 = lane < E ? cnt[lane] : 0, c1 = lane + 32 < E ? cnt[lane + 32] : 0;
+        int s0 = c0, s1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u0 = __shfl_up_sync(0xffffffffu, s0, o), u1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) { s0 += u0; s1 += u1; }
         }
-        p.offsets[E] = o;
-        p.offsets[E + 1] = o + (int)p.T;
-        p.counts[E] = (int)p.T;
-        *p.dec_ngroups = n;
+        const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+        s1 += tot0;
+        const int tot = __shfl_sync(0xffffffffu, s1, 31);
+        const unsigned b0 = __ballot_sync(0xffffffffu, c0 > 0), b1 = __ballot_sync(0xffffffffu, c1 > 0);
+        const unsigned lt = (1u << lane) - 1u;
+        if (lane < E) {
+            base[lane] = s0 - c0;
+            p.offsets[lane] = s0 - c0;
+            p.counts[lane] = c0;
+            if (c0) p.dec_groups[1 + __popc(b0 & lt)] = lane;
+        }
+        if (lane + 32 < E) {
+            base[lane + 32] = s1 - c1;
+            p.offsets[lane + 32] = s1 - c1;
+            p.counts[lane + 32] = c1;
+            if (c1) p.dec_groups[1 + __popc(b0) + __popc(b1 & lt)] = lane + 32;
+        }
+        const int nrouted = __popc(b0) + __popc(b1);
+        if (lane == 0) {
+            p.dec_groups[0] = E;
+            *p.dec_ngroups = 1 + nrouted;
+            p.offsets[E] = tot;
+            p.offsets[E + 1] = tot + (int)p.T;
+            p.counts[E] = (int)p.T;
+        }
     }
     __syncthreads();
     for (int s0 = 0; s0 < S; s0 += kRThreads) {
@@ -221,75 +253,78 @@ __device__ void permute_block(const Plan& p) {
 }
 
 // One cluster of `cs` CTAs handles all T <= 64 tokens; CTA `rank` the K rows
-// [rank ks, (rank + 1) ks) of W_r and x.  After the first cluster barrier
-// every CTA knows the activation scales (max over the cluster) and quantises
-// its slice; the owner CTA of token t (t mod cs) adds the partial logits in
-// rank order and runs gating and top-k; after the second barrier rank 0
-// builds the permutation (the barrier's release / acquire orders the owners'
-// writes of idx and gate before it).
+// [rank ks, (rank + 1) ks) of W_r and x (ks a multiple of 64).  Its partial
+// logits come from the tensor cores (W_r as exact BF16 pieces, each 16-wide K
+// step added in FP32).  After the first cluster barrier every CTA knows the
+// activation scales (max over the cluster) and quantises its slice; the owner
+// CTA of token t (t mod cs) adds the partial logits in rank order and runs
+// gating and top-k; after the second barrier rank 0 builds the permutation (the
+// barrier's release / acquire orders the owners' writes of idx and gate) and
+// asks L2 for the selected experts' weights.
 __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     const int d = p.d, E = p.E;
     const int ks = d / cs;
+    const int xrow = ks + 8;  // padded BF16 row of the x slice
     float* part = reinterpret_cast<float*>(smem);             // [kRTok][64] partial logits
     float* pmax = part + kRTok * 64;                          // [kRTok] partial absmax
     float* sxs = pmax + kRTok;                                // [kRTok] s_x
     uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + kRHeadBytes - 16);
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kRHeadBytes);  // [kRTok][ks]
-    float* ws = reinterpret_cast<float*>(xs + kRTok * ks);            // [ks][E]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kRHeadBytes);  // [kRTok][xrow]
+    uint8_t* ws = reinterpret_cast<uint8_t*>(xs + kRTok * xrow);      // ks / 64 chunks of W_r pieces
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
     const int rank = (int)cluster_rank();
     const int nt = (int)p.T;
     const int k0 = rank * ks;
+    const int mtiles = (nt + 15) >> 4;
     pdl_trigger();
 
-    // W_r rows and x slices of this CTA: bulk copies (ks * E * 4 and ks * 2 bytes, multiples of 16)
     if (tid == 0) {
         mbar_init(wbar, 1);
         fence_barrier_init();
-        const uint32_t wbytes = (uint32_t)ks * E * 4, xbytes = (uint32_t)ks * 2;
+        const uint32_t wbytes = (uint32_t)(ks / kRouterKChunk) * kRouterChunkBytes, xbytes = (uint32_t)ks * 2;
         mbar_expect_tx(wbar, wbytes + xbytes * nt);
-        bulk_load(ws, p.w_router + (int64_t)k0 * E, wbytes, wbar);
-        for (int t = 0; t < nt; ++t) bulk_load(xs + t * ks, p.x + (int64_t)t * d + k0, xbytes, wbar);
+        bulk_load(ws, reinterpret_cast<const uint8_t*>(p.w_router_split) + (size_t)(k0 / kRouterKChunk) * kRouterChunkBytes,
+                  wbytes, wbar);
+        for (int t = 0; t < nt; ++t) bulk_load(xs + t * xrow, p.x + (int64_t)t * d + k0, xbytes, wbar);
     }
-    // rows of absent tokens are zero (disjoint from the copies)
-    for (int i = nt * (ks / 8) + tid; i < kRTok * (ks / 8); i += kRThreads)
+    // rows of the last m16 tile beyond T are zero (disjoint from the copies)
+    for (int i = nt * (xrow / 8) + tid; i < mtiles * 16 * (xrow / 8); i += kRThreads)
         reinterpret_cast<uint4*>(xs)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
     const bool have = wait_bounded(wbar, 0);
     if (!have && tid == 0) set_error(p, 8);
-    {
-        // expert lane e, tokens tq + 4 q; FP32 sum over k ascending
-        const int e = tid & 63, tq = tid >> 6;
-        float acc[kRTok / 4];
+
+    // partial logits: work item (m16 tile of tokens, pair of n8 tiles of experts)
+    for (int it = warp; it < mtiles * 4; it += kRThreads / 32) {
+        const int m = it >> 2, np = it & 3;
+        float acc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+        if (have) {
+            const uint16_t* xa = xs + (m * 16 + gid) * xrow + 2 * t4;
+            for (int kk = 0; kk < ks; kk += 16) {
+                const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xa + kk);
+                const uint32_t a1 = *reinterpret_cast<const uint32_t*>(xa + 8 * xrow + kk);
+                const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xa + kk + 8);
+                const uint32_t a3 = *reinterpret_cast<const uint32_t*>(xa + 8 * xrow + kk + 8);
+                const uint16_t* wb = reinterpret_cast<const uint16_t*>(ws + (kk / kRouterKChunk) * kRouterChunkBytes) +
+                                     gid * kRouterRow + 2 * t4 + (kk % kRouterKChunk);
 #pragma unroll
-        for (int q = 0; q < kRTok / 4; ++q) acc[q] = 0.0f;
-        if (e < E && have && tq < nt) {
-            const float* w = ws + e;
-            for (int kk = 0; kk < ks; kk += 8) {
-                float wv[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) wv[u] = w[(kk + u) * E];
-#pragma unroll
-                for (int q = 0; q < kRTok / 4; ++q) {
-                    if (tq + 4 * q >= nt) continue;
-                    const uint4 xv = *reinterpret_cast<const uint4*>(xs + (tq + 4 * q) * ks + kk);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        acc[q] = fmaf(__uint_as_float(xw[u] << 16), wv[2 * u], acc[q]);
-                        acc[q] = fmaf(__uint_as_float(xw[u] & 0xffff0000u), wv[2 * u + 1], acc[q]);
-                    }
-                }
+                for (int j = 0; j < 2; ++j) router_kstep(acc[j], a0, a1, a2, a3, wb + (2 * np + j) * 8 * kRouterRow);
             }
         }
 #pragma unroll
-        for (int q = 0; q < kRTok / 4; ++q) part[(tq + 4 * q) * 64 + e] = acc[q];
+        for (int j = 0; j < 2; ++j) {
+            const int col = (2 * np + j) * 8 + 2 * t4;
+            part[(m * 16 + gid) * 64 + col] = acc[j][0];
+            part[(m * 16 + gid) * 64 + col + 1] = acc[j][1];
+            part[(m * 16 + gid + 8) * 64 + col] = acc[j][2];
+            part[(m * 16 + gid + 8) * 64 + col + 1] = acc[j][3];
+        }
     }
     for (int t = warp; t < nt; t += kRThreads / 32) {
         float m = 0.0f;
-        for (int i = lane; i < ks; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * ks + i])));
+        for (int i = lane; i < ks; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * xrow + i])));
         m = warp_max(m);
         if (lane == 0) pmax[t] = m;
     }
@@ -306,7 +341,7 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
     // K1 on this CTA's slice: codes of the shared-expert rows (rows Tk + t of xq)
     for (int i = tid; i < nt * (ks / 4); i += kRThreads) {
         const int t = i / (ks / 4), v = i % (ks / 4);
-        const uint16_t* xr = xs + t * ks + v * 4;
+        const uint16_t* xr = xs + t * xrow + v * 4;
         *reinterpret_cast<uint32_t*>(p.xq + (p.Tk + t) * d + k0 + v * 4) =
             pack_codes(bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), sxs[t]);
     }
@@ -513,6 +548,18 @@ expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnr
     if (rb0 >= nrb) return;
     const int nrows = shared ? (int)p.T : p.counts[g];
     const int64_t row0 = shared ? p.Tk : p.offsets[g];
+    if (GU && !DUMP && !shared && tid == 0 &&  // routed CTAs have waited for the routing here
+        (int64_t)(*p.dec_ngroups) * ((int64_t)p.d * p.h * 5 / 8) <= kDownPrefetchLimit) {
+        // this CTA's share of the group's down weights toward L2, for the next launch (only when all
+        // selected down weights fit easily in L2 next to the gate/up weights streaming through it)
+        const int nblk = (nrb + W - 1) / W;
+        const int64_t dbytes = (int64_t)p.d * hid * 5 / 8;
+        const int64_t per = ((dbytes / nblk) + 15) / 16 * 16;
+        const int64_t o0 = (int64_t)blk * per;
+        if (o0 < dbytes)
+            prefetch_range(p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8) + o0,
+                           o0 + per <= dbytes ? per : dbytes - o0);
+    }
     const int NJ = K / 64;
     const int cs = K + 32;
     const int ngr = K / 32;
@@ -726,12 +773,13 @@ int dec_max_tokens(int d, int hmax) {
 }
 
 // CTAs per router cluster: 16 (non-portable size) where the device runs it,
-// else 8, else 4; each CTA's K slice must be a multiple of 8 elements and its
-// x and W_r slices must fit in shared memory.  0: no size works.
+// else 8, 4, 2, 1; each CTA's K slice must be a multiple of 64 (whole chunks of
+// the W_r pieces) and its x and W_r slices must fit in shared memory.  0: no
+// size works (the decode path is then off).
 int dec_router_cluster(int d, int E) {
-    for (int cs = 16; cs >= 4; cs >>= 1) {
-        const size_t smem = dec::router_smem(d, cs, E);
-        if (d % (8 * cs) || smem > (size_t)dec::kSmemLimit) continue;
+    for (int cs = 16; cs >= 1; cs >>= 1) {
+        const size_t smem = dec::router_smem(d, cs);
+        if (d % (cs * kRouterKChunk) || smem > (size_t)dec::kSmemLimit) continue;
         if (dec::raise_smem((const void*)dec::router_decode_kernel, dec::g_router_smem, smem) != cudaSuccess) {
             cudaGetLastError();
             continue;
@@ -762,7 +810,7 @@ int dec_router_cluster(int d, int E) {
 
 cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    const size_t smem = dec::router_smem(p.d, cluster, p.E);
+    const size_t smem = dec::router_smem(p.d, cluster);
     cudaError_t e = dec::raise_smem((const void*)dec::router_decode_kernel, dec::g_router_smem, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};

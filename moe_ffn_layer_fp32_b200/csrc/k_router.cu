@@ -154,11 +154,11 @@ namespace rmma {
 
 constexpr int kTok = 128;                 // tokens per CTA (8 warps x 16)
 constexpr int kThreads = 256;
-constexpr int kKC = 64;                   // K per chunk
-constexpr int kRow = 72;                  // padded BF16 row of a chunk
+constexpr int kKC = kRouterKChunk;        // K per chunk
+constexpr int kRow = kRouterRow;          // padded BF16 row of a chunk
 constexpr int kXChunkBytes = kTok * kRow * 2;          // 18432
-constexpr int kWPieceBytes = 64 * kRow * 2;            // 9216
-constexpr int kWChunkBytes = 3 * kWPieceBytes;         // 27648
+constexpr int kWPieceBytes = kRouterPieceBytes;
+constexpr int kWChunkBytes = kRouterChunkBytes;
 constexpr int kStages = 2;
 constexpr int kLgRow = 65;                // padded logits row
 constexpr size_t kSmem = (size_t)kStages * (kXChunkBytes + kWChunkBytes);  // logits alias the stages
@@ -170,26 +170,6 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// D = A * B (C = 0), m16n8k16, BF16 inputs, FP32 result
-__device__ __forceinline__ void mma_bf16_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%10, %10, %10, %10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
-}
-
-// D += A * B, m16n8k16, BF16 inputs, FP32 accumulators
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ float bf16_abs(uint32_t bits16) { return fabsf(__uint_as_float(bits16 << 16)); }
 
@@ -252,18 +232,7 @@ __global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
             // ever sum 48 exact products, so their internal rounding stays far below FP32's
             // over the whole K range
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const uint16_t* wr = wb + n * 8 * kRow + kk;
-                float part[4];
-                mma_bf16_first(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes),
-                               *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes + 8));
-                mma_bf16(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes / 2),
-                         *reinterpret_cast<const uint32_t*>(wr + kWPieceBytes / 2 + 8));
-                mma_bf16(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr),
-                         *reinterpret_cast<const uint32_t*>(wr + 8));
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[n][i] = __fadd_rn(acc[n][i], part[i]);
-            }
+            for (int n = 0; n < 8; ++n) router_kstep(acc[n], a0, a1, a2, a3, wb + n * 8 * kRow + kk);
         }
         __syncthreads();  // the stage is refilled by the next iteration
     }

@@ -108,7 +108,51 @@ cudaError_t make_tensor_map(void* map, void* base, uint64_t inner_bytes, uint64_
 cudaError_t launch_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t* packed, float* scales,
                                  cudaStream_t s);
 
+// W_r as three BF16 pieces (hi + mid + lo = the FP32 weight), in K chunks of 64:
+// per chunk three pieces of [64 experts][72] BF16 (64 K values + 8 of padding
+// that keep the mma.sync fragment loads free of shared-memory bank conflicts).
+constexpr int kRouterKChunk = 64;
+constexpr int kRouterRow = 72;
+constexpr int kRouterPieceBytes = 64 * kRouterRow * 2;          // 9216
+constexpr int kRouterChunkBytes = 3 * kRouterPieceBytes;        // 27648
+
 // --- device helpers -------------------------------------------------------
+// D = A * B (C = 0), m16n8k16, BF16 inputs, FP32 result
+__device__ __forceinline__ void mma_bf16_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%10, %10, %10, %10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// D += A * B, m16n8k16, BF16 inputs, FP32 accumulators
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 16-wide K step of the router for an m16 x n8 tile: the partial of the step
+// (lo, mid, hi pieces on the tensor cores; they only ever sum 48 exact products)
+// added to the running logits with round-to-nearest FP32 additions.  `wr` points
+// at expert row n*8 + gid, column kk + 2*t4 of the hi piece of the chunk.
+__device__ __forceinline__ void router_kstep(float (&acc)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             const uint16_t* wr) {
+    float part[4];
+    mma_bf16_first(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr + kRouterPieceBytes),
+                   *reinterpret_cast<const uint32_t*>(wr + kRouterPieceBytes + 8));
+    mma_bf16(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr + kRouterPieceBytes / 2),
+             *reinterpret_cast<const uint32_t*>(wr + kRouterPieceBytes / 2 + 8));
+    mma_bf16(part, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(wr), *reinterpret_cast<const uint32_t*>(wr + 8));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = __fadd_rn(acc[i], part[i]);
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
 __device__ __forceinline__ float warp_max(float v) {
