@@ -48,7 +48,7 @@ using async::su32;
 constexpr int kJP = 640;
 constexpr int kStageJP = 4;                     // K-group pairs per bulk copy
 constexpr int kStageBytes = kStageJP * kJP;     // 2560
-constexpr int kRing = 3;                        // bulk copies in flight per warp
+constexpr int kRingMax = 4;                     // bulk copies in flight per warp (at most)
 constexpr int kMaxWarps = 8;
 constexpr int kMaxChunks = 8;                   // T <= 64 = 8 B operands of 8 tokens
 constexpr int kPassRows = 16;                   // rows of a group per pass (2 B operands)
@@ -371,11 +371,11 @@ struct WarpStream {
     const uint8_t* src;   // the warp's 16-row block in the decode layout
     uint8_t* ring;
     uint64_t* bars;
-    int NJ, nst, sc0;
+    int NJ, nst, sc0, nring;
     __device__ __forceinline__ void issue(int st) const {
         const int jp = NJ - st * kStageJP;
         const uint32_t bytes = (uint32_t)((jp < kStageJP ? jp : kStageJP) * kJP);
-        const int slot = (sc0 + st) % kRing;
+        const int slot = (sc0 + st) % nring;
         mbar_expect_tx(&bars[slot], bytes);
         bulk_load(ring + slot * kStageBytes, src + (int64_t)st * kStageBytes, bytes, &bars[slot]);
     }
@@ -396,15 +396,15 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
     const uint8_t* bbase = codes + (size_t)gid * cs + t4 * 8;
     for (int st = 0; st < S.nst; ++st) {
         const int sc = S.sc0 + st;
-        if (!wait_bounded(&S.bars[sc % kRing], (uint32_t)((sc / kRing) & 1))) {
+        if (!wait_bounded(&S.bars[sc % S.nring], (uint32_t)((sc / S.nring) & 1))) {
             if (lane == 0) set_error(p, 7);
             // let the copies in flight land before the CTA's shared memory goes away
-            const int issued = st + kRing < S.nst ? st + kRing : S.nst;
+            const int issued = st + S.nring < S.nst ? st + S.nring : S.nst;
             for (int s = st; s < issued; ++s)
-                wait_bounded(&S.bars[(S.sc0 + s) % kRing], (uint32_t)(((S.sc0 + s) / kRing) & 1));
+                wait_bounded(&S.bars[(S.sc0 + s) % S.nring], (uint32_t)(((S.sc0 + s) / S.nring) & 1));
             return false;
         }
-        const uint8_t* sb = S.ring + (sc % kRing) * kStageBytes;
+        const uint8_t* sb = S.ring + (sc % S.nring) * kStageBytes;
         const int njs = S.NJ - st * kStageJP < kStageJP ? S.NJ - st * kStageJP : kStageJP;
 #pragma unroll
         for (int q = 0; q < kStageJP; ++q) {
@@ -449,7 +449,7 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
             }
         }
         __syncwarp();
-        if (lane == 0 && st + kRing < S.nst) S.issue(st + kRing);
+        if (lane == 0 && st + S.nring < S.nst) S.issue(st + S.nring);
     }
     if (DUMP) return true;
 
@@ -508,10 +508,10 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
 // The group's rows go in passes of up to kPassRows; each pass stages their
 // codes (B-fragment order inside each 32-group) and streams the weights again
 // (from L2 after the first pass).  Shared memory: mbarriers | row scales |
-// W rings of kRing stages | codes [kPassRows][K + 32].
+// W rings of nring stages | codes [kPassRows][K + 32].
 template <bool GU, bool DUMP>
 __global__ void __launch_bounds__(kMaxWarps * 32)
-expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnrows)
+expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, int64_t dnrows)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     const int W = blockDim.x >> 5;
@@ -519,7 +519,7 @@ expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnr
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     float* shs = reinterpret_cast<float*>(smem + 256);
     uint8_t* ring = smem + kHeadBytes;
-    uint8_t* codes = ring + W * kRing * kStageBytes;
+    uint8_t* codes = ring + W * nring * kStageBytes;
 
     pdl_trigger();
     if (GU && !DUMP && !p.deterministic && p.y) {
@@ -569,13 +569,14 @@ expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnr
     S.src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
                 : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
             (int64_t)rb * NJ * kJP;
-    S.ring = ring + warp * kRing * kStageBytes;
-    S.bars = bars + warp * kRing;
+    S.ring = ring + warp * nring * kStageBytes;
+    S.bars = bars + warp * kRingMax;
     S.NJ = NJ;
     S.nst = (NJ + kStageJP - 1) / kStageJP;
     S.sc0 = 0;
+    S.nring = nring;
     if (lane == 0) {
-        for (int s = 0; s < kRing; ++s) mbar_init(&S.bars[s], 1);
+        for (int s = 0; s < nring; ++s) mbar_init(&S.bars[s], 1);
         fence_barrier_init();
     }
     __syncwarp();
@@ -589,7 +590,7 @@ expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnr
         const int64_t rrow0 = row0 + prow0;
         if (pass > 0) __syncthreads();  // every warp is done with the previous pass's codes
         if (alive && lane == 0)
-            for (int s = 0; s < kRing && s < S.nst; ++s) S.issue(s);
+            for (int s = 0; s < nring && s < S.nst; ++s) S.issue(s);
         if (pass == 0 && shared) pdl_wait();  // weights are in flight; now the previous launch's outputs
 
         // codes of this pass's rows, zero rows up to a multiple of 8
@@ -608,6 +609,8 @@ expert_decode_kernel(Plan p, int nbpg, int32_t* dump, int64_t drow0, int64_t dnr
                 dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
             }
         } else {
+            // requantise the group's SwiGLU rows: s_h = absmax / 127 (the absmax was built by the
+            // gate/up CTAs with atomicMax); one CTA per group also records h_q and s_h
             for (int i = tid; i < nch * 8; i += blockDim.x)
                 shs[i] = i < prows ? __fdiv_rn(__uint_as_float(p.amax_h[rrow0 + i]), 127.0f) : 0.0f;
             __syncthreads();
@@ -723,9 +726,16 @@ int sm_count() {
     return n[dev];
 }
 
-size_t expert_smem(int W, int64_t T, int K) {
+size_t expert_smem(int W, int64_t T, int K, int nring) {
     const int64_t rows = T < kPassRows ? T : kPassRows;
-    return (size_t)kHeadBytes + (size_t)W * kRing * kStageBytes + (size_t)((rows + 7) / 8) * 8 * (K + 32);
+    return (size_t)kHeadBytes + (size_t)W * nring * kStageBytes + (size_t)((rows + 7) / 8) * 8 * (K + 32);
+}
+
+// Stages in flight per warp: all of a row block's stages when they are at most kRingMax,
+// else 3 (keeps two 8-warp CTAs per SM).
+int pick_ring(int K) {
+    const int nst = (K / 64 + kStageJP - 1) / kStageJP;
+    return nst <= kRingMax ? nst : 3;
 }
 
 // warps per CTA: as many as keep at least two CTAs per SM busy
@@ -742,7 +752,8 @@ cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t 
     const int max_nrb = GU ? p.hmax / 8 : p.d / 16;
     const int W = pick_warps((int64_t)gmax * max_nrb);
     const int nbpg = (max_nrb + W - 1) / W;
-    const size_t smem = expert_smem(W, p.T, GU ? p.d : p.hmax);
+    const int nring = pick_ring(GU ? p.d : p.hmax);
+    const size_t smem = expert_smem(W, p.T, GU ? p.d : p.hmax, nring);
     auto kern = dump ? expert_decode_kernel<GU, true> : expert_decode_kernel<GU, false>;
     static int granted[2][64] = {};
     cudaError_t e = raise_smem((const void*)kern, granted[dump ? 1 : 0], smem);
@@ -757,7 +768,7 @@ cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t 
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p, nbpg, dump, r0, nr);
+    return cudaLaunchKernelEx(&cfg, kern, p, nbpg, nring, dump, r0, nr);
 }
 
 }  // namespace
@@ -768,7 +779,7 @@ bool dec_supported(int d, int h, int hs) { return d % 64 == 0 && h % 64 == 0 && 
 int dec_max_tokens(int d, int hmax) {
     const int K = d > hmax ? d : hmax;
     int T = dec::kMaxT;
-    while (T > 0 && dec::expert_smem(dec::kMaxWarps, T, K) > (size_t)dec::kSmemLimit) T -= 8;
+    while (T > 0 && dec::expert_smem(dec::kMaxWarps, T, K, dec::kRingMax) > (size_t)dec::kSmemLimit) T -= 8;
     return T;
 }
 

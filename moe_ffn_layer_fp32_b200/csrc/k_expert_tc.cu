@@ -12,25 +12,27 @@
 //            same 64 hidden features, so one MMA per K group yields both
 //            halves of SwiGLU; K = d_model.
 //   down:    128 output features; K = hidden size of the group's expert.
-// Roles (20 warps):
-//   warp 0      producer: 1-D bulk copy of the packed INT4 weight tile
-//               (pre-tiled at load time, 8 KB per 128-K stage) and a 2-D TMA
-//               load (128B swizzle) of the 128 x 128 INT8 activation tile,
-//               running ahead across tile boundaries;
+// Roles (18 warps):
+//   warp 0      producer: one 1-D bulk copy of the weight stage (128 rows x
+//               128 K as INT8 holding 16 x the INT4 code, already in the
+//               canonical K-major SW128 layout: expanded once at load time,
+//               twice the INT4 bytes, so no warp unpacks in the hot loop) and
+//               a 2-D TMA load (128B swizzle) of the 128 x 128 INT8 activation
+//               tile, running ahead across tile boundaries;
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=128,
 //               K=32, INT8 x INT8 -> INT32), one instruction per 32-element
 //               K group into one of 4 TMEM buffers of 128 columns, handed
 //               over to the promotion warps two groups (a pair of buffers) at
 //               a time;
-//   warps 2-3   unpack INT4 -> INT8 into the canonical K-major SW128 layout;
-//   warps 4-19  promotion: read each group's INT32 partials from TMEM and
+//   warps 2-17  promotion: read each group's INT32 partials from TMEM and
 //               accumulate acc = fma(float(P_j), s_j, acc) in registers
 //               (4 warpgroups x 32 token columns, one weight row per thread),
 //               then the tile's epilogue, which overlaps the MMAs of the next
 //               tile.  After reading a buffer they refill it with the bit
-//               pattern of 1.5 * 2^23; the next MMA accumulates onto it, so
-//               the INT32 result P arrives as the float 1.5 * 2^23 + P
-//               (exact for |P| < 2^22) and one exact subtraction converts it.
+//               pattern of 1.5 * 2^19; the next MMA accumulates 16 P onto it
+//               (the weights enter as 16 x their code), so the INT32 result
+//               arrives as the float 1.5 * 2^19 + P (exact for |16 P| < 2^22)
+//               and one exact subtraction converts it.
 // The exact INT32 group partial is needed because every 32-element group of K
 // has its own FP32 weight scale; the promotion order (j ascending, fused
 // multiply-add) is the oracle's, so the FP32 result is identical to it.
@@ -48,26 +50,24 @@ namespace tc {
 constexpr int BM = 128;                    // weight rows per tile
 constexpr int BN = kTcTileRows;            // token rows per tile (128)
 constexpr int BK = 128;                    // K elements (bytes of INT8) per stage
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kBufs = 4;                   // TMEM accumulator buffers, 128 columns each
 constexpr int kPairs = kBufs / 2;          // buffers are handed over two at a time
 constexpr int kPromoWarpgroups = 4;        // each covers 32 token columns of all 128 weight rows
 constexpr int kPromoThreads = kPromoWarpgroups * 128;
-constexpr int kThreads = 128 + kPromoThreads;   // producer, MMA, 2 unpack warps, promotion warps
+constexpr int kThreads = 64 + kPromoThreads;    // producer, MMA, promotion warps
 constexpr int kCols = BN / kPromoWarpgroups;    // token columns per promotion thread
 
-constexpr int kUnpackThreads = 64;
-constexpr int kAPackedBytes = BM * BK / 2; // 8 KB
-constexpr int kAI8Bytes = BM * BK;         // 16 KB
+constexpr int kAI8Bytes = BM * BK;         // 16 KB: the weight stage image (INT8, SW128)
 constexpr int kBBytes = BN * BK;           // 16 KB
-constexpr int kStageBytes = kAI8Bytes + kBBytes + kAPackedBytes;
+constexpr int kStageBytes = kAI8Bytes + kBBytes;
 constexpr int kXchBytes = BM * BN * 4;     // finished FP32 tile handed to the epilogue, [column][row]
 constexpr long long kTimeoutClk = 4000000000ll;  // about 2 s of SM clock
 
 enum Epi { kEpiSwiGLU = 0, kEpiCombine = 1 };
 
 constexpr int kTInfo = 4;                  // tile-info ring entries
-constexpr int kTInfoConsumers = 1 + 2 + kPromoWarpgroups * 4;  // MMA lane, unpack warps, promotion warps
+constexpr int kTInfoConsumers = 1 + kPromoWarpgroups * 4;  // MMA lane, promotion warps
 
 // What every role needs to know about one tile, gathered by the producer warp
 // ahead of time (tile decode, per-column data, the first two group scales).
@@ -80,9 +80,8 @@ struct TileInfo {
 };
 
 struct Smem {
-    // stage buffers are carved from the 1024-aligned base: [A_i8 | B | A_packed] x kStages
+    // stage buffers are carved from the 1024-aligned base: [A_i8 | B] x kStages
     uint64_t full[kStages];
-    uint64_t unpacked[kStages];
     uint64_t empty[kStages];
     uint64_t accf[kPairs];   // a pair of buffers holds two finished groups
     uint64_t acce[kPairs];   // a pair of buffers has been read and preset again
@@ -154,7 +153,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
 // kind::i8: signed A and B, S32 accumulator, both K-major, M = 128, N = BN.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-// D += A * B (the accumulator holds the preset 1.5 * 2^23 bit pattern)
+// D += A * B (the accumulator holds the preset 1.5 * 2^19 bit pattern)
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -210,12 +209,16 @@ __device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
-constexpr float kMagic = 12582912.0f;
+// The weights enter the MMA as 16 x their INT4 code (the code in the high nibble
+// of a byte), so a group's result is 16 P.  TMEM is preset with the bit pattern
+// of 1.5 * 2^19, whose float ulp is 1/16: the float with bits (preset + 16 P) is
+// exactly 1.5 * 2^19 + P for |16 P| < 2^22 (|P| <= 32 * 8 * 127).
+constexpr uint32_t kMagicBits = 0x49400000u;  // 1.5 * 2^19
+constexpr float kMagic = 786432.0f;
 
 // Two columns at once with paired FP32 instructions (each half is an ordinary IEEE
 // operation, so the results equal the scalar ones):
-// (a0, a1) = fma((float(v0) - 1.5 * 2^23, float(v1) - 1.5 * 2^23), s, (a0, a1))
+// (a0, a1) = fma((float(v0) - 1.5 * 2^19, float(v1) - 1.5 * 2^19), s, (a0, a1))
 __device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32_t v1, float s) {
     asm("{\n\t.reg .b64 t, acc, sc, mg;\n\t"
         "mov.b64 t, {%2, %3};\n\t"
@@ -226,23 +229,13 @@ __device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32
         "fma.rn.f32x2 acc, t, sc, acc;\n\t"
         "mov.b64 {%0, %1}, acc;\n\t}"
         : "+f"(a0), "+f"(a1)
-        : "r"(v0), "r"(v1), "f"(s), "f"(12582912.0f));
-}
-
-// exact int32 -> float for |v| < 2^22: integer add into the mantissa of 1.5 * 2^23
-__device__ __forceinline__ float exact_i2f(int32_t v) { return __int_as_float(v + 0x4B400000) - 12582912.0f; }
-
-// 8 packed nibbles stored as [v0 v4 v1 v5 v2 v6 v3 v7] -> signed bytes (v0..v3), (v4..v7)
-__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t& lo, uint32_t& hi) {
-    const uint32_t l = w & 0x0f0f0f0fu, h = (w >> 4) & 0x0f0f0f0fu;
-    lo = l | ((l & 0x08080808u) * 0x1eu);
-    hi = h | ((h & 0x08080808u) * 0x1eu);
+        : "r"(v0), "r"(v1), "f"(s), "f"(kMagic));
 }
 
 struct TcArgs {
-    const uint8_t* wtiles;  // pre-tiled packed weights of the expert kind (gate/up or down)
+    const uint8_t* wtiles;  // weight stage images (INT8, SW128) of the expert kind (gate/up or down)
     const float* stiles;    // pre-tiled group scales
-    int64_t w_expert_stride_tiles;  // tiles (of kAPackedBytes) per routed expert
+    int64_t w_expert_stride_tiles;  // stage images (of kAI8Bytes) per routed expert
     int mblocks_routed;     // weight-row blocks of a routed expert (gate/up: h/64, down: d/128)
     int mblocks_shared;
     int ks_routed;          // K stages of a routed expert (gate/up: d/128, down: h/128)
@@ -296,6 +289,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem* 
 }
 
 template <int kEpi, bool kDump>
+// 18 warps: the SM sub-partitions holding 5 of them bound a thread to 96 registers
 __global__ void __launch_bounds__(kThreads, 1)
 expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a)
 {
@@ -315,7 +309,6 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm->full[s], 1);
-            mbar_init(&sm->unpacked[s], kUnpackThreads);
             mbar_init(&sm->empty[s], 1);
         }
         for (int b = 0; b < kPairs; ++b) {
@@ -391,9 +384,8 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                         break;
                     }
                     uint8_t* st = stages + s * kStageBytes;
-                    mbar_expect_tx(&sm->full[s], kAPackedBytes + kBBytes);
-                    bulk_load(st + kAI8Bytes + kBBytes, a.wtiles + ((int64_t)t.tile0 + ks) * kAPackedBytes, kAPackedBytes,
-                              &sm->full[s]);
+                    mbar_expect_tx(&sm->full[s], kAI8Bytes + kBBytes);
+                    bulk_load(st, a.wtiles + ((int64_t)t.tile0 + ks) * kAI8Bytes, kAI8Bytes, &sm->full[s]);
                     tma_load_2d(st + kAI8Bytes, &bmap, ks * BK, t.row0, &sm->full[s]);
                 }
             }
@@ -417,7 +409,7 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                 if (end) break;
                 for (int ks = 0; ks < nks && ok; ++ks, ++sc) {
                     const int s = sc % kStages;
-                    if (!mbar_wait(&sm->unpacked[s], (sc / kStages) & 1, sm, ef, 2)) { ok = false; break; }
+                    if (!mbar_wait(&sm->full[s], (sc / kStages) & 1, sm, ef, 2)) { ok = false; break; }
                     tc_after_sync();
                     uint8_t* st = stages + s * kStageBytes;
                     const uint64_t ad = smem_desc_sw128(st);
@@ -440,45 +432,9 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
             // every MMA issued has completed before TMEM is released
             if (pc > 0) mbar_wait_drain(&sm->accf[(pc - 1) & 1], ((pc - 1) >> 1) & 1);
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ INT4 -> INT8 unpack
-        const int t = tid - 64;
-        int sc = 0, tcount = 0;
-        bool ok = true;
-        while (ok) {
-            const int tb = tcount % kTInfo;
-            if (!warp_wait(&sm->tfull[tb], (tcount / kTInfo) & 1, sm, ef, 8)) break;
-            const int nks = sm->ti[tb].nks, end = sm->ti[tb].end;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->tempty[tb]);
-            ++tcount;
-            if (end) break;
-            for (int ks = 0; ks < nks; ++ks, ++sc) {
-                const int s = sc % kStages;
-                if (!mbar_wait(&sm->full[s], (sc / kStages) & 1, sm, ef, 4)) { ok = false; break; }
-                uint8_t* st = stages + s * kStageBytes;
-                const uint8_t* src = st + kAI8Bytes + kBBytes;
-#pragma unroll 2
-                for (int i = 0; i < (BM * BK / 2 / 16) / kUnpackThreads; ++i) {
-                    const int q = i * kUnpackThreads + t;   // 16-byte chunk of packed data (one K group of one row)
-                    const int row = q >> 2, c = q & 3;
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + row * 64 + c * 16);
-                    uint4 o0, o1;
-                    unpack_word(w.x, o0.x, o0.y);
-                    unpack_word(w.y, o0.z, o0.w);
-                    unpack_word(w.z, o1.x, o1.y);
-                    unpack_word(w.w, o1.z, o1.w);
-                    uint8_t* rowp = st + row * 128;
-                    *reinterpret_cast<uint4*>(rowp + (((2 * c) ^ (row & 7)) << 4)) = o0;
-                    *reinterpret_cast<uint4*>(rowp + (((2 * c + 1) ^ (row & 7)) << 4)) = o1;
-                }
-                fence_proxy_async();
-                mbar_arrive(&sm->unpacked[s]);
-            }
-        }
     } else {
         // ------------------------------------------------------------ promotion + epilogue
-        const int pw = warp - 4;            // 0..15
+        const int pw = warp - 2;            // 0..15
         const int wg = pw >> 2;             // token-column quarter
         const int quarter = warp & 3;       // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;  // weight row of this thread (0..127)
@@ -541,7 +497,7 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                             const int cc = col0 + c;
                             const int64_t grow = (int64_t)row0 + cc;
                             if (cc >= nr || grow < a.drow0 || grow >= a.drow0 + a.dnrows) continue;
-                            const int32_t pv = (int32_t)((c < 16 ? v[c & 15] : w[c & 15]) - (int32_t)kMagicBits);
+                            const int32_t pv = ((int32_t)(c < 16 ? v[c & 15] : w[c & 15]) - (int32_t)kMagicBits) >> 4;
                             if (kEpi == kEpiSwiGLU) {
                                 const int f = mb * 64 + (row & 63);
                                 const int n = row < 64 ? f : p.hmax + f;
@@ -609,20 +565,23 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
 }
 
 // --------------------------------------------------------------- weight re-tiling (load time)
-// gate/up tile (g, fb, ks): 128 rows x 64 bytes; rows 0..63 gate rows fb*64.., rows 64..127 the up rows of the
-// same features; bytes [ks*64, ks*64+64) of each interchange row with every 32-bit word's nibbles reordered
-// to [v0 v4 v1 v5 v2 v6 v3 v7].  Scales (g, fb, j): 128 floats, one per tile row.
-__device__ __forceinline__ uint32_t interleave_nibbles(uint32_t w) {
-    uint32_t o = 0;
+// gate/up stage (g, fb, ks): 128 rows x 128 K; rows 0..63 are gate rows fb*64 .. fb*64+63, rows 64..127 the up
+// rows of the same features; down stage (g, mb, ks): output rows mb*128 ..  Each row holds K values
+// ks*128 .. ks*128+127 as bytes 16 x code, its 16-byte chunk c stored at chunk c ^ (row & 7) (the 128-byte
+// swizzle the MMA's shared-memory descriptor expects at a 1024-byte aligned stage).  Scales (g, fb, j): 128
+// floats, one per stage row.
+
+// 8 nibbles (K order, low nibble first) -> 8 bytes 16 x code: (K 0..3), (K 4..7)
+__device__ __forceinline__ void expand_nibbles(uint32_t v, uint32_t& a, uint32_t& b) {
+    a = b = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        o |= ((w >> (4 * i)) & 15u) << (8 * i);
-        o |= ((w >> (4 * (i + 4))) & 15u) << (8 * i + 4);
+        a |= ((v >> (4 * i)) & 15u) << (8 * i + 4);
+        b |= ((v >> (4 * (i + 4))) & 15u) << (8 * i + 4);
     }
-    return o;
 }
 
-// one thread per 16-byte chunk of a tile row
+// one thread per 16-byte chunk of packed codes (32 K values) of a stage row
 __global__ void retile_weights_kernel(const uint8_t* __restrict__ src, const float* __restrict__ ssrc,
                                       uint8_t* __restrict__ dst, float* __restrict__ sdst, int E, int K_routed,
                                       int K_shared, int rows_routed, int rows_shared, int gate_up, int h, int hs,
@@ -630,7 +589,7 @@ __global__ void retile_weights_kernel(const uint8_t* __restrict__ src, const flo
 {
     const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (q >= total_chunks) return;
-    // q -> (expert, tile, row, chunk)
+    // q -> (expert, stage, row, chunk)
     const int64_t per_routed = (int64_t)rows_routed / BM * (K_routed / BK) * BM * 4;  // chunks of a routed expert
     int g;
     int64_t r;
@@ -653,11 +612,16 @@ __global__ void retile_weights_kernel(const uint8_t* __restrict__ src, const flo
     const int64_t src_expert_bytes = src_rows_routed * ((int64_t)K_routed / 2);
     const uint8_t* s = src + (int64_t)g * src_expert_bytes + srow * src_row_bytes + (int64_t)ks * 64 + chunk * 16;
     const uint4 w = *reinterpret_cast<const uint4*>(s);
-    const uint4 o = make_uint4(interleave_nibbles(w.x), interleave_nibbles(w.y), interleave_nibbles(w.z),
-                               interleave_nibbles(w.w));
+    uint4 o0, o1;  // K 32 chunk + 0..15 and 16..31
+    expand_nibbles(w.x, o0.x, o0.y);
+    expand_nibbles(w.y, o0.z, o0.w);
+    expand_nibbles(w.z, o1.x, o1.y);
+    expand_nibbles(w.w, o1.z, o1.w);
     const int64_t dst_tiles_routed = (int64_t)rows_routed / BM * (K_routed / BK);
     const int64_t dtile = (int64_t)g * dst_tiles_routed + tile;
-    reinterpret_cast<uint4*>(dst + dtile * kAPackedBytes + trow * 64)[chunk] = o;
+    uint4* row = reinterpret_cast<uint4*>(dst + dtile * kAI8Bytes + trow * 128);
+    row[(2 * chunk) ^ (trow & 7)] = o0;
+    row[(2 * chunk + 1) ^ (trow & 7)] = o1;
     // scale of group (ks*4 + chunk) of this row
     const int64_t src_expert_scales = src_rows_routed * ((int64_t)K_routed / kGroup);
     const float sc = ssrc[(int64_t)g * src_expert_scales + srow * (K / kGroup) + ks * 4 + chunk];

@@ -428,9 +428,9 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
         }
     }
     if (h->use_tc) {
-        ALLOC(w_gate_up_t, h->n_gu_bytes);
+        ALLOC(w_gate_up_t, 2 * h->n_gu_bytes);  // INT8 stage images: twice the packed INT4 bytes
         ALLOC(s_gate_up_t, h->n_gu_scales);
-        ALLOC(w_down_t, h->n_d_bytes);
+        ALLOC(w_down_t, 2 * h->n_d_bytes);
         ALLOC(s_down_t, h->n_d_scales);
         if (e == cudaSuccess) e = make_tensor_map(h->tmap_xq, h->xq, (uint64_t)d, (uint64_t)R, (uint64_t)d);
         if (e == cudaSuccess) e = make_tensor_map(h->tmap_hq, h->hq, (uint64_t)h->hmax, (uint64_t)R, (uint64_t)h->hmax);
