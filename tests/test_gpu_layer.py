@@ -117,6 +117,25 @@ def test_decode_hot_groups_of_64_rows():
     assert out["counts"][[5, 9, 33, 58]].tolist() == [64] * 4
 
 
+@pytest.mark.parametrize("decode", [True, False], ids=["decode", "prefill"])
+def test_top8_of_16_experts_64_tokens(decode):
+    # top-8: 512 routing slots at T = 64 (two scatter rounds in the decode router's permutation)
+    lw = synth.draw_layer(256, 128, E=16, seed=48)
+    q = oracle.quantize_layer(lw, k=8)
+    x = synth.draw_x(64, 256, seed=49)
+    rep, out = _full_check(q, x, partial_rows=[0, 100, 511, 512, 575], decode=decode)
+    assert out["counts"][:16].sum() == 512
+
+
+def test_decode_every_expert_selected():
+    # k = E: every token runs every routed expert (the full mixture)
+    lw = synth.draw_layer(256, 128, E=4, seed=50)
+    q = oracle.quantize_layer(lw, k=4)
+    x = synth.draw_x(33, 256, seed=51)
+    rep, out = _full_check(q, x, partial_rows=[0, 131, 132, 164])
+    assert out["counts"].tolist() == [33] * 5
+
+
 def test_decode_shared_expert_wider_than_routed():
     lw = synth.draw_layer(256, 64, seed=46, shared_hidden=256)
     q = oracle.quantize_layer(lw)
