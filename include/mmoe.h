@@ -261,8 +261,8 @@ mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_m
  *     on the GPU (different streams, or different host threads) race on the
  *     array and corrupt each other's results: order them on one stream.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
- * Errors: INVALID_ARG (bad config, NULL or host weight pointers, T < 0, the
- * scratch limit), CUDA. */
+ * Errors: INVALID_ARG (bad config, NULL or host weight pointers, T < 0, NULL
+ * or not 16-byte aligned x or y, the scratch limit), CUDA. */
 #define MMOE_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
 
 mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weights* w, const uint16_t* x_bf16,

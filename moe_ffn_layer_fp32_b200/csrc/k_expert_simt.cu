@@ -221,18 +221,24 @@ __global__ void __launch_bounds__(kThreads) down_simt_kernel(Plan p, int32_t* du
 }
 
 // y[t] = o(shared row of t) + sum_j gate[t, j] * o(row of slot j), in that order
+// (4 consecutive outputs per thread; d_model is a multiple of 32 and the rows 16-byte aligned)
 __global__ void __launch_bounds__(kThreads) combine_kernel(Plan p)
 {
-    const int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (i >= p.T * p.d) return;
-    const int64_t t = i / p.d;
-    const int m = (int)(i % p.d);
-    float y = p.obuf[(p.Tk + t) * p.d + m];
+    const int64_t i4 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i4 >= p.T * p.d / 4) return;
+    const int64_t t = i4 * 4 / p.d;
+    const int m = (int)(i4 * 4 % p.d);
+    float4 y = *reinterpret_cast<const float4*>(p.obuf + (p.Tk + t) * p.d + m);
     for (int j = 0; j < p.k; ++j) {
         const int64_t r = p.slot_row[t * p.k + j];
-        y = __fadd_rn(y, __fmul_rn(p.gate[t * p.k + j], p.obuf[r * p.d + m]));
+        const float g = p.gate[t * p.k + j];
+        const float4 o = *reinterpret_cast<const float4*>(p.obuf + r * p.d + m);
+        y.x = __fadd_rn(y.x, __fmul_rn(g, o.x));
+        y.y = __fadd_rn(y.y, __fmul_rn(g, o.y));
+        y.z = __fadd_rn(y.z, __fmul_rn(g, o.z));
+        y.w = __fadd_rn(y.w, __fmul_rn(g, o.w));
     }
-    p.y[i] = y;
+    *reinterpret_cast<float4*>(p.y + i4 * 4) = y;
 }
 
 }  // namespace
@@ -266,7 +272,7 @@ cudaError_t launch_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t ro
 
 cudaError_t launch_combine(const Plan& p, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    const int64_t n = p.T * p.d;
+    const int64_t n = p.T * p.d / 4;
     combine_kernel<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }

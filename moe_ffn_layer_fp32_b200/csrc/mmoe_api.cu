@@ -691,6 +691,8 @@ mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weigh
     if (T < 0) return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be >= 0", (long long)T);
     if (T == 0) return MMOE_OK;
     if (!x || !y) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
+        return fail(MMOE_ERR_INVALID_ARG, "x and y must be 16-byte aligned");
 
     Plan p{};
     p.d = cfg->d_model;
