@@ -147,10 +147,16 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
 mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, float* y, void* stream,
                          int32_t* topk_idx, float* topk_gate, int32_t* expert_counts);
 
-/* The same layer with HOST buffers: copies x (host, BF16 bits [T, d_model])
- * to the handle's staging buffer, runs mmoe_forward, copies y back to the
- * host buffer and waits for the stream.  The copies use one cudaMemcpyAsync
- * each.  Errors: as mmoe_forward. */
+/* The same layer with HOST buffers: x (host, BF16 bits [T, d_model]) in,
+ * y (host, FP32 [T, d_model]) out; returns when y is written.  A batch of
+ * T >= 16384 tokens runs as 2 to 4 chunks of at least 8192 tokens: chunk i's
+ * x is copied on an internal stream, mmoe_forward runs on `stream` after that
+ * copy, and its y is copied back on a second internal stream, so copies and
+ * the layer overlap.  Each token's output depends on that token alone, so y
+ * equals that of one unsplit forward.  Pinned host memory makes the copies
+ * asynchronous; pageable memory works but overlaps less.  `stream` is ordered
+ * after both internal streams on return.  The inspection functions below then
+ * describe the last chunk.  Errors: as mmoe_forward. */
 mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_bf16_host, int64_t T, float* y_host,
                               void* stream);
 

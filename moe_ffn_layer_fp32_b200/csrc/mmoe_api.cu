@@ -2,6 +2,7 @@
 // workspace, weight loading and the stream-ordered forward pass.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -55,6 +56,13 @@ struct DeviceGuard {
     }
 };
 
+// mmoe_forward_host splits a batch into up to kHostChunksMax chunks of at
+// least kHostChunkMinTokens tokens (boundaries on multiples of 128 tokens), so
+// that the copies of one chunk overlap the layer on another.  Every token's
+// output depends on that token alone, so the split leaves y unchanged.
+constexpr int kHostChunksMax = 4;
+constexpr int64_t kHostChunkMinTokens = 8192;
+
 }  // namespace
 
 struct mmoe_handle {
@@ -94,6 +102,10 @@ struct mmoe_handle {
     float* obuf = nullptr;
     uint16_t* x_stage = nullptr;
     float* y_stage = nullptr;
+    // mmoe_forward_host: copy streams and the events that order chunks against the compute stream
+    cudaStream_t s_h2d = nullptr, s_d2h = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_done = nullptr;
+    cudaEvent_t ev_in[kHostChunksMax] = {}, ev_out[kHostChunksMax] = {};
     // tensor-core path: pre-tiled weights, tensor maps of xq / hq, error flag
     bool use_tc = false;
     uint8_t* w_gate_up_t = nullptr;
@@ -146,6 +158,14 @@ void free_all(mmoe_handle* h) {
     for (void* p : ptrs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);
+    for (cudaStream_t st : {h->s_h2d, h->s_d2h})
+        if (st) cudaStreamDestroy(st);
+    for (cudaEvent_t ev : {h->ev_start, h->ev_done})
+        if (ev) cudaEventDestroy(ev);
+    for (int i = 0; i < kHostChunksMax; ++i) {
+        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+        if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    }
 }
 
 mmoe_status check_config(const mmoe_config* c) {
@@ -552,13 +572,52 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T,
         MMOE_CUDA(dalloc(&h->x_stage, (size_t)h->max_tokens * d), "staging allocation");
         MMOE_CUDA(dalloc(&h->y_stage, (size_t)h->max_tokens * d), "staging allocation");
     }
-    MMOE_CUDA(cudaMemcpyAsync(h->x_stage, x_host, (size_t)T * d * sizeof(uint16_t), cudaMemcpyHostToDevice, s),
-              "copy x to the device");
-    mmoe_status st = mmoe_forward(h, h->x_stage, T, h->y_stage, stream, nullptr, nullptr, nullptr);
+    if (!h->s_h2d) {
+        MMOE_CUDA(cudaStreamCreateWithFlags(&h->s_h2d, cudaStreamNonBlocking), "copy stream");
+        MMOE_CUDA(cudaStreamCreateWithFlags(&h->s_d2h, cudaStreamNonBlocking), "copy stream");
+        for (cudaEvent_t* ev : {&h->ev_start, &h->ev_done})
+            MMOE_CUDA(cudaEventCreateWithFlags(ev, cudaEventDisableTiming), "copy event");
+        for (int i = 0; i < kHostChunksMax; ++i) {
+            MMOE_CUDA(cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming), "copy event");
+            MMOE_CUDA(cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming), "copy event");
+        }
+    }
+    const int nch = (int)std::max<int64_t>(1, std::min<int64_t>(kHostChunksMax, T / kHostChunkMinTokens));
+    int64_t bound[kHostChunksMax + 1];
+    for (int i = 0; i <= nch; ++i) bound[i] = i == nch ? T : (T * i / nch) / 128 * 128;
+    // copies start after the caller's earlier work on `stream`
+    MMOE_CUDA(cudaEventRecord(h->ev_start, s), "event record");
+    MMOE_CUDA(cudaStreamWaitEvent(h->s_h2d, h->ev_start, 0), "stream wait");
+    MMOE_CUDA(cudaStreamWaitEvent(h->s_d2h, h->ev_start, 0), "stream wait");
+    for (int i = 0; i < nch; ++i) {
+        const int64_t t0 = bound[i], Ti = bound[i + 1] - bound[i];
+        MMOE_CUDA(cudaMemcpyAsync(h->x_stage + t0 * d, x_host + t0 * d, (size_t)Ti * d * sizeof(uint16_t),
+                                  cudaMemcpyHostToDevice, h->s_h2d),
+                  "copy x to the device");
+        MMOE_CUDA(cudaEventRecord(h->ev_in[i], h->s_h2d), "event record");
+    }
+    mmoe_status st = MMOE_OK;
+    for (int i = 0; i < nch && st == MMOE_OK; ++i) {
+        const int64_t t0 = bound[i], Ti = bound[i + 1] - bound[i];
+        MMOE_CUDA(cudaStreamWaitEvent(s, h->ev_in[i], 0), "stream wait");
+        st = mmoe_forward(h, h->x_stage + t0 * d, Ti, h->y_stage + t0 * d, stream, nullptr, nullptr, nullptr);
+        if (st != MMOE_OK) break;
+        MMOE_CUDA(cudaEventRecord(h->ev_out[i], s), "event record");
+        MMOE_CUDA(cudaStreamWaitEvent(h->s_d2h, h->ev_out[i], 0), "stream wait");
+        MMOE_CUDA(cudaMemcpyAsync(y_host + t0 * d, h->y_stage + t0 * d, (size_t)Ti * d * sizeof(float),
+                                  cudaMemcpyDeviceToHost, h->s_d2h),
+                  "copy y to the host");
+    }
+    // `stream` is left ordered after both copy streams, whatever happened above
+    cudaError_t e1 = cudaEventRecord(h->ev_done, h->s_h2d);
+    if (e1 == cudaSuccess) e1 = cudaStreamWaitEvent(s, h->ev_done, 0);
+    cudaError_t e2 = cudaEventRecord(h->ev_done, h->s_d2h);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(s, h->ev_done, 0);
+    cudaError_t e3 = cudaStreamSynchronize(s);
     if (st != MMOE_OK) return st;
-    MMOE_CUDA(cudaMemcpyAsync(y_host, h->y_stage, (size_t)T * d * sizeof(float), cudaMemcpyDeviceToHost, s),
-              "copy y to the host");
-    MMOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    MMOE_CUDA(e1, "stream order");
+    MMOE_CUDA(e2, "stream order");
+    MMOE_CUDA(e3, "stream synchronize");
     return MMOE_OK;
 }
 

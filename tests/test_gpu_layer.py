@@ -201,6 +201,28 @@ def test_forward_host_matches_device():
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_forward_host_chunked_equals_one_forward(pinned):
+    # 3 * 8192 + 77 tokens: the host entry point splits the batch into three
+    # chunks whose copies overlap the layer; y must equal one unsplit forward.
+    w, q = workload("c0")
+    T = 3 * 8192 + 77
+    x = synth.workload_x(w, T=T)
+    L = gu.make_gpu_layer(q, T, deterministic=True)
+    a = gu.run_gpu(L, q, x, stages=False)["y"]
+    if pinned:
+        hx = torch.empty((T, w.d), dtype=torch.int16, pin_memory=True)
+        hx.numpy()[:] = x.view(np.int16)
+        hy = torch.full((T, w.d), float("nan"), dtype=torch.float32, pin_memory=True)
+        b = L.forward_host(hx.numpy().view(np.uint16), hy.numpy())
+    else:
+        b = L.forward_host(x)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    # the stream passed in is ordered after the copies: a device forward right after sees its own x
+    c = gu.run_gpu(L, q, x[:100], stages=False)["y"]
+    assert np.array_equal(c.view(np.uint32), a[:100].view(np.uint32))
+
+
 def test_errors_on_device():
     w, q = workload("c0")
     from moe_ffn_layer_fp32_b200.layer import MoELayer
