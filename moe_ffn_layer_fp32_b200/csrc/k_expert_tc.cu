@@ -28,11 +28,12 @@
 //               accumulate acc = fma(float(P_j), s_j, acc) in registers
 //               (4 warpgroups x 32 token columns, one weight row per thread),
 //               then the tile's epilogue, which overlaps the MMAs of the next
-//               tile.  After reading a buffer they refill it with the bit
-//               pattern of 1.5 * 2^19; the next MMA accumulates 16 P onto it
-//               (the weights enter as 16 x their code), so the INT32 result
-//               arrives as the float 1.5 * 2^19 + P (exact for |16 P| < 2^22)
-//               and one exact subtraction converts it.
+//               tile.  Each group is one MMA that overwrites its buffer, so a
+//               pair of buffers goes back to the MMA as soon as it has been
+//               read.  The weights enter as 16 x their code, so a partial
+//               arrives as 16 P; added as an integer to the bit pattern of
+//               1.5 * 2^19 it is the float 1.5 * 2^19 + P (exact for
+//               |16 P| < 2^22), and one exact subtraction converts it.
 // The exact INT32 group partial is needed because every 32-element group of K
 // has its own FP32 weight scale; the promotion order (j ascending, fused
 // multiply-add) is the oracle's, so the FP32 result is identical to it.
@@ -84,7 +85,7 @@ struct Smem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t accf[kPairs];   // a pair of buffers holds two finished groups
-    uint64_t acce[kPairs];   // a pair of buffers has been read and preset again
+    uint64_t acce[kPairs];   // a pair of buffers has been read (free for the next MMAs)
     uint64_t tfull[kTInfo];  // tile info written
     uint64_t tempty[kTInfo]; // tile info no longer needed
     uint32_t tmem_base;
@@ -152,13 +153,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
 // kind::i8: signed A and B, S32 accumulator, both K-major, M = 128, N = BN.
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-// D += A * B (the accumulator holds the preset 1.5 * 2^19 bit pattern)
+// D = A * B: a 32-element K group is exactly one instruction, so the buffer
+// receives that group's partial alone and needs no clearing in between.
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(1)
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(0)
         : "memory");
 }
 
@@ -178,27 +180,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, int32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-        "%1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // The weights enter the MMA as 16 x their INT4 code (the code in the high nibble
-// of a byte), so a group's result is 16 P.  TMEM is preset with the bit pattern
-// of 1.5 * 2^19, whose float ulp is 1/16: the float with bits (preset + 16 P) is
-// exactly 1.5 * 2^19 + P for |16 P| < 2^22 (|P| <= 32 * 8 * 127).
+// of a byte), so a group's result is v = 16 P.  Added as an integer to the bit
+// pattern of 1.5 * 2^19, whose float ulp is 1/16, it gives the bits of the float
+// 1.5 * 2^19 + P exactly (|16 P| < 2^22 since |P| <= 32 * 8 * 127), and one exact
+// subtraction leaves P.
 constexpr uint32_t kMagicBits = 0x49400000u;  // 1.5 * 2^19
 constexpr float kMagic = 786432.0f;
 
-// Two columns at once with paired FP32 instructions (each half is an ordinary IEEE
-// operation, so the results equal the scalar ones):
-// (a0, a1) = fma((float(v0) - 1.5 * 2^19, float(v1) - 1.5 * 2^19), s, (a0, a1))
+// Two columns at once, the FP32 steps as paired instructions (each half is an
+// ordinary IEEE operation, so the results equal the scalar ones):
+// (a0, a1) = fma((P0, P1), s, (a0, a1)) with P = float(bits(1.5 * 2^19) + v) - 1.5 * 2^19
 __device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32_t v1, float s) {
+    const uint32_t b0 = (uint32_t)v0 + kMagicBits, b1 = (uint32_t)v1 + kMagicBits;
     asm("{\n\t.reg .b64 t, acc, sc, mg;\n\t"
         "mov.b64 t, {%2, %3};\n\t"
         "mov.b64 acc, {%0, %1};\n\t"
@@ -208,7 +203,7 @@ __device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32
         "fma.rn.f32x2 acc, t, sc, acc;\n\t"
         "mov.b64 {%0, %1}, acc;\n\t}"
         : "+f"(a0), "+f"(a1)
-        : "r"(v0), "r"(v1), "f"(s), "f"(kMagic));
+        : "r"(b0), "r"(b1), "f"(s), "f"(kMagic));
 }
 
 struct TcArgs {
@@ -419,15 +414,7 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
         const int row = quarter * 32 + lane;  // weight row of this thread (0..127)
         const int col0 = wg * kCols;
         const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)col0;
-        // preset every buffer; this is completion 0 of both acce barriers
-#pragma unroll
-        for (int b = 0; b < kBufs; ++b) {
-            tmem_st16_const(tl + b * 128, kMagicBits);
-            tmem_st16_const(tl + b * 128 + 16, kMagicBits);
-        }
-        tmem_wait_st();
-        tc_before_sync();
-        __syncwarp();
+        // every buffer starts free: completion 0 of both acce barriers
         if (lane == 0)
             for (int b = 0; b < kPairs; ++b) mbar_arrive(&sm->acce[b]);
         int pc = 0, tcount = 0;
@@ -453,19 +440,23 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                 }
                 if (!warp_wait(&sm->accf[b], (pc >> 1) & 1, sm, ef, 5)) { ok = false; break; }
                 tc_after_sync();
+                // both halves of a group leave TMEM behind one wait; the pair goes back to the MMA
+                // as soon as its second group has been read, before that group's arithmetic
 #pragma unroll 1
                 for (int gg = 0; gg < 2; ++gg) {
                     const float sc = gg ? sb : sa;
                     const uint32_t ta = tl + (2 * b + gg) * 128;
                     int32_t v[16], w[16];
                     tmem_ld16(ta, v);
-                    tmem_wait_ld();
-                    tmem_st16_const(ta, kMagicBits);
-#pragma unroll
-                    for (int c = 0; c < 16; c += 2) promote2(acc[c], acc[c + 1], v[c], v[c + 1], sc);
                     tmem_ld16(ta + 16, w);
                     tmem_wait_ld();
-                    tmem_st16_const(ta + 16, kMagicBits);
+                    if (gg == 1) {
+                        tc_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm->acce[b]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; c += 2) promote2(acc[c], acc[c + 1], v[c], v[c + 1], sc);
 #pragma unroll
                     for (int c = 0; c < 16; c += 2) promote2(acc[16 + c], acc[17 + c], w[c], w[c + 1], sc);
                     if (kDump) {
@@ -476,7 +467,7 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                             const int cc = col0 + c;
                             const int64_t grow = (int64_t)row0 + cc;
                             if (cc >= nr || grow < a.drow0 || grow >= a.drow0 + a.dnrows) continue;
-                            const int32_t pv = ((int32_t)(c < 16 ? v[c & 15] : w[c & 15]) - (int32_t)kMagicBits) >> 4;
+                            const int32_t pv = (c < 16 ? v[c & 15] : w[c & 15]) >> 4;
                             if (kEpi == kEpiSwiGLU) {
                                 const int f = mb * 64 + (row & 63);
                                 const int n = row < 64 ? f : p.hmax + f;
@@ -488,10 +479,6 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                         }
                     }
                 }
-                tmem_wait_st();
-                tc_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->acce[b]);
             }
             if (!ok || *reinterpret_cast<volatile int*>(&sm->abort)) break;
             // epilogue: park the tile in shared memory ([column][row]), then each warpgroup finishes its columns
