@@ -149,7 +149,8 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, floa
 
 /* The same layer with HOST buffers: x (host, BF16 bits [T, d_model]) in,
  * y (host, FP32 [T, d_model]) out; returns when y is written.  A batch of
- * T >= 16384 tokens runs as 2 to 4 chunks of at least 8192 tokens: chunk i's
+ * T >= 16384 tokens runs as n = min(4, T / 8192) chunks (for n >= 3 the first
+ * and last are a third the size of the others): chunk i's
  * x is copied on an internal stream, mmoe_forward runs on `stream` after that
  * copy, and its y is copied back on a second internal stream, so copies and
  * the layer overlap.  Each token's output depends on that token alone, so y

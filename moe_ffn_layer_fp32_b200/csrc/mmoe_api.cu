@@ -56,10 +56,11 @@ struct DeviceGuard {
     }
 };
 
-// mmoe_forward_host splits a batch into up to kHostChunksMax chunks of at
-// least kHostChunkMinTokens tokens (boundaries on multiples of 128 tokens), so
-// that the copies of one chunk overlap the layer on another.  Every token's
-// output depends on that token alone, so the split leaves y unchanged.
+// mmoe_forward_host splits a batch of T tokens into n = min(kHostChunksMax,
+// T / kHostChunkMinTokens) chunks (boundaries on multiples of 128 tokens; for
+// n >= 3 the first and last chunks are a third of the others), so that the
+// copies of one chunk overlap the layer on another.  Every token's output
+// depends on that token alone, so the split leaves y unchanged.
 constexpr int kHostChunksMax = 4;
 constexpr int64_t kHostChunkMinTokens = 8192;
 
@@ -583,8 +584,16 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T,
         }
     }
     const int nch = (int)std::max<int64_t>(1, std::min<int64_t>(kHostChunksMax, T / kHostChunkMinTokens));
+    // chunk weights 1, 3, ..., 3, 1: short first and last chunks shorten the copy-in before the first
+    // forward and the copy-out after the last one
     int64_t bound[kHostChunksMax + 1];
-    for (int i = 0; i <= nch; ++i) bound[i] = i == nch ? T : (T * i / nch) / 128 * 128;
+    const int64_t wsum = nch < 3 ? nch : 3 * nch - 4;
+    int64_t wacc = 0;
+    bound[0] = 0;
+    for (int i = 0; i < nch; ++i) {
+        wacc += (nch < 3 || i == 0 || i == nch - 1) ? 1 : 3;
+        bound[i + 1] = i == nch - 1 ? T : (T * wacc / wsum) / 128 * 128;
+    }
     // copies start after the caller's earlier work on `stream`
     MMOE_CUDA(cudaEventRecord(h->ev_start, s), "event record");
     MMOE_CUDA(cudaStreamWaitEvent(h->s_h2d, h->ev_start, 0), "stream wait");
