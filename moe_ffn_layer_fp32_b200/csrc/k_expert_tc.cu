@@ -206,6 +206,15 @@ __device__ __forceinline__ void promote2(float& a0, float& a1, int32_t v0, int32
         : "r"(b0), "r"(b1), "f"(s), "f"(kMagic));
 }
 
+// SwiGLU of one feature from its gate and up sums and the token's activation scale:
+// silu(g sx) * (u sx), silu(v) = v / (1 + exp(-v)), each step an IEEE FP32 operation
+__device__ __forceinline__ float swiglu(float g, float u, float sx) {
+    const float gv = __fmul_rn(g, sx);
+    const float uv = __fmul_rn(u, sx);
+    const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+    return __fmul_rn(silu, uv);
+}
+
 struct TcArgs {
     const uint8_t* wtiles;  // weight stage images (INT8, SW128) of the expert kind (gate/up or down)
     const float* stiles;    // pre-tiled group scales
@@ -488,31 +497,48 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
             for (int c = 0; c < kCols; ++c) xch[(col0 + c) * BM + row] = acc[c];
             asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");
             if (!kDump) {
+                // warp `quarter` of the warpgroup finishes token columns cq .. cq + 7 of the warpgroup's 32,
+                // reading whole columns of the exchange buffer and storing 16 bytes per lane
+                const int cq = col0 + quarter * (kCols / 4);
                 if (kEpi == kEpiSwiGLU) {
                     // rows 0..63 hold the gate of feature mb*64 + row, rows 64..127 the up of the same feature;
-                    // thread (row) finishes feature row & 63 for half of the warpgroup's columns
-                    const int fl = row & 63;
-                    const int f = mb * 64 + fl;
-                    const int cbeg = col0 + (row >> 6) * (kCols / 2);
+                    // lanes 0-15 take one column, lanes 16-31 the next, each lane features 4 (lane & 15) .. + 3
+                    const int fl4 = 4 * (lane & 15);
+                    float* out = p.act + (int64_t)row0 * p.hmax + mb * 64 + fl4;
 #pragma unroll 1
-                    for (int cc = cbeg; cc < cbeg + kCols / 2; ++cc) {
+                    for (int c = lane >> 4; c < kCols / 4; c += 2) {
+                        const int cc = cq + c;
                         if (cc >= nr) break;
                         const float sx = ti.colf[cc];
-                        const float gv = __fmul_rn(xch[cc * BM + fl], sx);
-                        const float uv = __fmul_rn(xch[cc * BM + 64 + fl], sx);
-                        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
-                        p.act[((int64_t)row0 + cc) * p.hmax + f] = __fmul_rn(silu, uv);
+                        const float4 g4 = *reinterpret_cast<const float4*>(&xch[cc * BM + fl4]);
+                        const float4 u4 = *reinterpret_cast<const float4*>(&xch[cc * BM + 64 + fl4]);
+                        float4 r;
+                        r.x = swiglu(g4.x, u4.x, sx);
+                        r.y = swiglu(g4.y, u4.y, sx);
+                        r.z = swiglu(g4.z, u4.z, sx);
+                        r.w = swiglu(g4.w, u4.w, sx);
+                        *reinterpret_cast<float4*>(out + (int64_t)cc * p.hmax) = r;
                     }
                 } else {
-                    const int m = mb * BM + row;
-#pragma unroll 1
-                    for (int cc = col0; cc < col0 + kCols; ++cc) {
+                    // lane l covers outputs mb*128 + 4 l .. + 3 of each column
+                    const int m4 = mb * BM + 4 * lane;
+#pragma unroll 2
+                    for (int c = 0; c < kCols / 4; ++c) {
+                        const int cc = cq + c;
                         if (cc >= nr) break;
-                        const float o = __fmul_rn(xch[cc * BM + row], ti.colf[cc]);
+                        const float f = ti.colf[cc];
+                        const float4 v = *reinterpret_cast<const float4*>(&xch[cc * BM + 4 * lane]);
+                        const float4 o = make_float4(__fmul_rn(v.x, f), __fmul_rn(v.y, f), __fmul_rn(v.z, f),
+                                                     __fmul_rn(v.w, f));
                         if (p.deterministic) {
-                            p.obuf[((int64_t)row0 + cc) * p.d + m] = o;
+                            *reinterpret_cast<float4*>(p.obuf + ((int64_t)row0 + cc) * p.d + m4) = o;
                         } else {
-                            atomicAdd(p.y + (int64_t)ti.colrow[cc] * p.d + m, __fmul_rn(ti.colg[cc], o));
+                            const float g = ti.colg[cc];
+                            float* yr = p.y + (int64_t)ti.colrow[cc] * p.d + m4;
+                            atomicAdd(yr, __fmul_rn(g, o.x));
+                            atomicAdd(yr + 1, __fmul_rn(g, o.y));
+                            atomicAdd(yr + 2, __fmul_rn(g, o.z));
+                            atomicAdd(yr + 3, __fmul_rn(g, o.w));
                         }
                     }
                 }
