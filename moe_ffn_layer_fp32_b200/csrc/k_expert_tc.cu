@@ -27,8 +27,9 @@
 //   warps 2-17  promotion: read each group's INT32 partials from TMEM and
 //               accumulate acc = fma(float(P_j), s_j, acc) in registers
 //               (4 warpgroups x 32 token columns, one weight row per thread),
-//               then the tile's epilogue, which overlaps the MMAs of the next
-//               tile.  Each group is one MMA that overwrites its buffer, so a
+//               then park the finished tile in shared memory; its epilogue
+//               runs one step after each buffer pair of the next tile, while
+//               the warps would otherwise wait for the MMA.  Each group is one MMA that overwrites its buffer, so a
 //               pair of buffers goes back to the MMA as soon as it has been
 //               read.  The weights enter as 16 x their code, so a partial
 //               arrives as 16 P; added as an integer to the bit pattern of
@@ -271,6 +272,56 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem* 
     return __shfl_sync(0xffffffffu, ok, 0);
 }
 
+// One step of a parked tile's epilogue for one promotion warp: the warp of
+// lane quarter `quarter` in the warpgroup whose token columns start at col0
+// finishes columns cq .. cq + 7 (cq = col0 + 8 quarter) in kEpiSteps steps,
+// reading whole columns of the exchange buffer ([column][row]) and storing
+// 16 bytes per lane.
+template <int kEpi>
+constexpr int kEpiSteps = kEpi == kEpiSwiGLU ? kCols / 8 : kCols / 4;
+
+template <int kEpi>
+__device__ __forceinline__ void epilogue_step(const Plan& p, const TileInfo& ti, const float* xch, int col0,
+                                              int quarter, int lane, int step) {
+    const int cq = col0 + quarter * (kCols / 4);
+    const int nr = ti.nr, mb = ti.mb;
+    const int64_t row0 = ti.row0;
+    if (kEpi == kEpiSwiGLU) {
+        // rows 0..63 hold the gate of feature mb*64 + row, rows 64..127 the up of the same feature;
+        // lanes 0-15 take column cq + 2 step, lanes 16-31 the next, each lane features 4 (lane & 15) .. + 3
+        const int fl4 = 4 * (lane & 15);
+        const int cc = cq + 2 * step + (lane >> 4);
+        if (cc >= nr) return;
+        const float sx = ti.colf[cc];
+        const float4 g4 = *reinterpret_cast<const float4*>(&xch[cc * BM + fl4]);
+        const float4 u4 = *reinterpret_cast<const float4*>(&xch[cc * BM + 64 + fl4]);
+        float4 r;
+        r.x = swiglu(g4.x, u4.x, sx);
+        r.y = swiglu(g4.y, u4.y, sx);
+        r.z = swiglu(g4.z, u4.z, sx);
+        r.w = swiglu(g4.w, u4.w, sx);
+        *reinterpret_cast<float4*>(p.act + (row0 + cc) * p.hmax + mb * 64 + fl4) = r;
+    } else {
+        // column cq + step; lane l covers outputs mb*128 + 4 l .. + 3
+        const int cc = cq + step;
+        if (cc >= nr) return;
+        const int m4 = mb * BM + 4 * lane;
+        const float f = ti.colf[cc];
+        const float4 v = *reinterpret_cast<const float4*>(&xch[cc * BM + 4 * lane]);
+        const float4 o = make_float4(__fmul_rn(v.x, f), __fmul_rn(v.y, f), __fmul_rn(v.z, f), __fmul_rn(v.w, f));
+        if (p.deterministic) {
+            *reinterpret_cast<float4*>(p.obuf + (row0 + cc) * p.d + m4) = o;
+        } else {
+            const float g = ti.colg[cc];
+            float* yr = p.y + (int64_t)ti.colrow[cc] * p.d + m4;
+            atomicAdd(yr, __fmul_rn(g, o.x));
+            atomicAdd(yr + 1, __fmul_rn(g, o.y));
+            atomicAdd(yr + 2, __fmul_rn(g, o.z));
+            atomicAdd(yr + 3, __fmul_rn(g, o.w));
+        }
+    }
+}
+
 template <int kEpi, bool kDump>
 // 18 warps: the SM sub-partitions holding 5 of them bound a thread to 96 registers
 __global__ void __launch_bounds__(kThreads, 1)
@@ -427,6 +478,7 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
         if (lane == 0)
             for (int b = 0; b < kPairs; ++b) mbar_arrive(&sm->acce[b]);
         int pc = 0, tcount = 0;
+        int ptb = -1, pstep = 0;  // tile-info slot of the parked tile whose epilogue is pending, next step
         bool ok = true;
         while (ok) {
             const int tb = tcount % kTInfo;
@@ -488,65 +540,42 @@ expert_gemm_tc_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, TcArgs a
                         }
                     }
                 }
+                // one step of the previous tile's epilogue while the MMAs of the next pair run
+                if (!kDump && ptb >= 0) {
+                    epilogue_step<kEpi>(p, sm->ti[ptb], xch, col0, quarter, lane, pstep);
+                    if (++pstep == kEpiSteps<kEpi>) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm->tempty[ptb]);
+                        ptb = -1;
+                    }
+                }
             }
             if (!ok || *reinterpret_cast<volatile int*>(&sm->abort)) break;
-            // epilogue: park the tile in shared memory ([column][row]), then each warpgroup finishes its columns
+            // the rest of the previous tile's epilogue (a K loop shorter than its steps)
+            if (ptb >= 0) {
+                for (; pstep < kEpiSteps<kEpi>; ++pstep) epilogue_step<kEpi>(p, sm->ti[ptb], xch, col0, quarter, lane, pstep);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->tempty[ptb]);
+                ptb = -1;
+            }
+            // park the tile in shared memory ([column][row]); its epilogue runs during the next tile's pairs
             const int named = 1 + wg;
             asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");  // previous tile's readers are done
 #pragma unroll
             for (int c = 0; c < kCols; ++c) xch[(col0 + c) * BM + row] = acc[c];
             asm volatile("bar.sync %0, %1;" ::"r"(named), "r"(128) : "memory");
-            if (!kDump) {
-                // warp `quarter` of the warpgroup finishes token columns cq .. cq + 7 of the warpgroup's 32,
-                // reading whole columns of the exchange buffer and storing 16 bytes per lane
-                const int cq = col0 + quarter * (kCols / 4);
-                if (kEpi == kEpiSwiGLU) {
-                    // rows 0..63 hold the gate of feature mb*64 + row, rows 64..127 the up of the same feature;
-                    // lanes 0-15 take one column, lanes 16-31 the next, each lane features 4 (lane & 15) .. + 3
-                    const int fl4 = 4 * (lane & 15);
-                    float* out = p.act + (int64_t)row0 * p.hmax + mb * 64 + fl4;
-#pragma unroll 1
-                    for (int c = lane >> 4; c < kCols / 4; c += 2) {
-                        const int cc = cq + c;
-                        if (cc >= nr) break;
-                        const float sx = ti.colf[cc];
-                        const float4 g4 = *reinterpret_cast<const float4*>(&xch[cc * BM + fl4]);
-                        const float4 u4 = *reinterpret_cast<const float4*>(&xch[cc * BM + 64 + fl4]);
-                        float4 r;
-                        r.x = swiglu(g4.x, u4.x, sx);
-                        r.y = swiglu(g4.y, u4.y, sx);
-                        r.z = swiglu(g4.z, u4.z, sx);
-                        r.w = swiglu(g4.w, u4.w, sx);
-                        *reinterpret_cast<float4*>(out + (int64_t)cc * p.hmax) = r;
-                    }
-                } else {
-                    // lane l covers outputs mb*128 + 4 l .. + 3 of each column
-                    const int m4 = mb * BM + 4 * lane;
-#pragma unroll 2
-                    for (int c = 0; c < kCols / 4; ++c) {
-                        const int cc = cq + c;
-                        if (cc >= nr) break;
-                        const float f = ti.colf[cc];
-                        const float4 v = *reinterpret_cast<const float4*>(&xch[cc * BM + 4 * lane]);
-                        const float4 o = make_float4(__fmul_rn(v.x, f), __fmul_rn(v.y, f), __fmul_rn(v.z, f),
-                                                     __fmul_rn(v.w, f));
-                        if (p.deterministic) {
-                            *reinterpret_cast<float4*>(p.obuf + ((int64_t)row0 + cc) * p.d + m4) = o;
-                        } else {
-                            const float g = ti.colg[cc];
-                            float* yr = p.y + (int64_t)ti.colrow[cc] * p.d + m4;
-                            atomicAdd(yr, __fmul_rn(g, o.x));
-                            atomicAdd(yr + 1, __fmul_rn(g, o.y));
-                            atomicAdd(yr + 2, __fmul_rn(g, o.z));
-                            atomicAdd(yr + 3, __fmul_rn(g, o.w));
-                        }
-                    }
-                }
+            if (kDump) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->tempty[tb]);
+            } else {
+                ptb = tb;
+                pstep = 0;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->tempty[tb]);
             ++tcount;
         }
+        // the last parked tile's epilogue
+        if (ok && ptb >= 0 && !*reinterpret_cast<volatile int*>(&sm->abort))
+            for (; pstep < kEpiSteps<kEpi>; ++pstep) epilogue_step<kEpi>(p, sm->ti[ptb], xch, col0, quarter, lane, pstep);
     }
 
     __syncthreads();
