@@ -29,9 +29,10 @@
 //               (4 warpgroups x 32 token columns, one weight row per thread),
 //               then park the finished tile in shared memory; its epilogue
 //               runs one step after each buffer pair of the next tile, while
-//               the warps would otherwise wait for the MMA.  Each group is one MMA that overwrites its buffer, so a
-//               pair of buffers goes back to the MMA as soon as it has been
-//               read.  The weights enter as 16 x their code, so a partial
+//               the warps would otherwise wait for the MMA.  Each group is
+//               one MMA that overwrites its buffer, so a pair of buffers goes
+//               back to the MMA as soon as it has been read.  The weights
+//               enter as 16 x their code, so a partial
 //               arrives as 16 P; added as an integer to the bit pattern of
 //               1.5 * 2^19 it is the float 1.5 * 2^19 + P (exact for
 //               |16 P| < 2^22), and one exact subtraction converts it.
