@@ -212,6 +212,13 @@ mmoe_status mmoe_debug_copy_stage(mmoe_handle* h, int32_t stage, void* dst, size
 mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int64_t nrows, int32_t* dst,
                                 void* stream);
 
+/* The chunks mmoe_forward_host splits a T-token batch into (host only, no
+ * device call): writes n + 1 boundaries 0 = bounds[0] < ... < bounds[n] = T
+ * (for T > 0; T = 0 gives n = 1, bounds {0, 0}) to the host array `bounds`
+ * of `cap` entries and n to `*n`.  Errors: INVALID_ARG (T < 0, NULL pointer,
+ * cap < n + 1). */
+mmoe_status mmoe_debug_host_chunks(int64_t T, int64_t* bounds, int32_t cap, int32_t* n);
+
 /* ---- per-stage timing ------------------------------------------------------
  * While profiling is enabled, every forward records a CUDA event pair on its
  * own stream around each stage's kernels.  mmoe_profile_read waits for those

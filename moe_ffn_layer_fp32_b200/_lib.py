@@ -27,7 +27,7 @@ STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAG
 # every symbol include/mmoe.h declares
 EXPORTS = ("mmoe_create", "mmoe_load_quantized_weights", "mmoe_forward", "mmoe_forward_host", "mmoe_destroy",
            "mmoe_last_error", "mmoe_quantize_int4", "mmoe_debug_copy_stage", "mmoe_debug_partials",
-           "mmoe_profile_enable", "mmoe_profile_read", "mmoe_forward_static_scratch")
+           "mmoe_profile_enable", "mmoe_profile_read", "mmoe_forward_static_scratch", "mmoe_debug_host_chunks")
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
@@ -78,6 +78,7 @@ def lib() -> C.CDLL:
     L.mmoe_profile_enable.argtypes = [vp, i32]
     L.mmoe_profile_read.argtypes = [vp, vp, vp, i32]
     L.mmoe_forward_static_scratch.argtypes = [C.POINTER(Config), C.POINTER(Weights), vp, i64, vp, vp]
+    L.mmoe_debug_host_chunks.argtypes = [i64, vp, i32, vp]
     for name in EXPORTS:
         if name != "mmoe_last_error":
             getattr(L, name).restype = st

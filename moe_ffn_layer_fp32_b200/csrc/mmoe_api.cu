@@ -64,6 +64,20 @@ struct DeviceGuard {
 constexpr int kHostChunksMax = 4;
 constexpr int64_t kHostChunkMinTokens = 8192;
 
+// Chunk boundaries of a T-token host-buffer forward: bound[0] = 0 < ... <
+// bound[n] = T (T > 0), chunk weights 1, 3, ..., 3, 1 for n >= 3.  Returns n.
+int host_chunk_bounds(int64_t T, int64_t (&bound)[kHostChunksMax + 1]) {
+    const int nch = (int)std::max<int64_t>(1, std::min<int64_t>(kHostChunksMax, T / kHostChunkMinTokens));
+    const int64_t wsum = nch < 3 ? nch : 3 * nch - 4;
+    int64_t wacc = 0;
+    bound[0] = 0;
+    for (int i = 0; i < nch; ++i) {
+        wacc += (nch < 3 || i == 0 || i == nch - 1) ? 1 : 3;
+        bound[i + 1] = i == nch - 1 ? T : (T * wacc / wsum) / 128 * 128;
+    }
+    return nch;
+}
+
 }  // namespace
 
 struct mmoe_handle {
@@ -583,17 +597,10 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T,
             MMOE_CUDA(cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming), "copy event");
         }
     }
-    const int nch = (int)std::max<int64_t>(1, std::min<int64_t>(kHostChunksMax, T / kHostChunkMinTokens));
-    // chunk weights 1, 3, ..., 3, 1: short first and last chunks shorten the copy-in before the first
-    // forward and the copy-out after the last one
+    // short first and last chunks shorten the copy-in before the first forward and the copy-out
+    // after the last one
     int64_t bound[kHostChunksMax + 1];
-    const int64_t wsum = nch < 3 ? nch : 3 * nch - 4;
-    int64_t wacc = 0;
-    bound[0] = 0;
-    for (int i = 0; i < nch; ++i) {
-        wacc += (nch < 3 || i == 0 || i == nch - 1) ? 1 : 3;
-        bound[i + 1] = i == nch - 1 ? T : (T * wacc / wsum) / 128 * 128;
-    }
+    const int nch = host_chunk_bounds(T, bound);
     // copies start after the caller's earlier work on `stream`
     MMOE_CUDA(cudaEventRecord(h->ev_start, s), "event record");
     MMOE_CUDA(cudaStreamWaitEvent(h->s_h2d, h->ev_start, 0), "stream wait");
@@ -627,6 +634,17 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T,
     MMOE_CUDA(e1, "stream order");
     MMOE_CUDA(e2, "stream order");
     MMOE_CUDA(e3, "stream synchronize");
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_debug_host_chunks(int64_t T, int64_t* bounds, int32_t cap, int32_t* n) {
+    if (T < 0) return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be >= 0", (long long)T);
+    if (!bounds || !n) return fail(MMOE_ERR_INVALID_ARG, "bounds or n is NULL");
+    int64_t b[kHostChunksMax + 1];
+    const int nch = host_chunk_bounds(T, b);
+    if (cap < nch + 1) return fail(MMOE_ERR_INVALID_ARG, "cap=%d: %d boundaries needed", (int)cap, nch + 1);
+    for (int i = 0; i <= nch; ++i) bounds[i] = b[i];
+    *n = nch;
     return MMOE_OK;
 }
 

@@ -92,3 +92,42 @@ def test_static_scratch_forward_validates_before_any_device_work(L):
     assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, -1, fake, None) == 1
     assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, 0, fake, None) == 0
     assert L.mmoe_forward_static_scratch(None, C.byref(w), fake, 1, fake, None) == 1
+
+
+def host_chunks(L, T, cap=8):
+    b = (C.c_int64 * cap)()
+    n = C.c_int32()
+    assert L.mmoe_debug_host_chunks(T, b, cap, C.byref(n)) == 0
+    return list(b[:n.value + 1])
+
+
+@pytest.mark.parametrize("T", [0, 1, 64, 65, 8191, 8192, 16383, 16384, 16385, 24576, 24653, 32767, 32768, 32832,
+                               40000, 65536, 100003, 1 << 20])
+def test_host_forward_chunks(L, T):
+    # the split of a host-buffer forward: ordered, complete, on 128-token boundaries, with
+    # n = min(4, T // 8192) chunks and end chunks a third of the middle ones when n >= 3
+    b = host_chunks(L, T)
+    n = len(b) - 1
+    assert n == max(1, min(4, T // 8192))
+    assert b[0] == 0 and b[-1] == T
+    assert all(x % 128 == 0 for x in b[1:-1])
+    sizes = [b[i + 1] - b[i] for i in range(n)]
+    if T > 0:
+        assert all(s > 0 for s in sizes)
+    if n >= 2:
+        assert min(sizes) > 64  # every chunk stays on the prefill kernels, like the unsplit batch
+    if n >= 3:
+        unit = T / (3 * n - 4)
+        for i, s in enumerate(sizes):
+            w = 1 if i in (0, n - 1) else 3
+            assert abs(s - w * unit) <= 256, (i, s, w * unit)
+
+
+def test_host_chunks_rejects_bad_arguments(L):
+    b = (C.c_int64 * 8)()
+    n = C.c_int32()
+    assert L.mmoe_debug_host_chunks(-1, b, 8, C.byref(n)) == 1
+    assert L.mmoe_debug_host_chunks(40000, None, 8, C.byref(n)) == 1
+    assert L.mmoe_debug_host_chunks(40000, b, 8, None) == 1
+    assert L.mmoe_debug_host_chunks(40000, b, 4, C.byref(n)) == 1  # 4 chunks need 5 boundaries
+    assert b"cap" in L.mmoe_last_error()
