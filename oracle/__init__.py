@@ -25,15 +25,20 @@ _SO = os.path.join(_BUILD, "liboracle.so")
 GROUP = 32
 
 
+def compile_oracle(src: str, out: str) -> None:
+    """gcc -O2 with OpenMP over tokens and no fused multiply-adds: the oracle's build flags."""
+    cmd = ["gcc", "-O2", "-march=native", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+           "-std=c11", "-Wall", "-shared", "-fPIC", "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+
+
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (OpenMP over tokens, no fused multiply-adds)."""
+    """Compile the oracle (see compile_oracle) into oracle/_build if it is out of date."""
     if not force and os.path.exists(_SO) and os.path.getmtime(_SO) >= os.path.getmtime(_SRC):
         return _SO
     os.makedirs(_BUILD, exist_ok=True)
     tmp = _SO + f".{os.getpid()}.tmp"
-    cmd = ["gcc", "-O2", "-march=native", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
-    subprocess.run(cmd, check=True)
+    compile_oracle(_SRC, tmp)
     os.replace(tmp, _SO)
     return _SO
 
@@ -57,7 +62,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = C.CDLL(build())
+        # MMOE_ORACLE_SO: another build of the oracle source (the pin tests' mutation check
+        # points it at copies with one planted mistake each)
+        _lib = C.CDLL(os.environ.get("MMOE_ORACLE_SO") or build())
         i64, vp = C.c_int64, C.c_void_p
         _lib.oracle_quantize_int4.argtypes = [vp, i64, i64, vp, vp]
         _lib.oracle_quantize_act.argtypes = [vp, i64, i64, vp, vp]
