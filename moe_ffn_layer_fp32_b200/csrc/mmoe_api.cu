@@ -572,6 +572,37 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     return MMOE_OK;
 }
 
+namespace {
+
+// The copy streams and events of mmoe_forward_host, created all or nothing.
+mmoe_status ensure_host_copy_state(mmoe_handle* h) {
+    if (h->s_h2d) return MMOE_OK;
+    cudaStream_t a = nullptr, b = nullptr;
+    cudaEvent_t ev[2 + 2 * kHostChunksMax] = {};
+    cudaError_t e = cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking);
+    for (cudaEvent_t& x : ev)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+        if (a) cudaStreamDestroy(a);
+        if (b) cudaStreamDestroy(b);
+        for (cudaEvent_t x : ev)
+            if (x) cudaEventDestroy(x);
+        return cuda_fail(e, "copy streams and events");
+    }
+    h->s_h2d = a;
+    h->s_d2h = b;
+    h->ev_start = ev[0];
+    h->ev_done = ev[1];
+    for (int i = 0; i < kHostChunksMax; ++i) {
+        h->ev_in[i] = ev[2 + i];
+        h->ev_out[i] = ev[2 + kHostChunksMax + i];
+    }
+    return MMOE_OK;
+}
+
+}  // namespace
+
 mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T, float* y_host, void* stream) {
     if (!h) return fail(MMOE_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0 || T > h->max_tokens)
@@ -583,57 +614,63 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_host, int64_t T,
     DeviceGuard dg(h->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t d = h->cfg.d_model;
-    if (!h->x_stage) {
-        MMOE_CUDA(dalloc(&h->x_stage, (size_t)h->max_tokens * d), "staging allocation");
-        MMOE_CUDA(dalloc(&h->y_stage, (size_t)h->max_tokens * d), "staging allocation");
-    }
-    if (!h->s_h2d) {
-        MMOE_CUDA(cudaStreamCreateWithFlags(&h->s_h2d, cudaStreamNonBlocking), "copy stream");
-        MMOE_CUDA(cudaStreamCreateWithFlags(&h->s_d2h, cudaStreamNonBlocking), "copy stream");
-        for (cudaEvent_t* ev : {&h->ev_start, &h->ev_done})
-            MMOE_CUDA(cudaEventCreateWithFlags(ev, cudaEventDisableTiming), "copy event");
-        for (int i = 0; i < kHostChunksMax; ++i) {
-            MMOE_CUDA(cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming), "copy event");
-            MMOE_CUDA(cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming), "copy event");
-        }
-    }
+    if (!h->x_stage) MMOE_CUDA(dalloc(&h->x_stage, (size_t)h->max_tokens * d), "staging allocation");
+    if (!h->y_stage) MMOE_CUDA(dalloc(&h->y_stage, (size_t)h->max_tokens * d), "staging allocation");
+    const mmoe_status cs = ensure_host_copy_state(h);
+    if (cs != MMOE_OK) return cs;
     // short first and last chunks shorten the copy-in before the first forward and the copy-out
     // after the last one
     int64_t bound[kHostChunksMax + 1];
     const int nch = host_chunk_bounds(T, bound);
+    // The first failure is kept and ends the enqueueing, but the copy streams are always joined
+    // and waited for, so that no copy touches x_host or y_host after this call returns.
+    cudaError_t ce = cudaSuccess;
+    const char* what = "";
+    auto ok = [&](cudaError_t e, const char* w) {
+        if (ce == cudaSuccess && e != cudaSuccess) {
+            ce = e;
+            what = w;
+        }
+        return ce == cudaSuccess;
+    };
     // copies start after the caller's earlier work on `stream`
-    MMOE_CUDA(cudaEventRecord(h->ev_start, s), "event record");
-    MMOE_CUDA(cudaStreamWaitEvent(h->s_h2d, h->ev_start, 0), "stream wait");
-    MMOE_CUDA(cudaStreamWaitEvent(h->s_d2h, h->ev_start, 0), "stream wait");
-    for (int i = 0; i < nch; ++i) {
+    bool go = ok(cudaEventRecord(h->ev_start, s), "event record") &&
+              ok(cudaStreamWaitEvent(h->s_h2d, h->ev_start, 0), "stream wait") &&
+              ok(cudaStreamWaitEvent(h->s_d2h, h->ev_start, 0), "stream wait");
+    for (int i = 0; go && i < nch; ++i) {
         const int64_t t0 = bound[i], Ti = bound[i + 1] - bound[i];
-        MMOE_CUDA(cudaMemcpyAsync(h->x_stage + t0 * d, x_host + t0 * d, (size_t)Ti * d * sizeof(uint16_t),
-                                  cudaMemcpyHostToDevice, h->s_h2d),
-                  "copy x to the device");
-        MMOE_CUDA(cudaEventRecord(h->ev_in[i], h->s_h2d), "event record");
+        go = ok(cudaMemcpyAsync(h->x_stage + t0 * d, x_host + t0 * d, (size_t)Ti * d * sizeof(uint16_t),
+                                cudaMemcpyHostToDevice, h->s_h2d),
+                "copy x to the device") &&
+             ok(cudaEventRecord(h->ev_in[i], h->s_h2d), "event record");
     }
     mmoe_status st = MMOE_OK;
-    for (int i = 0; i < nch && st == MMOE_OK; ++i) {
+    for (int i = 0; go && i < nch; ++i) {
         const int64_t t0 = bound[i], Ti = bound[i + 1] - bound[i];
-        MMOE_CUDA(cudaStreamWaitEvent(s, h->ev_in[i], 0), "stream wait");
+        if (!ok(cudaStreamWaitEvent(s, h->ev_in[i], 0), "stream wait")) break;
         st = mmoe_forward(h, h->x_stage + t0 * d, Ti, h->y_stage + t0 * d, stream, nullptr, nullptr, nullptr);
         if (st != MMOE_OK) break;
-        MMOE_CUDA(cudaEventRecord(h->ev_out[i], s), "event record");
-        MMOE_CUDA(cudaStreamWaitEvent(h->s_d2h, h->ev_out[i], 0), "stream wait");
-        MMOE_CUDA(cudaMemcpyAsync(y_host + t0 * d, h->y_stage + t0 * d, (size_t)Ti * d * sizeof(float),
-                                  cudaMemcpyDeviceToHost, h->s_d2h),
-                  "copy y to the host");
+        go = ok(cudaEventRecord(h->ev_out[i], s), "event record") &&
+             ok(cudaStreamWaitEvent(h->s_d2h, h->ev_out[i], 0), "stream wait") &&
+             ok(cudaMemcpyAsync(y_host + t0 * d, h->y_stage + t0 * d, (size_t)Ti * d * sizeof(float),
+                                cudaMemcpyDeviceToHost, h->s_d2h),
+                "copy y to the host");
     }
     // `stream` is left ordered after both copy streams, whatever happened above
-    cudaError_t e1 = cudaEventRecord(h->ev_done, h->s_h2d);
-    if (e1 == cudaSuccess) e1 = cudaStreamWaitEvent(s, h->ev_done, 0);
-    cudaError_t e2 = cudaEventRecord(h->ev_done, h->s_d2h);
-    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(s, h->ev_done, 0);
-    cudaError_t e3 = cudaStreamSynchronize(s);
+    cudaError_t j1 = cudaEventRecord(h->ev_done, h->s_h2d);
+    if (j1 == cudaSuccess) j1 = cudaStreamWaitEvent(s, h->ev_done, 0);
+    cudaError_t j2 = cudaEventRecord(h->ev_done, h->s_d2h);
+    if (j2 == cudaSuccess) j2 = cudaStreamWaitEvent(s, h->ev_done, 0);
+    const cudaError_t w1 = cudaStreamSynchronize(h->s_h2d);
+    const cudaError_t w2 = cudaStreamSynchronize(h->s_d2h);
+    const cudaError_t w3 = cudaStreamSynchronize(s);
     if (st != MMOE_OK) return st;
-    MMOE_CUDA(e1, "stream order");
-    MMOE_CUDA(e2, "stream order");
-    MMOE_CUDA(e3, "stream synchronize");
+    ok(j1, "stream order");
+    ok(j2, "stream order");
+    ok(w1, "stream synchronize");
+    ok(w2, "stream synchronize");
+    ok(w3, "stream synchronize");
+    if (ce != cudaSuccess) return cuda_fail(ce, what);
     return MMOE_OK;
 }
 
