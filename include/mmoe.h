@@ -127,7 +127,9 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out);
 /* Copies the weights into the handle's buffers and re-tiles them into the
  * kernels' layouts (stream-ordered, asynchronous).  The caller keeps
  * ownership of `w` and may free or reuse it once the stream has reached this
- * point.  May be called again to replace the weights.
+ * point.  May be called again to replace the weights.  A call that fails
+ * after its argument checks leaves the handle unloaded: forwards return
+ * NOT_LOADED until a load succeeds.
  * Errors: INVALID_ARG (NULL pointer, bias presence not matching the config), CUDA. */
 mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, void* stream);
 

@@ -488,6 +488,8 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
         return fail(MMOE_ERR_INVALID_ARG, "the config has a router bias but router_bias is NULL");
     if (w->on_device != 0 && w->on_device != 1) return fail(MMOE_ERR_INVALID_ARG, "on_device must be 0 or 1");
     DeviceGuard dg(h->device);
+    // a load that fails part way leaves a mix of old and new weights: unloaded until one succeeds
+    h->loaded = false;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const cudaMemcpyKind kind = w->on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
     const size_t d = h->cfg.d_model, E = h->cfg.n_experts;
