@@ -151,17 +151,22 @@ __global__ void __launch_bounds__(kThreads) requant_kernel(Plan p)
     const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     if (row >= p.R) return;
     const int hid = row >= p.Tk ? p.hs : p.h;
-    const float* a = p.act + row * p.hmax;
+    // 16 bytes per lane: rows start on 4 * hmax bytes and hid is a multiple of 32
+    const float4* a4 = reinterpret_cast<const float4*>(p.act + row * p.hmax);
     float m = 0.0f;
-    for (int i = lane; i < hid; i += 32) m = fmaxf(m, fabsf(a[i]));
+#pragma unroll 4
+    for (int i = lane; i < hid / 4; i += 32) {
+        const float4 v = a4[i];
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
     m = warp_max(m);
     const float s = __fdiv_rn(m, 127.0f);
-    int8_t* q = p.hq + row * p.hmax;
-    for (int i = lane * 4; i < hid; i += 128) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) w |= (uint32_t)(quant_i8(a[i + u], s) & 0xff) << (8 * u);
-        *reinterpret_cast<uint32_t*>(q + i) = w;
+    uint32_t* q = reinterpret_cast<uint32_t*>(p.hq + row * p.hmax);
+#pragma unroll 4
+    for (int i = lane; i < hid / 4; i += 32) {
+        const float4 v = a4[i];
+        q[i] = (uint32_t)(quant_i8(v.x, s) & 0xff) | (uint32_t)(quant_i8(v.y, s) & 0xff) << 8 |
+               (uint32_t)(quant_i8(v.z, s) & 0xff) << 16 | (uint32_t)(quant_i8(v.w, s) & 0xff) << 24;
     }
     if (lane == 0) p.sh[row] = s;
 }
