@@ -24,7 +24,8 @@
  *     makes the copies asynchronous, pageable memory is accepted too).
  *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy
  *     default stream.  Work is enqueued on it in order; no function except
- *     mmoe_forward_host, mmoe_create and mmoe_destroy waits for the GPU.
+ *     mmoe_forward_host, mmoe_create, mmoe_destroy and mmoe_profile_read
+ *     waits for the GPU.
  *   - A handle is not thread-safe: one forward at a time per handle.
  *   - Arguments are checked before anything is launched; a rejected call
  *     leaves the handle and every buffer untouched.
