@@ -74,9 +74,10 @@ def lib():
         _lib.oracle_moe_layer.argtypes = [C.POINTER(_Layer), vp, i64, vp, C.POINTER(_Dumps)]
         _lib.oracle_moe_tokens.argtypes = [C.POINTER(_Layer), vp, i64, vp, i64, vp]
         _lib.oracle_num_threads.argtypes = []
+        _lib.oracle_set_num_threads.argtypes = [C.c_int]
         for f in ("oracle_quantize_int4", "oracle_quantize_act", "oracle_router",
                   "oracle_expert_gate_up", "oracle_expert_down", "oracle_moe_layer",
-                  "oracle_moe_tokens", "oracle_num_threads"):
+                  "oracle_moe_tokens", "oracle_num_threads", "oracle_set_num_threads"):
             getattr(_lib, f).restype = C.c_int
     return _lib
 
@@ -87,6 +88,11 @@ def _p(a):
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """OpenMP threads of the following oracle calls; returns the count now in effect."""
+    return int(lib().oracle_set_num_threads(int(n)))
 
 
 def quantize_int4(W: np.ndarray):
@@ -185,7 +191,7 @@ def router(q: QuantizedLayer, x_bf16: np.ndarray):
     gate = np.zeros((T, q.k), np.float32)
     L = q.struct()
     if lib().oracle_router(C.byref(L), _p(x), T, _p(logits), _p(probs), _p(idx), _p(gate)):
-        raise MemoryError
+        raise ValueError("oracle_router: invalid layer description or allocation failure")
     return logits, probs, idx, gate
 
 

@@ -44,7 +44,8 @@ typedef struct {
     int64_t hs;       /* hidden size of the shared expert */
     int64_t E;        /* routed experts (60) */
     int64_t k;        /* experts per token (4) */
-    int64_t gating;   /* 0: softmax over E, no renormalisation; 1: sigmoid, top-k normalised */
+    int64_t gating;   /* 0: softmax over E, no renormalisation; 1: sigmoid, top-k normalised;
+                         2: as 1 with the bias added to the scores for the selection only */
     const float* w_router;     /* [d, E] row-major */
     const float* router_bias;  /* [E] or NULL */
     const uint8_t* w_gate_up;  /* expert g at byte g*2h*d/2: [2*hid][d/2], rows 0..hid-1 gate, then up */
@@ -161,20 +162,29 @@ int oracle_quantize_act(const uint16_t* x, int64_t T, int64_t d, int8_t* xq, flo
 /* ---------------------------------------------------------------------------
  * FP32 router of one token ("MoE training stability techniques": router in
  * FP32; Eq. (*): top-k by router score).
- *   l_e = fp32( sum_i x_i * W_r[i, e] ) + b_e
- *   gating 0: p = softmax over all E, gate_j = p[idx_j] (no renormalisation)
- *   gating 1: p_e = sigmoid(l_e), gate_j = p[idx_j] / sum_j' p[idx_j']
- *   idx = the k largest l_e, the lower index first among equal logits.
+ *   gating 0: l_e = fp32( sum_i x_i * W_r[i, e] ) + b_e,
+ *             p = softmax over all E, gate_j = p[idx_j] (no renormalisation),
+ *             idx = the k largest l_e;
+ *   gating 1: l_e as for gating 0, p_e = sigmoid(l_e),
+ *             gate_j = p[idx_j] / sum_j' p[idx_j'], idx = the k largest l_e;
+ *   gating 2: the auxiliary-loss-free balancing bias ("MoE training stability
+ *             techniques": a per-expert bias, adjusted from the load
+ *             imbalance, with no extra loss): l_e = fp32( sum_i x_i W_r[i, e] )
+ *             without the bias, p_e = sigmoid(l_e), idx = the k largest of the
+ *             FP32 sums p_e + b_e, gate_j = p[idx_j] / sum_j' p[idx_j'] -- the
+ *             bias moves the selection but never enters a gate.
+ * Among equal keys the lower expert index comes first.
  * ------------------------------------------------------------------------- */
 static void router_token(const oracle_layer* L, const float* xf, float* logits, float* probs,
                          int32_t* idx, float* gate)
 {
     const int64_t d = L->d, E = L->E, k = L->k;
+    float key[64];
     for (int64_t e = 0; e < E; ++e) {
         double acc = 0.0;
         for (int64_t i = 0; i < d; ++i) acc += (double)xf[i] * (double)L->w_router[i * E + e];
         float l = (float)acc;
-        if (L->router_bias) l = l + L->router_bias[e];
+        if (L->router_bias && L->gating != 2) l = l + L->router_bias[e];
         logits[e] = l;
     }
     if (L->gating == 0) {
@@ -187,6 +197,8 @@ static void router_token(const oracle_layer* L, const float* xf, float* logits, 
     } else {
         for (int64_t e = 0; e < E; ++e) probs[e] = (float)(1.0 / (1.0 + exp(-(double)logits[e])));
     }
+    for (int64_t e = 0; e < E; ++e)
+        key[e] = L->gating == 2 ? (L->router_bias ? probs[e] + L->router_bias[e] : probs[e]) : logits[e];
     for (int64_t j = 0; j < k; ++j) {
         int64_t best = -1;
         for (int64_t e = 0; e < E; ++e) {
@@ -194,7 +206,7 @@ static void router_token(const oracle_layer* L, const float* xf, float* logits, 
             for (int64_t jj = 0; jj < j; ++jj)
                 if (idx[jj] == e) taken = 1;
             if (taken) continue;
-            if (best < 0 || logits[e] > logits[best]) best = e;
+            if (best < 0 || key[e] > key[best]) best = e;
         }
         idx[j] = (int32_t)best;
     }
@@ -207,9 +219,12 @@ static void router_token(const oracle_layer* L, const float* xf, float* logits, 
     }
 }
 
+static int check_layer(const oracle_layer* L);
+
 int oracle_router(const oracle_layer* L, const uint16_t* x, int64_t T, float* logits, float* probs,
                   int32_t* idx, float* gate)
 {
+    if (check_layer(L) || T < 0) return -1;
     int err = 0;
 #pragma omp parallel reduction(| : err)
     {
@@ -367,9 +382,9 @@ done:
 
 static int check_layer(const oracle_layer* L)
 {
-    if (!L || L->d <= 0 || L->h <= 0 || L->hs <= 0 || L->E <= 0 || L->k <= 0 || L->k > L->E) return -1;
+    if (!L || L->d <= 0 || L->h <= 0 || L->hs <= 0 || L->E <= 0 || L->E > 64 || L->k <= 0 || L->k > L->E) return -1;
     if (L->d % ORACLE_GROUP || L->h % ORACLE_GROUP || L->hs % ORACLE_GROUP) return -1;
-    if (L->gating != 0 && L->gating != 1) return -1;
+    if (L->gating < 0 || L->gating > 2) return -1;
     return 0;
 }
 
@@ -404,6 +419,20 @@ int oracle_num_threads(void)
     extern int omp_get_max_threads(void);
     return omp_get_max_threads();
 #else
+    return 1;
+#endif
+}
+
+/* Threads of the following calls (the CPU baseline is timed on one core and on all of them). */
+int oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    (void)n;
     return 1;
 #endif
 }

@@ -275,6 +275,86 @@ def test_sigmoid_gating_normalised():
     assert np.array_equal(oracle.router(q0, x)[2], idx), "selection is the same for any monotone gate"
 
 
+def _sel_bias_routing_ref(q, x):
+    """Selection-only bias routing (gating 2) from an independent float64 matmul: logits without
+    the bias, p = sigmoid, key = FP32(p + b), stable top-k of the key, gates = p / sum over the
+    selected.  Returns (logits32, probs32, key32, idx, gate)."""
+    l64 = bf16_to_f64(x) @ q.w_router.astype(np.float64)
+    l32 = l64.astype(np.float32)
+    p32 = (1.0 / (1.0 + np.exp(-l32.astype(np.float64)))).astype(np.float32)
+    key = (p32 + q.router_bias.astype(np.float32)).astype(np.float32)
+    idx = np.argsort(-key, axis=1, kind="stable")[:, :q.k]
+    sel = np.take_along_axis(p32.astype(np.float64), idx, axis=1)
+    return l32, p32, key, idx, sel / sel.sum(axis=1, keepdims=True)
+
+
+def test_selection_bias_moves_selection_not_gates():
+    # gating 2 (auxiliary-loss-free balancing): the per-expert bias joins the sigmoid score only to
+    # pick the top-k; the reported logits exclude it and the gates are the unbiased scores,
+    # normalised over the selected experts
+    w = synth.WORKLOADS["c0"]
+    lw = synth.draw_layer(w.d, w.h, seed=5, bias_coef=0.25)
+    q = oracle.quantize_layer(lw, gating=2)
+    x = synth.draw_x(256, w.d, seed=6)
+    logits, probs, idx, gate = oracle.router(q, x)
+    l32, p32, key, idx_ref, gate_ref = _sel_bias_routing_ref(q, x)
+    assert np.max(np.abs(logits - l32)) < 1e-5                 # no bias in the logits
+    assert np.allclose(probs, p32, atol=1e-7)
+    # the oracle's selection from its own scores: the top-k of p + b (exact), lower index first on ties
+    own_key = (probs + lw.router_bias.astype(np.float32)).astype(np.float32)
+    assert np.array_equal(idx, np.argsort(-own_key, axis=1, kind="stable")[:, :q.k])
+    srt = -np.sort(-key, axis=1)
+    clear = srt[:, q.k - 1] - srt[:, q.k] > 1e-5               # away from the selection margin
+    assert clear.mean() > 0.9
+    assert np.array_equal(idx[clear], idx_ref[clear])
+    assert np.allclose(gate.sum(axis=1), 1.0, atol=1e-6)
+    assert np.max(np.abs(gate[clear] - gate_ref[clear])) < 1e-6
+    # the bias really moves the selection: without it the top-k differs on most tokens
+    q1 = oracle.quantize_layer(synth.LayerWeights(d=lw.d, h=lw.h, hs=lw.hs, E=lw.E, w_router=lw.w_router,
+                                                  router_bias=None, w_gate_up=lw.w_gate_up, w_down=lw.w_down),
+                               gating=1)
+    idx1 = oracle.router(q1, x)[2]
+    assert np.mean(np.any(np.sort(idx1, axis=1) != np.sort(idx, axis=1), axis=1)) > 0.5
+
+
+def test_selection_bias_zero_equals_sigmoid_gating():
+    # with a zero bias the key is the sigmoid score, a monotone function of the logit: the same
+    # experts and gates as gating 1 (no two scores of these tokens round to the same FP32 value)
+    w = synth.WORKLOADS["c0"]
+    lw = synth.workload_layer(w)
+    lw0 = synth.LayerWeights(d=lw.d, h=lw.h, hs=lw.hs, E=lw.E, w_router=lw.w_router,
+                             router_bias=np.zeros(lw.E, np.float32), w_gate_up=lw.w_gate_up, w_down=lw.w_down)
+    x = synth.workload_x(w)
+    _, p2, i2, g2 = oracle.router(oracle.quantize_layer(lw0, gating=2), x)
+    _, _, i1, g1 = oracle.router(oracle.quantize_layer(lw, gating=1), x)
+    assert all(len(set(r.tolist())) == len(r) for r in p2)
+    assert np.array_equal(i1, i2) and np.array_equal(g1, g2)
+
+
+def test_selection_bias_layer_brute_force():
+    # the whole layer with gating 2 against the dense float64 brute force, routed by the
+    # independent reference above
+    w = synth.WORKLOADS["c0"]
+    lw = synth.draw_layer(w.d, w.h, seed=7, bias_coef=1.5)
+    q = oracle.quantize_layer(lw, gating=2)
+    x = synth.draw_x(32, w.d, seed=8)
+    y, D = oracle.moe_layer(q, x, dumps=True)
+    _, _, key, idx_ref, gate_ref = _sel_bias_routing_ref(q, x)
+    srt = -np.sort(-key, axis=1)
+    assert np.all(srt[:, q.k - 1] - srt[:, q.k] > 1e-6)
+    assert np.array_equal(D["idx"], idx_ref)
+    assert np.max(np.abs(D["gate"] - gate_ref)) < 1e-6
+    # the expert side (SwiGLU codes, down projection) is pinned by the brute-force test of gating 0;
+    # here the layer is recombined from the oracle's own codes with the reference routing and gates
+    yref = np.zeros((x.shape[0], q.d))
+    for t in range(x.shape[0]):
+        for s in range(q.k + 1):
+            g = q.E if s == q.k else int(idx_ref[t, s])
+            o = brute_down(q, g, D["hq"][t, s], float(D["sh"][t, s]))
+            yref[t] += o if s == q.k else gate_ref[t, s] * o
+    assert np.max(np.abs(y - yref)) <= 1e-5 * np.abs(yref).max()
+
+
 # ---------------------------------------------------------------------------
 # brute force over all experts
 # ---------------------------------------------------------------------------

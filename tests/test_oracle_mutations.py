@@ -27,9 +27,16 @@ MUTATIONS = {
                             "for (int64_t m = 0; m < d; ++m) yrow[m] = 0.5f * o[m];"),
     "gates_reversed": ("float prod = gate[s] * o[m];", "float prod = gate[k - 1 - s] * o[m];"),
     # router (section on the FP32 router; softmax without renormalisation)
-    "router_bias_missing": ("if (L->router_bias) l = l + L->router_bias[e];", ""),
-    "tie_goes_to_high_index": ("if (best < 0 || logits[e] > logits[best]) best = e;",
-                               "if (best < 0 || logits[e] >= logits[best]) best = e;"),
+    "router_bias_missing": ("if (L->router_bias && L->gating != 2) l = l + L->router_bias[e];", ""),
+    "tie_goes_to_high_index": ("if (best < 0 || key[e] > key[best]) best = e;",
+                               "if (best < 0 || key[e] >= key[best]) best = e;"),
+    # selection-only bias (gating 2, auxiliary-loss-free balancing)
+    "sel_bias_enters_logit": ("if (L->router_bias && L->gating != 2) l = l + L->router_bias[e];",
+                              "if (L->router_bias) l = l + L->router_bias[e];"),
+    "sel_bias_ignored": ("key[e] = L->gating == 2 ? (L->router_bias ? probs[e] + L->router_bias[e] : probs[e])",
+                         "key[e] = L->gating == 2 ? (L->router_bias ? probs[e] : probs[e])"),
+    "sel_bias_on_logit": ("key[e] = L->gating == 2 ? (L->router_bias ? probs[e] + L->router_bias[e] : probs[e])",
+                          "key[e] = L->gating == 2 ? (L->router_bias ? logits[e] + L->router_bias[e] : probs[e])"),
     "softmax_renormalised": ("for (int64_t j = 0; j < k; ++j) gate[j] = probs[idx[j]];",
                              "double ss = 0; for (int64_t j = 0; j < k; ++j) ss += probs[idx[j]]; "
                              "for (int64_t j = 0; j < k; ++j) gate[j] = (float)(probs[idx[j]] / ss);"),
