@@ -32,11 +32,17 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer prefill tokens/s & decode us/layer; % of INT8-TC / HBM roofline"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# prefill gate/up GEMM, from one ncu capture of this bench command on B200
-# (`--metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:expert_gemm_tc`);
-# valid only while that kernel is unchanged.
-GATE_UP_TRAFFIC_BYTES = {"c4": 625195264 + 621898240}
+# prefill gate/up GEMM per workload, from one ncu capture on B200, keyed by the
+# first 16 hex digits of the SHA-256 of the GEMM's source file at the time of the
+# capture: a figure is reported only while that file is unchanged.
+GATE_UP_TRAFFIC_BYTES = {}
+GEMM_SOURCE = os.path.join(ROOT, "moe_ffn_layer_fp32_b200", "csrc", "k_expert_f16.cu")
 L2_BYTES = 126 * 1024 * 1024
+# Peaks when MEASURED_PEAKS.json is absent: an earlier measurement on this machine (bf16 dense burst,
+# HBM copy bandwidth)
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+PREFILL_EXTRAS = ("c2", "c3a", "c3b", "s2048")
 
 
 def parse_args(argv=None):
@@ -50,6 +56,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-sweep", action="store_true", help="skip the 24-layer decode sweep (T=1 and T=8)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU work budget of the oracle sample")
+    ap.add_argument("--no-extras", action="store_true", help="skip the c2, c3a, c3b and MobileMoE-S prefill lines")
     return ap.parse_args(argv)
 
 
@@ -147,6 +154,33 @@ def layer_counts(w, T):
     return gu_ops, dn_ops
 
 
+def gemm_source_hash():
+    import hashlib
+    with open(GEMM_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, HBM GB/s, source note)."""
+    try:
+        pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return (float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                float(pk["hbm_gbs"]), "measured")
+    except (OSError, KeyError, ValueError, TypeError):
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def quantized_on_device(w, device, layer=0):
     """Seeded FP32 weights (synth) quantised on the GPU by the library's Eq. (6) kernel."""
     from moe_ffn_layer_fp32_b200.run_case import quantized_weights
@@ -157,16 +191,17 @@ def weight_bytes(w, experts):
     return sum((3 * w.d * (w.h if g < w.E else w.hs)) * 0.625 for g in experts)
 
 
-def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8)):
-    """The decode workload: 24 distinct layers (d_model=1024, h=512; 1.44 GB of INT4 weights and scales, far
-    beyond L2) run back to back, layer l+1 reading layer l's y cast to BF16, captured once as a CUDA graph.
-    Step s feeds a fresh seeded x (seed 10^6 + s) to layer 0.  Returns us/layer and GB/s per token count."""
+def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8), name="c1"):
+    """A decode workload: 24 distinct layers (c1: d_model=1024, h=512, 1.44 GB of INT4 weights and scales;
+    s1: the MobileMoE-S shape; both far beyond L2) run back to back, layer l+1 reading layer l's y cast to
+    BF16, captured once as a CUDA graph.  Step s feeds a fresh seeded x to layer 0.  Returns us/layer and
+    GB/s per token count."""
     import numpy as np
     import torch
 
     from moe_ffn_layer_fp32_b200 import synth
     from moe_ffn_layer_fp32_b200.layer import MoELayer
-    w = synth.WORKLOADS["c1"]
+    w = synth.WORKLOADS[name]
     layers = []
     for l in range(w.layers):
         tensors, lw = quantized_on_device(w, dev, l)
@@ -217,7 +252,7 @@ def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8)):
         nbytes /= w.layers
         gbs = nbytes / (us_layer * 1e-6) / 1e9
         out[f"T{T}"] = {"us_per_layer": us_layer, "bytes_per_layer": nbytes, "achieved_gbs": gbs,
-                        "hbm_frac": gbs / hbm_gbs, "launches_per_layer": 3}
+                        "hbm_frac": gbs / hbm_gbs, "hbm_peak_gbs": hbm_gbs, "launches_per_layer": 3}
         del g
     for L in layers:
         L.close()
@@ -227,8 +262,9 @@ def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8)):
 # --------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # --------------------------------------------------------------------------
-def oracle_rate(w, budget_s, lw=None):
-    """Tokens/s of the CPU oracle on a bounded sample of the workload's tokens."""
+def oracle_rate(w, budget_s, lw=None, threads=None):
+    """Tokens/s of the CPU oracle on a bounded sample of the workload's tokens (all host cores, or
+    `threads` of them)."""
     import numpy as np
 
     import oracle
@@ -236,7 +272,8 @@ def oracle_rate(w, budget_s, lw=None):
     if lw is None:
         lw = synth.workload_layer(w)
     q = oracle.quantize_layer(lw)
-    cores = oracle.num_threads()
+    all_cores = os.cpu_count() or 1
+    cores = oracle.set_num_threads(threads if threads else all_cores)
     x = synth.workload_x(w, T=min(w.T, 4096))
     n = max(2, cores)
     t0 = time.perf_counter()
@@ -278,6 +315,73 @@ def run_reference(args):
 # --------------------------------------------------------------------------
 # the GPU arm
 # --------------------------------------------------------------------------
+def gemm_roofline(w, T, ms_gate_up, ms_down, int8_peak_tops, bf16_peak_tflops, note):
+    """Achieved INT8-equivalent TOP/s of the two expert GEMMs (2 ops per MAC of the INT8 x INT4 product)
+    against the dense INT8 tensor-core peak (2 x the bf16 peak), and against the f16 tensor-core peak
+    their kind::f16 MMAs run at."""
+    gu_ops, dn_ops = layer_counts(w, T)
+    out = {}
+    for name, ops, ms in (("gate_up", gu_ops, ms_gate_up), ("down", dn_ops, ms_down)):
+        if not ms:
+            continue
+        tops = ops / (ms / 1e3) / 1e12
+        out[name] = {"ms": ms, "ops": ops, "achieved_tops": tops, "frac_int8_peak": tops / int8_peak_tops,
+                     "frac_f16_pipe_peak": tops / bf16_peak_tflops}
+    out["peak_int8_tops"] = int8_peak_tops
+    out["peak_note"] = note
+    return out
+
+
+def measure_prefill(name, dev, steps, warmup, peaks):
+    """One extra prefill workload: per-forward device time (L2 flushed before every forward, so the
+    weights come from HBM), tokens/s, per-stage times, the GEMMs' tensor-core fractions and the
+    router's HBM fraction."""
+    import numpy as np
+    import torch
+
+    from moe_ffn_layer_fp32_b200 import synth
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    bf16_burst, _, hbm, note = peaks
+    w = synth.WORKLOADS[name]
+    tensors, lw = quantized_on_device(w, dev)
+    L = MoELayer(w.d, w.h, shared_hidden=w.hs, n_experts=w.E, top_k=w.k, max_tokens=w.T,
+                 has_router_bias=lw.router_bias is not None, device=dev.index)
+    L.load(*tensors)
+    del tensors
+    x = torch.from_numpy(synth.workload_x(w).view(np.int16)).to(dev).view(torch.bfloat16)
+    y = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
+    counts = torch.zeros(w.E + 1, dtype=torch.int32, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        L.forward(x, y)
+    torch.cuda.synchronize(dev)
+    L.profile(True)
+    times = []
+    for _ in range(steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        L.forward(x, y, expert_counts=counts)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    prof = L.profile_read()
+    L.profile(False)
+    ms = statistics.median(a.elapsed_time(b) for a, b in times)
+    st = {k: v[1] / steps for k, v in prof.items() if v[0] or v[1]}
+    c = counts.cpu().numpy()
+    L.close()
+    router_bytes = w.T * w.d * 2 * 2 + w.T * w.d * 2 + w.d * w.E * 4   # x read twice, f16 codes, W_r
+    out = {"workload": w.desc, "tokens": w.T, "ms": ms, "tokens_per_s": w.T / (ms / 1e3), "stages_ms": st,
+           "gemm": gemm_roofline(w, w.T, st.get("gate_up"), st.get("down"), 2.0 * bf16_burst, bf16_burst, note),
+           "router_hbm_frac": (router_bytes / (st["router"] / 1e3) / 1e9 / hbm) if st.get("router") else None,
+           "expert_rows_max_over_min_nonzero": float(c[:w.E].max() / max(1, c[:w.E][c[:w.E] > 0].min())),
+           "experts_without_tokens": int((c[:w.E] == 0).sum()),
+           "l2": "flushed (a 252 MB write) before every forward"}
+    return out
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -367,28 +471,26 @@ def run_ours(args):
     tmax, units = aggregate(elapsed, tokens_per_step * args.steps, dist, dev)
     launches = sum(v[0] for v in prof_p.values()) + sum(v[0] for v in prof_d.values())
 
-    # dominant kernel: the prefill gate/up GEMM (INT8 x INT4 -> INT32, tensor-bound)
+    # dominant kernel: the prefill gate/up GEMM (INT8 x INT4 products with exact integer group sums on the
+    # tensor cores).  Its timed region is 0.1 s long, so the burst peak is the denominator.
+    bf16_burst, bf16_sust, hbm, peak_src = load_peaks()
+    int8_peak = 2.0 * bf16_burst
     gu_ops, dn_ops = layer_counts(w, Tp)
     n_gu, ms_gu = prof_p["gate_up"]
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-        int8_peak = 2.0 * float(peaks["bf16_tflops_sustained"])
-        peak_note = "measured cuBLAS bf16 sustained x 2 (nominal int8/bf16 ratio)"
-    except (OSError, KeyError, ValueError):
-        int8_peak = 2.0 * 1400.0
-        peak_note = "fallback 1.4 PFLOP/s bf16 sustained x 2"
     gu_avg_s = (ms_gu / max(n_gu, 1)) / 1e3
     achieved = gu_ops / gu_avg_s / 1e12 if gu_avg_s > 0 else 0.0
-    traffic = GATE_UP_TRAFFIC_BYTES.get(w.name)
-    roofline = {"kernel": "gate_up (prefill)", "bound": "tensor", "achieved": achieved, "peak": int8_peak,
-                "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": traffic, "traffic_unit": "bytes per launch (ncu)",
-                "op_dtype": "int8",
-                "peak_source": peak_note, "ops_per_launch": gu_ops, "avg_launch_ms": gu_avg_s * 1e3}
+    traffic = GATE_UP_TRAFFIC_BYTES.get(gemm_source_hash(), {}).get(w.name)
+    roofline = {"kernel": "gate_up (prefill, expert_gemm_f16_kernel)", "bound": "tensor", "achieved": achieved,
+                "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak, "traffic": traffic,
+                "traffic_unit": "bytes per launch (ncu, this GEMM source)", "op_dtype": "int8",
+                "peak_source": f"{peak_src} bf16 dense burst x 2 (nominal int8/bf16 ratio); of {peak_src}",
+                "frac_f16_pipe_peak": achieved / bf16_burst, "ops_per_launch": gu_ops,
+                "avg_launch_ms": gu_avg_s * 1e3}
+    peaks = {"bf16_tflops_burst": bf16_burst, "bf16_tflops_sustained": bf16_sust, "hbm_gbs": hbm,
+             "source": peak_src}
 
     decode = None
     if dec:
-        hbm = float(peaks.get("hbm_gbs", 6650.0))
         idx = idx_d.cpu().numpy()
         experts = sorted(set(idx.ravel().tolist()) | {w.E})
         dbytes = weight_bytes(w, experts) + w.d * w.E * 4
@@ -431,16 +533,29 @@ def run_ours(args):
                "h2d_bytes_per_step": (Tp + Td) * w.d * 2, "d2h_bytes_per_step": (Tp + Td) * w.d * 4,
                "api": "mmoe_forward_host (pinned host x and y)"}
 
-    sweep = None
+    sweep = sweep_s = None
     if not args.no_decode_sweep:
-        sweep = decode_sweep(dev, args.steps, args.warmup, float(peaks.get("hbm_gbs", 6650.0)))
+        sweep = decode_sweep(dev, args.steps, args.warmup, hbm)
+        sweep_s = decode_sweep(dev, args.steps, args.warmup, hbm, token_counts=(1,), name="s1")
+
+    # the other prefill workloads, each its own short measurement (outside the timed step above)
+    extras = {}
+    if not args.no_extras:
+        for name in PREFILL_EXTRAS:
+            extras[name] = measure_prefill(name, dev, max(3, args.steps), max(3, args.warmup),
+                                           (bf16_burst, bf16_sust, hbm, peak_src))
+        extras["c4"] = {"gemm": gemm_roofline(w, Tp, prof_p["gate_up"][1] / args.steps, prof_p["down"][1] / args.steps,
+                                              int8_peak, bf16_burst, peak_src)}
 
     clk = clocks.stop() if clocks else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, n, dt = oracle_rate(w, args.cpu_seconds, lw)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"first {n} prefill tokens of {w.name} ({dt:.1f} s of CPU work)"}
+        rate1, _, n1, dt1 = oracle_rate(w, max(2.0, args.cpu_seconds / 4), lw, threads=1)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+               "sample": f"first {n} prefill tokens of {w.name} ({dt:.1f} s of CPU work)",
+               "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
+                               "sample": f"first {n1} prefill tokens of {w.name} ({dt1:.1f} s)"}}
 
     if dist is not None:
         dist.barrier()
@@ -461,6 +576,9 @@ def run_ours(args):
                     "stages_ms": {k: v[1] / args.steps for k, v in prof_p.items() if v[0] or v[1]}},
         "decode": decode,
         "decode_sweep": sweep,
+        "decode_sweep_s_shape": sweep_s,
+        "prefill_workloads": extras,
+        "peaks": peaks,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -52,8 +52,10 @@ typedef enum {
     MMOE_ERR_UNIMPLEMENTED = 6  /* a valid request this build does not serve */
 } mmoe_status;
 
-/* Router gating.  Selection is always the top-k of the FP32 biased logits,
- * the lower expert index first among equal logits; only the gate differs. */
+/* Router gating.  Selection is the top-k of the FP32 biased logits for
+ * gating 0 and 1 (the lower expert index first among equal logits; the two
+ * select the same experts and differ in the gates), and of the biased
+ * sigmoid scores for gating 2. */
 typedef enum {
     /* p = softmax over all experts, gate_j = p[idx_j], no renormalisation
      * (the gating the layer benchmark fixes) */
@@ -61,7 +63,16 @@ typedef enum {
     /* p_e = sigmoid(l_e), gate_j = p[idx_j] / sum_j' p[idx_j'] ("sigmoid
      * gating with per-token top-k normalisation", section "MoE training
      * stability techniques") */
-    MMOE_GATE_SIGMOID_TOPK_NORM = 1
+    MMOE_GATE_SIGMOID_TOPK_NORM = 1,
+    /* as MMOE_GATE_SIGMOID_TOPK_NORM, with the router bias (has_router_bias)
+     * used the way the auxiliary-loss-free load balancing uses it ("MoE
+     * training stability techniques": a per-expert bias adjusted from the
+     * load imbalance, with no extra loss): p_e = sigmoid(l_e) with l_e WITHOUT
+     * the bias, idx = top-k of the FP32 sums p_e + b_e (lower index first
+     * among equal sums), gate_j = p[idx_j] / sum_j' p[idx_j'].  The bias moves
+     * the selection only and never enters a gate; the logits reported by
+     * MMOE_STAGE_LOGITS exclude it. */
+    MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS = 2
 } mmoe_gating;
 
 /* mmoe_config.flags */
@@ -79,6 +90,11 @@ typedef enum {
 #define MMOE_FLAG_NO_DECODE 4u     /* never take the decode path: by default a forward with few tokens
                                       (T <= 64 where d_model and both hidden sizes are multiples of 64)
                                       runs the weight-streaming decode kernels; same results */
+#define MMOE_FLAG_TC_INT8 16u      /* prefill expert GEMMs on the INT8 tensor-core kind (tcgen05 kind::i8,
+                                      S32 group partials) instead of the default f16 kind (exact integer
+                                      group partials in FP32 accumulators, which the promotion reads
+                                      without a conversion; d_model a multiple of 256 and both hidden
+                                      sizes multiples of 128); same results, slower */
 
 typedef struct {
     int32_t d_model;        /* multiple of 32, 64 <= d_model <= 8192 */
@@ -89,7 +105,8 @@ typedef struct {
     int32_t group_size;     /* must be 32 (Eq. (6) group size) */
     int32_t max_tokens;     /* largest T a forward may pass, 1..2^20; sizes the workspace */
     int32_t gating;         /* mmoe_gating */
-    int32_t has_router_bias;/* 0 or 1: a per-expert FP32 bias added to the logits before gating */
+    int32_t has_router_bias;/* 0 or 1: a per-expert FP32 bias, added to the logits before gating
+                               (gating 0, 1) or to the sigmoid scores for the selection only (2) */
     uint32_t flags;         /* MMOE_FLAG_* */
 } mmoe_config;
 
@@ -191,7 +208,7 @@ mmoe_status mmoe_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t*
  *   MMOE_STAGE_SLOT_ROW int32 [T, top_k]    row of each (token, slot)
  *   MMOE_STAGE_HQ       int8  [R, hmax]     SwiGLU output codes (hmax = max hidden)
  *   MMOE_STAGE_SH       FP32  [R]           SwiGLU output scales
- *   MMOE_STAGE_LOGITS   FP32  [T, n_experts] biased router logits
+ *   MMOE_STAGE_LOGITS   FP32  [T, n_experts] router logits (biased for gating 0 and 1)
  * Errors: INVALID_ARG (unknown stage, bytes larger than the stage), CUDA. */
 typedef enum {
     MMOE_STAGE_XQ = 0,
@@ -221,6 +238,30 @@ mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int
  * of `cap` entries and n to `*n`.  Errors: INVALID_ARG (T < 0, NULL pointer,
  * cap < n + 1). */
 mmoe_status mmoe_debug_host_chunks(int64_t T, int64_t* bounds, int32_t cap, int32_t* n);
+
+/* Allocation-failure injection (tests): after `after` more device
+ * allocations by the library on the calling thread, the next one fails as if
+ * the device were out of memory (mmoe_create, the staging buffers of
+ * mmoe_forward_host); after = 0 fails the very next one, -1 turns the
+ * injection off.  It fires once, then turns itself off.  The failing call
+ * returns MMOE_ERR_OOM and frees whatever it had allocated.
+ * Errors: INVALID_ARG (after < -1). */
+mmoe_status mmoe_debug_fail_alloc(int64_t after);
+
+/* Failure detection without a GPU fault.  Sets how long (in SM clock
+ * cycles) a bounded device-side wait of the prefill tensor-core GEMMs
+ * (default kind) lasts before it gives up; clocks = 0 restores the default
+ * (4e9 cycles, about 2 s).  With stall_next = 1 the next forward that takes
+ * the prefill path makes one of those waits wait for a barrier that nothing
+ * signals, as a hung producer would: the wait runs out after `clocks`, the
+ * GEMM drains its copies in flight and exits without writing its outputs, and
+ * the following mmoe_forward (or mmoe_destroy) on the handle returns
+ * MMOE_ERR_TIMEOUT; later forwards run normally.  A caller has no reason to
+ * call this outside tests.
+ * Errors: INVALID_ARG (NULL handle, clocks < 0, stall_next not 0 or 1),
+ * UNIMPLEMENTED (stall_next = 1 on a handle without the default tensor-core
+ * GEMMs). */
+mmoe_status mmoe_debug_set_wait_limit(mmoe_handle* h, int64_t clocks, int32_t stall_next);
 
 /* ---- per-stage timing ------------------------------------------------------
  * While profiling is enabled, every forward records a CUDA event pair on its
@@ -264,22 +305,32 @@ mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_m
  * mmoe_forward.  All intermediate data lives in one array that the library
  * declares at file scope in device memory, MMOE_STATIC_SCRATCH_BYTES long;
  * every GPU that loads the library holds that array until the process exits.
- *   - Size limit: the scratch a call needs grows with T, d_model, the hidden
- *     sizes and top_k (about T*(top_k+1)*(d_model + 5*max_hidden) bytes, plus
- *     T*(top_k+1)*d_model*4 more with MMOE_FLAG_DETERMINISTIC); a call that
- *     needs more than the array holds is rejected with MMOE_ERR_INVALID_ARG
- *     before anything is launched.  cfg->max_tokens is not used.
+ *   - Kernels: the CUDA-core expert GEMMs (no re-tiled weight copies exist in
+ *     this mode).  The expert outputs are added in the fixed order of
+ *     mmoe_forward's prefill path (y bit-reproducible from run to run) unless
+ *     cfg->flags has MMOE_FLAG_ATOMIC_COMBINE, which adds them with atomics
+ *     and needs less scratch.
+ *   - Alignment: x, y, w_gate_up and w_down 16-byte aligned; w_router,
+ *     router_bias, s_gate_up and s_down 4-byte aligned (they are read in
+ *     place with vector loads).
+ *   - Size limit: T <= 2^20, and the scratch a call needs grows with T,
+ *     d_model, the hidden sizes and top_k: about
+ *     T*(top_k+1)*(d_model + 5*max_hidden) bytes, plus T*(top_k+1)*d_model*4
+ *     for the fixed-order combine.  A call that needs more than the array
+ *     holds is rejected with MMOE_ERR_INVALID_ARG before anything is
+ *     launched.  cfg->max_tokens is not used.
  *   - Set-up: the first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
  *     first call before any stream capture.
  *   - Sharing: every call on a device uses the same array and leaves its
  *     contents behind.  Each kernel writes every scratch word it later reads,
- *     so nothing needs clearing between calls, but calls whose work overlaps
- *     on the GPU (different streams, or different host threads) race on the
- *     array and corrupt each other's results: order them on one stream.
+ *     so nothing needs clearing between calls (also when T changes from one
+ *     call to the next), but calls whose work overlaps on the GPU (different
+ *     streams, or different host threads) race on the array and corrupt each
+ *     other's results: order them on one stream.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
- * Errors: INVALID_ARG (bad config, NULL or host weight pointers, T < 0, NULL
- * or not 16-byte aligned x or y, the scratch limit), CUDA. */
+ * Errors: INVALID_ARG (bad config, NULL, host or misaligned weight pointers,
+ * T < 0 or T > 2^20, NULL or misaligned x or y, the scratch limit), CUDA. */
 #define MMOE_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
 
 mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weights* w, const uint16_t* x_bf16,

@@ -17,17 +17,20 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "NOT_LOADED", 3: "OOM", 4: "CUDA",
 
 GATE_SOFTMAX = 0
 GATE_SIGMOID_TOPK_NORM = 1
+GATE_SIGMOID_TOPK_NORM_SEL_BIAS = 2
 FLAG_DETERMINISTIC = 1
 FLAG_CUDA_CORES = 2
 FLAG_NO_DECODE = 4
 FLAG_ATOMIC_COMBINE = 8
+FLAG_TC_INT8 = 16
 
 STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAGE_SH, STAGE_LOGITS = range(8)
 
 # every symbol include/mmoe.h declares
 EXPORTS = ("mmoe_create", "mmoe_load_quantized_weights", "mmoe_forward", "mmoe_forward_host", "mmoe_destroy",
            "mmoe_last_error", "mmoe_quantize_int4", "mmoe_debug_copy_stage", "mmoe_debug_partials",
-           "mmoe_profile_enable", "mmoe_profile_read", "mmoe_forward_static_scratch", "mmoe_debug_host_chunks")
+           "mmoe_profile_enable", "mmoe_profile_read", "mmoe_forward_static_scratch", "mmoe_debug_host_chunks",
+           "mmoe_debug_set_wait_limit", "mmoe_debug_fail_alloc")
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
@@ -79,6 +82,8 @@ def lib() -> C.CDLL:
     L.mmoe_profile_read.argtypes = [vp, vp, vp, i32]
     L.mmoe_forward_static_scratch.argtypes = [C.POINTER(Config), C.POINTER(Weights), vp, i64, vp, vp]
     L.mmoe_debug_host_chunks.argtypes = [i64, vp, i32, vp]
+    L.mmoe_debug_set_wait_limit.argtypes = [vp, i64, i32]
+    L.mmoe_debug_fail_alloc.argtypes = [i64]
     for name in EXPORTS:
         if name != "mmoe_last_error":
             getattr(L, name).restype = st

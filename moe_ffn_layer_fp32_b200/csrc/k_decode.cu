@@ -350,8 +350,8 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
         const float s0 = cluster_sum(&part[t * 64 + lane], cs);
         const float s1 = cluster_sum(&part[t * 64 + lane + 32], cs);
         float l0 = -INFINITY, l1 = -INFINITY;
-        if (lane < E) l0 = p.router_bias ? __fadd_rn(s0, p.router_bias[lane]) : s0;
-        if (lane + 32 < E) l1 = p.router_bias ? __fadd_rn(s1, p.router_bias[lane + 32]) : s1;
+        if (lane < E) l0 = biased_logit(p, s0, lane);
+        if (lane + 32 < E) l1 = biased_logit(p, s1, lane + 32);
         gate_topk_warp(p, t, l0, l1, lane);
         if (lane == 0) {
             p.sx[t] = sxs[t];

@@ -161,12 +161,23 @@ __global__ void __launch_bounds__(kThreads) requant_kernel(Plan p)
     }
     m = warp_max(m);
     const float s = __fdiv_rn(m, 127.0f);
-    uint32_t* q = reinterpret_cast<uint32_t*>(p.hq + row * p.hmax);
+    if (p.hq16) {
+        // f16 codes for the kind::f16 down GEMM
+        uint2* q = reinterpret_cast<uint2*>(p.hq16 + row * p.hmax);
 #pragma unroll 4
-    for (int i = lane; i < hid / 4; i += 32) {
-        const float4 v = a4[i];
-        q[i] = (uint32_t)(quant_i8(v.x, s) & 0xff) | (uint32_t)(quant_i8(v.y, s) & 0xff) << 8 |
-               (uint32_t)(quant_i8(v.z, s) & 0xff) << 16 | (uint32_t)(quant_i8(v.w, s) & 0xff) << 24;
+        for (int i = lane; i < hid / 4; i += 32) {
+            const float4 v = a4[i];
+            q[i] = make_uint2(code_f16(quant_i8(v.x, s)) | (code_f16(quant_i8(v.y, s)) << 16),
+                              code_f16(quant_i8(v.z, s)) | (code_f16(quant_i8(v.w, s)) << 16));
+        }
+    } else {
+        uint32_t* q = reinterpret_cast<uint32_t*>(p.hq + row * p.hmax);
+#pragma unroll 4
+        for (int i = lane; i < hid / 4; i += 32) {
+            const float4 v = a4[i];
+            q[i] = (uint32_t)(quant_i8(v.x, s) & 0xff) | (uint32_t)(quant_i8(v.y, s) & 0xff) << 8 |
+                   (uint32_t)(quant_i8(v.z, s) & 0xff) << 16 | (uint32_t)(quant_i8(v.w, s) & 0xff) << 24;
+        }
     }
     if (lane == 0) p.sh[row] = s;
 }

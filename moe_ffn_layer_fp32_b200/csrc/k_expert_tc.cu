@@ -674,7 +674,8 @@ cudaError_t launch_retile(const uint8_t* gu, const float* sgu, const uint8_t* dn
 
 size_t tensor_map_bytes() { return sizeof(CUtensorMap); }
 
-cudaError_t make_tensor_map(void* map_, void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_stride) {
+cudaError_t make_tensor_map(void* map_, void* base, uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
+                            int elem_bytes) {
     CUtensorMap* map = static_cast<CUtensorMap*>(map_);
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
@@ -685,13 +686,15 @@ cudaError_t make_tensor_map(void* map_, void* base, uint64_t inner_bytes, uint64
         if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    const cuuint64_t dims[2] = {inner_bytes, rows};
-    const cuuint64_t strides[1] = {row_stride};
-    const cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)tc::BN};
+    if (elem_bytes != 1 && elem_bytes != 2) return cudaErrorInvalidValue;
+    // boxes of 128 bytes (one swizzle row) x 128 rows
+    const cuuint64_t dims[2] = {inner_elems, rows};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), 128u};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = encode(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base,
+                        dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 

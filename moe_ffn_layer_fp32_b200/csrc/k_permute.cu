@@ -8,6 +8,8 @@
 //
 // Row order: routed rows grouped by expert, each expert's rows in ascending
 // (token, slot) order; then the T rows of the shared expert in token order.
+#include <algorithm>
+
 #include "mmoe_internal.cuh"
 
 namespace mmoe {
@@ -133,12 +135,32 @@ __global__ void __launch_bounds__(kThreads) gather_rows_kernel(Plan p)
     const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     if (row >= p.Tk) return;
     const int64_t t = p.row_src[row];
-    const uint4* src = reinterpret_cast<const uint4*>(p.xq + (p.Tk + t) * p.d);
-    uint4* dst = reinterpret_cast<uint4*>(p.xq + row * p.d);
-    for (int i = lane; i < p.d / 16; i += 32) dst[i] = src[i];
+    if (p.xq16) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.xq16 + (p.Tk + t) * p.d);
+        uint4* dst = reinterpret_cast<uint4*>(p.xq16 + row * p.d);
+        for (int i = lane; i < p.d / 8; i += 32) dst[i] = src[i];
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(p.xq + (p.Tk + t) * p.d);
+        uint4* dst = reinterpret_cast<uint4*>(p.xq + row * p.d);
+        for (int i = lane; i < p.d / 16; i += 32) dst[i] = src[i];
+    }
+}
+
+// f16 codes -> INT8 codes (both exact integers in [-127, 127])
+__global__ void codes_f16_to_i8_kernel(const uint16_t* __restrict__ src, int8_t* __restrict__ dst, int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = (int8_t)__half2int_rn(__ushort_as_half(src[i]));
 }
 
 }  // namespace
+
+cudaError_t launch_codes_f16_to_i8(const uint16_t* src, int8_t* dst, int64_t n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 4096);
+    codes_f16_to_i8_kernel<<<(unsigned)blocks, 256, 0, s>>>(src, dst, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_permute(const Plan& p, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;

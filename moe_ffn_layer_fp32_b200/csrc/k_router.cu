@@ -50,12 +50,17 @@ router_quant_kernel(Plan p)
         m = warp_max(m);
         const float s = __fdiv_rn(m, 127.0f);
         const int64_t t = t0 + tt;
-        int8_t* q = p.xq + (p.Tk + t) * d;
-        for (int i = lane * 4; i < d; i += 128) {
-            uint32_t w = 0;
+        if (p.xq16) {
+            uint16_t* q = p.xq16 + (p.Tk + t) * d;
+            for (int i = lane; i < d; i += 32) q[i] = (uint16_t)code_f16(quant_i8(bf16_to_f32(row[i]), s));
+        } else {
+            int8_t* q = p.xq + (p.Tk + t) * d;
+            for (int i = lane * 4; i < d; i += 128) {
+                uint32_t w = 0;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) w |= (uint32_t)(quant_i8(bf16_to_f32(row[i + u]), s) & 0xff) << (8 * u);
-            *reinterpret_cast<uint32_t*>(q + i) = w;
+                for (int u = 0; u < 4; ++u) w |= (uint32_t)(quant_i8(bf16_to_f32(row[i + u]), s) & 0xff) << (8 * u);
+                *reinterpret_cast<uint32_t*>(q + i) = w;
+            }
         }
         if (lane == 0) {
             p.sx[t] = s;
@@ -98,8 +103,7 @@ router_quant_kernel(Plan p)
             float l = __fadd_rn(__fadd_rn(__fadd_rn(part[(0 * TB + t) * 64 + e], part[(1 * TB + t) * 64 + e]),
                                           part[(2 * TB + t) * 64 + e]),
                                 part[(3 * TB + t) * 64 + e]);
-            if (p.router_bias) l = __fadd_rn(l, p.router_bias[e]);
-            lg[i] = l;
+            lg[i] = biased_logit(p, l, e);
         }
     }
     __syncthreads();
@@ -263,24 +267,37 @@ __global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
     for (int tt = warp; tt < nt; tt += kThreads / 32) {
         const int64_t t = t0 + tt;
         float l0 = -INFINITY, l1 = -INFINITY;
-        if (lane < E) l0 = p.router_bias ? __fadd_rn(lg[tt * kLgRow + lane], p.router_bias[lane]) : lg[tt * kLgRow + lane];
-        if (lane + 32 < E)
-            l1 = p.router_bias ? __fadd_rn(lg[tt * kLgRow + lane + 32], p.router_bias[lane + 32])
-                               : lg[tt * kLgRow + lane + 32];
+        if (lane < E) l0 = biased_logit(p, lg[tt * kLgRow + lane], lane);
+        if (lane + 32 < E) l1 = biased_logit(p, lg[tt * kLgRow + lane + 32], lane + 32);
         gate_topk_warp(p, t, l0, l1, lane);
         const float s = sxs[tt];
         const uint4* xr = reinterpret_cast<const uint4*>(p.x + t * d);
-        uint2* q = reinterpret_cast<uint2*>(p.xq + (p.Tk + t) * d);
-        for (int i = lane; i < d / 8; i += 32) {
-            const uint4 v = xr[i];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o[2] = {0u, 0u};
+        if (p.xq16) {
+            // f16 codes for the kind::f16 expert GEMMs
+            uint4* q = reinterpret_cast<uint4*>(p.xq16 + (p.Tk + t) * d);
+            for (int i = lane; i < d / 8; i += 32) {
+                const uint4 v = xr[i];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint32_t bits = (w[u >> 1] >> (16 * (u & 1))) & 0xffffu;
-                o[u >> 2] |= (uint32_t)(quant_i8(bf16_to_f32(bits), s) & 0xff) << (8 * (u & 3));
+                for (int u = 0; u < 4; ++u)
+                    o[u] = code_f16(quant_i8(bf16_to_f32(w[u] & 0xffffu), s)) |
+                           (code_f16(quant_i8(bf16_to_f32(w[u] >> 16), s)) << 16);
+                q[i] = make_uint4(o[0], o[1], o[2], o[3]);
             }
-            q[i] = make_uint2(o[0], o[1]);
+        } else {
+            uint2* q = reinterpret_cast<uint2*>(p.xq + (p.Tk + t) * d);
+            for (int i = lane; i < d / 8; i += 32) {
+                const uint4 v = xr[i];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[2] = {0u, 0u};
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t bits = (w[u >> 1] >> (16 * (u & 1))) & 0xffffu;
+                    o[u >> 2] |= (uint32_t)(quant_i8(bf16_to_f32(bits), s) & 0xff) << (8 * (u & 3));
+                }
+                q[i] = make_uint2(o[0], o[1]);
+            }
         }
         if (lane == 0) {
             p.sx[t] = s;

@@ -121,12 +121,19 @@ struct mmoe_handle {
     cudaStream_t s_h2d = nullptr, s_d2h = nullptr;
     cudaEvent_t ev_start = nullptr, ev_done = nullptr;
     cudaEvent_t ev_in[kHostChunksMax] = {}, ev_out[kHostChunksMax] = {};
-    // tensor-core path: pre-tiled weights, tensor maps of xq / hq, error flag
-    bool use_tc = false;
+    // tensor-core path: kind (kTcF16, kTcI8 or kTcNone), pre-tiled weights, f16 codes, tensor maps of the
+    // activation / SwiGLU codes, error flag and the limit of the bounded waits
+    int tc_kind = kTcNone;
     uint8_t* w_gate_up_t = nullptr;
     float* s_gate_up_t = nullptr;
     uint8_t* w_down_t = nullptr;
     float* s_down_t = nullptr;
+    uint16_t* w_gate_up_f16 = nullptr;
+    uint16_t* w_down_f16 = nullptr;
+    uint16_t* xq16 = nullptr;
+    uint16_t* hq16 = nullptr;
+    long long wait_limit = kDefaultWaitLimit;
+    bool stall_next = false;   // the next prefill forward injects a stall (mmoe_debug_set_wait_limit)
     alignas(64) unsigned char tmap_xq[128] = {};
     alignas(64) unsigned char tmap_hq[128] = {};
     int* err_host = nullptr;   // mapped pinned host memory; kernels write its device alias
@@ -156,9 +163,18 @@ struct mmoe_handle {
 
 namespace {
 
+// Allocation-failure injection (mmoe_debug_fail_alloc): the number of device
+// allocations this thread may still make before one fails; -1: never.
+thread_local int64_t g_fail_alloc_after = -1;
+
 template <class T>
 cudaError_t dalloc(T** p, size_t count) {
     *p = nullptr;
+    if (g_fail_alloc_after == 0) {
+        g_fail_alloc_after = -1;
+        return cudaErrorMemoryAllocation;
+    }
+    if (g_fail_alloc_after > 0) --g_fail_alloc_after;
     if (count == 0) count = 1;
     return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
 }
@@ -169,7 +185,7 @@ void free_all(mmoe_handle* h) {
                     h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
                     h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
                     h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->amax_h, h->dec_groups,
-                    h->dec_ngroups};
+                    h->dec_ngroups, h->w_gate_up_f16, h->w_down_f16, h->xq16, h->hq16};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);
@@ -200,11 +216,13 @@ mmoe_status check_config(const mmoe_config* c) {
     if (c->group_size != kGroup) return fail(MMOE_ERR_INVALID_ARG, "group_size=%d: must be 32", c->group_size);
     if (c->max_tokens < 1 || c->max_tokens > (1 << 20))
         return fail(MMOE_ERR_INVALID_ARG, "max_tokens=%d: must be in [1, 2^20]", c->max_tokens);
-    if (c->gating != MMOE_GATE_SOFTMAX && c->gating != MMOE_GATE_SIGMOID_TOPK_NORM)
+    if (c->gating != MMOE_GATE_SOFTMAX && c->gating != MMOE_GATE_SIGMOID_TOPK_NORM &&
+        c->gating != MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS)
         return fail(MMOE_ERR_INVALID_ARG, "gating=%d: unknown", c->gating);
     if (c->has_router_bias != 0 && c->has_router_bias != 1)
         return fail(MMOE_ERR_INVALID_ARG, "has_router_bias=%d: must be 0 or 1", c->has_router_bias);
-    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE | MMOE_FLAG_ATOMIC_COMBINE))
+    if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE | MMOE_FLAG_ATOMIC_COMBINE |
+                     MMOE_FLAG_TC_INT8))
         return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
     return MMOE_OK;
 }
@@ -250,14 +268,19 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.hq = h->hq;
     p.sh = h->sh;
     p.obuf = h->obuf;
-    p.use_tc = h->use_tc;
-    p.tile_rows = p.use_tc ? kTcTileRows : kTileRows;
+    p.tc_kind = h->tc_kind;
+    p.tile_rows = p.tc_kind != kTcNone ? kTcTileRows : kTileRows;
     p.max_tiles = max_tiles_for(T, c.top_k, c.n_experts, p.tile_rows);
     p.nchunks = (int)((p.Tk + kChunk - 1) / kChunk);
     p.w_gate_up_t = h->w_gate_up_t;
     p.s_gate_up_t = h->s_gate_up_t;
     p.w_down_t = h->w_down_t;
     p.s_down_t = h->s_down_t;
+    p.w_gate_up_f16 = h->w_gate_up_f16;
+    p.w_down_f16 = h->w_down_f16;
+    p.xq16 = h->xq16;
+    p.hq16 = h->hq16;
+    p.wait_limit = h->wait_limit;
     p.tmap_xq = h->tmap_xq;
     p.tmap_hq = h->tmap_hq;
     p.err = h->err_dev;
@@ -271,11 +294,19 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
 }
 
 cudaError_t run_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t r0, int64_t nr) {
-    return p.use_tc ? launch_gate_up_tc(p, s, dump, r0, nr) : launch_gate_up(p, s, dump, r0, nr);
+    switch (p.tc_kind) {
+        case kTcF16: return launch_gate_up_f16(p, s, dump, r0, nr);
+        case kTcI8: return launch_gate_up_tc(p, s, dump, r0, nr);
+        default: return launch_gate_up(p, s, dump, r0, nr);
+    }
 }
 
 cudaError_t run_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t r0, int64_t nr) {
-    return p.use_tc ? launch_down_tc(p, s, dump, r0, nr) : launch_down(p, s, dump, r0, nr);
+    switch (p.tc_kind) {
+        case kTcF16: return launch_down_f16(p, s, dump, r0, nr);
+        case kTcI8: return launch_down_tc(p, s, dump, r0, nr);
+        default: return launch_down(p, s, dump, r0, nr);
+    }
 }
 
 // A bounded device-side wait of an earlier call gave up: report it once and
@@ -404,6 +435,27 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     h->n_d_scales = (size_t)(E * hh + hs) * d / kGroup;
     const int64_t nchunks = (Tm * k + kChunk - 1) / kChunk;
 
+    // which kernels serve this handle: the decode path for few tokens, and for prefill the kind::f16
+    // tensor-core GEMMs (default), the kind::i8 ones (MMOE_FLAG_TC_INT8, or shapes only they take) or
+    // the CUDA-core ones
+    h->use_dec = !(cfg->flags & (MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE)) && dec_supported((int)d, (int)hh, (int)hs);
+    if (h->use_dec) {
+        h->dec_max_T = dec_max_tokens((int)d, h->hmax);
+        h->dec_cluster = dec_router_cluster((int)d, (int)E);
+        if (h->dec_max_T <= 0 || h->dec_cluster == 0) h->use_dec = false;
+    }
+    if (!(cfg->flags & MMOE_FLAG_CUDA_CORES)) {
+        const bool f16ok = f16tc_supported((int)d, (int)hh, (int)hs) && router_mma_supported((int)d, (int)E);
+        const bool i8ok = tc_supported((int)d, (int)hh, (int)hs);
+        if ((cfg->flags & MMOE_FLAG_TC_INT8) && i8ok) h->tc_kind = kTcI8;
+        else if (f16ok) h->tc_kind = kTcF16;
+        else if (i8ok) h->tc_kind = kTcI8;
+    }
+    // rows of the INT8 code buffers: every row when a prefill kernel set reads them, else only the
+    // decode path's
+    const int64_t Rd = h->use_dec ? (Tm < h->dec_max_T ? Tm : h->dec_max_T) * (k + 1) : 1;
+    const int64_t R8 = h->tc_kind == kTcF16 ? Rd : R;
+
     cudaError_t e = cudaSuccess;
 #define ALLOC(ptr, n) \
     if (e == cudaSuccess) e = dalloc(&h->ptr, (size_t)(n))
@@ -414,7 +466,7 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(s_gate_up, h->n_gu_scales);
     ALLOC(w_down, h->n_d_bytes);
     ALLOC(s_down, h->n_d_scales);
-    ALLOC(xq, R * d);
+    ALLOC(xq, R8 * d);
     ALLOC(sx, Tm);
     ALLOC(logits, Tm * E);
     ALLOC(idx, Tm * k);
@@ -429,17 +481,9 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(row_gate, R);
     ALLOC(slot_row, Tm * k);
     ALLOC(act, R * h->hmax);
-    ALLOC(hq, R * h->hmax);
+    ALLOC(hq, R8 * h->hmax);
     ALLOC(sh, R);
-    h->use_tc = !(cfg->flags & MMOE_FLAG_CUDA_CORES) && tc_supported((int)d, (int)hh, (int)hs);
-    h->use_dec = !(cfg->flags & (MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE)) && dec_supported((int)d, (int)hh, (int)hs);
     if (h->use_dec) {
-        h->dec_max_T = dec_max_tokens((int)d, h->hmax);
-        h->dec_cluster = dec_router_cluster((int)d, (int)E);
-        if (h->dec_max_T <= 0 || h->dec_cluster == 0) h->use_dec = false;
-    }
-    if (h->use_dec) {
-        const int64_t Rd = (Tm < h->dec_max_T ? Tm : h->dec_max_T) * (k + 1);
         ALLOC(w_gate_up_d, h->n_gu_bytes + h->n_gu_scales * 4);
         ALLOC(w_down_d, h->n_d_bytes + h->n_d_scales * 4);
         ALLOC(amax_h, Rd);
@@ -453,7 +497,7 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
         const bool prefill_possible = !h->use_dec || Tm > h->dec_max_T;
         if (det || (prefill_possible && !(cfg->flags & MMOE_FLAG_ATOMIC_COMBINE))) ALLOC(obuf, R * d);
     }
-    if (h->use_tc || h->use_dec) {
+    if (h->tc_kind != kTcNone || h->use_dec) {
         ALLOC(err_dev, 1);
         if (e == cudaSuccess) e = cudaMemset(h->err_dev, 0, sizeof(int));
         if (e == cudaSuccess) e = cudaHostAlloc(reinterpret_cast<void**>(&h->err_host), sizeof(int), cudaHostAllocMapped);
@@ -462,13 +506,24 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
             e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->err_host_dev), h->err_host, 0);
         }
     }
-    if (h->use_tc) {
+    if (h->tc_kind == kTcF16) {
+        ALLOC(w_gate_up_f16, f16tc_image_elems((int)d, (int)hh, (int)hs, (int)E, true));
+        ALLOC(s_gate_up_t, h->n_gu_scales);
+        ALLOC(w_down_f16, f16tc_image_elems((int)d, (int)hh, (int)hs, (int)E, false));
+        ALLOC(s_down_t, h->n_d_scales);
+        ALLOC(xq16, R * d);
+        ALLOC(hq16, R * h->hmax);
+        if (e == cudaSuccess) e = make_tensor_map(h->tmap_xq, h->xq16, (uint64_t)d, (uint64_t)R, (uint64_t)d * 2, 2);
+        if (e == cudaSuccess)
+            e = make_tensor_map(h->tmap_hq, h->hq16, (uint64_t)h->hmax, (uint64_t)R, (uint64_t)h->hmax * 2, 2);
+    } else if (h->tc_kind == kTcI8) {
         ALLOC(w_gate_up_t, 2 * h->n_gu_bytes);  // INT8 stage images: twice the packed INT4 bytes
         ALLOC(s_gate_up_t, h->n_gu_scales);
         ALLOC(w_down_t, 2 * h->n_d_bytes);
         ALLOC(s_down_t, h->n_d_scales);
-        if (e == cudaSuccess) e = make_tensor_map(h->tmap_xq, h->xq, (uint64_t)d, (uint64_t)R, (uint64_t)d);
-        if (e == cudaSuccess) e = make_tensor_map(h->tmap_hq, h->hq, (uint64_t)h->hmax, (uint64_t)R, (uint64_t)h->hmax);
+        if (e == cudaSuccess) e = make_tensor_map(h->tmap_xq, h->xq, (uint64_t)d, (uint64_t)R, (uint64_t)d, 1);
+        if (e == cudaSuccess)
+            e = make_tensor_map(h->tmap_hq, h->hq, (uint64_t)h->hmax, (uint64_t)R, (uint64_t)h->hmax, 1);
     }
 #undef ALLOC
     if (e != cudaSuccess) {
@@ -502,7 +557,12 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
     MMOE_CUDA(cudaMemcpyAsync(h->s_gate_up, w->s_gate_up, h->n_gu_scales * sizeof(float), kind, s), "copy s_gate_up");
     MMOE_CUDA(cudaMemcpyAsync(h->w_down, w->w_down, h->n_d_bytes, kind, s), "copy w_down");
     MMOE_CUDA(cudaMemcpyAsync(h->s_down, w->s_down, h->n_d_scales * sizeof(float), kind, s), "copy s_down");
-    if (h->use_tc)
+    if (h->tc_kind == kTcF16)
+        MMOE_CUDA(launch_retile_f16(h->w_gate_up, h->s_gate_up, h->w_down, h->s_down, h->w_gate_up_f16,
+                                    h->s_gate_up_t, h->w_down_f16, h->s_down_t, h->cfg.d_model, h->cfg.expert_hidden,
+                                    h->cfg.shared_hidden, h->cfg.n_experts, s),
+                  "weight re-tiling launch");
+    if (h->tc_kind == kTcI8)
         MMOE_CUDA(launch_retile(h->w_gate_up, h->s_gate_up, h->w_down, h->s_down, h->w_gate_up_t, h->s_gate_up_t,
                                 h->w_down_t, h->s_down_t, h->cfg.d_model, h->cfg.expert_hidden, h->cfg.shared_hidden,
                                 h->cfg.n_experts, s),
@@ -532,6 +592,11 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     if (fst != MMOE_OK) return fst;
     const bool dec = h->use_dec && T <= h->dec_max_T;
     Plan p = make_plan(h, x, T, y);
+    if (dec) {
+        // the decode kernels work on the INT8 code buffers
+        p.xq16 = nullptr;
+        p.hq16 = nullptr;
+    }
     // fixed-order combine: always in deterministic mode; on the prefill path unless atomics were asked for
     p.deterministic = (h->cfg.flags & MMOE_FLAG_DETERMINISTIC) ||
                       (!dec && !(h->cfg.flags & MMOE_FLAG_ATOMIC_COMBINE));
@@ -552,8 +617,11 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
         MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_quant(p, s); }),
                   "router/quantiser launch");
         MMOE_CUDA(run_stage(h, MMOE_PROF_PERMUTE, 4, s, [&] { return launch_permute(p, s); }), "permute launch");
+        p.debug_stall = h->stall_next && p.tc_kind == kTcF16 ? 1 : 0;
+        h->stall_next = false;
         MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return run_gate_up(p, s, nullptr, 0, 0); }),
                   "gate/up launch");
+        p.debug_stall = 0;
         MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
         MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return run_down(p, s, nullptr, 0, 0); }), "down launch");
     }
@@ -738,8 +806,14 @@ mmoe_status mmoe_debug_copy_stage(mmoe_handle* h, int32_t stage, void* dst, size
     }
     if (bytes > have) return fail(MMOE_ERR_INVALID_ARG, "stage %d holds %zu bytes, asked for %zu", stage, have, bytes);
     DeviceGuard dg(h->device);
-    MMOE_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, reinterpret_cast<cudaStream_t>(stream)),
-              "copy stage");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!h->last_dec && h->tc_kind == kTcF16 && (stage == MMOE_STAGE_XQ || stage == MMOE_STAGE_HQ)) {
+        // the kind::f16 path keeps these codes as f16: converted to INT8 on the way out
+        const uint16_t* src16 = stage == MMOE_STAGE_XQ ? h->xq16 + T * k * d : h->hq16;
+        MMOE_CUDA(launch_codes_f16_to_i8(src16, static_cast<int8_t*>(dst), (int64_t)bytes, s), "code conversion");
+        return MMOE_OK;
+    }
+    MMOE_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s), "copy stage");
     return MMOE_OK;
 }
 
@@ -757,12 +831,32 @@ mmoe_status mmoe_debug_partials(mmoe_handle* h, int32_t which, int64_t row0, int
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Plan p = make_plan(h, nullptr, h->last_T, nullptr);
     if (h->last_dec) {
-        if (which == 0) MMOE_CUDA(launch_gate_up_dec(p, s, dst, row0, nrows), "gate/up dump launch");
-        else MMOE_CUDA(launch_down_dec(p, s, dst, row0, nrows), "down dump launch");
+        Plan pd = p;
+        pd.xq16 = nullptr;
+        pd.hq16 = nullptr;
+        if (which == 0) MMOE_CUDA(launch_gate_up_dec(pd, s, dst, row0, nrows), "gate/up dump launch");
+        else MMOE_CUDA(launch_down_dec(pd, s, dst, row0, nrows), "down dump launch");
     } else {
         if (which == 0) MMOE_CUDA(run_gate_up(p, s, dst, row0, nrows), "gate/up dump launch");
         else MMOE_CUDA(run_down(p, s, dst, row0, nrows), "down dump launch");
     }
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_debug_fail_alloc(int64_t after) {
+    if (after < -1) return fail(MMOE_ERR_INVALID_ARG, "after=%lld: must be >= -1", (long long)after);
+    g_fail_alloc_after = after;
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_debug_set_wait_limit(mmoe_handle* h, int64_t clocks, int32_t stall_next) {
+    if (!h) return fail(MMOE_ERR_INVALID_ARG, "handle is NULL");
+    if (clocks < 0) return fail(MMOE_ERR_INVALID_ARG, "clocks=%lld: must be >= 0", (long long)clocks);
+    if (stall_next != 0 && stall_next != 1) return fail(MMOE_ERR_INVALID_ARG, "stall_next=%d: must be 0 or 1", stall_next);
+    if (stall_next && h->tc_kind != kTcF16)
+        return fail(MMOE_ERR_UNIMPLEMENTED, "an injected stall needs the kind::f16 tensor-core GEMMs on this handle");
+    h->wait_limit = clocks == 0 ? kDefaultWaitLimit : clocks;
+    h->stall_next = stall_next != 0;
     return MMOE_OK;
 }
 
@@ -813,7 +907,14 @@ mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weigh
     if (w->on_device != 1) return fail(MMOE_ERR_INVALID_ARG, "weights must be device pointers (on_device = 1)");
     if (cfg->has_router_bias && !w->router_bias)
         return fail(MMOE_ERR_INVALID_ARG, "the config has a router bias but router_bias is NULL");
-    if (T < 0) return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be >= 0", (long long)T);
+    // the weights are read in place by kernels that load the packed codes 16 bytes and the FP32
+    // arrays 4 bytes at a time
+    if ((reinterpret_cast<uintptr_t>(w->w_gate_up) | reinterpret_cast<uintptr_t>(w->w_down)) & 15)
+        return fail(MMOE_ERR_INVALID_ARG, "w_gate_up and w_down must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(w->w_router) | reinterpret_cast<uintptr_t>(w->router_bias) |
+         reinterpret_cast<uintptr_t>(w->s_gate_up) | reinterpret_cast<uintptr_t>(w->s_down)) & 3)
+        return fail(MMOE_ERR_INVALID_ARG, "w_router, router_bias, s_gate_up and s_down must be 4-byte aligned");
+    if (T < 0 || T > (1 << 20)) return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be in [0, 2^20]", (long long)T);
     if (T == 0) return MMOE_OK;
     if (!x || !y) return fail(MMOE_ERR_INVALID_ARG, "x or y is NULL");
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15)
@@ -830,7 +931,8 @@ mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weigh
     p.T = T;
     p.Tk = T * p.k;
     p.R = T * (p.k + 1);
-    p.deterministic = (cfg->flags & MMOE_FLAG_DETERMINISTIC) != 0;
+    // fixed-order combine unless atomics were asked for (as on mmoe_forward's prefill path)
+    p.deterministic = (cfg->flags & MMOE_FLAG_DETERMINISTIC) || !(cfg->flags & MMOE_FLAG_ATOMIC_COMBINE);
     p.w_router = w->w_router;
     p.router_bias = cfg->has_router_bias ? w->router_bias : nullptr;
     p.w_gate_up = w->w_gate_up;
@@ -839,7 +941,7 @@ mmoe_status mmoe_forward_static_scratch(const mmoe_config* cfg, const mmoe_weigh
     p.s_down = w->s_down;
     p.x = x;
     p.y = y;
-    p.use_tc = false;
+    p.tc_kind = kTcNone;
     p.tile_rows = kTileRows;
     p.max_tiles = max_tiles_for(T, p.k, p.E, p.tile_rows);
     p.nchunks = (int)((p.Tk + kChunk - 1) / kChunk);

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "mmoe.h"
@@ -15,6 +16,8 @@ constexpr int kMaxTopK = 8;
 constexpr int kChunk = 1024;        // routing slots per permutation block
 constexpr int kTileRows = 32;       // rows (token slots) per CUDA-core expert-GEMM tile
 constexpr int kTcTileRows = 128;    // rows per tensor-core expert-GEMM tile
+constexpr int kTcNone = 0, kTcF16 = 1, kTcI8 = 2;  // Plan::tc_kind
+constexpr long long kDefaultWaitLimit = 4000000000ll;  // about 2 s of SM clock
 
 // Everything a forward pass needs, as plain device pointers.
 struct Plan {
@@ -54,14 +57,21 @@ struct Plan {
     int64_t max_tiles;
     int nchunks;
     int tile_rows;          // kTileRows (CUDA-core GEMMs) or kTcTileRows (tensor-core GEMMs)
-    // tensor-core path
-    bool use_tc;
-    const uint8_t* w_gate_up_t;   // pre-tiled weights (tensor-core layout)
-    const float* s_gate_up_t;
+    // tensor-core path: kTcNone (CUDA-core GEMMs), kTcF16 (kind::f16, exact integer partials, the
+    // default) or kTcI8 (kind::i8, S32 partials)
+    int tc_kind;
+    const uint8_t* w_gate_up_t;   // kTcI8: INT8 stage images
+    const float* s_gate_up_t;     // pre-tiled group scales (both tensor-core kinds)
     const uint8_t* w_down_t;
     const float* s_down_t;
-    const void* tmap_xq;          // host pointers to CUtensorMap of xq and hq (128B-swizzled 128 x 128 boxes)
+    const uint16_t* w_gate_up_f16;  // kTcF16: f16 stage images
+    const uint16_t* w_down_f16;
+    uint16_t* xq16;               // kTcF16: [R, d] activation codes as f16 (replaces xq on that path)
+    uint16_t* hq16;               // kTcF16: [R, hmax] SwiGLU codes as f16 (replaces hq on that path)
+    const void* tmap_xq;          // host pointers to CUtensorMap of the activation and SwiGLU codes
     const void* tmap_hq;
+    long long wait_limit;         // SM clocks a bounded wait of the kind::f16 GEMMs lasts before giving up
+    int debug_stall;              // 1: the kind::f16 gate/up GEMM injects a stall (failure-detection tests)
     int* err;                     // device flag: a bounded wait gave up (later CTAs exit at once)
     int* err_host;                // device alias of the host-mapped copy of that flag
     // decode path (k_decode.cu)
@@ -88,7 +98,17 @@ cudaError_t launch_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t
 cudaError_t launch_requant(const Plan& p, cudaStream_t s);
 cudaError_t launch_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_combine(const Plan& p, cudaStream_t s);
-// tensor-core path (k_expert_tc.cu)
+// tensor-core path, kind::f16 (k_expert_f16.cu)
+bool f16tc_supported(int d, int h, int hs);
+size_t f16tc_image_elems(int d, int h, int hs, int E, bool gate_up);
+cudaError_t launch_gate_up_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
+cudaError_t launch_down_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
+cudaError_t launch_retile_f16(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
+                              uint16_t* gu_t, float* sgu_t, uint16_t* dn_t, float* sdn_t, int d, int h, int hs, int E,
+                              cudaStream_t s);
+// f16 codes (integers in [-127, 127]) -> INT8 codes, for the inspection entry point
+cudaError_t launch_codes_f16_to_i8(const uint16_t* src, int8_t* dst, int64_t n, cudaStream_t s);
+// tensor-core path, kind::i8 (k_expert_tc.cu)
 bool tc_supported(int d, int h, int hs);
 cudaError_t launch_gate_up_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_down_tc(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
@@ -104,7 +124,10 @@ cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_
 cudaError_t launch_retile_dec(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
                               uint8_t* gu_d, uint8_t* dn_d, int d, int h, int hs, int E, cudaStream_t s);
 size_t tensor_map_bytes();
-cudaError_t make_tensor_map(void* map, void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_stride);
+// 2-D tensor map of a row-major [rows, inner] matrix of 1- or 2-byte elements, 128-byte swizzle,
+// boxes of 128 bytes x 128 rows
+cudaError_t make_tensor_map(void* map, void* base, uint64_t inner_elems, uint64_t rows, uint64_t row_stride_bytes,
+                            int elem_bytes);
 cudaError_t launch_quantize_int4(const float* w, int64_t rows, int64_t K, uint8_t* packed, float* scales,
                                  cudaStream_t s);
 
@@ -155,6 +178,9 @@ __device__ __forceinline__ void router_kstep(float (&acc)[4], uint32_t a0, uint3
 
 __device__ __forceinline__ float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
+// f16 bit pattern of an integer code in [-2048, 2048] (exact)
+__device__ __forceinline__ uint32_t code_f16(int q) { return (uint32_t)__half_as_ushort(__int2half_rn(q)); }
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -176,9 +202,12 @@ __device__ __forceinline__ int quant_i8(float v, float s) {
 }
 
 // Gating and top-k of token t by one warp.  Lane l holds the logits of
-// experts l and l + 32 (-inf where the expert does not exist).  Softmax over
+// experts l and l + 32 (-inf where the expert does not exist); the router bias
+// is already in them for gating 0 and 1 and not for gating 2.  Softmax over
 // all experts (or per-expert sigmoid), then k rounds of a warp arg-max on
-// (logit descending, index ascending); writes logits (if kept), idx and gate.
+// (key descending, index ascending), the key being the logit, or for gating 2
+// the sigmoid score plus the bias (which then moves the selection but enters
+// no gate); writes logits (if kept), idx and gate.
 __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane) {
     const int E = p.E, k = p.k;
     const bool v0 = lane < E, v1 = lane + 32 < E;
@@ -198,16 +227,21 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
         p0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l0)));
         p1 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l1)));
     }
+    float k0 = l0, k1 = l1;
+    if (p.gating == MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS) {
+        k0 = v0 ? (p.router_bias ? __fadd_rn(p0, p.router_bias[lane]) : p0) : -INFINITY;
+        k1 = v1 ? (p.router_bias ? __fadd_rn(p1, p.router_bias[lane + 32]) : p1) : -INFINITY;
+    }
     bool taken0 = !v0, taken1 = !v1;
     int sel[kMaxTopK];
     float gsel[kMaxTopK];
     float gsum = 0.0f;
     for (int j = 0; j < k; ++j) {
-        // this lane's best untaken candidate, then a warp arg-max on (logit desc, index asc)
+        // this lane's best untaken candidate, then a warp arg-max on (key desc, index asc)
         float bv = -INFINITY;
         int bi = 1 << 30;
-        if (!taken0) { bv = l0; bi = lane; }
-        if (!taken1 && (l1 > bv || bi == (1 << 30))) { bv = l1; bi = lane + 32; }
+        if (!taken0) { bv = k0; bi = lane; }
+        if (!taken1 && (k1 > bv || bi == (1 << 30))) { bv = k1; bi = lane + 32; }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -230,6 +264,11 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
         p.idx[t * k + lane] = my;
         p.gate[t * k + lane] = g;
     }
+}
+
+// The router bias enters the logit for gating 0 and 1 (and only the selection key for gating 2).
+__device__ __forceinline__ float biased_logit(const Plan& p, float l, int e) {
+    return (p.router_bias && p.gating != MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS) ? __fadd_rn(l, p.router_bias[e]) : l;
 }
 
 }  // namespace mmoe

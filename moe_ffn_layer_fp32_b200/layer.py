@@ -57,13 +57,15 @@ class MoELayer:
     def __init__(self, d_model: int, expert_hidden: int, *, shared_hidden: int | None = None,
                  n_experts: int = 60, top_k: int = 4, max_tokens: int = 4096, gating: int = 0,
                  has_router_bias: bool = False, deterministic: bool = False, cuda_cores: bool = False,
-                 decode: bool = True, atomic_combine: bool = False, device: int = 0):
+                 decode: bool = True, atomic_combine: bool = False, tc_int8: bool = False, device: int = 0):
         """decode=False keeps small batches (T <= 64) on the prefill kernels instead of the
         weight-streaming decode kernels; cuda_cores=True runs every expert GEMM on CUDA cores;
-        atomic_combine=True adds the prefill expert outputs into y with atomics (no [R, d] workspace);
-        deterministic=True uses the fixed-order combine on the decode path too."""
+        tc_int8=True runs the prefill expert GEMMs on the kind::i8 tensor-core kernels instead of the
+        default kind::f16 ones; atomic_combine=True adds the prefill expert outputs into y with atomics
+        (no [R, d] workspace); deterministic=True uses the fixed-order combine on the decode path too."""
         flags = ((_lib.FLAG_DETERMINISTIC if deterministic else 0) | (_lib.FLAG_CUDA_CORES if cuda_cores else 0)
-                 | (0 if decode else _lib.FLAG_NO_DECODE) | (_lib.FLAG_ATOMIC_COMBINE if atomic_combine else 0))
+                 | (0 if decode else _lib.FLAG_NO_DECODE) | (_lib.FLAG_ATOMIC_COMBINE if atomic_combine else 0)
+                 | (_lib.FLAG_TC_INT8 if tc_int8 else 0))
         self.cfg = _lib.Config(d_model, n_experts, top_k, expert_hidden,
                                expert_hidden if shared_hidden is None else shared_hidden, GROUP, max_tokens,
                                gating, int(has_router_bias), flags)
@@ -118,6 +120,11 @@ class MoELayer:
             y = np.empty((T, self.cfg.d_model), dtype=np.float32)
         check(lib().mmoe_forward_host(self._h, _ptr(x), T, _ptr(y), _stream_ptr(stream)))
         return y
+
+    def set_wait_limit(self, clocks: int, stall_next: bool = False) -> None:
+        """SM clocks a bounded wait of the prefill tensor-core GEMMs lasts before giving up (0: default);
+        stall_next=True makes the next prefill forward stall on purpose (failure-detection tests)."""
+        check(lib().mmoe_debug_set_wait_limit(self._h, int(clocks), 1 if stall_next else 0))
 
     def profile(self, enable: bool) -> None:
         """Start (and clear) or stop per-stage event timing of the following forwards."""

@@ -42,6 +42,7 @@ def main(argv=None) -> int:
     ap.add_argument("--no-decode", action="store_true", help="keep T <= 64 on the prefill kernels")
     ap.add_argument("--cuda-cores", action="store_true")
     ap.add_argument("--deterministic", action="store_true")
+    ap.add_argument("--tc-int8", action="store_true", help="prefill GEMMs on the kind::i8 tensor-core kernels")
     args = ap.parse_args(argv)
 
     dev = torch.device("cuda", 0)
@@ -50,7 +51,7 @@ def main(argv=None) -> int:
     tensors, lw = quantized_weights(w, dev)
     L = MoELayer(w.d, w.h, shared_hidden=w.hs, n_experts=w.E, top_k=w.k, max_tokens=T,
                  has_router_bias=lw.router_bias is not None, decode=not args.no_decode,
-                 cuda_cores=args.cuda_cores, deterministic=args.deterministic)
+                 cuda_cores=args.cuda_cores, deterministic=args.deterministic, tc_int8=args.tc_int8)
     L.load(*tensors)
     del tensors
     x = torch.from_numpy(synth.workload_x(w, T=T).view(np.int16)).to(dev).view(torch.bfloat16)

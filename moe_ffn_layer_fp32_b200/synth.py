@@ -71,6 +71,12 @@ WORKLOADS: dict[str, Workload] = {
                    desc="large prefill: 4 x 8192 = 32768 tokens, d_model=2048, h=1024"),
     "c4dec": Workload("c4dec", T=64, d=2048, h=1024, x_seed=2,
                       desc="batched decode: T=64 on the d_model=2048, h=1024 weights"),
+    # The MobileMoE-S layer shape: 60 routed SwiGLU experts of 768 x 384 and one
+    # shared expert four times a routed one (hidden 1536), top-4.
+    "s2048": Workload("s2048", T=2048, d=768, h=384, shared_hidden=1536, weight_seed=3, x_seed=4,
+                      desc="MobileMoE-S layer, prefill: T=2048, d_model=768, h=384, shared hidden 1536"),
+    "s1": Workload("s1", T=1, d=768, h=384, shared_hidden=1536, layers=24, weight_seed=2000, x_seed=3 * 10**6,
+                   desc="MobileMoE-S layer, decode: T=1, d_model=768, h=384, shared hidden 1536, 24 layers"),
 }
 
 

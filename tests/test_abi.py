@@ -41,7 +41,7 @@ def valid_cfg(**kw):
 @pytest.mark.parametrize("kw", [dict(d_model=250), dict(d_model=32), dict(n_experts=0), dict(n_experts=65),
                                 dict(top_k=0), dict(top_k=9), dict(n_experts=3, top_k=4),
                                 dict(expert_hidden=100), dict(shared_hidden=0), dict(group_size=64),
-                                dict(max_tokens=0), dict(gating=2), dict(has_router_bias=2), dict(flags=16),
+                                dict(max_tokens=0), dict(gating=3), dict(has_router_bias=2), dict(flags=32),
                                 dict(flags=0x80000000)])
 def test_create_rejects_bad_config(L, kw):
     h = C.c_void_p()
@@ -92,6 +92,36 @@ def test_static_scratch_forward_validates_before_any_device_work(L):
     assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, -1, fake, None) == 1
     assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, 0, fake, None) == 0
     assert L.mmoe_forward_static_scratch(None, C.byref(w), fake, 1, fake, None) == 1
+    # more than 2^20 tokens: rejected before the scratch size is worked out
+    assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, (1 << 20) + 1, fake, None) == 1
+    assert b"2^20" in L.mmoe_last_error()
+
+
+@pytest.mark.parametrize("field,offset,msg", [("w_gate_up", 8, b"16-byte"), ("w_down", 4, b"16-byte"),
+                                              ("w_router", 2, b"4-byte"), ("router_bias", 1, b"4-byte"),
+                                              ("s_gate_up", 2, b"4-byte"), ("s_down", 3, b"4-byte")])
+def test_static_scratch_rejects_misaligned_weights(L, field, offset, msg):
+    # the weights are read in place with vector loads: a misaligned slice of a caller's pool is an
+    # argument error, found before anything is launched (no device is needed to see it)
+    cfg = valid_cfg(has_router_bias=1)
+    ptrs = {f: 0x10000 + 0x1000 * i for i, f in enumerate(("w_router", "router_bias", "w_gate_up", "s_gate_up",
+                                                            "w_down", "s_down"))}
+    ptrs[field] += offset
+    w = _lib.Weights(*[C.c_void_p(ptrs[f]) for f in ("w_router", "router_bias", "w_gate_up", "s_gate_up",
+                                                     "w_down", "s_down")], 1)
+    fake = C.c_void_p(0x1000)
+    assert L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(w), fake, 1, fake, None) == 1
+    assert msg in L.mmoe_last_error()
+
+
+def test_failure_injection_entry_points_validate(L):
+    # the allocation-failure and stall hooks of the failure-detection tests: arguments checked
+    # without a device; an armed allocation hook that never fires is turned off again
+    assert L.mmoe_debug_fail_alloc(-2) == 1
+    assert L.mmoe_debug_fail_alloc(3) == 0
+    assert L.mmoe_debug_fail_alloc(-1) == 0
+    assert L.mmoe_debug_set_wait_limit(None, 100, 1) == 1
+    assert b"NULL" in L.mmoe_last_error()
 
 
 def host_chunks(L, T, cap=8):

@@ -54,15 +54,15 @@ def test_quantizer_matches_oracle_bit_exact():
 
 
 def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False, decode=True,
-                atomic_combine=False):
+                atomic_combine=False, tc_int8=False):
     T = x.shape[0]
     L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic, cuda_cores=cuda_cores,
-                          decode=decode, atomic_combine=atomic_combine)
+                          decode=decode, atomic_combine=atomic_combine, tc_int8=tc_int8)
     out = gu.run_gpu(L, q, x)
     y, D = oracle.moe_layer(q, x, dumps=True)
     rep = {}
     assert np.array_equal(out["xq"], D["xq"]) and np.array_equal(out["sx"].view(np.uint32), D["sx"].view(np.uint32))
-    assert np.max(np.abs(out["logits"] - D["logits"])) <= 1e-5 * max(1.0, np.abs(D["logits"]).max())
+    assert np.max(np.abs(out["logits"] - D["logits"])) <= gu.LOGIT_TOL * max(1.0, np.abs(D["logits"]).max())
     gu.check_routing_and_permutation(q, out, D["idx"], D["gate"], D["probs"], rep, D["logits"])
     gu.check_hq(q, out, D, rep)
     gu.check_y(out["y"], y, rep)
@@ -72,17 +72,18 @@ def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, c
     return rep, out
 
 
-@pytest.mark.parametrize("path", ["decode", "tensor_cores", "cuda_cores"])
+@pytest.mark.parametrize("path", ["decode", "tensor_cores", "tensor_cores_i8", "cuda_cores"])
 @pytest.mark.parametrize("combine", ["atomic", "fixed_order"])
 def test_c0_all_stages(combine, path):
-    # T = 64 takes the decode kernels by default; the other two force the prefill kernels.
+    # T = 64 takes the decode kernels by default; the others force the prefill kernels: the
+    # kind::f16 tensor-core GEMMs (default), the kind::i8 ones, or the CUDA-core ones.
     # atomic: the decode path's default, forced on the prefill path; fixed_order: forced on the decode path
     w, q = workload("c0")
     x = synth.workload_x(w)
     R = w.T * (q.k + 1)
     rep, out = _full_check(q, x, combine == "fixed_order", partial_rows=range(0, R, 3),
                            cuda_cores=path == "cuda_cores", decode=path == "decode",
-                           atomic_combine=combine == "atomic")
+                           atomic_combine=combine == "atomic", tc_int8=path == "tensor_cores_i8")
     print("c0", path, rep)
 
 
@@ -184,6 +185,71 @@ def test_sigmoid_topk_normalised_gating():
     assert np.allclose(out["gate"].sum(axis=1), 1.0, atol=1e-6)
 
 
+@pytest.mark.parametrize("decode,T", [(True, 64), (False, 200)], ids=["decode", "prefill"])
+def test_selection_only_bias_gating(decode, T):
+    # gating 2: the router bias (auxiliary-loss-free balancing) moves the top-k of the sigmoid
+    # scores and enters no gate; the gates of a token sum to one
+    w = synth.WORKLOADS["c0"]
+    lw = synth.draw_layer(w.d, w.h, seed=60, bias_coef=0.25)
+    q = oracle.quantize_layer(lw, gating=2)
+    x = synth.draw_x(T, w.d, seed=61)
+    R = T * (q.k + 1)
+    rep, out = _full_check(q, x, decode=decode, partial_rows=[0, T * q.k - 1, T * q.k, R - 1])
+    assert np.allclose(out["gate"].sum(axis=1), 1.0, atol=1e-6)
+    print("selection bias", "decode" if decode else "prefill", rep)
+
+
+def _group_edge_rows(out, E):
+    """First and last row of every group that has rows (the shared group included)."""
+    off = out["offsets"]
+    rows = []
+    for g in range(E + 1):
+        if off[g + 1] > off[g]:
+            rows += [int(off[g]), int(off[g + 1]) - 1]
+    return sorted(set(rows))
+
+
+@pytest.mark.parametrize("decode,T", [(True, 1), (True, 8), (True, 64), (False, 300)],
+                         ids=["decode1", "decode8", "decode64", "prefill300"])
+def test_mobilemoe_s_shape(decode, T):
+    # the MobileMoE-S layer: d_model 768, 60 experts of hidden 384, shared expert hidden 1536 (4x)
+    w, q = workload("s2048")
+    x = synth.workload_x(w, T=T)
+    L = gu.make_gpu_layer(q, max(T, 1), decode=decode)
+    out = gu.run_gpu(L, q, x)
+    y, D = oracle.moe_layer(q, x, dumps=True)
+    rep = {}
+    assert np.array_equal(out["xq"], D["xq"])
+    gu.check_routing_and_permutation(q, out, D["idx"], D["gate"], D["probs"], rep, D["logits"])
+    gu.check_hq(q, out, D, rep)
+    gu.check_y(out["y"], y, rep)
+    gu.check_partials(L, q, out, _group_edge_rows(out, q.E))
+    L.close()
+    print("s shape", T, rep)
+
+
+def test_mobilemoe_s_prefill_2048():
+    w, q = workload("s2048")
+    x = synth.workload_x(w)
+    L = gu.make_gpu_layer(q, w.T)
+    out = gu.run_gpu(L, q, x)
+    y, D = oracle.moe_layer(q, x, dumps=True)
+    rep = {}
+    gu.check_routing_and_permutation(q, out, D["idx"], D["gate"], D["probs"], rep, D["logits"])
+    gu.check_hq(q, out, D, rep)
+    gu.check_y(out["y"], y, rep)
+    gu.check_partials(L, q, out, _group_edge_rows(out, q.E))
+    L.close()
+    print("s2048", rep)
+
+
+def test_c2_prefill_int8_tensor_cores():
+    # the kind::i8 GEMMs (MMOE_FLAG_TC_INT8) on the balanced prefill workload
+    w, q = workload("c2")
+    x = synth.workload_x(w, T=1024)
+    rep, out = _full_check(q, x, tc_int8=True, partial_rows=[0, 4095, 4096, 5119])
+
+
 def test_shared_expert_wider_than_routed():
     # MobileMoE's shared expert is 4x a routed expert (final-architecture paragraph)
     lw = synth.draw_layer(256, 64, seed=42, shared_hidden=256)
@@ -260,7 +326,10 @@ def test_c2_prefill():
     print("c2", rep)
 
 
-def _sampled_check(name, n_sample=192, T=None):
+def _sampled_check(name, n_sample=1024, T=None):
+    # full-size workloads: routing, permutation and activation codes on every token, y on
+    # n_sample seeded tokens (plus the first and the last), the INT32 partials of the first and
+    # last row of every group that has rows (hot and cold groups alike)
     w, q = workload(name)
     T = w.T if T is None else T
     x = synth.workload_x(w, T=T)
@@ -268,7 +337,7 @@ def _sampled_check(name, n_sample=192, T=None):
     out = gu.run_gpu(L, q, x)
     rep = {}
     logits, probs, idx, gate = oracle.router(q, x)
-    assert np.max(np.abs(out["logits"] - logits)) <= 1e-5 * max(1.0, np.abs(logits).max())
+    assert np.max(np.abs(out["logits"] - logits)) <= gu.LOGIT_TOL * max(1.0, np.abs(logits).max())
     gu.check_routing_and_permutation(q, out, idx, gate, probs, rep, logits)
     xq, sx = oracle.quantize_act(x)
     assert np.array_equal(out["xq"], xq) and np.array_equal(out["sx"], sx)
@@ -276,8 +345,9 @@ def _sampled_check(name, n_sample=192, T=None):
     toks = np.unique(np.concatenate([rng.choice(T, size=min(n_sample, T), replace=False), [0, T - 1]]))
     yref = oracle.moe_tokens(q, x, toks)
     gu.check_y(out["y"], yref, rep, rows=toks)
-    R = T * (q.k + 1)
-    gu.check_partials(L, q, out, [0, R // 3, T * q.k - 1, T * q.k, R - 1])
+    rows = _group_edge_rows(out, q.E)
+    rep["partial_rows"] = len(rows)
+    gu.check_partials(L, q, out, rows)
     L.close()
     return rep, out
 

@@ -40,8 +40,17 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-@pytest.mark.parametrize("name,deterministic", [("c0", False), ("c4dec", False), ("c4dec", True)])
-def test_static_scratch_forward_matches_mmoe_forward(name, deterministic):
+def _static_call(L, cfg, wts, x, T, d, dev):
+    y = torch.full((T, d), float("nan"), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    _lib.check(L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(wts), x.data_ptr(), T, y.data_ptr(), stream))
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("name,flags", [("c0", 0), ("c4dec", 0), ("c4dec", _lib.FLAG_DETERMINISTIC),
+                                        ("c4dec", _lib.FLAG_ATOMIC_COMBINE)])
+def test_static_scratch_forward_matches_mmoe_forward(name, flags):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     build.build()
@@ -53,28 +62,59 @@ def test_static_scratch_forward_matches_mmoe_forward(name, deterministic):
     x = torch.from_numpy(synth.workload_x(w).view(np.int16)).to(dev).view(torch.bfloat16)
     T = x.shape[0]
 
-    ref_layer = MoELayer(w.d, w.h, shared_hidden=w.hs, max_tokens=T, deterministic=deterministic,
-                         has_router_bias=tensors[1] is not None)
+    ref_layer = MoELayer(w.d, w.h, shared_hidden=w.hs, max_tokens=T,
+                         deterministic=bool(flags & _lib.FLAG_DETERMINISTIC), has_router_bias=tensors[1] is not None)
     ref_layer.load(*tensors)
     y_ref = ref_layer.forward(x)
     torch.cuda.synchronize()
 
-    cfg = _lib.Config(w.d, w.E, w.k, w.h, w.hs, 32, T, 0, int(tensors[1] is not None),
-                      _lib.FLAG_DETERMINISTIC if deterministic else 0)
+    cfg = _lib.Config(w.d, w.E, w.k, w.h, w.hs, 32, T, 0, int(tensors[1] is not None), flags)
     wts = _lib.Weights(*[_ptr(t) for t in tensors], 1)
-    stream = torch.cuda.current_stream(dev).cuda_stream
     scale = y_ref.abs().max().item()
     outs = []
     for _ in range(2):
-        y = torch.full((T, w.d), float("nan"), dtype=torch.float32, device=dev)
-        _lib.check(L.mmoe_forward_static_scratch(C.byref(cfg), C.byref(wts), x.data_ptr(), T, y.data_ptr(), stream))
-        torch.cuda.synchronize()
+        y = _static_call(L, cfg, wts, x, T, w.d, dev)
         err = (y - y_ref).abs().max().item()
         assert err <= Y_TOL * scale, (err, scale)
         outs.append(y)
     assert (outs[0] - outs[1]).abs().max().item() <= Y_TOL * scale
-    if deterministic:
+    if not flags & _lib.FLAG_ATOMIC_COMBINE:
+        # the fixed-order combine (the default) makes y bit-reproducible from call to call
         assert torch.equal(outs[0], outs[1])
+    ref_layer.close()
+
+
+@pytest.mark.parametrize("name,sizes,flags", [("c4dec", (64, 100, 64), 0),
+                                              ("c4dec", (64, 200, 64), _lib.FLAG_ATOMIC_COMBINE),
+                                              ("c3b", (37, 100, 37), 0)])
+def test_static_scratch_calls_of_changing_size(name, sizes, flags):
+    # A larger call moves every buffer inside the shared array; the smaller call after it finds
+    # the larger call's data where its own buffers now lie.  Each call must still match
+    # mmoe_forward on the same tokens.  c3b carries a per-expert router bias.
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    L = _lib.lib()
+    w = synth.WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    tensors = _device_weights(w, dev)
+    bias = tensors[1] is not None
+    assert bias == (w.bias_coef is not None)
+    Tmax = max(sizes)
+    ref_layer = MoELayer(w.d, w.h, shared_hidden=w.hs, max_tokens=Tmax, has_router_bias=bias)
+    ref_layer.load(*tensors)
+    wts = _lib.Weights(*[_ptr(t) for t in tensors], 1)
+    xs = torch.from_numpy(synth.workload_x(w, T=Tmax).view(np.int16)).to(dev).view(torch.bfloat16)
+    for T in sizes:
+        x = xs[:T].contiguous()
+        y_ref = ref_layer.forward(x)
+        torch.cuda.synchronize()
+        cfg = _lib.Config(w.d, w.E, w.k, w.h, w.hs, 32, T, 0, int(bias), flags)
+        y = _static_call(L, cfg, wts, x, T, w.d, dev)
+        scale = y_ref.abs().max().item()
+        err = (y - y_ref).abs().max().item()
+        assert err <= Y_TOL * scale, (T, err, scale)
     ref_layer.close()
 
 
