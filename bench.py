@@ -252,7 +252,9 @@ def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8), name="c1"):
         nbytes /= w.layers
         gbs = nbytes / (us_layer * 1e-6) / 1e9
         out[f"T{T}"] = {"us_per_layer": us_layer, "bytes_per_layer": nbytes, "achieved_gbs": gbs,
-                        "hbm_frac": gbs / hbm_gbs, "hbm_peak_gbs": hbm_gbs, "launches_per_layer": 3}
+                        "hbm_frac": gbs / hbm_gbs, "hbm_peak_gbs": hbm_gbs,
+                        "launches_per_layer": 1 if T <= 8 else 3,
+                        "kernels": "one-launch fused decode" if T <= 8 else "router, gate/up, down"}
         del g
     for L in layers:
         L.close()

@@ -90,6 +90,18 @@ typedef enum {
 #define MMOE_FLAG_NO_DECODE 4u     /* never take the decode path: by default a forward with few tokens
                                       (T <= 64 where d_model and both hidden sizes are multiples of 64)
                                       runs the weight-streaming decode kernels; same results */
+#define MMOE_FLAG_NO_FUSED_DECODE 32u /* a forward of at most 8 tokens on the decode path runs the layer as
+                                      one launch of a persistent grid by default (routing, gate/up and
+                                      down in one kernel, the next step of a token starting as soon as
+                                      what it needs is done); this flag keeps the three launches of the
+                                      larger decode batches; same results */
+#define MMOE_FLAG_FUSED_REQUANT 64u /* the prefill gate/up GEMM (default tensor-core kind) requantises its
+                                      SwiGLU output itself: the CTAs that hold the hidden-feature blocks of
+                                      a token tile form a cluster and exchange the per-token maxima through
+                                      distributed shared memory, so no FP32 SwiGLU buffer and no separate
+                                      requantisation pass exist (needs max hidden size <= 1024); same
+                                      results.  Off by default: measured on B200 it is slower than the
+                                      separate pass (c4 gate/up 6.9 ms against 2.9 + 0.17 ms) */
 #define MMOE_FLAG_TC_INT8 16u      /* prefill expert GEMMs on the INT8 tensor-core kind (tcgen05 kind::i8,
                                       S32 group partials) instead of the default f16 kind (exact integer
                                       group partials in FP32 accumulators, which the promotion reads
@@ -276,6 +288,7 @@ mmoe_status mmoe_debug_set_wait_limit(mmoe_handle* h, int64_t clocks, int32_t st
  *   MMOE_PROF_REQUANT   per-row requantisation of the SwiGLU output
  *   MMOE_PROF_DOWN      grouped down GEMM with the gate-weighted combine
  *   MMOE_PROF_COMBINE   deterministic combine
+ *   MMOE_PROF_DECODE_FUSED  the one-launch decode of up to 8 tokens (all of the above)
  * Errors: INVALID_ARG (n < 1, NULL arrays), CUDA. */
 enum {
     MMOE_PROF_ZERO_Y = 0,
@@ -285,6 +298,7 @@ enum {
     MMOE_PROF_REQUANT = 4,
     MMOE_PROF_DOWN = 5,
     MMOE_PROF_COMBINE = 6,
+    MMOE_PROF_DECODE_FUSED = 7,
     MMOE_PROF_STAGES = 8
 };
 

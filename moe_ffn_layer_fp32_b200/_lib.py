@@ -23,6 +23,8 @@ FLAG_CUDA_CORES = 2
 FLAG_NO_DECODE = 4
 FLAG_ATOMIC_COMBINE = 8
 FLAG_TC_INT8 = 16
+FLAG_NO_FUSED_DECODE = 32
+FLAG_FUSED_REQUANT = 64
 
 STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAGE_SH, STAGE_LOGITS = range(8)
 
@@ -34,7 +36,7 @@ EXPORTS = ("mmoe_create", "mmoe_load_quantized_weights", "mmoe_forward", "mmoe_f
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
-PROF_STAGES = ("zero_y", "router", "permute", "gate_up", "requant", "down", "combine", "unused")
+PROF_STAGES = ("zero_y", "router", "permute", "gate_up", "requant", "down", "combine", "decode_fused")
 
 
 class MMoEError(RuntimeError):

@@ -386,7 +386,7 @@ struct WarpStream {
 template <bool GU, bool DUMP, int NCH>
 __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs,
                                           const float* shs, int lane, int rb, int64_t rrow0, int prows,
-                                          int32_t* dump, int64_t drow0, int64_t dnrows)
+                                          int32_t* dump, int64_t drow0, int64_t dnrows, uint32_t* amax_rows)
 {
     const int gid = lane >> 2, t4 = lane & 3;
     float alo[NCH][2], ahi[NCH][2];
@@ -464,7 +464,7 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
                 const int64_t r = rrow0 + i;
                 float a = 0.0f;
                 if (valid) {
-                    const float sxr = p.sx[p.row_src[r]];
+                    const float sxr = shs[i];  // the row's activation scale, staged by the caller
                     const float gv = __fmul_rn(alo[c][q], sxr), uv = __fmul_rn(ahi[c][q], sxr);
                     const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
                     a = __fmul_rn(silu, uv);
@@ -474,7 +474,7 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-                if (valid && gid == 0) atomicMax(p.amax_h + r, __float_as_uint(m));
+                if (valid && gid == 0) atomicMax(amax_rows + i, __float_as_uint(m));
             }
         }
     } else {
@@ -492,8 +492,8 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
                     p.obuf[r * p.d + m0] = olo;
                     p.obuf[r * p.d + m0 + 8] = ohi;
                 } else {
-                    const float gt = p.row_gate[r];
-                    float* yr = p.y + (int64_t)p.row_src[r] * p.d;
+                    const float gt = __ldcg(p.row_gate + r);
+                    float* yr = p.y + (int64_t)__ldcg(p.row_src + r) * p.d;
                     atomicAdd(yr + m0, __fmul_rn(gt, olo));
                     atomicAdd(yr + m0 + 8, __fmul_rn(gt, ohi));
                 }
@@ -595,6 +595,7 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
 
         // codes of this pass's rows, zero rows up to a multiple of 8
         if (GU) {
+            for (int i = tid; i < nch * 8; i += blockDim.x) shs[i] = i < prows ? p.sx[p.row_src[rrow0 + i]] : 0.0f;
             for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
                 const int i = it / ngr, j = it % ngr;
                 uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
@@ -641,9 +642,308 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
         __syncthreads();
         if (alive)  // a warp that gave up keeps taking the CTA barriers but issues and computes nothing
             alive = nch == 1 ? warp_pass<GU, DUMP, 1>(p, S, codes, cs, shs, lane, rb, rrow0, prows, dump, drow0,
-                                                      dnrows)
+                                                      dnrows, p.amax_h + rrow0)
                              : warp_pass<GU, DUMP, 2>(p, S, codes, cs, shs, lane, rb, rrow0, prows, dump, drow0,
-                                                      dnrows);
+                                                      dnrows, p.amax_h + rrow0);
+    }
+}
+
+// ------------------------------------------------------------------ fused decode (T <= kFusedMaxT)
+// The whole layer for a handful of tokens in one launch of a persistent grid (every CTA resident at
+// once), so that no step waits for a kernel boundary:
+//   - every CTA quantises x itself (T rows of d values);
+//   - CTAs 0 .. rctas-1 each sum the FP32 router products of one slice of K for every token and store
+//     their partial logits; the last of them to finish (a ticket) adds the slices in rank order, runs
+//     gating, top-k and the permutation of the routing slots, clears y and publishes the routing;
+//   - the other CTAs work through a list of units (a group and a block of W weight-row blocks): the
+//     shared expert's gate/up units first (no routing needed), then the routed groups' gate/up units
+//     (after the routing), then every group's down units (after all gate/up units of that group).
+//     Each unit streams its weights exactly as the three-launch path does (a ring of bulk copies per
+//     warp, mma.sync m16n8k32 with the weights as A), the gate/up units record their rows' SwiGLU
+//     absmax per unit (no zeroed memory needed), the down units requantise from those and add
+//     gate * o into y.
+// Every wait on another CTA is a bounded spin on a counter in global memory; one that gives up raises
+// the handle's error flag and the CTA skips the rest of its units.  The last CTA to leave resets the
+// counters for the next launch.
+constexpr int kFusedMaxT = 8;
+constexpr int kFusedWarps = 8;
+constexpr int kFusedMaxRouterCtas = 64;
+// sync words: [0] router CTAs done, [1] routing published, [2] CTAs that left, [3 + slot] gate/up units done
+constexpr int kSyncWords = 3 + kMaxExperts + 1;
+
+struct FusedArgs {
+    uint32_t* sync;   // kSyncWords counters, zero at launch
+    float* part;      // [kFusedMaxRouterCtas][kFusedMaxT][64] partial logits
+    uint32_t* pamax;  // [gmax][nbpg_gu][16] per-unit SwiGLU absmax bits of each row of the group's pass
+    int rctas, nbpg_gu, nbpg_dn, nring, gmax;
+    long long limit;  // SM clocks of a bounded wait
+};
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Thread 0 waits (bounded) until *ctr >= target, then the whole block continues; false if it gave up.
+__device__ bool block_wait(const Plan& p, const FusedArgs& fa, const uint32_t* ctr, uint32_t target, int where,
+                           int* flag_smem) {
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        if (ld_acquire(ctr) < target) {
+            const long long t0 = clk();
+            while (ld_acquire(ctr) < target) {
+                if (clk() - t0 > fa.limit) {
+                    ok = 0;
+                    set_error(p, where);
+                    break;
+                }
+                __nanosleep(100);
+            }
+        }
+        *flag_smem = ok;
+    }
+    __syncthreads();
+    const int ok = *flag_smem;
+    __syncthreads();
+    return ok != 0;
+}
+
+__global__ void __launch_bounds__(kFusedWarps * 32) decode_fused_kernel(Plan p, FusedArgs fa)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = kFusedWarps, G = (int)gridDim.x;
+    const int T = (int)p.T, d = p.d, E = p.E;
+    // shared memory: mbarriers | shs | uamax | flags | router partials | x (BF16) | x codes | rings | codes
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                       // W * kRingMax
+    float* shs = reinterpret_cast<float*>(smem + 256);                       // [64]
+    uint32_t* uamax = reinterpret_cast<uint32_t*>(smem + 512);               // [16]
+    int* flags = reinterpret_cast<int*>(smem + 576);                          // [16]
+    float* rpart = reinterpret_cast<float*>(smem + 640);                      // [4][kFusedMaxT][64]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + 640 + 4 * kFusedMaxT * 64 * 4);
+    int8_t* xc = reinterpret_cast<int8_t*>(xs + kFusedMaxT * d);
+    uint8_t* ring = reinterpret_cast<uint8_t*>(xc + kFusedMaxT * d);         // 128-byte aligned (d % 64 == 0)
+    uint8_t* codes = ring + W * fa.nring * kStageBytes;
+    float* sxs = shs + 32;                                                    // [kFusedMaxT] activation scales
+
+    if (lane == 0) {
+        for (int s = 0; s < fa.nring; ++s) mbar_init(&bars[warp * kRingMax + s], 1);
+        fence_barrier_init();
+    }
+    if (tid < 16) flags[tid] = 0;
+    // x and its codes, in every CTA
+    {
+        const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
+        uint4* xs4 = reinterpret_cast<uint4*>(xs);
+        for (int i = tid; i < T * d / 8; i += blockDim.x) xs4[i] = x4[i];
+    }
+    __syncthreads();
+    for (int t = warp; t < T; t += W) {
+        float m = 0.0f;
+        for (int i = lane; i < d; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * d + i])));
+        m = warp_max(m);
+        if (lane == 0) sxs[t] = __fdiv_rn(m, 127.0f);
+    }
+    __syncthreads();
+    for (int i = tid; i < T * d; i += blockDim.x) xc[i] = (int8_t)quant_i8(bf16_to_f32(xs[i]), sxs[i / d]);
+    __syncthreads();
+    bool ok = true;
+
+    // ---------------------------------------------------------------- router
+    if ((int)blockIdx.x < fa.rctas) {
+        const int ks = d / fa.rctas, kq = ks / 4;
+        const int e = tid & 63, q = tid >> 6;
+        const int k0 = blockIdx.x * ks + q * kq;
+        float acc[kFusedMaxT];
+#pragma unroll
+        for (int t = 0; t < kFusedMaxT; ++t) acc[t] = 0.0f;
+        if (e < E)
+            for (int kk = k0; kk < k0 + kq; ++kk) {
+                const float w = __ldg(p.w_router + (int64_t)kk * E + e);
+#pragma unroll
+                for (int t = 0; t < kFusedMaxT; ++t)
+                    if (t < T) acc[t] = fmaf(bf16_to_f32(xs[t * d + kk]), w, acc[t]);
+            }
+#pragma unroll
+        for (int t = 0; t < kFusedMaxT; ++t) rpart[(q * kFusedMaxT + t) * 64 + e] = acc[t];
+        __syncthreads();
+        for (int i = tid; i < T * 64; i += blockDim.x) {
+            const int t = i / 64, ee = i % 64;
+            const float v = __fadd_rn(__fadd_rn(__fadd_rn(rpart[(0 * kFusedMaxT + t) * 64 + ee],
+                                                          rpart[(1 * kFusedMaxT + t) * 64 + ee]),
+                                                rpart[(2 * kFusedMaxT + t) * 64 + ee]),
+                                      rpart[(3 * kFusedMaxT + t) * 64 + ee]);
+            fa.part[((int64_t)blockIdx.x * kFusedMaxT + t) * 64 + ee] = v;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            flags[1] = atomicAdd(&fa.sync[0], 1u) == (uint32_t)(fa.rctas - 1);
+        }
+        __syncthreads();
+        if (flags[1]) {
+            // the last router CTA: logits (slices added in rank order), gating, top-k, permutation
+            __threadfence();
+            for (int t = warp; t < T; t += W) {
+                float l0 = -INFINITY, l1 = -INFINITY;
+                if (lane < E) {
+                    float sacc = 0.0f;
+                    for (int c = 0; c < fa.rctas; ++c)
+                        sacc = __fadd_rn(sacc, __ldcg(fa.part + ((int64_t)c * kFusedMaxT + t) * 64 + lane));
+                    l0 = biased_logit(p, sacc, lane);
+                }
+                if (lane + 32 < E) {
+                    float sacc = 0.0f;
+                    for (int c = 0; c < fa.rctas; ++c)
+                        sacc = __fadd_rn(sacc, __ldcg(fa.part + ((int64_t)c * kFusedMaxT + t) * 64 + lane + 32));
+                    l1 = biased_logit(p, sacc, lane + 32);
+                }
+                gate_topk_warp(p, t, l0, l1, lane);
+                if (lane == 0) {
+                    p.sx[t] = sxs[t];
+                    p.row_src[p.Tk + t] = t;
+                    p.row_gate[p.Tk + t] = 1.0f;
+                }
+            }
+            // codes of the shared-expert rows, kept for inspection like the three-launch path's
+            for (int i = tid; i < T * d / 4; i += blockDim.x)
+                reinterpret_cast<uint32_t*>(p.xq + p.Tk * d)[i] = reinterpret_cast<const uint32_t*>(xc)[i];
+            __syncthreads();
+            permute_block(p);
+            // y is cleared before any down unit adds into it
+            if (!p.deterministic) {
+                float4* y4 = reinterpret_cast<float4*>(p.y);
+                for (int i = tid; i < T * d / 4; i += blockDim.x) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicExch(&fa.sync[1], 1u);
+        }
+    }
+
+    // ---------------------------------------------------------------- units
+    const int nu_gu = fa.gmax * fa.nbpg_gu;
+    const int nu = nu_gu + fa.gmax * fa.nbpg_dn;
+    int wsc = 0;  // this warp's running stage count: its ring's phases carry over from unit to unit
+    int ngroups = 1;
+    bool routed = false;
+    for (int u = ((int)blockIdx.x + G - fa.rctas) % G; ok && u < nu; u += G) {
+        const bool GU = u < nu_gu;
+        const int uu = GU ? u : u - nu_gu;
+        const int nbpg = GU ? fa.nbpg_gu : fa.nbpg_dn;
+        const int gs = uu / nbpg, blk = uu % nbpg;
+        if ((gs > 0 || !GU) && !routed) {
+            if (!block_wait(p, fa, &fa.sync[1], 1u, 31, &flags[2])) { ok = false; break; }
+            routed = true;
+            ngroups = __ldcg(p.dec_ngroups);
+        }
+        if (gs >= ngroups) continue;  // (slot 0, the shared expert, always exists)
+        if (!GU && !block_wait(p, fa, &fa.sync[3 + gs], (uint32_t)fa.nbpg_gu, 32, &flags[3])) { ok = false; break; }
+        const int g = gs == 0 ? E : __ldcg(p.dec_groups + gs);
+        const int hid = g == E ? p.hs : p.h;
+        const int K = GU ? d : hid;
+        const int nrb = GU ? hid / 8 : d / 16;
+        const int nrows = gs == 0 ? T : __ldcg(p.counts + g);
+        const int64_t rrow0 = gs == 0 ? p.Tk : __ldcg(p.offsets + g);
+        const int NJ = K / 64, cs = K + 32, ngr = K / 32;
+        const int rb = blk * W + warp;
+        const bool wact = rb < nrb && nrows > 0;
+        if (GU) {
+            // codes of the group's rows (at most kFusedMaxT: one token selects an expert once), from
+            // this CTA's own x codes, zero rows up to 8
+            for (int it = tid; it < 8 * ngr; it += blockDim.x) {
+                const int i = it / ngr, j = it % ngr;
+                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+                if (i < nrows) {
+                    const int t = gs == 0 ? i : __ldcg(p.row_src + rrow0 + i);
+                    const uint4* s4 = reinterpret_cast<const uint4*>(xc + t * d + j * 32);
+                    u0 = s4[0];
+                    u1 = s4[1];
+                }
+                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
+                dst[0] = make_uint4(u0.x, u1.x, u0.y, u1.y);
+                dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
+            }
+            if (tid < 16) {
+                uamax[tid] = 0u;
+                // the rows' activation scales
+                const int t = tid < nrows ? (gs == 0 ? tid : __ldcg(p.row_src + rrow0 + tid)) : 0;
+                shs[tid] = tid < nrows ? sxs[t] : 0.0f;
+            }
+        } else {
+            // requantise the group's SwiGLU rows from the gate/up units' absmax
+            if (tid < 8) {
+                uint32_t m = 0u;
+                if (tid < nrows)
+                    for (int v = 0; v < fa.nbpg_gu; ++v)
+                        m = max(m, __ldcg(fa.pamax + ((int64_t)gs * fa.nbpg_gu + v) * 16 + tid));
+                shs[tid] = tid < nrows ? __fdiv_rn(__uint_as_float(m), 127.0f) : 0.0f;
+                if (blk == 0 && tid < nrows) {
+                    p.amax_h[rrow0 + tid] = m;
+                    p.sh[rrow0 + tid] = shs[tid];
+                }
+            }
+            __syncthreads();
+            for (int it = tid; it < 8 * ngr; it += blockDim.x) {
+                const int i = it / ngr, j = it % ngr;
+                uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                if (i < nrows) {
+                    const float sv = shs[i];
+                    const float4* a4 = reinterpret_cast<const float4*>(p.act + (rrow0 + i) * p.hmax + j * 32);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const float4 a = __ldcg(a4 + v);
+                        wv[v] = pack_codes(a.x, a.y, a.z, a.w, sv);
+                    }
+                    if (blk == 0) {
+                        uint4* q4 = reinterpret_cast<uint4*>(p.hq + (rrow0 + i) * p.hmax + j * 32);
+                        q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                    }
+                }
+                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
+                dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
+                dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+            }
+        }
+        __syncthreads();
+        if (wact) {
+            WarpStream S;
+            S.src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
+                        : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
+                    (int64_t)rb * NJ * kJP;
+            S.ring = ring + warp * fa.nring * kStageBytes;
+            S.bars = bars + warp * kRingMax;
+            S.NJ = NJ;
+            S.nst = (NJ + kStageJP - 1) / kStageJP;
+            S.sc0 = wsc;
+            S.nring = fa.nring;
+            if (lane == 0)
+                for (int s = 0; s < fa.nring && s < S.nst; ++s) S.issue(s);
+            const bool alive = GU ? warp_pass<true, false, 1>(p, S, codes, cs, shs, lane, rb, rrow0, nrows, nullptr,
+                                                              0, 0, uamax)
+                                  : warp_pass<false, false, 1>(p, S, codes, cs, shs, lane, rb, rrow0, nrows, nullptr,
+                                                               0, 0, uamax);
+            wsc += S.nst;
+            if (!alive) flags[4] = 1;
+        }
+        __syncthreads();
+        if (flags[4]) { ok = false; break; }
+        if (GU) {
+            // this unit's absmax of every row (zero for rows it did not touch), then the unit counts as done
+            if (tid < 16) fa.pamax[((int64_t)gs * fa.nbpg_gu + blk) * 16 + tid] = tid < nrows ? uamax[tid] : 0u;
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicAdd(&fa.sync[3 + gs], 1u);
+        }
+    }
+    // leave; the last CTA out resets the counters for the next launch
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(&fa.sync[2], 1u) == (uint32_t)(G - 1))
+            for (int i = 0; i < kSyncWords; ++i) fa.sync[i] = 0u;
     }
 }
 
@@ -771,8 +1071,54 @@ cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t 
     return cudaLaunchKernelEx(&cfg, kern, p, nbpg, nring, dump, r0, nr);
 }
 
+size_t fused_smem(int d, int K, int nring) {
+    return (size_t)640 + 4 * kFusedMaxT * 64 * 4 + (size_t)kFusedMaxT * d * 3 + (size_t)kFusedWarps * nring * kStageBytes +
+           (size_t)kPassRows * (K + 32);
+}
+
 }  // namespace
 }  // namespace dec
+
+int dec_fused_max_tokens() { return dec::kFusedMaxT; }
+
+bool dec_fused_supported(int d, int hmax) {
+    const int nring = std::max(dec::pick_ring(d), dec::pick_ring(hmax));
+    return dec::fused_smem(d, std::max(d, hmax), nring) <= (size_t)dec::kSmemLimit;
+}
+size_t dec_fused_sync_words() { return dec::kSyncWords; }
+size_t dec_fused_part_floats() { return (size_t)dec::kFusedMaxRouterCtas * dec::kFusedMaxT * 64; }
+size_t dec_fused_pamax_words(int d, int hmax, int E, int k) {
+    const int gmax = (dec::kFusedMaxT * k < E ? dec::kFusedMaxT * k : E) + 1;
+    const int nbpg_gu = (hmax / 8 + dec::kFusedWarps - 1) / dec::kFusedWarps;
+    (void)d;
+    return (size_t)gmax * nbpg_gu * 16;
+}
+
+cudaError_t launch_decode_fused(const Plan& p, uint32_t* sync, float* part, uint32_t* pamax, cudaStream_t s) {
+    if (p.T == 0) return cudaSuccess;
+    dec::FusedArgs fa{};
+    fa.sync = sync;
+    fa.part = part;
+    fa.pamax = pamax;
+    fa.rctas = std::max(1, std::min(p.d / 64, dec::kFusedMaxRouterCtas));
+    fa.nbpg_gu = (p.hmax / 8 + dec::kFusedWarps - 1) / dec::kFusedWarps;
+    fa.nbpg_dn = (p.d / 16 + dec::kFusedWarps - 1) / dec::kFusedWarps;
+    fa.nring = std::max(dec::pick_ring(p.d), dec::pick_ring(p.hmax));
+    fa.gmax = (int)std::min<int64_t>(p.Tk, p.E) + 1;
+    fa.limit = p.wait_limit;
+    const size_t smem = dec::fused_smem(p.d, std::max(p.d, p.hmax), fa.nring);
+    static int granted[64] = {};
+    cudaError_t e = dec::raise_smem((const void*)dec::decode_fused_kernel, granted, smem);
+    if (e != cudaSuccess) return e;
+    // every CTA resident at once (units wait on units of other CTAs)
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dec::decode_fused_kernel, dec::kFusedWarps * 32, smem);
+    if (e != cudaSuccess) return e;
+    const int G = dec::sm_count() * std::min(occ, 2);
+    if (occ < 1 || G < fa.rctas) return cudaErrorInvalidConfiguration;
+    dec::decode_fused_kernel<<<G, dec::kFusedWarps * 32, smem, s>>>(p, fa);
+    return cudaGetLastError();
+}
 
 bool dec_supported(int d, int h, int hs) { return d % 64 == 0 && h % 64 == 0 && hs % 64 == 0; }
 

@@ -52,6 +52,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
+
 #include "mmoe_internal.cuh"
 #include "sm100_tc.cuh"
 
@@ -66,16 +68,25 @@ constexpr int kStages = 4;
 constexpr int kBufs = 2;                   // TMEM buffers of 2 x BN columns
 constexpr int kBufCols = 2 * BN;
 constexpr int kTmemCols = kBufs * kBufCols;
-constexpr int kPromoWarps = 8;
-constexpr int kPromoWarp0 = 4;             // promotion warps are warpgroups 1 and 2
+#ifndef MMOE_F16_PROMO_WARPS
+#define MMOE_F16_PROMO_WARPS 8
+#endif
+// 8 or 16: two or four per SM sub-partition.  Measured on c4 (gate/up, down): 2.90 / 1.54 ms with 8,
+// 2.80 / 1.95 ms with 16 (32 token columns per thread); the build uses 8.
+constexpr int kPromoWarps = MMOE_F16_PROMO_WARPS;
+constexpr int kPromoWarp0 = 4;             // promotion warps are the warpgroups after the first
 constexpr int kThreads = 128 + kPromoWarps * 32;
-// Register split (setmaxnreg): the launch gives every thread 168 registers (384 x 168 = 64512 of the
-// SM's 65536); warpgroup 0 (producer, MMA issuer, two idle warps) drops to 32 and the two promotion
-// warpgroups rise to 232: 128 x 32 + 256 x 232 = 63488 <= 64512.
+// Register split (setmaxnreg): the launch gives every thread kRegsLaunch registers (what fits the SM's
+// 65536 when the sub-partition with the most warps holds ceil(warps / 4) of them); warpgroup 0
+// (producer, MMA issuer, two idle warps) drops to 32 and the promotion warpgroups rise to kRegsHigh.
+constexpr int kRegsLaunch = kPromoWarps == 8 ? 168 : 96;
 constexpr int kRegsLow = 32;
-constexpr int kRegsHigh = 232;
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * 168, "register split");
-constexpr int kCols = BN / 2;              // token columns per promotion thread (per half)
+constexpr int kRegsHigh = kPromoWarps == 8 ? 232 : 112;
+static_assert(kPromoWarps == 8 || kPromoWarps == 16, "8 or 16 promotion warps");
+static_assert(128 * kRegsLow + kPromoWarps * 32 * kRegsHigh <= kThreads * kRegsLaunch, "register split");
+constexpr int kColGroups = kPromoWarps / 4;  // token-column groups (one warp per lane quarter each)
+constexpr int kCols = BN / kColGroups;     // token columns per promotion thread (per half)
+constexpr int kChunks = 2 * kCols / 16;    // 16-column TMEM loads per thread and group (both halves)
 
 constexpr int kImgBytes = BMH * BK * 2;    // one half's weight stage image: 16 KB
 constexpr int kBBytes = BN * BK * 2;       // activation-code tile: 16 KB
@@ -86,12 +97,15 @@ constexpr uint32_t kIdesc = tc5::idesc_f16(BN);
 
 enum Epi { kEpiSwiGLU = 0, kEpiDown = 1 };
 
+constexpr int kMaxCluster = 8;             // CTAs sharing a token tile when the requantisation is fused
+
 constexpr int kTInfo = 4;                  // tile-info ring entries
 constexpr int kTInfoConsumers = 1 + kPromoWarps;  // MMA lane, promotion warps
 
 // What every role needs to know about one tile, gathered by the producer warp.
 struct TileInfo {
     int row0, nr, mb, nks, tile0, end;
+    int skip;            // fused requantisation: this CTA has no feature block of the tile's group
     float colf[BN];      // per token column: activation scale (gate/up) or SwiGLU scale (down)
     float colg[BN];      // per token column: gate of the row (down)
     int colrow[BN];      // per token column: token id (down)
@@ -105,10 +119,17 @@ struct Smem {
     uint64_t tfull[kTInfo];
     uint64_t tempty[kTInfo];
     uint64_t never;          // signalled by nothing: the injected stall of the failure-detection tests
+    uint64_t xbar[2];        // fused requantisation: the cluster's per-token maxima of a tile have arrived
+    uint64_t pbar;           // fused requantisation: the promotion warps' two meeting points of a tile
     uint32_t tmem_base;
     int abort;
     TileInfo ti[kTInfo];
+    // fused requantisation: per-token |SwiGLU| maxima of this CTA's 128 features, per TMEM lane quarter,
+    // and the maxima received from every CTA of the cluster (two tiles in flight)
+    uint32_t amax_part[4][BN];
+    alignas(16) float recv[2][kMaxCluster][BN];  // written with 16-byte st.async: 16-byte aligned
 };
+static_assert(offsetof(Smem, recv) % 16 == 0, "st.async needs 16-byte aligned destinations");
 
 using async::bulk_load;
 using async::clk;
@@ -172,6 +193,7 @@ struct Args {
     int ks_routed;          // K stages of a routed expert (gate/up: d/64, down: h/64)
     int ks_shared;
     int fblocks;            // weight-row tiles per token tile in the launch (the larger of the two)
+    int cluster;            // fused requantisation: CTAs per cluster (= fblocks), else 1
     int32_t* dump;          // optional INT32 partial dump
     int64_t drow0, dnrows;
 };
@@ -199,6 +221,31 @@ __device__ __forceinline__ Tile decode_tile(const Plan& p, const Args& a, int L)
     // half 0 is image block 2 mb, half 1 block 2 mb + 1; each block has nks stage images
     t.tile0 = (int)(t.g * a.expert_stride) + 2 * fb * t.nks;
     return t;
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(async::su32(p)), "r"(rank));
+    return a;
+}
+
+// 16 bytes into a peer's shared memory, counted on the peer's mbarrier as bytes of its transaction.
+__device__ __forceinline__ void st_async_peer(uint32_t dst, uint32_t bar, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(dst),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
+                 : "memory");
 }
 
 // acc[c] = fma((P[2c], P[2c+1]), (s, s), acc[c]) for 8 pairs of columns: the
@@ -240,7 +287,7 @@ __device__ __forceinline__ void dump16(const Plan& p, const Args& a, const TileI
     }
 }
 
-template <int kEpi, bool kDump>
+template <int kEpi, bool kDump, bool kFuse>
 __global__ void __launch_bounds__(kThreads, 1)
 expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
 {
@@ -249,10 +296,18 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
     uint8_t* stages = base;
     Smem* sm = reinterpret_cast<Smem*>(base + kStages * kStageBytes);
 
-    // nothing to do after an earlier wait gave up
-    if (p.err && *reinterpret_cast<volatile int*>(p.err)) return;
-    const int total = (*p.tile_count) * a.fblocks;
-    if ((int)blockIdx.x >= total) return;
+    // Fused requantisation: the CTAs of a cluster share each token tile, rank r taking feature block r;
+    // they all walk the same tiles and leave together (no early exit: peers write into each other's
+    // shared memory until the final cluster barrier).
+    const int C = kFuse ? a.cluster : 1;
+    const int crank = kFuse ? (int)cluster_ctarank() : 0;
+    const int cid = (int)blockIdx.x / C, ncl = (int)gridDim.x / C;
+    if (!kFuse) {
+        // nothing to do after an earlier wait gave up
+        if (p.err && *reinterpret_cast<volatile int*>(p.err)) return;
+    }
+    const int total = kFuse ? *p.tile_count : (*p.tile_count) * a.fblocks;
+    if (!kFuse && (int)blockIdx.x >= total) return;
     const ErrFlags ef{p.err, p.err_host, p.wait_limit};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -270,6 +325,9 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
             mbar_init(&sm->tempty[b], kTInfoConsumers);
         }
         mbar_init(&sm->never, 1);
+        mbar_init(&sm->xbar[0], 1);
+        mbar_init(&sm->xbar[1], 1);
+        mbar_init(&sm->pbar, kPromoWarps);
         sm->abort = 0;
         fence_barrier_init();
     }
@@ -279,6 +337,8 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
     }
     __syncthreads();
     tc5::after_sync();
+    // the peers' barriers exist before anyone signals them
+    if (kFuse) cluster_sync_all();
     const uint32_t tmem = sm->tmem_base;
     if (warp < kPromoWarp0) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
@@ -286,13 +346,15 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
             // ------------------------------------------------------------ producer (whole warp)
             int sc = 0, tcount = 0;
             bool ok = true;
-            for (int L = blockIdx.x; ok; L += gridDim.x) {
+            for (int L = kFuse ? cid : (int)blockIdx.x; ok; L += kFuse ? ncl : (int)gridDim.x) {
                 Tile t{};
                 const bool last = L >= total;  // past the last tile: publish the end marker and stop
                 if (!last) {
-                    if (lane == 0) t = decode_tile(p, a, L);
+                    // fused: token tile L, feature block = cluster rank
+                    if (lane == 0) t = decode_tile(p, a, kFuse ? L * a.fblocks + crank : L);
                     t.valid = __shfl_sync(0xffffffffu, t.valid, 0);
-                    if (!t.valid) continue;
+                    if (!t.valid && !kFuse) continue;
+                    if (!t.valid) t.nks = 0;  // published with no K stages: the CTA joins the exchange only
                     t.mb = __shfl_sync(0xffffffffu, t.mb, 0);
                     t.nks = __shfl_sync(0xffffffffu, t.nks, 0);
                     t.nr = __shfl_sync(0xffffffffu, t.nr, 0);
@@ -307,6 +369,7 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
                 TileInfo& ti = sm->ti[b];
                 if (lane == 0) {
                     ti.end = last ? 1 : 0;
+                    ti.skip = (!last && !t.valid) ? 1 : 0;
                     ti.row0 = t.row0; ti.nr = t.nr; ti.mb = t.mb; ti.nks = t.nks; ti.tile0 = t.tile0;
                 }
                 if (!last) {
@@ -393,7 +456,7 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
         // ------------------------------------------------------------ promotion + epilogue
         const int pw = warp - kPromoWarp0;    // 0..7
-        const int hc = pw >> 2;               // token-column half
+        const int hc = pw >> 2;               // token-column group
         const int quarter = warp & 3;         // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;  // weight row of this thread within each half
         const int col0 = hc * kCols;
@@ -408,7 +471,7 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
             if (!warp_wait(&sm->tfull[tb], (tcount / kTInfo) & 1, sm, ef, 19)) break;
             const TileInfo& ti = sm->ti[tb];
             if (ti.end) break;
-            const int nks = ti.nks, nr = ti.nr, mb = ti.mb;
+            const int nks = ti.nks, nr = ti.nr, mb = ti.mb, skip = ti.skip;
             const int64_t row0 = ti.row0;
             // group scales: half 0 at sp[j * 128], half 1 at sp[half1 + j * 128]
             const float* sp = a.simg + (size_t)ti.tile0 * (kGroupsPerStage * BMH) + row;
@@ -417,7 +480,11 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
 #pragma unroll
             for (int c = 0; c < kCols / 2; ++c) acc0[c] = acc1[c] = make_float2(0.0f, 0.0f);
             const int ng = nks * kGroupsPerStage;
-            float s0 = __ldg(sp), s1 = __ldg(sp + half1);
+            float s0 = 0.0f, s1 = 0.0f;
+            if (ng > 0) {
+                s0 = __ldg(sp);
+                s1 = __ldg(sp + half1);
+            }
             for (int j = 0; j < ng; ++j, ++pc) {
                 const int b = pc & 1;
                 float n0 = 0.0f, n1 = 0.0f;
@@ -428,26 +495,28 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
                 if (!warp_wait(&sm->accf[b], (pc >> 1) & 1, sm, ef, 15)) { ok = false; break; }
                 tc5::after_sync();
                 const uint32_t ta = tl + b * kBufCols;
-                // eight loads of 16 columns (four per half), each overlapped with the promotion of the
+                // loads of 16 columns (half 0, then half 1), each overlapped with the promotion of the
                 // one before; the buffer goes back to the MMA as soon as the last has landed
+                constexpr int kPerHalf = kChunks / 2;
                 uint32_t va[16], vb[16];
                 tc5::tmem_ld16(ta, va);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
+                for (int ch = 0; ch < kChunks; ++ch) {
                     uint32_t (&cur)[16] = (ch & 1) ? vb : va;
                     uint32_t (&nxt)[16] = (ch & 1) ? va : vb;
                     tc5::tmem_wait_ld(cur);
-                    if (ch < 7) {
+                    if (ch < kChunks - 1) {
                         const int nc = ch + 1;
-                        tc5::tmem_ld16(ta + (nc >> 2) * BN + (nc & 3) * 16, nxt);
+                        tc5::tmem_ld16(ta + (nc / kPerHalf) * BN + (nc % kPerHalf) * 16, nxt);
                     } else {
                         tc5::before_sync();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sm->acce[b]);
                     }
-                    float2* acc = (ch >> 2) ? acc1 : acc0;
-                    promote8(acc + (ch & 3) * 8, cur, (ch >> 2) ? s1 : s0);
-                    if (kDump) dump16<kEpi>(p, a, ti, ch >> 2, row, col0 + (ch & 3) * 16, cur, j);
+                    const int half = ch / kPerHalf;
+                    float2* acc = half ? acc1 : acc0;
+                    promote8(acc + (ch % kPerHalf) * 8, cur, half ? s1 : s0);
+                    if (kDump) dump16<kEpi>(p, a, ti, half, row, col0 + (ch % kPerHalf) * 16, cur, j);
                 }
                 s0 = n0;
                 s1 = n1;
@@ -457,6 +526,71 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
             // The inspection launch (kDump) runs the same K loop with the partials' stores added and no
             // epilogue: its plan has no output buffers.
             if (kDump) {
+            } else if (kEpi == kEpiSwiGLU && kFuse) {
+                // SwiGLU in registers (kept in acc0), then the per-token requantisation over all
+                // hidden features: this CTA's maxima over its 128 features (a warp reduction per
+                // column, then the four lane quarters through shared memory), sent to every CTA of
+                // the cluster, the cluster's maximum, the codes of this CTA's features
+                const int slot = tcount & 1;
+#pragma unroll
+                for (int c = 0; c < kCols; ++c) {
+                    const int cc = col0 + c;
+                    const float g = (c & 1) ? acc0[c >> 1].y : acc0[c >> 1].x;
+                    const float u = (c & 1) ? acc1[c >> 1].y : acc1[c >> 1].x;
+                    const float av = (!skip && cc < nr) ? swiglu(g, u, ti.colf[cc]) : 0.0f;
+                    if (c & 1) acc0[c >> 1].y = av;
+                    else acc0[c >> 1].x = av;
+                }
+                uint32_t mine[kCols / 32];
+#pragma unroll
+                for (int c = 0; c < kCols; ++c) {
+                    const float av = (c & 1) ? acc0[c >> 1].y : acc0[c >> 1].x;
+                    const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(av)));
+                    if ((c & 31) == lane) mine[c >> 5] = m;
+                }
+#pragma unroll
+                for (int i = 0; i < kCols / 32; ++i) sm->amax_part[quarter][col0 + 32 * i + lane] = mine[i];
+                // every promotion warp has written its maxima: the first of the tile's two phases of pbar
+                // (a bounded wait, unlike a named barrier, so that a warp that gave up cannot hang the rest)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->pbar);
+                if (!warp_wait(&sm->pbar, 0, sm, ef, 22)) { ok = false; break; }
+                mbar_try_wait(&sm->pbar, 0);  // this lane's own acquire of the phase
+                const int pt = pw * 32 + lane;  // 0 .. promotion threads - 1
+                if (pt == 0) mbar_expect_tx(&sm->xbar[slot], (uint32_t)(C * BN * 4));
+                if (pt < C * 32) {
+                    // thread pt sends columns 4 (pt % 32) .. + 3 to cluster rank pt / 32
+                    const int c4 = 4 * (pt & 31);
+                    uint32_t v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        v[i] = max(max(sm->amax_part[0][c4 + i], sm->amax_part[1][c4 + i]),
+                                   max(sm->amax_part[2][c4 + i], sm->amax_part[3][c4 + i]));
+                    const uint32_t dst = (uint32_t)(pt >> 5);
+                    st_async_peer(peer_addr(&sm->recv[slot][crank][c4], dst), peer_addr(&sm->xbar[slot], dst), v[0],
+                                  v[1], v[2], v[3]);
+                }
+                // every sender has read the maxima before the next tile overwrites them: the second phase
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->pbar);
+                if (!warp_wait(&sm->pbar, 1, sm, ef, 23)) { ok = false; break; }
+                if (!warp_wait(&sm->xbar[slot], (tcount >> 1) & 1, sm, ef, 21)) { ok = false; break; }
+                mbar_try_wait(&sm->xbar[slot], (tcount >> 1) & 1);  // this lane's own acquire of the phase
+                if (!skip) {
+                    uint16_t* out = p.hq16 + row0 * p.hmax + mb * BMH + row;
+#pragma unroll
+                    for (int c = 0; c < kCols; ++c) {
+                        const int cc = col0 + c;
+                        float m = 0.0f;
+                        for (int r = 0; r < C; ++r) m = fmaxf(m, sm->recv[slot][r][cc]);
+                        const float sh = __fdiv_rn(m, 127.0f);
+                        const float av = (c & 1) ? acc0[c >> 1].y : acc0[c >> 1].x;
+                        if (cc < nr) {
+                            out[(int64_t)cc * p.hmax] = (uint16_t)code_f16(quant_i8(av, sh));
+                            if (crank == 0 && quarter == 0 && lane == (c & 31)) p.sh[row0 + cc] = sh;
+                        }
+                    }
+                }
             } else if (kEpi == kEpiSwiGLU) {
                 float* out = p.act + row0 * p.hmax + mb * BMH + row;
 #pragma unroll
@@ -497,6 +631,8 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
     }
 
     __syncthreads();
+    // no CTA of a cluster leaves while a peer may still write into its shared memory
+    if (kFuse) cluster_sync_all();
     if (warp == 1) {
         tc5::after_sync();
         tc5::tmem_dealloc(tmem, kTmemCols);
@@ -601,17 +737,73 @@ static int sm_count_f16() {
     return n[dev];
 }
 
-template <int kEpi, bool kDump>
+int f16tc_fused_clusters(int c);
+
+template <int kEpi, bool kDump, bool kFuse>
 static cudaError_t launch_f16(const Plan& p, cudaStream_t s, const CUtensorMap* map, tf::Args a) {
-    auto kern = tf::expert_gemm_f16_kernel<kEpi, kDump>;
+    auto kern = tf::expert_gemm_f16_kernel<kEpi, kDump, kFuse>;
     const size_t smem = f16tc_smem_bytes();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    // persistent: one CTA per SM (never more CTAs than the largest possible tile count)
-    const int64_t upper = p.max_tiles * (int64_t)a.fblocks;
-    const unsigned grid = (unsigned)(upper < sm_count_f16() ? upper : sm_count_f16());
-    kern<<<grid, tf::kThreads, smem, s>>>(*map, p, a);
-    return cudaGetLastError();
+    if (!kFuse) {
+        // persistent: one CTA per SM (never more CTAs than the largest possible tile count)
+        a.cluster = 1;
+        const int64_t upper = p.max_tiles * (int64_t)a.fblocks;
+        const unsigned grid = (unsigned)(upper < sm_count_f16() ? upper : sm_count_f16());
+        kern<<<grid, tf::kThreads, smem, s>>>(*map, p, a);
+        return cudaGetLastError();
+    }
+    // fused requantisation: clusters of fblocks CTAs, as many as the device holds at once (each CTA
+    // takes a whole SM), never more than the largest possible token-tile count
+    a.cluster = a.fblocks;
+    const int ncl_max = f16tc_fused_clusters(a.fblocks);
+    if (ncl_max <= 0) return cudaErrorNotSupported;
+    const int64_t ncl = p.max_tiles < ncl_max ? p.max_tiles : ncl_max;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(ncl * a.cluster), 1, 1);
+    cfg.blockDim = dim3(tf::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)a.cluster;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, *map, p, a);
+}
+
+// Clusters of `c` CTAs of the fused gate/up GEMM that fit on the device at once (0: none); queried
+// once per device and cluster size.
+int f16tc_fused_clusters(int c) {
+    static int cache[64][tf::kMaxCluster + 1] = {};
+    static bool done[64][tf::kMaxCluster + 1] = {};
+    if (c < 1 || c > tf::kMaxCluster) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (done[dev][c]) return cache[dev][c];
+    auto kern = tf::expert_gemm_f16_kernel<tf::kEpiSwiGLU, false, true>;
+    const size_t smem = f16tc_smem_bytes();
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)c, 1, 1);
+        cfg.blockDim = dim3(tf::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = (unsigned)c;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    cache[dev][c] = n;
+    done[dev][c] = true;
+    return n;
 }
 
 cudaError_t launch_gate_up_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
@@ -628,7 +820,9 @@ cudaError_t launch_gate_up_f16(const Plan& p, cudaStream_t s, int32_t* dump, int
     a.drow0 = row0;
     a.dnrows = nrows;
     const CUtensorMap* map = static_cast<const CUtensorMap*>(p.tmap_xq);
-    return dump ? launch_f16<tf::kEpiSwiGLU, true>(p, s, map, a) : launch_f16<tf::kEpiSwiGLU, false>(p, s, map, a);
+    if (dump) return launch_f16<tf::kEpiSwiGLU, true, false>(p, s, map, a);
+    return p.fuse_requant ? launch_f16<tf::kEpiSwiGLU, false, true>(p, s, map, a)
+                          : launch_f16<tf::kEpiSwiGLU, false, false>(p, s, map, a);
 }
 
 cudaError_t launch_down_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
@@ -645,7 +839,7 @@ cudaError_t launch_down_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_
     a.drow0 = row0;
     a.dnrows = nrows;
     const CUtensorMap* map = static_cast<const CUtensorMap*>(p.tmap_hq);
-    return dump ? launch_f16<tf::kEpiDown, true>(p, s, map, a) : launch_f16<tf::kEpiDown, false>(p, s, map, a);
+    return dump ? launch_f16<tf::kEpiDown, true, false>(p, s, map, a) : launch_f16<tf::kEpiDown, false, false>(p, s, map, a);
 }
 
 }  // namespace mmoe

@@ -134,6 +134,7 @@ struct mmoe_handle {
     uint16_t* hq16 = nullptr;
     long long wait_limit = kDefaultWaitLimit;
     bool stall_next = false;   // the next prefill forward injects a stall (mmoe_debug_set_wait_limit)
+    bool fuse_requant = false; // kind::f16: the gate/up GEMM requantises the SwiGLU output itself (clusters)
     alignas(64) unsigned char tmap_xq[128] = {};
     alignas(64) unsigned char tmap_hq[128] = {};
     int* err_host = nullptr;   // mapped pinned host memory; kernels write its device alias
@@ -149,6 +150,12 @@ struct mmoe_handle {
     uint32_t* amax_h = nullptr;
     int32_t* dec_groups = nullptr;
     int32_t* dec_ngroups = nullptr;
+    // fused one-launch decode: synchronisation words (kept zero between launches), router partials,
+    // per-unit SwiGLU absmax
+    bool use_dec_fused = false;
+    uint32_t* dec_sync = nullptr;
+    float* dec_part = nullptr;
+    uint32_t* dec_pamax = nullptr;
     // per-stage timing (mmoe_profile_*)
     struct ProfRec {
         int stage, launches;
@@ -185,7 +192,8 @@ void free_all(mmoe_handle* h) {
                     h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
                     h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
                     h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->amax_h, h->dec_groups,
-                    h->dec_ngroups, h->w_gate_up_f16, h->w_down_f16, h->xq16, h->hq16};
+                    h->dec_ngroups, h->w_gate_up_f16, h->w_down_f16, h->xq16, h->hq16, h->dec_sync,
+                    h->dec_part, h->dec_pamax};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);
@@ -222,7 +230,7 @@ mmoe_status check_config(const mmoe_config* c) {
     if (c->has_router_bias != 0 && c->has_router_bias != 1)
         return fail(MMOE_ERR_INVALID_ARG, "has_router_bias=%d: must be 0 or 1", c->has_router_bias);
     if (c->flags & ~(MMOE_FLAG_DETERMINISTIC | MMOE_FLAG_CUDA_CORES | MMOE_FLAG_NO_DECODE | MMOE_FLAG_ATOMIC_COMBINE |
-                     MMOE_FLAG_TC_INT8))
+                     MMOE_FLAG_TC_INT8 | MMOE_FLAG_NO_FUSED_DECODE | MMOE_FLAG_FUSED_REQUANT))
         return fail(MMOE_ERR_INVALID_ARG, "flags=0x%x: unknown bits", c->flags);
     return MMOE_OK;
 }
@@ -281,6 +289,7 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.xq16 = h->xq16;
     p.hq16 = h->hq16;
     p.wait_limit = h->wait_limit;
+    p.fuse_requant = h->fuse_requant;
     p.tmap_xq = h->tmap_xq;
     p.tmap_hq = h->tmap_hq;
     p.err = h->err_dev;
@@ -317,6 +326,8 @@ mmoe_status check_device_flag(mmoe_handle* h, cudaStream_t s) {
     if (v == 0) return MMOE_OK;
     *reinterpret_cast<volatile int*>(h->err_host) = 0;
     cudaMemsetAsync(h->err_dev, 0, sizeof(int), s);
+    // a fused decode that gave up may have left its synchronisation words set
+    if (h->dec_sync) cudaMemsetAsync(h->dec_sync, 0, dec_fused_sync_words() * sizeof(uint32_t), s);
     return fail(MMOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (site %d); its results were not written", v);
 }
 
@@ -455,6 +466,14 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     // decode path's
     const int64_t Rd = h->use_dec ? (Tm < h->dec_max_T ? Tm : h->dec_max_T) * (k + 1) : 1;
     const int64_t R8 = h->tc_kind == kTcF16 ? Rd : R;
+    // with MMOE_FLAG_FUSED_REQUANT the SwiGLU requantisation runs inside the kind::f16 gate/up GEMM when
+    // one cluster of CTAs can hold all hidden-feature blocks of a token tile (at most 8 blocks of 128)
+    // and the device fits such clusters; the FP32 SwiGLU buffer then serves only the decode rows
+    if (h->tc_kind == kTcF16 && (cfg->flags & MMOE_FLAG_FUSED_REQUANT)) {
+        const int fb = h->hmax / 128;
+        h->fuse_requant = fb >= 1 && fb <= 8 && f16tc_fused_clusters(fb) > 0;
+    }
+    const int64_t Ract = h->fuse_requant ? Rd : R;
 
     cudaError_t e = cudaSuccess;
 #define ALLOC(ptr, n) \
@@ -480,7 +499,7 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(row_src, R);
     ALLOC(row_gate, R);
     ALLOC(slot_row, Tm * k);
-    ALLOC(act, R * h->hmax);
+    ALLOC(act, Ract * h->hmax);
     ALLOC(hq, R8 * h->hmax);
     ALLOC(sh, R);
     if (h->use_dec) {
@@ -489,6 +508,13 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
         ALLOC(amax_h, Rd);
         ALLOC(dec_groups, E + 1);
         ALLOC(dec_ngroups, 1);
+        h->use_dec_fused = !(cfg->flags & MMOE_FLAG_NO_FUSED_DECODE) && dec_fused_supported((int)d, h->hmax);
+        if (h->use_dec_fused) {
+            ALLOC(dec_sync, dec_fused_sync_words());
+            ALLOC(dec_part, dec_fused_part_floats());
+            ALLOC(dec_pamax, dec_fused_pamax_words((int)d, h->hmax, (int)E, (int)k));
+            if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, dec_fused_sync_words() * sizeof(uint32_t));
+        }
     }
     if (e == cudaSuccess) {
         // the fixed-order combine needs the per-row outputs: always in deterministic mode, and by
@@ -600,7 +626,13 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     // fixed-order combine: always in deterministic mode; on the prefill path unless atomics were asked for
     p.deterministic = (h->cfg.flags & MMOE_FLAG_DETERMINISTIC) ||
                       (!dec && !(h->cfg.flags & MMOE_FLAG_ATOMIC_COMBINE));
-    if (dec) {
+    const bool fused = dec && h->use_dec_fused && T <= dec_fused_max_tokens() && !p.deterministic;
+    if (fused) {
+        // the whole layer in one launch (routing, gate/up, down, the combine into y)
+        MMOE_CUDA(run_stage(h, MMOE_PROF_DECODE_FUSED, 1, s,
+                            [&] { return launch_decode_fused(p, h->dec_sync, h->dec_part, h->dec_pamax, s); }),
+                  "fused decode launch");
+    } else if (dec) {
         // decode path: router + permutation, gate/up (also clears y), down
         MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_dec(p, h->dec_cluster, s); }),
                   "decode router launch");
@@ -622,7 +654,8 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
         MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return run_gate_up(p, s, nullptr, 0, 0); }),
                   "gate/up launch");
         p.debug_stall = 0;
-        MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
+        if (!p.fuse_requant)
+            MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
         MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return run_down(p, s, nullptr, 0, 0); }), "down launch");
     }
     if (p.deterministic)

@@ -72,6 +72,7 @@ struct Plan {
     const void* tmap_hq;
     long long wait_limit;         // SM clocks a bounded wait of the kind::f16 GEMMs lasts before giving up
     int debug_stall;              // 1: the kind::f16 gate/up GEMM injects a stall (failure-detection tests)
+    bool fuse_requant;            // kind::f16: the gate/up GEMM writes the SwiGLU codes itself (clusters)
     int* err;                     // device flag: a bounded wait gave up (later CTAs exit at once)
     int* err_host;                // device alias of the host-mapped copy of that flag
     // decode path (k_decode.cu)
@@ -100,6 +101,7 @@ cudaError_t launch_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t ro
 cudaError_t launch_combine(const Plan& p, cudaStream_t s);
 // tensor-core path, kind::f16 (k_expert_f16.cu)
 bool f16tc_supported(int d, int h, int hs);
+int f16tc_fused_clusters(int c);  // clusters of c CTAs of the fused gate/up GEMM the device holds at once
 size_t f16tc_image_elems(int d, int h, int hs, int E, bool gate_up);
 cudaError_t launch_gate_up_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_down_f16(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
@@ -119,6 +121,14 @@ bool dec_supported(int d, int h, int hs);
 int dec_max_tokens(int d, int hmax);
 int dec_router_cluster(int d, int E);
 cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s);
+// the fused one-launch decode of up to dec_fused_max_tokens() tokens, with its synchronisation words
+// (zero before the first launch; the kernel leaves them zero), router partials and per-unit absmax
+int dec_fused_max_tokens();
+bool dec_fused_supported(int d, int hmax);
+size_t dec_fused_sync_words();
+size_t dec_fused_part_floats();
+size_t dec_fused_pamax_words(int d, int hmax, int E, int k);
+cudaError_t launch_decode_fused(const Plan& p, uint32_t* sync, float* part, uint32_t* pamax, cudaStream_t s);
 cudaError_t launch_gate_up_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_retile_dec(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,

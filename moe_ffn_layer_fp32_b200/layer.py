@@ -57,15 +57,19 @@ class MoELayer:
     def __init__(self, d_model: int, expert_hidden: int, *, shared_hidden: int | None = None,
                  n_experts: int = 60, top_k: int = 4, max_tokens: int = 4096, gating: int = 0,
                  has_router_bias: bool = False, deterministic: bool = False, cuda_cores: bool = False,
-                 decode: bool = True, atomic_combine: bool = False, tc_int8: bool = False, device: int = 0):
+                 decode: bool = True, atomic_combine: bool = False, tc_int8: bool = False,
+                 fused_decode: bool = True, fused_requant: bool = False, device: int = 0):
         """decode=False keeps small batches (T <= 64) on the prefill kernels instead of the
         weight-streaming decode kernels; cuda_cores=True runs every expert GEMM on CUDA cores;
         tc_int8=True runs the prefill expert GEMMs on the kind::i8 tensor-core kernels instead of the
-        default kind::f16 ones; atomic_combine=True adds the prefill expert outputs into y with atomics
+        default kind::f16 ones; fused_decode=False keeps batches of at most 8 tokens on the three-launch
+        decode kernels instead of the one-launch decode; fused_requant=True requantises the SwiGLU output
+        inside the prefill gate/up GEMM (thread-block clusters); atomic_combine=True adds the prefill expert outputs into y with atomics
         (no [R, d] workspace); deterministic=True uses the fixed-order combine on the decode path too."""
         flags = ((_lib.FLAG_DETERMINISTIC if deterministic else 0) | (_lib.FLAG_CUDA_CORES if cuda_cores else 0)
                  | (0 if decode else _lib.FLAG_NO_DECODE) | (_lib.FLAG_ATOMIC_COMBINE if atomic_combine else 0)
-                 | (_lib.FLAG_TC_INT8 if tc_int8 else 0))
+                 | (_lib.FLAG_TC_INT8 if tc_int8 else 0) | (0 if fused_decode else _lib.FLAG_NO_FUSED_DECODE)
+                 | (_lib.FLAG_FUSED_REQUANT if fused_requant else 0))
         self.cfg = _lib.Config(d_model, n_experts, top_k, expert_hidden,
                                expert_hidden if shared_hidden is None else shared_hidden, GROUP, max_tokens,
                                gating, int(has_router_bias), flags)

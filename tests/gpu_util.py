@@ -23,11 +23,13 @@ def x_to_device(x_np: np.ndarray) -> torch.Tensor:
 
 
 def make_gpu_layer(q: oracle.QuantizedLayer, max_tokens: int, deterministic: bool = False, cuda_cores: bool = False,
-                   decode: bool = True, atomic_combine: bool = False, tc_int8: bool = False):
+                   decode: bool = True, atomic_combine: bool = False, tc_int8: bool = False,
+                   fused_decode: bool = True, fused_requant: bool = False):
     from moe_ffn_layer_fp32_b200.layer import MoELayer
     L = MoELayer(q.d, q.h, shared_hidden=q.hs, n_experts=q.E, top_k=q.k, max_tokens=max_tokens,
                  gating=q.gating, has_router_bias=q.router_bias is not None, deterministic=deterministic,
-                 cuda_cores=cuda_cores, decode=decode, atomic_combine=atomic_combine, tc_int8=tc_int8)
+                 cuda_cores=cuda_cores, decode=decode, atomic_combine=atomic_combine, tc_int8=tc_int8,
+                 fused_decode=fused_decode, fused_requant=fused_requant)
     L.load(q.w_router, q.router_bias, q.w_gate_up, q.s_gate_up, q.w_down, q.s_down)
     return L
 

@@ -41,7 +41,7 @@ def valid_cfg(**kw):
 @pytest.mark.parametrize("kw", [dict(d_model=250), dict(d_model=32), dict(n_experts=0), dict(n_experts=65),
                                 dict(top_k=0), dict(top_k=9), dict(n_experts=3, top_k=4),
                                 dict(expert_hidden=100), dict(shared_hidden=0), dict(group_size=64),
-                                dict(max_tokens=0), dict(gating=3), dict(has_router_bias=2), dict(flags=32),
+                                dict(max_tokens=0), dict(gating=3), dict(has_router_bias=2), dict(flags=128),
                                 dict(flags=0x80000000)])
 def test_create_rejects_bad_config(L, kw):
     h = C.c_void_p()

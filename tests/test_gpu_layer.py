@@ -54,10 +54,11 @@ def test_quantizer_matches_oracle_bit_exact():
 
 
 def _full_check(q, x, deterministic=False, partial_rows=None, max_tokens=None, cuda_cores=False, decode=True,
-                atomic_combine=False, tc_int8=False):
+                atomic_combine=False, tc_int8=False, fused_decode=True, fused_requant=False):
     T = x.shape[0]
     L = gu.make_gpu_layer(q, max_tokens or max(T, 1), deterministic=deterministic, cuda_cores=cuda_cores,
-                          decode=decode, atomic_combine=atomic_combine, tc_int8=tc_int8)
+                          decode=decode, atomic_combine=atomic_combine, tc_int8=tc_int8, fused_decode=fused_decode,
+                          fused_requant=fused_requant)
     out = gu.run_gpu(L, q, x)
     y, D = oracle.moe_layer(q, x, dumps=True)
     rep = {}
@@ -104,6 +105,31 @@ def test_ragged_token_counts(T, decode):
     rep, out = _full_check(q, x, max_tokens=512, partial_rows=[0, T * q.k - 1, T * q.k, T * (q.k + 1) - 1],
                            decode=decode)
     assert out["counts"][q.E] == T
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+@pytest.mark.parametrize("fused", [True, False], ids=["one_launch", "three_launches"])
+def test_small_decode_batches_both_kernel_sets(T, fused):
+    # up to 8 tokens run as one launch of a persistent grid by default; the three-launch kernels give
+    # the same results
+    w, q = workload("c0")
+    x = synth.draw_x(T, w.d, seed=200 + T)
+    R = T * (q.k + 1)
+    rep, out = _full_check(q, x, max_tokens=64, partial_rows=range(R), fused_decode=fused)
+    assert out["counts"][q.E] == T
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_c1_decode_one_launch_matches_three_launches(T):
+    # the decode workload's shapes (d_model 1024, hidden 512): both kernel sets against the oracle,
+    # and against each other (the same expert outputs, added into y in a different order)
+    w = synth.WORKLOADS["c1"]
+    q = oracle.quantize_layer(synth.workload_layer(w, 5))
+    x = synth.workload_x(w, step=5, T=T)
+    _, a = _full_check(q, x, max_tokens=64, fused_decode=True)
+    _, b = _full_check(q, x, max_tokens=64, fused_decode=False)
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["hq"], b["hq"])
+    assert np.max(np.abs(a["y"] - b["y"])) <= 1e-5 * np.abs(b["y"]).max()
 
 
 def test_decode_hot_groups_of_64_rows():
@@ -241,6 +267,17 @@ def test_mobilemoe_s_prefill_2048():
     gu.check_partials(L, q, out, _group_edge_rows(out, q.E))
     L.close()
     print("s2048", rep)
+
+
+@pytest.mark.parametrize("name,T", [("c0", 200), ("c2", 1024), ("c3b", 600)])
+def test_prefill_fused_requantisation(name, T):
+    # MMOE_FLAG_FUSED_REQUANT: the gate/up GEMM's clusters (1, 4 and 6 CTAs here) exchange the
+    # per-token maxima and write the SwiGLU codes themselves
+    w, q = workload(name)
+    x = synth.workload_x(w, T=T)
+    R = T * (q.k + 1)
+    rep, out = _full_check(q, x, fused_requant=True, partial_rows=[0, T * q.k - 1, T * q.k, R - 1])
+    print("fused requant", name, rep)
 
 
 def test_c2_prefill_int8_tensor_cores():
