@@ -35,7 +35,11 @@ METRIC = "MoE-layer prefill tokens/s & decode us/layer; % of INT8-TC / HBM roofl
 # prefill gate/up GEMM per workload, from one ncu capture on B200, keyed by the
 # first 16 hex digits of the SHA-256 of the GEMM's source file at the time of the
 # capture: a figure is reported only while that file is unchanged.
-GATE_UP_TRAFFIC_BYTES = {}
+GATE_UP_TRAFFIC_BYTES = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:expert_gemm_f16 (1 pass):
+    # c2 157.09 + 9.36 MB, c4 1.22 GB + 635.09 MB
+    "b012fadf693f5309": {"c2": 166_450_000, "c4": 1_855_090_000},
+}
 GEMM_SOURCE = os.path.join(ROOT, "moe_ffn_layer_fp32_b200", "csrc", "k_expert_f16.cu")
 L2_BYTES = 126 * 1024 * 1024
 # Peaks when MEASURED_PEAKS.json is absent: an earlier measurement on this machine (bf16 dense burst,
