@@ -364,47 +364,53 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
 }
 
 // ------------------------------------------------------------------ experts
-// One warp's weight stream for one pass: stage st (0 .. nst-1) of the pass is
-// global stage sc0 + st of the warp's ring, so slot and phase carry over
-// between passes.
+// One warp's weight stream: `npass` passes over blocks `pstride` bytes apart
+// (0: the same block again), each of nst stages.  Stage sc of the stream (from
+// 0) is stage sc % nst of pass sc / nst and lands in ring slot (base + sc) %
+// nring, so slot and phase carry over from stream to stream when `base` is the
+// warp's running stage count.  A pass consumes stages sc0 .. sc0 + nst - 1 and
+// refills the ring with stages below ntot.
 struct WarpStream {
-    const uint8_t* src;   // the warp's 16-row block in the decode layout
+    const uint8_t* src;   // the warp's first 16-row block in the decode layout
     uint8_t* ring;
     uint64_t* bars;
-    int NJ, nst, sc0, nring;
-    __device__ __forceinline__ void issue(int st) const {
+    int64_t pstride;
+    int NJ, nst, sc0, nring, ntot, base;
+    __device__ __forceinline__ int slot(int sc) const { return (base + sc) % nring; }
+    __device__ __forceinline__ uint32_t parity(int sc) const { return (uint32_t)(((base + sc) / nring) & 1); }
+    __device__ __forceinline__ void issue(int sc) const {
+        const int st = sc % nst;
         const int jp = NJ - st * kStageJP;
         const uint32_t bytes = (uint32_t)((jp < kStageJP ? jp : kStageJP) * kJP);
-        const int slot = (sc0 + st) % nring;
-        mbar_expect_tx(&bars[slot], bytes);
-        bulk_load(ring + slot * kStageBytes, src + (int64_t)st * kStageBytes, bytes, &bars[slot]);
+        mbar_expect_tx(&bars[slot(sc)], bytes);
+        bulk_load(ring + slot(sc) * kStageBytes, src + (int64_t)(sc / nst) * pstride + (int64_t)st * kStageBytes, bytes,
+                  &bars[slot(sc)]);
     }
 };
 
-// The GEMV of one warp over one pass of up to 8 * NCH rows, then its
-// epilogue.  Returns false if a bounded wait gave up (nothing is written).
+// The K loop of one warp over one pass of up to 8 * NCH rows: the accumulators
+// of its 16 weight rows (A rows 0-7 in alo, 8-15 in ahi) for every row column.
+// Returns false if a bounded wait gave up (the copies in flight have landed).
 template <bool GU, bool DUMP, int NCH>
-__device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs,
-                                          const float* shs, int lane, int rb, int64_t rrow0, int prows,
-                                          int32_t* dump, int64_t drow0, int64_t dnrows, uint32_t* amax_rows)
+__device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs, int lane,
+                                          int rb, int64_t rrow0, int prows, int32_t* dump, int64_t drow0,
+                                          int64_t dnrows, float (&alo)[NCH][2], float (&ahi)[NCH][2])
 {
     const int gid = lane >> 2, t4 = lane & 3;
-    float alo[NCH][2], ahi[NCH][2];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) alo[c][0] = alo[c][1] = ahi[c][0] = ahi[c][1] = 0.0f;
     const int ng = p.d / kGroup, ngh = p.hmax / kGroup;
     const uint8_t* bbase = codes + (size_t)gid * cs + t4 * 8;
     for (int st = 0; st < S.nst; ++st) {
         const int sc = S.sc0 + st;
-        if (!wait_bounded(&S.bars[sc % S.nring], (uint32_t)((sc / S.nring) & 1))) {
+        if (!wait_bounded(&S.bars[S.slot(sc)], S.parity(sc))) {
             if (lane == 0) set_error(p, 7);
             // let the copies in flight land before the CTA's shared memory goes away
-            const int issued = st + S.nring < S.nst ? st + S.nring : S.nst;
-            for (int s = st; s < issued; ++s)
-                wait_bounded(&S.bars[(S.sc0 + s) % S.nring], (uint32_t)(((S.sc0 + s) / S.nring) & 1));
+            const int issued = sc + S.nring < S.ntot ? sc + S.nring : S.ntot;
+            for (int s = sc; s < issued; ++s) wait_bounded(&S.bars[S.slot(s)], S.parity(s));
             return false;
         }
-        const uint8_t* sb = S.ring + (sc % S.nring) * kStageBytes;
+        const uint8_t* sb = S.ring + S.slot(sc) * kStageBytes;
         const int njs = S.NJ - st * kStageJP < kStageJP ? S.NJ - st * kStageJP : kStageJP;
 #pragma unroll
         for (int q = 0; q < kStageJP; ++q) {
@@ -449,8 +455,29 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
             }
         }
         __syncwarp();
-        if (lane == 0 && st + S.nring < S.nst) S.issue(st + S.nring);
+        if (lane == 0 && sc + S.nring < S.ntot) S.issue(sc + S.nring);
     }
+    return true;
+}
+
+// SwiGLU of row i's gate and up accumulators (the row's activation scale sxr applied to both)
+__device__ __forceinline__ float swiglu_row(float g, float u, float sxr) {
+    const float gv = __fmul_rn(g, sxr), uv = __fmul_rn(u, sxr);
+    const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+    return __fmul_rn(silu, uv);
+}
+
+// The GEMV of one warp over one pass of up to 8 * NCH rows, then its
+// epilogue.  Returns false if a bounded wait gave up (nothing is written).
+template <bool GU, bool DUMP, int NCH>
+__device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs,
+                                          const float* shs, int lane, int rb, int64_t rrow0, int prows,
+                                          int32_t* dump, int64_t drow0, int64_t dnrows, uint32_t* amax_rows)
+{
+    const int gid = lane >> 2, t4 = lane & 3;
+    float alo[NCH][2], ahi[NCH][2];
+    if (!warp_gemv<GU, DUMP, NCH>(p, S, codes, cs, lane, rb, rrow0, prows, dump, drow0, dnrows, alo, ahi))
+        return false;
     if (DUMP) return true;
 
     if (GU) {
@@ -464,10 +491,7 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
                 const int64_t r = rrow0 + i;
                 float a = 0.0f;
                 if (valid) {
-                    const float sxr = shs[i];  // the row's activation scale, staged by the caller
-                    const float gv = __fmul_rn(alo[c][q], sxr), uv = __fmul_rn(ahi[c][q], sxr);
-                    const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
-                    a = __fmul_rn(silu, uv);
+                    a = swiglu_row(alo[c][q], ahi[c][q], shs[i]);  // shs: the rows' activation scales
                     p.act[r * p.hmax + n] = a;
                 }
                 float m = fabsf(a);
@@ -575,6 +599,10 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
     S.nst = (NJ + kStageJP - 1) / kStageJP;
     S.sc0 = 0;
     S.nring = nring;
+    S.pstride = 0;  // every pass of rows streams the same block again (from L2 after the first)
+    S.base = 0;
+    const int npass = (nrows + kPassRows - 1) / kPassRows;
+    S.ntot = npass * S.nst;  // the ring runs on into the next pass
     if (lane == 0) {
         for (int s = 0; s < nring; ++s) mbar_init(&S.bars[s], 1);
         fence_barrier_init();
@@ -582,15 +610,14 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
     __syncwarp();
     const bool keep = blk == 0 && !DUMP;  // one CTA per group records h_q and s_h
     bool alive = wact;                    // false once this warp's bounded wait gave up
-    const int npass = (nrows + kPassRows - 1) / kPassRows;
     for (int pass = 0; pass < npass; ++pass, S.sc0 += S.nst) {
         const int prow0 = pass * kPassRows;
         const int prows = nrows - prow0 < kPassRows ? nrows - prow0 : kPassRows;
         const int nch = (prows + 7) >> 3;
         const int64_t rrow0 = row0 + prow0;
         if (pass > 0) __syncthreads();  // every warp is done with the previous pass's codes
-        if (alive && lane == 0)
-            for (int s = 0; s < nring && s < S.nst; ++s) S.issue(s);
+        if (pass == 0 && alive && lane == 0)
+            for (int s = 0; s < nring && s < S.ntot; ++s) S.issue(s);
         if (pass == 0 && shared) pdl_wait();  // weights are in flight; now the previous launch's outputs
 
         // codes of this pass's rows, zero rows up to a multiple of 8
@@ -648,303 +675,488 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
     }
 }
 
-// ------------------------------------------------------------------ fused decode (T <= kFusedMaxT)
-// The whole layer for a handful of tokens in one launch of a persistent grid (every CTA resident at
-// once), so that no step waits for a kernel boundary:
-//   - every CTA quantises x itself (T rows of d values);
-//   - CTAs 0 .. rctas-1 each sum the FP32 router products of one slice of K for every token and store
-//     their partial logits; the last of them to finish (a ticket) adds the slices in rank order, runs
-//     gating, top-k and the permutation of the routing slots, clears y and publishes the routing;
-//   - the other CTAs work through a list of units (a group and a block of W weight-row blocks): the
-//     shared expert's gate/up units first (no routing needed), then the routed groups' gate/up units
-//     (after the routing), then every group's down units (after all gate/up units of that group).
-//     Each unit streams its weights exactly as the three-launch path does (a ring of bulk copies per
-//     warp, mma.sync m16n8k32 with the weights as A), the gate/up units record their rows' SwiGLU
-//     absmax per unit (no zeroed memory needed), the down units requantise from those and add
-//     gate * o into y.
-// Every wait on another CTA is a bounded spin on a counter in global memory; one that gives up raises
-// the handle's error flag and the CTA skips the rest of its units.  The last CTA to leave resets the
-// counters for the next launch.
-constexpr int kFusedMaxT = 8;
-constexpr int kFusedWarps = 8;
-constexpr int kFusedMaxRouterCtas = 64;
-// sync words: [0] router CTAs done, [1] routing published, [2] CTAs that left, [3 + slot] gate/up units done
-constexpr int kSyncWords = 3 + kMaxExperts + 1;
+// ------------------------------------------------------------------ one-launch decode (T <= kCMaxT)
+// The whole layer for a handful of tokens in one launch of clusters of CS CTAs, with no CTA ever
+// waiting on another cluster:
+//   - every CTA computes the activation scales of all tokens and the FP32 router products of its
+//     K slice (d / CS rows of W_r) for every token; the slices' partial logits go to every CTA of the
+//     cluster through distributed shared memory and, after a cluster barrier, each CTA adds them in
+//     rank order (the same sums in every CTA of every cluster), then runs gating, top-k and the
+//     permutation of the routing slots itself;
+//   - the groups with rows (the shared expert first, then the selected experts in ascending order)
+//     go to the clusters in turn; CTA r of a cluster takes the weight-row blocks r W + w, r W + w + CS W,
+//     ... of the group's gate/up and then of its down weights, streamed as in the three-launch path
+//     (a ring of bulk copies per warp, mma.sync m16n8k32 with the weights as A).  Each warp's down
+//     stream starts as soon as its gate/up blocks are done;
+//   - each CTA writes the SwiGLU values of its hidden features into every CTA's copy of the group's
+//     rows (distributed shared memory); after one cluster barrier every CTA requantises the whole rows
+//     itself (absmax / 127 and the INT8 codes, as K4's requantisation) for its down blocks;
+//   - the down outputs go to a row buffer.  Per token and CTA rank a counter in global memory counts
+//     the k + 1 contributions; the CTA that brings the last one adds them in the fixed order of
+//     Eq. (*) (shared expert, then the selected experts in top-k order) over its rank's output
+//     columns and resets the counter.
+// The only waits are for this CTA's own bulk copies (bounded) and the cluster barriers, which every
+// CTA of a cluster reaches equally often; the clusters need not be resident at the same time.
+constexpr int kCMaxT = 8;
+constexpr int kCWarps = 8;
+constexpr int kCThreads = kCWarps * 32;
+constexpr int kCMaxCS = 16;
+constexpr int kCMaxSlots = kCMaxT * kMaxTopK;
 
-struct FusedArgs {
-    uint32_t* sync;   // kSyncWords counters, zero at launch
-    float* part;      // [kFusedMaxRouterCtas][kFusedMaxT][64] partial logits
-    uint32_t* pamax;  // [gmax][nbpg_gu][16] per-unit SwiGLU absmax bits of each row of the group's pass
-    int rctas, nbpg_gu, nbpg_dn, nring, gmax;
-    long long limit;  // SM clocks of a bounded wait
+struct CArgs {
+    uint32_t* cnt;        // [kCMaxT][CS] contribution counters, zero at launch (the last user resets one)
+    float* obuf;          // [kCMaxT * (kMaxTopK + 1)][d] expert outputs, rows as in the permutation
+    int32_t* out_idx;     // optional copies of the routing for the caller: [T, k]
+    float* out_gate;      // [T, k]
+    int32_t* out_counts;  // [E + 1]
+    // dynamic shared memory offsets
+    int off_x, off_codes, off_act, off_u;
 };
 
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-    return v;
+struct CShared {
+    uint64_t bars[kCWarps * kRingMax];
+    uint64_t wbar, xbar;
+    float sxs[kCMaxT];             // activation scales of the tokens
+    float shs[8];                  // per row of the current group: activation scale, then SwiGLU scale
+    float keys[kCWarps][64];       // top-k: each warp's copy of its token's selection keys
+    float selp[kCWarps][kMaxTopK]; //   and the probabilities of the selected experts
+    int idx[kCMaxSlots];
+    float gate[kCMaxSlots];
+    int slot_row[kCMaxSlots];
+    int row_tok[kCMaxSlots];       // routed row -> token
+    int cnt[kMaxExperts];
+    int offs[kMaxExperts + 2];
+    int groups[kMaxExperts + 1];
+    int nslots;
+    int last[8];
+};
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t peer_addr(const void* p, int rank) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(su32(p)), "r"(rank));
+    return a;
+}
+__device__ __forceinline__ void st_peer(const void* p, int rank, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_addr(p, rank)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_peer(const void* p, int rank, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(peer_addr(p, rank)), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
-// Thread 0 waits (bounded) until *ctr >= target, then the whole block continues; false if it gave up.
-__device__ bool block_wait(const Plan& p, const FusedArgs& fa, const uint32_t* ctr, uint32_t target, int where,
-                           int* flag_smem) {
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        if (ld_acquire(ctr) < target) {
-            const long long t0 = clk();
-            while (ld_acquire(ctr) < target) {
-                if (clk() - t0 > fa.limit) {
-                    ok = 0;
-                    set_error(p, where);
-                    break;
-                }
-                __nanosleep(100);
-            }
-        }
-        *flag_smem = ok;
-    }
-    __syncthreads();
-    const int ok = *flag_smem;
-    __syncthreads();
-    return ok != 0;
-}
+// number of passes pi >= 0 with first + pi * step < n
+__device__ __forceinline__ int npasses(int first, int step, int n) { return first < n ? (n - first + step - 1) / step : 0; }
 
-__global__ void __launch_bounds__(kFusedWarps * 32) decode_fused_kernel(Plan p, FusedArgs fa)
+template <int CS>
+__global__ void __launch_bounds__(kCThreads) decode_cluster_kernel(Plan p, CArgs ca)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int W = kFusedWarps, G = (int)gridDim.x;
-    const int T = (int)p.T, d = p.d, E = p.E;
-    // shared memory: mbarriers | shs | uamax | flags | router partials | x (BF16) | x codes | rings | codes
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);                       // W * kRingMax
-    float* shs = reinterpret_cast<float*>(smem + 256);                       // [64]
-    uint32_t* uamax = reinterpret_cast<uint32_t*>(smem + 512);               // [16]
-    int* flags = reinterpret_cast<int*>(smem + 576);                          // [16]
-    float* rpart = reinterpret_cast<float*>(smem + 640);                      // [4][kFusedMaxT][64]
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + 640 + 4 * kFusedMaxT * 64 * 4);
-    int8_t* xc = reinterpret_cast<int8_t*>(xs + kFusedMaxT * d);
-    uint8_t* ring = reinterpret_cast<uint8_t*>(xc + kFusedMaxT * d);         // 128-byte aligned (d % 64 == 0)
-    uint8_t* codes = ring + W * fa.nring * kStageBytes;
-    float* sxs = shs + 32;                                                    // [kFusedMaxT] activation scales
+    __shared__ CShared st;
+    constexpr int W = kCWarps;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, t4 = lane & 3;
+    const int T = (int)p.T, d = p.d, E = p.E, k = p.k, Tk = (int)p.Tk;
+    const int rank = (int)cluster_rank();
+    const int cid = (int)blockIdx.x / CS, ncl = (int)gridDim.x / CS;
+    const int ks = d / CS;
+    const bool keeper = cid == 0 && rank == 0;  // writes the routing and permutation for inspection
+    float* part_recv = reinterpret_cast<float*>(smem);                       // [CS][kCMaxT][64]
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + ca.off_x); // [T][d]
+    uint8_t* codes = smem + ca.off_codes;                                    // [8][max(d, hmax) + 32]
+    float* act_all = reinterpret_cast<float*>(smem + ca.off_act);            // [8 rows][hmax] SwiGLU values
+    uint8_t* ring = smem + ca.off_u;                                         // W_r slice, then the rings
+    const float* wr = reinterpret_cast<const float*>(ring);
 
-    if (lane == 0) {
-        for (int s = 0; s < fa.nring; ++s) mbar_init(&bars[warp * kRingMax + s], 1);
+    // first half of a cluster barrier: this CTA has started (its shared memory may be written by peers
+    // once the second half has been waited for)
+    cluster_arrive_relaxed();
+    pdl_trigger();
+    if (tid == 0) {
+        for (int i = 0; i < W * kRingMax; ++i) mbar_init(&st.bars[i], 1);
+        mbar_init(&st.wbar, 1);
+        mbar_init(&st.xbar, 1);
         fence_barrier_init();
+        // this CTA's K slice of W_r, rows [rank ks, (rank + 1) ks): weights, not outputs of the previous launch
+        const uint32_t wbytes = (uint32_t)(ks * E * 4);
+        mbar_expect_tx(&st.wbar, wbytes);
+        bulk_load(ring, p.w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
     }
-    if (tid < 16) flags[tid] = 0;
-    // x and its codes, in every CTA
-    {
-        const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
-        uint4* xs4 = reinterpret_cast<uint4*>(xs);
-        for (int i = tid; i < T * d / 8; i += blockDim.x) xs4[i] = x4[i];
+    if (cid == 0 && tid == 32) {
+        // the shared expert (slot 0, this cluster's first group) toward L2: this CTA's gate/up and down blocks
+        const int NJ = d / 64, NJd = p.hs / 64, nrb = p.hs / 8, nrbd = d / 16;
+        for (int b0 = rank * W; b0 < nrb; b0 += CS * W)
+            prefetch_range(p.w_gate_up_d + (int64_t)E * ((int64_t)p.h * d * 5 / 4) + (int64_t)b0 * NJ * kJP,
+                           (int64_t)min(W, nrb - b0) * NJ * kJP);
+        for (int b0 = rank * W; b0 < nrbd; b0 += CS * W)
+            prefetch_range(p.w_down_d + (int64_t)E * ((int64_t)d * p.h * 5 / 8) + (int64_t)b0 * NJd * kJP,
+                           (int64_t)min(W, nrbd - b0) * NJd * kJP);
     }
-    __syncthreads();
+    __syncthreads();  // the mbarriers are initialised
+    pdl_wait();       // x, and the buffers the previous launch used
+    if (tid == 0) {
+        const uint32_t xbytes = (uint32_t)(T * d * 2);
+        mbar_expect_tx(&st.xbar, xbytes);
+        bulk_load(smem + ca.off_x, p.x, xbytes, &st.xbar);
+    }
+    bool ok = wait_bounded(&st.xbar, 0);
     for (int t = warp; t < T; t += W) {
         float m = 0.0f;
         for (int i = lane; i < d; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * d + i])));
         m = warp_max(m);
-        if (lane == 0) sxs[t] = __fdiv_rn(m, 127.0f);
+        if (lane == 0) st.sxs[t] = __fdiv_rn(m, 127.0f);
     }
-    __syncthreads();
-    for (int i = tid; i < T * d; i += blockDim.x) xc[i] = (int8_t)quant_i8(bf16_to_f32(xs[i]), sxs[i / d]);
-    __syncthreads();
-    bool ok = true;
+    ok = wait_bounded(&st.wbar, 0) && ok;
+    if (!ok && tid == 0) set_error(p, 40);
 
     // ---------------------------------------------------------------- router
-    if ((int)blockIdx.x < fa.rctas) {
-        const int ks = d / fa.rctas, kq = ks / 4;
-        const int e = tid & 63, q = tid >> 6;
-        const int k0 = blockIdx.x * ks + q * kq;
-        float acc[kFusedMaxT];
+    // thread (q, e): FP32 products of K rows [q ks / 4, (q + 1) ks / 4) of the slice, each token, four K
+    // rows per step (kq is a multiple of 4)
+    {
+        const int e = tid & 63, q = tid >> 6, kq = ks / 4;
+        float acc[kCMaxT];
 #pragma unroll
-        for (int t = 0; t < kFusedMaxT; ++t) acc[t] = 0.0f;
-        if (e < E)
-            for (int kk = k0; kk < k0 + kq; ++kk) {
-                const float w = __ldg(p.w_router + (int64_t)kk * E + e);
+        for (int t = 0; t < kCMaxT; ++t) acc[t] = 0.0f;
+        if (e < E && ok) {
+            const uint16_t* xk = xs + rank * ks + q * kq;
+            const float* wk = wr + (q * kq) * E + e;
+#pragma unroll 2
+            for (int kk = 0; kk < kq; kk += 4) {
+                const float w0 = wk[kk * E], w1 = wk[(kk + 1) * E], w2 = wk[(kk + 2) * E], w3 = wk[(kk + 3) * E];
 #pragma unroll
-                for (int t = 0; t < kFusedMaxT; ++t)
-                    if (t < T) acc[t] = fmaf(bf16_to_f32(xs[t * d + kk]), w, acc[t]);
+                for (int t = 0; t < kCMaxT; ++t)
+                    if (t < T) {
+                        const uint2 xv = *reinterpret_cast<const uint2*>(xk + t * d + kk);
+                        acc[t] = fmaf(bf16_to_f32(xv.x & 0xffffu), w0, acc[t]);
+                        acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w1, acc[t]);
+                        acc[t] = fmaf(bf16_to_f32(xv.y & 0xffffu), w2, acc[t]);
+                        acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w3, acc[t]);
+                    }
             }
-#pragma unroll
-        for (int t = 0; t < kFusedMaxT; ++t) rpart[(q * kFusedMaxT + t) * 64 + e] = acc[t];
-        __syncthreads();
-        for (int i = tid; i < T * 64; i += blockDim.x) {
-            const int t = i / 64, ee = i % 64;
-            const float v = __fadd_rn(__fadd_rn(__fadd_rn(rpart[(0 * kFusedMaxT + t) * 64 + ee],
-                                                          rpart[(1 * kFusedMaxT + t) * 64 + ee]),
-                                                rpart[(2 * kFusedMaxT + t) * 64 + ee]),
-                                      rpart[(3 * kFusedMaxT + t) * 64 + ee]);
-            fa.part[((int64_t)blockIdx.x * kFusedMaxT + t) * 64 + ee] = v;
         }
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            flags[1] = atomicAdd(&fa.sync[0], 1u) == (uint32_t)(fa.rctas - 1);
+        float* rq = act_all;  // scratch until the first group's SwiGLU: [4][kCMaxT][64]
+#pragma unroll
+        for (int t = 0; t < kCMaxT; ++t) rq[(q * kCMaxT + t) * 64 + e] = acc[t];
+    }
+    __syncthreads();
+    cluster_wait();  // every CTA of the cluster has started
+    for (int i = tid; i < T * 16; i += kCThreads) {
+        const int t = i >> 4, e4 = (i & 15) * 4;
+        const float* rq = act_all;
+        float v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int o = t * 64 + e4 + c;
+            v[c] = __fadd_rn(__fadd_rn(__fadd_rn(rq[o], rq[kCMaxT * 64 + o]), rq[2 * kCMaxT * 64 + o]),
+                             rq[3 * kCMaxT * 64 + o]);
         }
-        __syncthreads();
-        if (flags[1]) {
-            // the last router CTA: logits (slices added in rank order), gating, top-k, permutation
-            __threadfence();
-            for (int t = warp; t < T; t += W) {
-                float l0 = -INFINITY, l1 = -INFINITY;
-                if (lane < E) {
-                    float sacc = 0.0f;
-                    for (int c = 0; c < fa.rctas; ++c)
-                        sacc = __fadd_rn(sacc, __ldcg(fa.part + ((int64_t)c * kFusedMaxT + t) * 64 + lane));
-                    l0 = biased_logit(p, sacc, lane);
-                }
-                if (lane + 32 < E) {
-                    float sacc = 0.0f;
-                    for (int c = 0; c < fa.rctas; ++c)
-                        sacc = __fadd_rn(sacc, __ldcg(fa.part + ((int64_t)c * kFusedMaxT + t) * 64 + lane + 32));
-                    l1 = biased_logit(p, sacc, lane + 32);
-                }
-                gate_topk_warp(p, t, l0, l1, lane);
-                if (lane == 0) {
-                    p.sx[t] = sxs[t];
-                    p.row_src[p.Tk + t] = t;
-                    p.row_gate[p.Tk + t] = 1.0f;
-                }
+        const float4 v4 = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll 4
+        for (int c = 0; c < CS; ++c) st_peer(part_recv + (rank * kCMaxT + t) * 64 + e4, c, v4);
+    }
+    cluster_sync();  // every slice's partial logits are here
+    for (int t = warp; t < T; t += W) {
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int c = 0; c < CS; ++c) {
+            s0 = __fadd_rn(s0, part_recv[(c * kCMaxT + t) * 64 + lane]);
+            s1 = __fadd_rn(s1, part_recv[(c * kCMaxT + t) * 64 + lane + 32]);
+        }
+        const float l0 = lane < E ? biased_logit(p, s0, lane) : -INFINITY;
+        const float l1 = lane + 32 < E ? biased_logit(p, s1, lane + 32) : -INFINITY;
+        gate_topk_rank(p, t, l0, l1, lane, st.keys[warp], st.selp[warp], st.idx, st.gate, keeper ? p.logits : nullptr);
+    }
+    __syncthreads();
+    // ---------------------------------------------------------------- permutation (warp 0)
+    if (warp == 0) {
+        // per-expert counts (experts lane, lane + 32) and each slot's rank among the earlier slots of its
+        // expert (slots lane, lane + 32), by one pass over the slots
+        const int s0 = lane, s1 = lane + 32;
+        const int e0 = s0 < Tk ? st.idx[s0] : -1, e1 = s1 < Tk ? st.idx[s1] : -1;
+        int c0 = 0, c1 = 0, r0 = 0, r1 = 0;
+#pragma unroll 4
+        for (int sl = 0; sl < Tk; ++sl) {
+            const int e = st.idx[sl];
+            c0 += e == lane;
+            c1 += e == lane + 32;
+            r0 += sl < s0 && e == e0;
+            r1 += sl < s1 && e == e1;
+        }
+        if (lane >= E) c0 = 0;
+        if (lane + 32 >= E) c1 = 0;
+        st.cnt[lane] = c0;
+        st.cnt[lane + 32] = c1;
+        int i0 = c0, i1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
+            if (lane >= o) { i0 += u0; i1 += u1; }
+        }
+        i1 += __shfl_sync(0xffffffffu, i0, 31);
+        const unsigned lt = (1u << lane) - 1u;
+        const unsigned b0 = __ballot_sync(0xffffffffu, c0 > 0), b1 = __ballot_sync(0xffffffffu, c1 > 0);
+        st.offs[lane] = i0 - c0;
+        st.offs[lane + 32] = i1 - c1;
+        if (c0) st.groups[1 + __popc(b0 & lt)] = lane;
+        if (c1) st.groups[1 + __popc(b0) + __popc(b1 & lt)] = lane + 32;
+        __syncwarp();
+        if (lane == 0) {
+            st.groups[0] = E;
+            st.nslots = 1 + __popc(b0) + __popc(b1);
+            st.offs[E] = Tk;
+            st.offs[E + 1] = Tk + T;
+        }
+        __syncwarp();
+        if (e0 >= 0) {
+            const int r = st.offs[e0] + r0;
+            st.slot_row[s0] = r;
+            st.row_tok[r] = s0 / k;
+        }
+        if (e1 >= 0) {
+            const int r = st.offs[e1] + r1;
+            st.slot_row[s1] = r;
+            st.row_tok[r] = s1 / k;
+        }
+    }
+    __syncthreads();
+    if (keeper) {
+        // the routing and the permutation, as the three-launch path leaves them
+        for (int i = tid; i < Tk; i += kCThreads) {
+            p.idx[i] = st.idx[i];
+            p.gate[i] = st.gate[i];
+            p.slot_row[i] = st.slot_row[i];
+            p.row_src[st.slot_row[i]] = i / k;
+            p.row_gate[st.slot_row[i]] = st.gate[i];
+            if (ca.out_idx) ca.out_idx[i] = st.idx[i];
+            if (ca.out_gate) ca.out_gate[i] = st.gate[i];
+        }
+        for (int t = tid; t < T; t += kCThreads) {
+            p.sx[t] = st.sxs[t];
+            p.row_src[Tk + t] = t;
+            p.row_gate[Tk + t] = 1.0f;
+        }
+        for (int e = tid; e <= E + 1; e += kCThreads) {
+            p.offsets[e] = st.offs[e];
+            if (e <= E) {
+                const int c = e < E ? st.cnt[e] : T;
+                p.counts[e] = c;
+                if (ca.out_counts) ca.out_counts[e] = c;
             }
-            // codes of the shared-expert rows, kept for inspection like the three-launch path's
-            for (int i = tid; i < T * d / 4; i += blockDim.x)
-                reinterpret_cast<uint32_t*>(p.xq + p.Tk * d)[i] = reinterpret_cast<const uint32_t*>(xc)[i];
-            __syncthreads();
-            permute_block(p);
-            // y is cleared before any down unit adds into it
-            if (!p.deterministic) {
-                float4* y4 = reinterpret_cast<float4*>(p.y);
-                for (int i = tid; i < T * d / 4; i += blockDim.x) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicExch(&fa.sync[1], 1u);
+        }
+        for (int i = tid; i < st.nslots; i += kCThreads) p.dec_groups[i] = st.groups[i];
+        if (tid == 0) *p.dec_ngroups = st.nslots;
+    }
+    if (cid == 0) {
+        // the shared rows' activation codes (this CTA's K slice), kept for inspection
+        for (int i = tid; i < T * (ks / 4); i += kCThreads) {
+            const int t = i / (ks / 4), v = i % (ks / 4);
+            const uint16_t* xr = xs + t * d + rank * ks + v * 4;
+            *reinterpret_cast<uint32_t*>(p.xq + (int64_t)(Tk + t) * d + rank * ks + v * 4) =
+                pack_codes(bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), st.sxs[t]);
         }
     }
 
-    // ---------------------------------------------------------------- units
-    const int nu_gu = fa.gmax * fa.nbpg_gu;
-    const int nu = nu_gu + fa.gmax * fa.nbpg_dn;
-    int wsc = 0;  // this warp's running stage count: its ring's phases carry over from unit to unit
-    int ngroups = 1;
-    bool routed = false;
-    for (int u = ((int)blockIdx.x + G - fa.rctas) % G; ok && u < nu; u += G) {
-        const bool GU = u < nu_gu;
-        const int uu = GU ? u : u - nu_gu;
-        const int nbpg = GU ? fa.nbpg_gu : fa.nbpg_dn;
-        const int gs = uu / nbpg, blk = uu % nbpg;
-        if ((gs > 0 || !GU) && !routed) {
-            if (!block_wait(p, fa, &fa.sync[1], 1u, 31, &flags[2])) { ok = false; break; }
-            routed = true;
-            ngroups = __ldcg(p.dec_ngroups);
+    // ---------------------------------------------------------------- the groups of this cluster
+    const int nslots = st.nslots;
+    const int nring = kRingMax;
+    const int rb0 = rank * W + warp;  // this warp's first row block of every stream
+    if (tid == 32) {
+        // every down block of this CTA's groups toward L2 now, and the gate/up blocks of all but the
+        // first (whose streams start at once)
+        for (int s = cid; s < nslots; s += ncl) {
+            const int g = st.groups[s];
+            const int hid = g == E ? p.hs : p.h;
+            const int NJ = d / 64, NJd = hid / 64, nrb = hid / 8, nrbd = d / 16;
+            for (int b = rank * W; b < nrbd; b += CS * W)
+                prefetch_range(p.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)b * NJd * kJP,
+                               (int64_t)min(W, nrbd - b) * NJd * kJP);
+            if (s != cid)
+                for (int b = rank * W; b < nrb; b += CS * W)
+                    prefetch_range(p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * d * 5 / 4) + (int64_t)b * NJ * kJP,
+                                   (int64_t)min(W, nrb - b) * NJ * kJP);
         }
-        if (gs >= ngroups) continue;  // (slot 0, the shared expert, always exists)
-        if (!GU && !block_wait(p, fa, &fa.sync[3 + gs], (uint32_t)fa.nbpg_gu, 32, &flags[3])) { ok = false; break; }
-        const int g = gs == 0 ? E : __ldcg(p.dec_groups + gs);
-        const int hid = g == E ? p.hs : p.h;
-        const int K = GU ? d : hid;
-        const int nrb = GU ? hid / 8 : d / 16;
-        const int nrows = gs == 0 ? T : __ldcg(p.counts + g);
-        const int64_t rrow0 = gs == 0 ? p.Tk : __ldcg(p.offsets + g);
-        const int NJ = K / 64, cs = K + 32, ngr = K / 32;
-        const int rb = blk * W + warp;
-        const bool wact = rb < nrb && nrows > 0;
-        if (GU) {
-            // codes of the group's rows (at most kFusedMaxT: one token selects an expert once), from
-            // this CTA's own x codes, zero rows up to 8
-            for (int it = tid; it < 8 * ngr; it += blockDim.x) {
-                const int i = it / ngr, j = it % ngr;
-                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
-                if (i < nrows) {
-                    const int t = gs == 0 ? i : __ldcg(p.row_src + rrow0 + i);
-                    const uint4* s4 = reinterpret_cast<const uint4*>(xc + t * d + j * 32);
-                    u0 = s4[0];
-                    u1 = s4[1];
-                }
-                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
-                dst[0] = make_uint4(u0.x, u1.x, u0.y, u1.y);
-                dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
-            }
-            if (tid < 16) {
-                uamax[tid] = 0u;
-                // the rows' activation scales
-                const int t = tid < nrows ? (gs == 0 ? tid : __ldcg(p.row_src + rrow0 + tid)) : 0;
-                shs[tid] = tid < nrows ? sxs[t] : 0.0f;
-            }
-        } else {
-            // requantise the group's SwiGLU rows from the gate/up units' absmax
-            if (tid < 8) {
-                uint32_t m = 0u;
-                if (tid < nrows)
-                    for (int v = 0; v < fa.nbpg_gu; ++v)
-                        m = max(m, __ldcg(fa.pamax + ((int64_t)gs * fa.nbpg_gu + v) * 16 + tid));
-                shs[tid] = tid < nrows ? __fdiv_rn(__uint_as_float(m), 127.0f) : 0.0f;
-                if (blk == 0 && tid < nrows) {
-                    p.amax_h[rrow0 + tid] = m;
-                    p.sh[rrow0 + tid] = shs[tid];
-                }
-            }
-            __syncthreads();
-            for (int it = tid; it < 8 * ngr; it += blockDim.x) {
-                const int i = it / ngr, j = it % ngr;
-                uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                if (i < nrows) {
-                    const float sv = shs[i];
-                    const float4* a4 = reinterpret_cast<const float4*>(p.act + (rrow0 + i) * p.hmax + j * 32);
+    }
+    int wsc = 0;      // this warp's running stage count (ring slot and phase)
+    bool alive = ok;  // false once one of this warp's bounded waits gave up
+    WarpStream S;
+    S.ring = ring + warp * nring * kStageBytes;
+    S.bars = st.bars + warp * kRingMax;
+    S.nring = nring;
+    for (int s = cid; s < nslots; s += ncl) {
+        const int g = st.groups[s];
+        const bool shared = g == E;
+        const int hid = shared ? p.hs : p.h;
+        const int nrows = shared ? T : st.cnt[g];
+        const int row0 = shared ? Tk : st.offs[g];
+        // -------------------------------------------------- gate/up: blocks of 8 gate + 8 up rows
+        const int nrb = hid / 8, NJ = d / 64, csz = d + 32, ngr = d / 32;
+        const int np = npasses(rb0, CS * W, nrb);
+        S.src = p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * d * 5 / 4) + (int64_t)rb0 * NJ * kJP;
+        S.pstride = (int64_t)CS * W * NJ * kJP;
+        S.NJ = NJ;
+        S.nst = (NJ + kStageJP - 1) / kStageJP;
+        S.ntot = np * S.nst;
+        S.base = wsc;
+        if (alive && lane == 0)
+            for (int i = 0; i < nring && i < S.ntot; ++i) S.issue(i);
+        // the rows' activation codes, zero rows up to 8
+        for (int it = tid; it < 8 * ngr; it += kCThreads) {
+            const int i = it / ngr, j = it % ngr;
+            uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (i < nrows) {
+                const int t = shared ? i : st.row_tok[row0 + i];
+                const float sx = st.sxs[t];
+                const uint2* x2 = reinterpret_cast<const uint2*>(xs + t * d + j * 32);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const float4 a = __ldcg(a4 + v);
-                        wv[v] = pack_codes(a.x, a.y, a.z, a.w, sv);
-                    }
-                    if (blk == 0) {
-                        uint4* q4 = reinterpret_cast<uint4*>(p.hq + (rrow0 + i) * p.hmax + j * 32);
-                        q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                        q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                    }
+                for (int v = 0; v < 8; ++v) {
+                    const uint2 u = x2[v];
+                    wv[v] = pack_codes(bf16_to_f32(u.x & 0xffffu), bf16_to_f32(u.x >> 16), bf16_to_f32(u.y & 0xffffu),
+                                       bf16_to_f32(u.y >> 16), sx);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
-                dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
-                dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * csz + j * 32);
+            dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
+            dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+        }
+        if (tid < 8) st.shs[tid] = tid < nrows ? st.sxs[shared ? tid : st.row_tok[row0 + tid]] : 0.0f;
+        __syncthreads();
+        for (int pi = 0; pi < np; ++pi) {
+            const int rb = rb0 + pi * CS * W;
+            float alo[1][2], ahi[1][2];
+            S.sc0 = pi * S.nst;
+            if (alive)
+                alive = warp_gemv<true, false, 1>(p, S, codes, csz, lane, rb, row0, nrows, nullptr, 0, 0, alo, ahi);
+            // SwiGLU of rows 2 t4, 2 t4 + 1 at feature n, into every CTA's copy of the rows (and into act)
+            const int n = rb * 8 + gid;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int i = 2 * t4 + q;
+                if (i >= nrows) continue;
+                const float a = alive ? swiglu_row(alo[0][q], ahi[0][q], st.shs[i]) : 0.0f;
+                p.act[(int64_t)(row0 + i) * p.hmax + n] = a;
+#pragma unroll 4
+                for (int c = 0; c < CS; ++c) st_peer(act_all + i * p.hmax + n, c, __float_as_uint(a));
             }
         }
-        __syncthreads();
-        if (wact) {
-            WarpStream S;
-            S.src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
-                        : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
-                    (int64_t)rb * NJ * kJP;
-            S.ring = ring + warp * fa.nring * kStageBytes;
-            S.bars = bars + warp * kRingMax;
-            S.NJ = NJ;
-            S.nst = (NJ + kStageJP - 1) / kStageJP;
-            S.sc0 = wsc;
-            S.nring = fa.nring;
-            if (lane == 0)
-                for (int s = 0; s < fa.nring && s < S.nst; ++s) S.issue(s);
-            const bool alive = GU ? warp_pass<true, false, 1>(p, S, codes, cs, shs, lane, rb, rrow0, nrows, nullptr,
-                                                              0, 0, uamax)
-                                  : warp_pass<false, false, 1>(p, S, codes, cs, shs, lane, rb, rrow0, nrows, nullptr,
-                                                               0, 0, uamax);
-            wsc += S.nst;
-            if (!alive) flags[4] = 1;
+        wsc += S.ntot;
+        // this warp's down blocks start streaming now
+        const int nrbd = d / 16, NJd = hid / 64, cszd = hid + 32, ngh = hid / 32;
+        const int npd = npasses(rb0, CS * W, nrbd);
+        WarpStream D = S;
+        D.src = p.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)rb0 * NJd * kJP;
+        D.pstride = (int64_t)CS * W * NJd * kJP;
+        D.NJ = NJd;
+        D.nst = (NJd + kStageJP - 1) / kStageJP;
+        D.ntot = npd * D.nst;
+        D.base = wsc;
+        __syncwarp();
+        if (alive && lane == 0)
+            for (int i = 0; i < nring && i < D.ntot; ++i) D.issue(i);
+        // -------------------------------------------------- requantisation of the whole rows, in every CTA
+        cluster_sync();  // every CTA's SwiGLU features are in every CTA's copy
+        if (warp < nrows) {
+            float m = 0.0f;
+            for (int n = lane; n < hid; n += 32) m = fmaxf(m, fabsf(act_all[warp * p.hmax + n]));
+            m = warp_max(m);
+            if (lane == 0) {
+                const float sv = __fdiv_rn(m, 127.0f);
+                st.shs[warp] = sv;
+                if (rank == 0) {
+                    p.amax_h[row0 + warp] = __float_as_uint(m);
+                    p.sh[row0 + warp] = sv;
+                }
+            }
+        } else if (warp < 8 && lane == 0) {
+            st.shs[warp] = 0.0f;
         }
         __syncthreads();
-        if (flags[4]) { ok = false; break; }
-        if (GU) {
-            // this unit's absmax of every row (zero for rows it did not touch), then the unit counts as done
-            if (tid < 16) fa.pamax[((int64_t)gs * fa.nbpg_gu + blk) * 16 + tid] = tid < nrows ? uamax[tid] : 0u;
-            __threadfence();
+        for (int it = tid; it < 8 * ngh; it += kCThreads) {
+            const int i = it / ngh, j = it % ngh;
+            uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (i < nrows) {
+                const float sv = st.shs[i];
+                const float4* a4 = reinterpret_cast<const float4*>(act_all + i * p.hmax + j * 32);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 a = a4[v];
+                    wv[v] = pack_codes(a.x, a.y, a.z, a.w, sv);
+                }
+                if (rank == 0) {
+                    uint4* q4 = reinterpret_cast<uint4*>(p.hq + (int64_t)(row0 + i) * p.hmax + j * 32);
+                    q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+                }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cszd + j * 32);
+            dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
+            dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+        }
+        // before this cluster's next group, no CTA may write its SwiGLU values into a copy whose codes
+        // are still being taken
+        if (s + ncl < nslots)
+            cluster_sync();
+        else
             __syncthreads();
-            if (tid == 0) atomicAdd(&fa.sync[3 + gs], 1u);
+        // -------------------------------------------------- down: blocks of 16 output rows
+        for (int pi = 0; pi < npd; ++pi) {
+            const int rb = rb0 + pi * CS * W;
+            float alo[1][2], ahi[1][2];
+            D.sc0 = pi * D.nst;
+            if (alive)
+                alive = warp_gemv<false, false, 1>(p, D, codes, cszd, lane, rb, row0, nrows, nullptr, 0, 0, alo, ahi);
+            const int m0 = rb * 16 + gid;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int i = 2 * t4 + q;
+                if (i >= nrows) continue;
+                const float sv = st.shs[i];
+                ca.obuf[(int64_t)(row0 + i) * d + m0] = __fmul_rn(alo[0][q], sv);
+                ca.obuf[(int64_t)(row0 + i) * d + m0 + 8] = __fmul_rn(ahi[0][q], sv);
+            }
+        }
+        wsc += D.ntot;
+        // -------------------------------------------------- combine of the tokens whose last contribution this is
+        __threadfence();
+        __syncthreads();
+        if (tid < 8) {
+            int t = -1;
+            if (tid < nrows) {
+                const int tt = shared ? tid : st.row_tok[row0 + tid];
+                if (atomicAdd(ca.cnt + tt * CS + rank, 1u) == (uint32_t)k) t = tt;
+            }
+            st.last[tid] = t;
+        }
+        __syncthreads();
+        const int npdmax = npasses(rank * W, CS * W, nrbd);
+        for (int i = 0; i < 8; ++i) {
+            const int t = st.last[i];
+            if (t < 0) continue;
+            __threadfence();
+            for (int it = tid; it < npdmax * W * 4; it += kCThreads) {
+                const int pi = it / (W * 4), w = (it >> 2) % W, c4 = it & 3;
+                const int rb = rank * W + w + pi * CS * W;
+                if (rb >= nrbd) continue;
+                const int m = rb * 16 + c4 * 4;
+                float4 yv = __ldcg(reinterpret_cast<const float4*>(ca.obuf + (int64_t)(Tk + t) * d + m));
+                for (int j = 0; j < k; ++j) {
+                    const float gj = st.gate[t * k + j];
+                    const float4 o =
+                        __ldcg(reinterpret_cast<const float4*>(ca.obuf + (int64_t)st.slot_row[t * k + j] * d + m));
+                    yv.x = __fadd_rn(yv.x, __fmul_rn(gj, o.x));
+                    yv.y = __fadd_rn(yv.y, __fmul_rn(gj, o.y));
+                    yv.z = __fadd_rn(yv.z, __fmul_rn(gj, o.z));
+                    yv.w = __fadd_rn(yv.w, __fmul_rn(gj, o.w));
+                }
+                *reinterpret_cast<float4*>(p.y + (int64_t)t * d + m) = yv;
+            }
+            if (tid == 0) ca.cnt[t * CS + rank] = 0u;
         }
     }
-    // leave; the last CTA out resets the counters for the next launch
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        if (atomicAdd(&fa.sync[2], 1u) == (uint32_t)(G - 1))
-            for (int i = 0; i < kSyncWords; ++i) fa.sync[i] = 0u;
-    }
+    if (!alive && lane == 0) set_error(p, 41);
 }
 
 // INT4 interchange layout -> decode layout (see the top of this file).  For
@@ -1071,53 +1283,115 @@ cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t 
     return cudaLaunchKernelEx(&cfg, kern, p, nbpg, nring, dump, r0, nr);
 }
 
-size_t fused_smem(int d, int K, int nring) {
-    return (size_t)640 + 4 * kFusedMaxT * 64 * 4 + (size_t)kFusedMaxT * d * 3 + (size_t)kFusedWarps * nring * kStageBytes +
-           (size_t)kPassRows * (K + 32);
+size_t align128(size_t v) { return (v + 127) / 128 * 128; }
+
+// Dynamic shared memory of the one-launch decode and its offsets: partial logits from every CTA of
+// the cluster | x (BF16, up to kCMaxT tokens) | operand buffer of 8 rows | SwiGLU values of this CTA's
+// features (also the router's scratch) | the W_r slice, then the rings.
+size_t cluster_layout(int d, int h, int hs, int E, int CS, CArgs* ca) {
+    const int hmax = h > hs ? h : hs;
+    size_t o = align128((size_t)CS * kCMaxT * 64 * 4);
+    const size_t off_x = o;
+    o = align128(o + (size_t)kCMaxT * d * 2);
+    const size_t off_codes = o;
+    o = align128(o + (size_t)8 * ((d > hmax ? d : hmax) + 32));
+    const size_t off_act = o;
+    o = align128(o + std::max((size_t)8 * hmax * 4, (size_t)4 * kCMaxT * 64 * 4));
+    const size_t off_u = o;
+    o += std::max((size_t)(d / CS) * E * 4, (size_t)kCWarps * kRingMax * kStageBytes);
+    if (ca) {
+        ca->off_x = (int)off_x;
+        ca->off_codes = (int)off_codes;
+        ca->off_act = (int)off_act;
+        ca->off_u = (int)off_u;
+    }
+    return o;
+}
+
+template <int CS>
+cudaLaunchConfig_t cluster_config(size_t smem, int nclusters, cudaStream_t s, cudaLaunchAttribute (&at)[2]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nclusters * CS), 1, 1);
+    cfg.blockDim = dim3(kCThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    return cfg;
+}
+
+// Clusters of CS CTAs of the one-launch decode the device holds at once for this shape (0: none).
+template <int CS>
+int cluster_capacity(int d, int h, int hs, int E) {
+    if (d % (CS * 16)) return 0;  // each CTA's K slice of the router: a multiple of 16 rows
+    const size_t smem = cluster_layout(d, h, hs, E, CS, nullptr);
+    if (smem + sizeof(CShared) > (size_t)kSmemLimit) return 0;
+    static int granted[64] = {};
+    if (raise_smem((const void*)decode_cluster_kernel<CS>, granted, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (CS > 8 && cudaFuncSetAttribute(decode_cluster_kernel<CS>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                      cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchAttribute at[2];
+    cudaLaunchConfig_t cfg = cluster_config<CS>(smem, 1, nullptr, at);
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_cluster_kernel<CS>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
 }  // namespace
 }  // namespace dec
 
-int dec_fused_max_tokens() { return dec::kFusedMaxT; }
+int dec_fused_max_tokens() { return dec::kCMaxT; }
 
-bool dec_fused_supported(int d, int hmax) {
-    const int nring = std::max(dec::pick_ring(d), dec::pick_ring(hmax));
-    return dec::fused_smem(d, std::max(d, hmax), nring) <= (size_t)dec::kSmemLimit;
-}
-size_t dec_fused_sync_words() { return dec::kSyncWords; }
-size_t dec_fused_part_floats() { return (size_t)dec::kFusedMaxRouterCtas * dec::kFusedMaxT * 64; }
-size_t dec_fused_pamax_words(int d, int hmax, int E, int k) {
-    const int gmax = (dec::kFusedMaxT * k < E ? dec::kFusedMaxT * k : E) + 1;
-    const int nbpg_gu = (hmax / 8 + dec::kFusedWarps - 1) / dec::kFusedWarps;
-    (void)d;
-    return (size_t)gmax * nbpg_gu * 16;
+DecFusedShape dec_fused_shape(int d, int h, int hs, int E) {
+    DecFusedShape r{};
+    if (E > kMaxExperts || d % 64 || h % 64 || hs % 64) return r;
+    r.clusters8 = dec::cluster_capacity<8>(d, h, hs, E);
+    r.clusters16 = dec::cluster_capacity<16>(d, h, hs, E);
+    return r;
 }
 
-cudaError_t launch_decode_fused(const Plan& p, uint32_t* sync, float* part, uint32_t* pamax, cudaStream_t s) {
+size_t dec_fused_counter_words() { return (size_t)dec::kCMaxT * dec::kCMaxCS; }
+size_t dec_fused_obuf_floats(int d) { return (size_t)dec::kCMaxT * (kMaxTopK + 1) * d; }
+
+cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
+                                int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    dec::FusedArgs fa{};
-    fa.sync = sync;
-    fa.part = part;
-    fa.pamax = pamax;
-    fa.rctas = std::max(1, std::min(p.d / 64, dec::kFusedMaxRouterCtas));
-    fa.nbpg_gu = (p.hmax / 8 + dec::kFusedWarps - 1) / dec::kFusedWarps;
-    fa.nbpg_dn = (p.d / 16 + dec::kFusedWarps - 1) / dec::kFusedWarps;
-    fa.nring = std::max(dec::pick_ring(p.d), dec::pick_ring(p.hmax));
-    fa.gmax = (int)std::min<int64_t>(p.Tk, p.E) + 1;
-    fa.limit = p.wait_limit;
-    const size_t smem = dec::fused_smem(p.d, std::max(p.d, p.hmax), fa.nring);
-    static int granted[64] = {};
-    cudaError_t e = dec::raise_smem((const void*)dec::decode_fused_kernel, granted, smem);
-    if (e != cudaSuccess) return e;
-    // every CTA resident at once (units wait on units of other CTAs)
-    int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dec::decode_fused_kernel, dec::kFusedWarps * 32, smem);
-    if (e != cudaSuccess) return e;
-    const int G = dec::sm_count() * std::min(occ, 2);
-    if (occ < 1 || G < fa.rctas) return cudaErrorInvalidConfiguration;
-    dec::decode_fused_kernel<<<G, dec::kFusedWarps * 32, smem, s>>>(p, fa);
-    return cudaGetLastError();
+    if (p.T > dec::kCMaxT) return cudaErrorInvalidValue;
+    dec::CArgs ca{};
+    ca.cnt = cnt;
+    ca.obuf = obuf;
+    ca.out_idx = out_idx;
+    ca.out_gate = out_gate;
+    ca.out_counts = out_counts;
+    // 16-CTA clusters when one or two tokens leave few groups and every warp of such a cluster has a
+    // row block of a routed expert; else 8
+    const bool big = shape.clusters16 > 0 && p.T <= 2 && std::min(p.h / 8, p.d / 16) >= 16 * dec::kCWarps;
+    cudaLaunchAttribute at[2];
+    if (big) {
+        const size_t smem = dec::cluster_layout(p.d, p.h, p.hs, p.E, 16, &ca);
+        cudaLaunchConfig_t cfg = dec::cluster_config<16>(smem, shape.clusters16, s, at);
+        return cudaLaunchKernelEx(&cfg, dec::decode_cluster_kernel<16>, p, ca);
+    }
+    if (shape.clusters8 <= 0) return cudaErrorInvalidConfiguration;
+    const size_t smem = dec::cluster_layout(p.d, p.h, p.hs, p.E, 8, &ca);
+    cudaLaunchConfig_t cfg = dec::cluster_config<8>(smem, shape.clusters8, s, at);
+    return cudaLaunchKernelEx(&cfg, dec::decode_cluster_kernel<8>, p, ca);
 }
 
 bool dec_supported(int d, int h, int hs) { return d % 64 == 0 && h % 64 == 0 && hs % 64 == 0; }

@@ -153,9 +153,9 @@ struct mmoe_handle {
     // fused one-launch decode: synchronisation words (kept zero between launches), router partials,
     // per-unit SwiGLU absmax
     bool use_dec_fused = false;
-    uint32_t* dec_sync = nullptr;
-    float* dec_part = nullptr;
-    uint32_t* dec_pamax = nullptr;
+    DecFusedShape dec_shape = {};
+    uint32_t* dec_sync = nullptr;  // the one-launch decode's per-token contribution counters
+    float* dec_obuf = nullptr;     // its expert-output rows
     // per-stage timing (mmoe_profile_*)
     struct ProfRec {
         int stage, launches;
@@ -193,7 +193,7 @@ void free_all(mmoe_handle* h) {
                     h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
                     h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->amax_h, h->dec_groups,
                     h->dec_ngroups, h->w_gate_up_f16, h->w_down_f16, h->xq16, h->hq16, h->dec_sync,
-                    h->dec_part, h->dec_pamax};
+                    h->dec_obuf};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     if (h->err_host) cudaFreeHost(h->err_host);
@@ -326,8 +326,8 @@ mmoe_status check_device_flag(mmoe_handle* h, cudaStream_t s) {
     if (v == 0) return MMOE_OK;
     *reinterpret_cast<volatile int*>(h->err_host) = 0;
     cudaMemsetAsync(h->err_dev, 0, sizeof(int), s);
-    // a fused decode that gave up may have left its synchronisation words set
-    if (h->dec_sync) cudaMemsetAsync(h->dec_sync, 0, dec_fused_sync_words() * sizeof(uint32_t), s);
+    // a one-launch decode that gave up may have left contribution counters set
+    if (h->dec_sync) cudaMemsetAsync(h->dec_sync, 0, dec_fused_counter_words() * sizeof(uint32_t), s);
     return fail(MMOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (site %d); its results were not written", v);
 }
 
@@ -508,12 +508,14 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
         ALLOC(amax_h, Rd);
         ALLOC(dec_groups, E + 1);
         ALLOC(dec_ngroups, 1);
-        h->use_dec_fused = !(cfg->flags & MMOE_FLAG_NO_FUSED_DECODE) && dec_fused_supported((int)d, h->hmax);
+        if (!(cfg->flags & MMOE_FLAG_NO_FUSED_DECODE)) {
+            h->dec_shape = dec_fused_shape((int)d, (int)cfg->expert_hidden, (int)cfg->shared_hidden, (int)E);
+            h->use_dec_fused = h->dec_shape.clusters8 > 0;
+        }
         if (h->use_dec_fused) {
-            ALLOC(dec_sync, dec_fused_sync_words());
-            ALLOC(dec_part, dec_fused_part_floats());
-            ALLOC(dec_pamax, dec_fused_pamax_words((int)d, h->hmax, (int)E, (int)k));
-            if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, dec_fused_sync_words() * sizeof(uint32_t));
+            ALLOC(dec_sync, dec_fused_counter_words());
+            ALLOC(dec_obuf, dec_fused_obuf_floats((int)d));
+            if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, dec_fused_counter_words() * sizeof(uint32_t));
         }
     }
     if (e == cudaSuccess) {
@@ -626,12 +628,16 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
     // fixed-order combine: always in deterministic mode; on the prefill path unless atomics were asked for
     p.deterministic = (h->cfg.flags & MMOE_FLAG_DETERMINISTIC) ||
                       (!dec && !(h->cfg.flags & MMOE_FLAG_ATOMIC_COMBINE));
-    const bool fused = dec && h->use_dec_fused && T <= dec_fused_max_tokens() && !p.deterministic;
+    const bool fused = dec && h->use_dec_fused && T <= dec_fused_max_tokens();
     if (fused) {
-        // the whole layer in one launch (routing, gate/up, down, the combine into y)
+        // the whole layer in one launch (routing, gate/up, down, the fixed-order combine into y); it also
+        // writes the caller's copies of the routing
         MMOE_CUDA(run_stage(h, MMOE_PROF_DECODE_FUSED, 1, s,
-                            [&] { return launch_decode_fused(p, h->dec_sync, h->dec_part, h->dec_pamax, s); }),
-                  "fused decode launch");
+                            [&] {
+                                return launch_decode_fused(p, h->dec_shape, h->dec_sync, h->dec_obuf, topk_idx,
+                                                           topk_gate, expert_counts, s);
+                            }),
+                  "one-launch decode");
     } else if (dec) {
         // decode path: router + permutation, gate/up (also clears y), down
         MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_dec(p, h->dec_cluster, s); }),
@@ -658,15 +664,15 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
             MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }), "requant launch");
         MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return run_down(p, s, nullptr, 0, 0); }), "down launch");
     }
-    if (p.deterministic)
+    if (p.deterministic && !fused)
         MMOE_CUDA(run_stage(h, MMOE_PROF_COMBINE, 1, s, [&] { return launch_combine(p, s); }), "combine launch");
-    if (topk_idx)
+    if (topk_idx && !fused)
         MMOE_CUDA(cudaMemcpyAsync(topk_idx, h->idx, (size_t)p.Tk * sizeof(int32_t), cudaMemcpyDeviceToDevice, s),
                   "copy topk_idx");
-    if (topk_gate)
+    if (topk_gate && !fused)
         MMOE_CUDA(cudaMemcpyAsync(topk_gate, h->gate, (size_t)p.Tk * sizeof(float), cudaMemcpyDeviceToDevice, s),
                   "copy topk_gate");
-    if (expert_counts)
+    if (expert_counts && !fused)
         MMOE_CUDA(cudaMemcpyAsync(expert_counts, h->counts, (size_t)(p.E + 1) * sizeof(int32_t),
                                   cudaMemcpyDeviceToDevice, s),
                   "copy expert_counts");

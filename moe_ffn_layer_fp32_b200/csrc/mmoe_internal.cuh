@@ -121,14 +121,19 @@ bool dec_supported(int d, int h, int hs);
 int dec_max_tokens(int d, int hmax);
 int dec_router_cluster(int d, int E);
 cudaError_t launch_router_dec(const Plan& p, int cluster, cudaStream_t s);
-// the fused one-launch decode of up to dec_fused_max_tokens() tokens, with its synchronisation words
-// (zero before the first launch; the kernel leaves them zero), router partials and per-unit absmax
+// the one-launch decode of up to dec_fused_max_tokens() tokens: clusters of 8 or 16 CTAs (how many
+// of each the device holds at once for a shape; 0 where that size does not fit), per-token
+// contribution counters (zero before the first launch; every launch leaves them zero) and a small
+// row buffer of expert outputs
+struct DecFusedShape {
+    int clusters8, clusters16;
+};
 int dec_fused_max_tokens();
-bool dec_fused_supported(int d, int hmax);
-size_t dec_fused_sync_words();
-size_t dec_fused_part_floats();
-size_t dec_fused_pamax_words(int d, int hmax, int E, int k);
-cudaError_t launch_decode_fused(const Plan& p, uint32_t* sync, float* part, uint32_t* pamax, cudaStream_t s);
+DecFusedShape dec_fused_shape(int d, int h, int hs, int E);
+size_t dec_fused_counter_words();
+size_t dec_fused_obuf_floats(int d);
+cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
+                                int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s);
 cudaError_t launch_gate_up_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_retile_dec(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
@@ -218,14 +223,12 @@ __device__ __forceinline__ int quant_i8(float v, float s) {
 // (key descending, index ascending), the key being the logit, or for gating 2
 // the sigmoid score plus the bias (which then moves the selection but enters
 // no gate); writes logits (if kept), idx and gate.
-__device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane) {
-    const int E = p.E, k = p.k;
+// The gating probabilities of experts lane and lane + 32 and their selection keys (the logit, or for
+// gating 2 the sigmoid score plus the bias; -inf where the expert does not exist).
+__device__ __forceinline__ void gate_probs_keys(const Plan& p, float l0, float l1, int lane, float& p0, float& p1,
+                                                float& k0, float& k1) {
+    const int E = p.E;
     const bool v0 = lane < E, v1 = lane + 32 < E;
-    if (p.logits) {
-        if (v0) p.logits[t * E + lane] = l0;
-        if (v1) p.logits[t * E + lane + 32] = l1;
-    }
-    float p0, p1;
     if (p.gating == MMOE_GATE_SOFTMAX) {
         const float mx = warp_max(fmaxf(l0, l1));
         const float e0 = v0 ? expf(__fsub_rn(l0, mx)) : 0.0f;
@@ -237,11 +240,24 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
         p0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l0)));
         p1 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-l1)));
     }
-    float k0 = l0, k1 = l1;
+    k0 = l0;
+    k1 = l1;
     if (p.gating == MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS) {
         k0 = v0 ? (p.router_bias ? __fadd_rn(p0, p.router_bias[lane]) : p0) : -INFINITY;
         k1 = v1 ? (p.router_bias ? __fadd_rn(p1, p.router_bias[lane + 32]) : p1) : -INFINITY;
     }
+}
+
+__device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane, int32_t* idx,
+                                               float* gate, float* logits) {
+    const int E = p.E, k = p.k;
+    const bool v0 = lane < E, v1 = lane + 32 < E;
+    if (logits) {
+        if (v0) logits[t * E + lane] = l0;
+        if (v1) logits[t * E + lane + 32] = l1;
+    }
+    float p0, p1, k0, k1;
+    gate_probs_keys(p, l0, l1, lane, p0, p1, k0, k1);
     bool taken0 = !v0, taken1 = !v1;
     int sel[kMaxTopK];
     float gsel[kMaxTopK];
@@ -271,9 +287,58 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
         for (int j = 0; j < k; ++j)
             if (j == lane) { my = sel[j]; g = gsel[j]; }
         if (p.gating != MMOE_GATE_SOFTMAX) g = __fdiv_rn(g, gsum);
-        p.idx[t * k + lane] = my;
-        p.gate[t * k + lane] = g;
+        idx[t * k + lane] = my;
+        gate[t * k + lane] = g;
     }
+}
+
+__device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane) {
+    gate_topk_warp(p, t, l0, l1, lane, p.idx, p.gate, p.logits);
+}
+
+// The same gating and top-k as gate_topk_warp (the same probabilities and the same order: key
+// descending, the lower index first among equal keys), with each expert's position found by counting
+// the experts ahead of it in a copy of the keys in shared memory (`keys`: 64 floats, `selp`: k floats,
+// both private to the warp) instead of k rounds of warp arg-max.
+__device__ __forceinline__ void gate_topk_rank(const Plan& p, int64_t t, float l0, float l1, int lane, float* keys,
+                                               float* selp, int32_t* idx, float* gate, float* logits) {
+    const int E = p.E, k = p.k;
+    const bool v0 = lane < E, v1 = lane + 32 < E;
+    if (logits) {
+        if (v0) logits[t * E + lane] = l0;
+        if (v1) logits[t * E + lane + 32] = l1;
+    }
+    float p0, p1, k0, k1;
+    gate_probs_keys(p, l0, l1, lane, p0, p1, k0, k1);
+    keys[lane] = k0;
+    keys[lane + 32] = k1;
+    __syncwarp();
+    int r0 = 0, r1 = 0;
+#pragma unroll 4
+    for (int e = 0; e < E; ++e) {
+        const float ke = keys[e];
+        r0 += (ke > k0) || (ke == k0 && e < lane);
+        r1 += (ke > k1) || (ke == k1 && e < lane + 32);
+    }
+    if (v0 && r0 < k) {
+        idx[t * k + r0] = lane;
+        selp[r0] = p0;
+    }
+    if (v1 && r1 < k) {
+        idx[t * k + r1] = lane + 32;
+        selp[r1] = p1;
+    }
+    __syncwarp();
+    if (lane < k) {
+        float g = selp[lane];
+        if (p.gating != MMOE_GATE_SOFTMAX) {
+            float gsum = 0.0f;
+            for (int j = 0; j < k; ++j) gsum = __fadd_rn(gsum, selp[j]);
+            g = __fdiv_rn(g, gsum);
+        }
+        gate[t * k + lane] = g;
+    }
+    __syncwarp();
 }
 
 // The router bias enters the logit for gating 0 and 1 (and only the selection key for gating 2).
