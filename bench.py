@@ -247,19 +247,45 @@ def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8), name="c1"):
             g.replay()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        us_layer = e0.elapsed_time(e1) * 1e3 / (steps * w.layers)
+        us_sep = e0.elapsed_time(e1) * 1e3 / (steps * w.layers)
         # algorithmic bytes of the last step: the distinct experts each layer selected, the shared one, W_r
         nbytes = 0.0
         for l in range(w.layers):
             ex = sorted(set(idx[l].cpu().numpy().ravel().tolist()) | {w.E})
             nbytes += weight_bytes(w, ex) + w.d * w.E * 4
         nbytes /= w.layers
+        del g
+        # the same stack through mmoe_forward_chain: for up to 8 tokens one launch runs all layers (layer
+        # l + 1 rounding layer l's y to BF16 itself); the same outputs bit for bit
+        MoELayer.forward_chain(layers, xs[0], ys)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            MoELayer.forward_chain(layers, xs[0], ys)
+        for s in range(warmup):
+            xs[0].copy_(x0[s])
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for s in range(steps):
+            xs[0].copy_(x0[warmup + s])
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        us_layer = e0.elapsed_time(e1) * 1e3 / (steps * w.layers)
+        del g
         gbs = nbytes / (us_layer * 1e-6) / 1e9
+        one = T <= 8
         out[f"T{T}"] = {"us_per_layer": us_layer, "bytes_per_layer": nbytes, "achieved_gbs": gbs,
                         "hbm_frac": gbs / hbm_gbs, "hbm_peak_gbs": hbm_gbs,
-                        "launches_per_layer": 1 if T <= 8 else 3,
-                        "kernels": "one-launch fused decode" if T <= 8 else "router, gate/up, down"}
-        del g
+                        "api": "mmoe_forward_chain (24 layers)",
+                        "launches_per_layer": 1.0 / w.layers if one else 4,
+                        "kernels": ("one launch of the one-launch decode for the 24-layer stack" if one
+                                    else "router, gate/up, down and a BF16 rounding per layer"),
+                        "us_per_layer_separate_forwards": us_sep,
+                        "separate_forwards": ("mmoe_forward per layer (one launch each) and a torch BF16 copy"
+                                              if one else "mmoe_forward per layer (three launches) and a torch "
+                                              "BF16 copy")}
     for L in layers:
         L.close()
     return out

@@ -91,10 +91,11 @@ typedef enum {
                                       (T <= 64 where d_model and both hidden sizes are multiples of 64)
                                       runs the weight-streaming decode kernels; same results */
 #define MMOE_FLAG_NO_FUSED_DECODE 32u /* a forward of at most 8 tokens on the decode path runs the layer as
-                                      one launch of a persistent grid by default (routing, gate/up and
-                                      down in one kernel, the next step of a token starting as soon as
-                                      what it needs is done); this flag keeps the three launches of the
-                                      larger decode batches; same results */
+                                      one launch of thread-block clusters by default (each cluster routes
+                                      the tokens itself and computes whole experts; y is added in the
+                                      fixed order of Eq. (*)); this flag keeps the three launches of the
+                                      larger decode batches; the same routing and codes, y within
+                                      FP32 rounding of the router's summation order */
 #define MMOE_FLAG_FUSED_REQUANT 64u /* the prefill gate/up GEMM (default tensor-core kind) requantises its
                                       SwiGLU output itself: the CTAs that hold the hidden-feature blocks of
                                       a token tile form a cluster and exchange the per-token maxima through
@@ -192,6 +193,30 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, floa
  * describe the last chunk.  Errors: as mmoe_forward. */
 mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_bf16_host, int64_t T, float* y_host,
                               void* stream);
+
+/* Layers one after another on the same tokens, as in a decoder stack: layer 0
+ * reads x (BF16, device, [T, d_model]); layer l + 1 reads layer l's y rounded
+ * to BF16 (round to nearest even); y_layers[l] (device, FP32 [T, d_model], each
+ * 16-byte aligned) receives layer l's y.  layers[l] is the handle of layer l
+ * (host array of n_layers handles; y_layers likewise a host array of device
+ * pointers).  Every handle must be loaded, on the same device and created with
+ * the same d_model, n_experts, top_k, expert_hidden, shared_hidden and gating.
+ * When layer 0's handle runs the one-launch decode and T <= 8, the whole stack
+ * is ONE launch: its clusters move from layer to layer, each layer's router
+ * starting once every column of the previous layer's y has been combined (a
+ * bounded wait on a counter in global memory: TIMEOUT on the next call if it
+ * gave up), with the next layer's router weights and shared expert fetched
+ * during the current layer.  That launch uses layer 0's workspace; the
+ * inspection functions of the other handles are not updated.  Otherwise each
+ * layer is one mmoe_forward on its own handle, with the BF16 rounding of y in
+ * between.  Either way each layer's y equals that of mmoe_forward on the
+ * rounded input, within FP32 rounding of the router's summation order.
+ * Errors: INVALID_ARG (n_layers outside [1, MMOE_MAX_CHAIN_LAYERS], NULL or
+ * mismatched handles, T outside [0, max_tokens] of any handle, NULL or
+ * misaligned pointers), NOT_LOADED, TIMEOUT, OOM, CUDA. */
+#define MMOE_MAX_CHAIN_LAYERS 32
+mmoe_status mmoe_forward_chain(mmoe_handle* const* layers, int32_t n_layers, const uint16_t* x_bf16, int64_t T,
+                               float* const* y_layers, void* stream);
 
 /* Waits for the handle's pending work, frees everything it owns and the
  * handle itself.  NULL is accepted (no-op). */

@@ -32,7 +32,8 @@ STAGE_XQ, STAGE_SX, STAGE_OFFSETS, STAGE_ROW_SRC, STAGE_SLOT_ROW, STAGE_HQ, STAG
 EXPORTS = ("mmoe_create", "mmoe_load_quantized_weights", "mmoe_forward", "mmoe_forward_host", "mmoe_destroy",
            "mmoe_last_error", "mmoe_quantize_int4", "mmoe_debug_copy_stage", "mmoe_debug_partials",
            "mmoe_profile_enable", "mmoe_profile_read", "mmoe_forward_static_scratch", "mmoe_debug_host_chunks",
-           "mmoe_debug_set_wait_limit", "mmoe_debug_fail_alloc")
+           "mmoe_debug_set_wait_limit", "mmoe_debug_fail_alloc", "mmoe_forward_chain")
+MAX_CHAIN_LAYERS = 32
 
 STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 
@@ -86,6 +87,7 @@ def lib() -> C.CDLL:
     L.mmoe_debug_host_chunks.argtypes = [i64, vp, i32, vp]
     L.mmoe_debug_set_wait_limit.argtypes = [vp, i64, i32]
     L.mmoe_debug_fail_alloc.argtypes = [i64]
+    L.mmoe_forward_chain.argtypes = [C.POINTER(vp), i32, vp, i64, C.POINTER(vp), vp]
     for name in EXPORTS:
         if name != "mmoe_last_error":
             getattr(L, name).restype = st

@@ -26,6 +26,8 @@
 //  3. expert_decode_kernel<down>: requantises its group's rows from that
 //     absmax in the prologue, then the same streaming GEMV; the epilogue adds
 //     gate * o into y (or stores o for the fixed-order combine).
+#include <cuda_bf16.h>
+
 #include <algorithm>
 
 #include "mmoe_internal.cuh"
@@ -702,15 +704,28 @@ constexpr int kCWarps = 8;
 constexpr int kCThreads = kCWarps * 32;
 constexpr int kCMaxCS = 16;
 constexpr int kCMaxSlots = kCMaxT * kMaxTopK;
+constexpr int kMaxChain = kDecChainMax;
+
+// One layer's weights and outputs (the layers of one launch share every shape).
+struct LayerW {
+    const float* w_router;
+    const float* router_bias;
+    const uint8_t* w_gate_up_d;
+    const uint8_t* w_down_d;
+    float* y;             // [T, d]
+    int32_t* out_idx;     // optional copies of the routing for the caller: [T, k]
+    float* out_gate;      // [T, k]
+    int32_t* out_counts;  // [E + 1]
+};
 
 struct CArgs {
     uint32_t* cnt;        // [kCMaxT][CS] contribution counters, zero at launch (the last user resets one)
     float* obuf;          // [kCMaxT * (kMaxTopK + 1)][d] expert outputs, rows as in the permutation
-    int32_t* out_idx;     // optional copies of the routing for the caller: [T, k]
-    float* out_gate;      // [T, k]
-    int32_t* out_counts;  // [E + 1]
-    // dynamic shared memory offsets
-    int off_x, off_codes, off_act, off_u;
+    uint32_t* chain;      // [2]: y columns combined over the launch, CTAs that left (zero at launch; reset by
+                          // the last CTA to leave)
+    int nl;               // layers in this launch; layer l + 1 reads layer l's y rounded to BF16
+    int off_x, off_codes, off_act, off_wr, off_u;  // dynamic shared memory offsets
+    LayerW layers[kMaxChain];
 };
 
 struct CShared {
@@ -718,8 +733,8 @@ struct CShared {
     uint64_t wbar, xbar;
     float sxs[kCMaxT];             // activation scales of the tokens
     float shs[8];                  // per row of the current group: activation scale, then SwiGLU scale
-    float keys[kCWarps][64];       // top-k: each warp's copy of its token's selection keys
-    float selp[kCWarps][kMaxTopK]; //   and the probabilities of the selected experts
+    float keys[kCMaxT][64];        // top-k: each token's selection keys
+    float probs[kCMaxT][64];       //   and gating probabilities
     int idx[kCMaxSlots];
     float gate[kCMaxSlots];
     int slot_row[kCMaxSlots];
@@ -729,6 +744,7 @@ struct CShared {
     int groups[kMaxExperts + 1];
     int nslots;
     int last[8];
+    int flag;
 };
 
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -750,11 +766,53 @@ __device__ __forceinline__ void st_peer(const void* p, int rank, float4 v) {
                  : "memory");
 }
 
+// position of word v (features 4v .. 4v + 3) of a 32-element group in the B-fragment order of an operand
+// row: words 0, 4, 1, 5, 2, 6, 3, 7
+__device__ __forceinline__ int bfrag_pos(int v) { return v < 4 ? 2 * v : 2 * (v - 4) + 1; }
+
 // number of passes pi >= 0 with first + pi * step < n
 __device__ __forceinline__ int npasses(int first, int step, int n) { return first < n ? (n - first + step - 1) / step : 0; }
 
+// two floats rounded to BF16 (round to nearest even; finite inputs), packed low | high << 16
+__device__ __forceinline__ uint32_t bf16_pair_rn(float a, float b) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// The shared expert of a layer toward L2: this CTA's gate/up and down row blocks (one thread).
 template <int CS>
-__global__ void __launch_bounds__(kCThreads) decode_cluster_kernel(Plan p, CArgs ca)
+__device__ void prefetch_shared_expert(const Plan& p, const LayerW& Lw, int rank) {
+    const int W = kCWarps, d = p.d, E = p.E;
+    const int NJ = d / 64, NJd = p.hs / 64, nrb = p.hs / 8, nrbd = d / 16;
+    for (int b0 = rank * W; b0 < nrb; b0 += CS * W)
+        prefetch_range(Lw.w_gate_up_d + (int64_t)E * ((int64_t)p.h * d * 5 / 4) + (int64_t)b0 * NJ * kJP,
+                       (int64_t)min(W, nrb - b0) * NJ * kJP);
+    for (int b0 = rank * W; b0 < nrbd; b0 += CS * W)
+        prefetch_range(Lw.w_down_d + (int64_t)E * ((int64_t)d * p.h * 5 / 8) + (int64_t)b0 * NJd * kJP,
+                       (int64_t)min(W, nrbd - b0) * NJd * kJP);
+}
+
+// The gate/up weight stream of one warp over group g of a layer: row blocks rb0, rb0 + CS W, ...
+template <int CS>
+__device__ __forceinline__ void gu_stream(WarpStream& S, const Plan& p, const LayerW& Lw, int g, int rb0, int base) {
+    const int hid = g == p.E ? p.hs : p.h, nrb = hid / 8, NJ = p.d / 64;
+    const int np = npasses(rb0, CS * kCWarps, nrb);
+    S.src = Lw.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4) + (int64_t)rb0 * NJ * kJP;
+    S.pstride = (int64_t)CS * kCWarps * NJ * kJP;
+    S.NJ = NJ;
+    S.nst = (NJ + kStageJP - 1) / kStageJP;
+    S.ntot = np * S.nst;
+    S.base = base;
+}
+
+template <int CS>
+__global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CArgs ca)
 {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ CShared st;
@@ -766,11 +824,12 @@ __global__ void __launch_bounds__(kCThreads) decode_cluster_kernel(Plan p, CArgs
     const int ks = d / CS;
     const bool keeper = cid == 0 && rank == 0;  // writes the routing and permutation for inspection
     float* part_recv = reinterpret_cast<float*>(smem);                       // [CS][kCMaxT][64]
-    const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem + ca.off_x); // [T][d]
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + ca.off_x);             // [T][d]
     uint8_t* codes = smem + ca.off_codes;                                    // [8][max(d, hmax) + 32]
     float* act_all = reinterpret_cast<float*>(smem + ca.off_act);            // [8 rows][hmax] SwiGLU values
-    uint8_t* ring = smem + ca.off_u;                                         // W_r slice, then the rings
-    const float* wr = reinterpret_cast<const float*>(ring);
+    float* wr = reinterpret_cast<float*>(smem + ca.off_wr);                  // this CTA's slice of W_r
+    uint8_t* ring = smem + ca.off_u;                                         // the warps' rings
+    const uint32_t wbytes = (uint32_t)(ks * E * 4);
 
     // first half of a cluster barrier: this CTA has started (its shared memory may be written by peers
     // once the second half has been waited for)
@@ -781,382 +840,454 @@ __global__ void __launch_bounds__(kCThreads) decode_cluster_kernel(Plan p, CArgs
         mbar_init(&st.wbar, 1);
         mbar_init(&st.xbar, 1);
         fence_barrier_init();
-        // this CTA's K slice of W_r, rows [rank ks, (rank + 1) ks): weights, not outputs of the previous launch
-        const uint32_t wbytes = (uint32_t)(ks * E * 4);
+        // layer 0's K slice of W_r, rows [rank ks, (rank + 1) ks): weights, not outputs of the previous launch
         mbar_expect_tx(&st.wbar, wbytes);
-        bulk_load(ring, p.w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
+        bulk_load(wr, ca.layers[0].w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
     }
-    if (cid == 0 && tid == 32) {
-        // the shared expert (slot 0, this cluster's first group) toward L2: this CTA's gate/up and down blocks
-        const int NJ = d / 64, NJd = p.hs / 64, nrb = p.hs / 8, nrbd = d / 16;
-        for (int b0 = rank * W; b0 < nrb; b0 += CS * W)
-            prefetch_range(p.w_gate_up_d + (int64_t)E * ((int64_t)p.h * d * 5 / 4) + (int64_t)b0 * NJ * kJP,
-                           (int64_t)min(W, nrb - b0) * NJ * kJP);
-        for (int b0 = rank * W; b0 < nrbd; b0 += CS * W)
-            prefetch_range(p.w_down_d + (int64_t)E * ((int64_t)d * p.h * 5 / 8) + (int64_t)b0 * NJd * kJP,
-                           (int64_t)min(W, nrbd - b0) * NJd * kJP);
-    }
+    if (cid == 0 && tid == 32) prefetch_shared_expert<CS>(p, ca.layers[0], rank);
     __syncthreads();  // the mbarriers are initialised
     pdl_wait();       // x, and the buffers the previous launch used
-    if (tid == 0) {
-        const uint32_t xbytes = (uint32_t)(T * d * 2);
-        mbar_expect_tx(&st.xbar, xbytes);
-        bulk_load(smem + ca.off_x, p.x, xbytes, &st.xbar);
-    }
-    bool ok = wait_bounded(&st.xbar, 0);
-    for (int t = warp; t < T; t += W) {
-        float m = 0.0f;
-        for (int i = lane; i < d; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * d + i])));
-        m = warp_max(m);
-        if (lane == 0) st.sxs[t] = __fdiv_rn(m, 127.0f);
-    }
-    ok = wait_bounded(&st.wbar, 0) && ok;
-    if (!ok && tid == 0) set_error(p, 40);
-
-    // ---------------------------------------------------------------- router
-    // thread (q, e): FP32 products of K rows [q ks / 4, (q + 1) ks / 4) of the slice, each token, four K
-    // rows per step (kq is a multiple of 4)
-    {
-        const int e = tid & 63, q = tid >> 6, kq = ks / 4;
-        float acc[kCMaxT];
-#pragma unroll
-        for (int t = 0; t < kCMaxT; ++t) acc[t] = 0.0f;
-        if (e < E && ok) {
-            const uint16_t* xk = xs + rank * ks + q * kq;
-            const float* wk = wr + (q * kq) * E + e;
-#pragma unroll 2
-            for (int kk = 0; kk < kq; kk += 4) {
-                const float w0 = wk[kk * E], w1 = wk[(kk + 1) * E], w2 = wk[(kk + 2) * E], w3 = wk[(kk + 3) * E];
-#pragma unroll
-                for (int t = 0; t < kCMaxT; ++t)
-                    if (t < T) {
-                        const uint2 xv = *reinterpret_cast<const uint2*>(xk + t * d + kk);
-                        acc[t] = fmaf(bf16_to_f32(xv.x & 0xffffu), w0, acc[t]);
-                        acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w1, acc[t]);
-                        acc[t] = fmaf(bf16_to_f32(xv.y & 0xffffu), w2, acc[t]);
-                        acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w3, acc[t]);
-                    }
-            }
-        }
-        float* rq = act_all;  // scratch until the first group's SwiGLU: [4][kCMaxT][64]
-#pragma unroll
-        for (int t = 0; t < kCMaxT; ++t) rq[(q * kCMaxT + t) * 64 + e] = acc[t];
-    }
-    __syncthreads();
-    cluster_wait();  // every CTA of the cluster has started
-    for (int i = tid; i < T * 16; i += kCThreads) {
-        const int t = i >> 4, e4 = (i & 15) * 4;
-        const float* rq = act_all;
-        float v[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int o = t * 64 + e4 + c;
-            v[c] = __fadd_rn(__fadd_rn(__fadd_rn(rq[o], rq[kCMaxT * 64 + o]), rq[2 * kCMaxT * 64 + o]),
-                             rq[3 * kCMaxT * 64 + o]);
-        }
-        const float4 v4 = make_float4(v[0], v[1], v[2], v[3]);
-#pragma unroll 4
-        for (int c = 0; c < CS; ++c) st_peer(part_recv + (rank * kCMaxT + t) * 64 + e4, c, v4);
-    }
-    cluster_sync();  // every slice's partial logits are here
-    for (int t = warp; t < T; t += W) {
-        float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-        for (int c = 0; c < CS; ++c) {
-            s0 = __fadd_rn(s0, part_recv[(c * kCMaxT + t) * 64 + lane]);
-            s1 = __fadd_rn(s1, part_recv[(c * kCMaxT + t) * 64 + lane + 32]);
-        }
-        const float l0 = lane < E ? biased_logit(p, s0, lane) : -INFINITY;
-        const float l1 = lane + 32 < E ? biased_logit(p, s1, lane + 32) : -INFINITY;
-        gate_topk_rank(p, t, l0, l1, lane, st.keys[warp], st.selp[warp], st.idx, st.gate, keeper ? p.logits : nullptr);
-    }
-    __syncthreads();
-    // ---------------------------------------------------------------- permutation (warp 0)
-    if (warp == 0) {
-        // per-expert counts (experts lane, lane + 32) and each slot's rank among the earlier slots of its
-        // expert (slots lane, lane + 32), by one pass over the slots
-        const int s0 = lane, s1 = lane + 32;
-        const int e0 = s0 < Tk ? st.idx[s0] : -1, e1 = s1 < Tk ? st.idx[s1] : -1;
-        int c0 = 0, c1 = 0, r0 = 0, r1 = 0;
-#pragma unroll 4
-        for (int sl = 0; sl < Tk; ++sl) {
-            const int e = st.idx[sl];
-            c0 += e == lane;
-            c1 += e == lane + 32;
-            r0 += sl < s0 && e == e0;
-            r1 += sl < s1 && e == e1;
-        }
-        if (lane >= E) c0 = 0;
-        if (lane + 32 >= E) c1 = 0;
-        st.cnt[lane] = c0;
-        st.cnt[lane + 32] = c1;
-        int i0 = c0, i1 = c1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
-            if (lane >= o) { i0 += u0; i1 += u1; }
-        }
-        i1 += __shfl_sync(0xffffffffu, i0, 31);
-        const unsigned lt = (1u << lane) - 1u;
-        const unsigned b0 = __ballot_sync(0xffffffffu, c0 > 0), b1 = __ballot_sync(0xffffffffu, c1 > 0);
-        st.offs[lane] = i0 - c0;
-        st.offs[lane + 32] = i1 - c1;
-        if (c0) st.groups[1 + __popc(b0 & lt)] = lane;
-        if (c1) st.groups[1 + __popc(b0) + __popc(b1 & lt)] = lane + 32;
-        __syncwarp();
-        if (lane == 0) {
-            st.groups[0] = E;
-            st.nslots = 1 + __popc(b0) + __popc(b1);
-            st.offs[E] = Tk;
-            st.offs[E + 1] = Tk + T;
-        }
-        __syncwarp();
-        if (e0 >= 0) {
-            const int r = st.offs[e0] + r0;
-            st.slot_row[s0] = r;
-            st.row_tok[r] = s0 / k;
-        }
-        if (e1 >= 0) {
-            const int r = st.offs[e1] + r1;
-            st.slot_row[s1] = r;
-            st.row_tok[r] = s1 / k;
-        }
-    }
-    __syncthreads();
-    if (keeper) {
-        // the routing and the permutation, as the three-launch path leaves them
-        for (int i = tid; i < Tk; i += kCThreads) {
-            p.idx[i] = st.idx[i];
-            p.gate[i] = st.gate[i];
-            p.slot_row[i] = st.slot_row[i];
-            p.row_src[st.slot_row[i]] = i / k;
-            p.row_gate[st.slot_row[i]] = st.gate[i];
-            if (ca.out_idx) ca.out_idx[i] = st.idx[i];
-            if (ca.out_gate) ca.out_gate[i] = st.gate[i];
-        }
-        for (int t = tid; t < T; t += kCThreads) {
-            p.sx[t] = st.sxs[t];
-            p.row_src[Tk + t] = t;
-            p.row_gate[Tk + t] = 1.0f;
-        }
-        for (int e = tid; e <= E + 1; e += kCThreads) {
-            p.offsets[e] = st.offs[e];
-            if (e <= E) {
-                const int c = e < E ? st.cnt[e] : T;
-                p.counts[e] = c;
-                if (ca.out_counts) ca.out_counts[e] = c;
-            }
-        }
-        for (int i = tid; i < st.nslots; i += kCThreads) p.dec_groups[i] = st.groups[i];
-        if (tid == 0) *p.dec_ngroups = st.nslots;
-    }
-    if (cid == 0) {
-        // the shared rows' activation codes (this CTA's K slice), kept for inspection
-        for (int i = tid; i < T * (ks / 4); i += kCThreads) {
-            const int t = i / (ks / 4), v = i % (ks / 4);
-            const uint16_t* xr = xs + t * d + rank * ks + v * 4;
-            *reinterpret_cast<uint32_t*>(p.xq + (int64_t)(Tk + t) * d + rank * ks + v * 4) =
-                pack_codes(bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), st.sxs[t]);
-        }
-    }
-
-    // ---------------------------------------------------------------- the groups of this cluster
-    const int nslots = st.nslots;
-    const int nring = kRingMax;
+    bool ok = true;
+    int wsc = 0;      // this warp's running stage count (ring slot and phase), over all layers
+    bool alive = true;  // false once one of this warp's bounded waits gave up
+    WarpStream S;
+    S.ring = ring + warp * kRingMax * kStageBytes;
+    S.bars = st.bars + warp * kRingMax;
+    S.nring = kRingMax;
     const int rb0 = rank * W + warp;  // this warp's first row block of every stream
-    if (tid == 32) {
-        // every down block of this CTA's groups toward L2 now, and the gate/up blocks of all but the
-        // first (whose streams start at once)
+
+    for (int l = 0; l < ca.nl; ++l) {
+        const LayerW& Lw = ca.layers[l];
+        // ------------------------------------------------------------ this layer's x
+        if (l == 0) {
+            if (tid == 0) {
+                const uint32_t xbytes = (uint32_t)(T * d * 2);
+                mbar_expect_tx(&st.xbar, xbytes);
+                bulk_load(xs, p.x, xbytes, &st.xbar);
+            }
+            ok = wait_bounded(&st.xbar, 0) && ok;
+        } else {
+            // every combine of layer l - 1 is done, so its y is complete; x = its BF16 rounding
+            if (tid == 0) {
+                int good = 1;
+                const uint32_t target = (uint32_t)(l * T * CS);
+                if (ld_acquire(ca.chain) < target) {
+                    const long long t0 = clk();
+                    while (ld_acquire(ca.chain) < target) {
+                        if (clk() - t0 > p.wait_limit) {
+                            good = 0;
+                            set_error(p, 42);
+                            break;
+                        }
+                    }
+                }
+                st.flag = good;
+            }
+            __syncthreads();
+            ok = ok && st.flag;
+            const float4* y4 = reinterpret_cast<const float4*>(ca.layers[l - 1].y);
+            uint2* x2 = reinterpret_cast<uint2*>(xs);
+            for (int i = tid; i < T * d / 4; i += kCThreads) {
+                const float4 v = __ldcg(y4 + i);
+                x2[i] = make_uint2(bf16_pair_rn(v.x, v.y), bf16_pair_rn(v.z, v.w));
+            }
+            __syncthreads();
+        }
+        // activation scales: warp t, the absmax of token t over d
+        for (int t = warp; t < T; t += W) {
+            float m = 0.0f;
+            for (int i = lane; i < d; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * d + i])));
+            m = warp_max(m);
+            if (lane == 0) st.sxs[t] = __fdiv_rn(m, 127.0f);
+        }
+        ok = wait_bounded(&st.wbar, (uint32_t)(l & 1)) && ok;
+        if (!ok && tid == 0) set_error(p, 40);
+
+        // ------------------------------------------------------------ router
+        // thread (q, e): FP32 products of K rows [q ks / 4, (q + 1) ks / 4) of the slice, each token, four K
+        // rows per step (kq is a multiple of 4)
+        {
+            const int e = tid & 63, q = tid >> 6, kq = ks / 4;
+            float acc[kCMaxT];
+#pragma unroll
+            for (int t = 0; t < kCMaxT; ++t) acc[t] = 0.0f;
+            if (e < E && ok) {
+                const uint16_t* xk = xs + rank * ks + q * kq;
+                const float* wk = wr + (q * kq) * E + e;
+#pragma unroll 2
+                for (int kk = 0; kk < kq; kk += 4) {
+                    const float w0 = wk[kk * E], w1 = wk[(kk + 1) * E], w2 = wk[(kk + 2) * E], w3 = wk[(kk + 3) * E];
+#pragma unroll
+                    for (int t = 0; t < kCMaxT; ++t)
+                        if (t < T) {
+                            const uint2 xv = *reinterpret_cast<const uint2*>(xk + t * d + kk);
+                            acc[t] = fmaf(bf16_to_f32(xv.x & 0xffffu), w0, acc[t]);
+                            acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w1, acc[t]);
+                            acc[t] = fmaf(bf16_to_f32(xv.y & 0xffffu), w2, acc[t]);
+                            acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w3, acc[t]);
+                        }
+                }
+            }
+            float* rq = act_all;  // scratch until the first group's SwiGLU: [4][kCMaxT][64]
+#pragma unroll
+            for (int t = 0; t < kCMaxT; ++t) rq[(q * kCMaxT + t) * 64 + e] = acc[t];
+        }
+        __syncthreads();
+        if (l + 1 < ca.nl && tid == 0) {
+            // every thread is done with this layer's W_r slice: the next layer's goes in now
+            mbar_expect_tx(&st.wbar, wbytes);
+            bulk_load(wr, ca.layers[l + 1].w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
+        }
+        if (l == 0) cluster_wait();  // every CTA of the cluster has started
+        for (int i = tid; i < T * 16; i += kCThreads) {
+            const int t = i >> 4, e4 = (i & 15) * 4;
+            const float* rq = act_all;
+            float v[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int o = t * 64 + e4 + c;
+                v[c] = __fadd_rn(__fadd_rn(__fadd_rn(rq[o], rq[kCMaxT * 64 + o]), rq[2 * kCMaxT * 64 + o]),
+                                 rq[3 * kCMaxT * 64 + o]);
+            }
+            const float4 v4 = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll 4
+            for (int c = 0; c < CS; ++c) st_peer(part_recv + (rank * kCMaxT + t) * 64 + e4, c, v4);
+        }
+        cluster_sync();  // every slice's partial logits are here
+        // gating: warp t adds token t's slices in rank order and computes its probabilities and keys
+        for (int t = warp; t < T; t += W) {
+            float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+            for (int c = 0; c < CS; ++c) {
+                s0 = __fadd_rn(s0, part_recv[(c * kCMaxT + t) * 64 + lane]);
+                s1 = __fadd_rn(s1, part_recv[(c * kCMaxT + t) * 64 + lane + 32]);
+            }
+            const float l0 = lane < E ? biased_logit(p, Lw.router_bias, s0, lane) : -INFINITY;
+            const float l1 = lane + 32 < E ? biased_logit(p, Lw.router_bias, s1, lane + 32) : -INFINITY;
+            if (keeper && p.logits) {
+                if (lane < E) p.logits[t * E + lane] = l0;
+                if (lane + 32 < E) p.logits[t * E + lane + 32] = l1;
+            }
+            float p0, p1, k0, k1;
+            gate_probs_keys(p, Lw.router_bias, l0, l1, lane, p0, p1, k0, k1);
+            st.keys[t][lane] = k0;
+            st.keys[t][lane + 32] = k1;
+            st.probs[t][lane] = p0;
+            st.probs[t][lane + 32] = p1;
+        }
+        __syncwarp();
+        // top-k: an expert's position is the number of experts ahead of it (key descending, the lower index
+        // first among equal keys); warp t counts for token t, experts lane and lane + 32
+        for (int t = warp; t < T; t += W) {
+            const float k0 = st.keys[t][lane], k1 = st.keys[t][lane + 32];
+            int r0 = 0, r1 = 0;
+#pragma unroll 4
+            for (int f = 0; f < E; ++f) {
+                const float kf = st.keys[t][f];
+                r0 += (kf > k0) || (kf == k0 && f < lane);
+                r1 += (kf > k1) || (kf == k1 && f < lane + 32);
+            }
+            if (lane < E && r0 < k) {
+                st.idx[t * k + r0] = lane;
+                st.gate[t * k + r0] = st.probs[t][lane];
+            }
+            if (lane + 32 < E && r1 < k) {
+                st.idx[t * k + r1] = lane + 32;
+                st.gate[t * k + r1] = st.probs[t][lane + 32];
+            }
+        }
+        __syncthreads();
+        if (p.gating != MMOE_GATE_SOFTMAX && tid < T) {
+            // top-k normalisation, the selected probabilities added in top-k order
+            float gsum = 0.0f;
+            for (int j = 0; j < k; ++j) gsum = __fadd_rn(gsum, st.gate[tid * k + j]);
+            for (int j = 0; j < k; ++j) st.gate[tid * k + j] = __fdiv_rn(st.gate[tid * k + j], gsum);
+        }
+        __syncthreads();
+        // ------------------------------------------------------------ permutation (warp 0)
+        if (warp == 0) {
+            // per-expert counts (experts lane, lane + 32) and each slot's rank among the earlier slots of its
+            // expert (slots lane, lane + 32), by one pass over the slots
+            const int s0 = lane, s1 = lane + 32;
+            const int e0 = s0 < Tk ? st.idx[s0] : -1, e1 = s1 < Tk ? st.idx[s1] : -1;
+            int c0 = 0, c1 = 0, r0 = 0, r1 = 0;
+#pragma unroll 4
+            for (int sl = 0; sl < Tk; ++sl) {
+                const int e = st.idx[sl];
+                c0 += e == lane;
+                c1 += e == lane + 32;
+                r0 += sl < s0 && e == e0;
+                r1 += sl < s1 && e == e1;
+            }
+            if (lane >= E) c0 = 0;
+            if (lane + 32 >= E) c1 = 0;
+            st.cnt[lane] = c0;
+            st.cnt[lane + 32] = c1;
+            int i0 = c0, i1 = c1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u0 = __shfl_up_sync(0xffffffffu, i0, o), u1 = __shfl_up_sync(0xffffffffu, i1, o);
+                if (lane >= o) { i0 += u0; i1 += u1; }
+            }
+            i1 += __shfl_sync(0xffffffffu, i0, 31);
+            const unsigned lt = (1u << lane) - 1u;
+            const unsigned b0 = __ballot_sync(0xffffffffu, c0 > 0), b1 = __ballot_sync(0xffffffffu, c1 > 0);
+            st.offs[lane] = i0 - c0;
+            st.offs[lane + 32] = i1 - c1;
+            if (c0) st.groups[1 + __popc(b0 & lt)] = lane;
+            if (c1) st.groups[1 + __popc(b0) + __popc(b1 & lt)] = lane + 32;
+            __syncwarp();
+            if (lane == 0) {
+                st.groups[0] = E;
+                st.nslots = 1 + __popc(b0) + __popc(b1);
+                st.offs[E] = Tk;
+                st.offs[E + 1] = Tk + T;
+            }
+            __syncwarp();
+            if (e0 >= 0) {
+                const int r = st.offs[e0] + r0;
+                st.slot_row[s0] = r;
+                st.row_tok[r] = s0 / k;
+            }
+            if (e1 >= 0) {
+                const int r = st.offs[e1] + r1;
+                st.slot_row[s1] = r;
+                st.row_tok[r] = s1 / k;
+            }
+        }
+        __syncthreads();
+        // this cluster's first group's gate/up weights start streaming at once
+        const int nslots = st.nslots;
+        if (cid < nslots) {
+            gu_stream<CS>(S, p, Lw, st.groups[cid], rb0, wsc);
+            if (alive && lane == 0)
+                for (int i = 0; i < kRingMax && i < S.ntot; ++i) S.issue(i);
+        }
+        if (keeper) {
+            // the routing and the permutation, as the three-launch path leaves them (of the last layer)
+            for (int i = tid; i < Tk; i += kCThreads) {
+                p.idx[i] = st.idx[i];
+                p.gate[i] = st.gate[i];
+                p.slot_row[i] = st.slot_row[i];
+                p.row_src[st.slot_row[i]] = i / k;
+                p.row_gate[st.slot_row[i]] = st.gate[i];
+                if (Lw.out_idx) Lw.out_idx[i] = st.idx[i];
+                if (Lw.out_gate) Lw.out_gate[i] = st.gate[i];
+            }
+            for (int t = tid; t < T; t += kCThreads) {
+                p.sx[t] = st.sxs[t];
+                p.row_src[Tk + t] = t;
+                p.row_gate[Tk + t] = 1.0f;
+            }
+            for (int e = tid; e <= E + 1; e += kCThreads) {
+                p.offsets[e] = st.offs[e];
+                if (e <= E) {
+                    const int c = e < E ? st.cnt[e] : T;
+                    p.counts[e] = c;
+                    if (Lw.out_counts) Lw.out_counts[e] = c;
+                }
+            }
+            for (int i = tid; i < st.nslots; i += kCThreads) p.dec_groups[i] = st.groups[i];
+            if (tid == 0) *p.dec_ngroups = st.nslots;
+        }
+        if (cid == 0) {
+            // the shared rows' activation codes (this CTA's K slice), kept for inspection
+            for (int i = tid; i < T * (ks / 4); i += kCThreads) {
+                const int t = i / (ks / 4), v = i % (ks / 4);
+                const uint16_t* xr = xs + t * d + rank * ks + v * 4;
+                *reinterpret_cast<uint32_t*>(p.xq + (int64_t)(Tk + t) * d + rank * ks + v * 4) = pack_codes(
+                    bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), st.sxs[t]);
+            }
+        }
+
+        // ------------------------------------------------------------ the groups of this cluster
+        if (tid == 32) {
+            // every down block of this CTA's groups toward L2 now, and the gate/up blocks of all but the
+            // first (whose streams start at once); the next layer's shared expert after them
+            for (int s = cid; s < nslots; s += ncl) {
+                const int g = st.groups[s];
+                const int hid = g == E ? p.hs : p.h;
+                const int NJ = d / 64, NJd = hid / 64, nrb = hid / 8, nrbd = d / 16;
+                for (int b = rank * W; b < nrbd; b += CS * W)
+                    prefetch_range(Lw.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)b * NJd * kJP,
+                                   (int64_t)min(W, nrbd - b) * NJd * kJP);
+                if (s != cid)
+                    for (int b = rank * W; b < nrb; b += CS * W)
+                        prefetch_range(Lw.w_gate_up_d + (int64_t)g * ((int64_t)p.h * d * 5 / 4) + (int64_t)b * NJ * kJP,
+                                       (int64_t)min(W, nrb - b) * NJ * kJP);
+            }
+            if (l + 1 < ca.nl && cid == 0) prefetch_shared_expert<CS>(p, ca.layers[l + 1], rank);
+        }
         for (int s = cid; s < nslots; s += ncl) {
             const int g = st.groups[s];
-            const int hid = g == E ? p.hs : p.h;
-            const int NJ = d / 64, NJd = hid / 64, nrb = hid / 8, nrbd = d / 16;
-            for (int b = rank * W; b < nrbd; b += CS * W)
-                prefetch_range(p.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)b * NJd * kJP,
-                               (int64_t)min(W, nrbd - b) * NJd * kJP);
-            if (s != cid)
-                for (int b = rank * W; b < nrb; b += CS * W)
-                    prefetch_range(p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * d * 5 / 4) + (int64_t)b * NJ * kJP,
-                                   (int64_t)min(W, nrb - b) * NJ * kJP);
-        }
-    }
-    int wsc = 0;      // this warp's running stage count (ring slot and phase)
-    bool alive = ok;  // false once one of this warp's bounded waits gave up
-    WarpStream S;
-    S.ring = ring + warp * nring * kStageBytes;
-    S.bars = st.bars + warp * kRingMax;
-    S.nring = nring;
-    for (int s = cid; s < nslots; s += ncl) {
-        const int g = st.groups[s];
-        const bool shared = g == E;
-        const int hid = shared ? p.hs : p.h;
-        const int nrows = shared ? T : st.cnt[g];
-        const int row0 = shared ? Tk : st.offs[g];
-        // -------------------------------------------------- gate/up: blocks of 8 gate + 8 up rows
-        const int nrb = hid / 8, NJ = d / 64, csz = d + 32, ngr = d / 32;
-        const int np = npasses(rb0, CS * W, nrb);
-        S.src = p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * d * 5 / 4) + (int64_t)rb0 * NJ * kJP;
-        S.pstride = (int64_t)CS * W * NJ * kJP;
-        S.NJ = NJ;
-        S.nst = (NJ + kStageJP - 1) / kStageJP;
-        S.ntot = np * S.nst;
-        S.base = wsc;
-        if (alive && lane == 0)
-            for (int i = 0; i < nring && i < S.ntot; ++i) S.issue(i);
-        // the rows' activation codes, zero rows up to 8
-        for (int it = tid; it < 8 * ngr; it += kCThreads) {
-            const int i = it / ngr, j = it % ngr;
-            uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (i < nrows) {
-                const int t = shared ? i : st.row_tok[row0 + i];
-                const float sx = st.sxs[t];
-                const uint2* x2 = reinterpret_cast<const uint2*>(xs + t * d + j * 32);
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const uint2 u = x2[v];
-                    wv[v] = pack_codes(bf16_to_f32(u.x & 0xffffu), bf16_to_f32(u.x >> 16), bf16_to_f32(u.y & 0xffffu),
-                                       bf16_to_f32(u.y >> 16), sx);
-                }
+            const bool shared = g == E;
+            const int hid = shared ? p.hs : p.h;
+            const int nrows = shared ? T : st.cnt[g];
+            const int row0 = shared ? Tk : st.offs[g];
+            // -------------------------------------------------- gate/up: blocks of 8 gate + 8 up rows
+            const int nrb = hid / 8, csz = d + 32, ngr = d / 32;
+            const int np = npasses(rb0, CS * W, nrb);
+            if (s != cid) {  // (the first group's stream was started right after the routing)
+                gu_stream<CS>(S, p, Lw, g, rb0, wsc);
+                if (alive && lane == 0)
+                    for (int i = 0; i < kRingMax && i < S.ntot; ++i) S.issue(i);
             }
-            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * csz + j * 32);
-            dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
-            dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
-        }
-        if (tid < 8) st.shs[tid] = tid < nrows ? st.sxs[shared ? tid : st.row_tok[row0 + tid]] : 0.0f;
-        __syncthreads();
-        for (int pi = 0; pi < np; ++pi) {
-            const int rb = rb0 + pi * CS * W;
-            float alo[1][2], ahi[1][2];
-            S.sc0 = pi * S.nst;
-            if (alive)
-                alive = warp_gemv<true, false, 1>(p, S, codes, csz, lane, rb, row0, nrows, nullptr, 0, 0, alo, ahi);
-            // SwiGLU of rows 2 t4, 2 t4 + 1 at feature n, into every CTA's copy of the rows (and into act)
-            const int n = rb * 8 + gid;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int i = 2 * t4 + q;
-                if (i >= nrows) continue;
-                const float a = alive ? swiglu_row(alo[0][q], ahi[0][q], st.shs[i]) : 0.0f;
-                p.act[(int64_t)(row0 + i) * p.hmax + n] = a;
-#pragma unroll 4
-                for (int c = 0; c < CS; ++c) st_peer(act_all + i * p.hmax + n, c, __float_as_uint(a));
-            }
-        }
-        wsc += S.ntot;
-        // this warp's down blocks start streaming now
-        const int nrbd = d / 16, NJd = hid / 64, cszd = hid + 32, ngh = hid / 32;
-        const int npd = npasses(rb0, CS * W, nrbd);
-        WarpStream D = S;
-        D.src = p.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)rb0 * NJd * kJP;
-        D.pstride = (int64_t)CS * W * NJd * kJP;
-        D.NJ = NJd;
-        D.nst = (NJd + kStageJP - 1) / kStageJP;
-        D.ntot = npd * D.nst;
-        D.base = wsc;
-        __syncwarp();
-        if (alive && lane == 0)
-            for (int i = 0; i < nring && i < D.ntot; ++i) D.issue(i);
-        // -------------------------------------------------- requantisation of the whole rows, in every CTA
-        cluster_sync();  // every CTA's SwiGLU features are in every CTA's copy
-        if (warp < nrows) {
-            float m = 0.0f;
-            for (int n = lane; n < hid; n += 32) m = fmaxf(m, fabsf(act_all[warp * p.hmax + n]));
-            m = warp_max(m);
-            if (lane == 0) {
-                const float sv = __fdiv_rn(m, 127.0f);
-                st.shs[warp] = sv;
-                if (rank == 0) {
-                    p.amax_h[row0 + warp] = __float_as_uint(m);
-                    p.sh[row0 + warp] = sv;
+            // the rows' activation codes (one word of four per item, at its place in the B-fragment order of
+            // its 32-group), zero rows up to 8
+            for (int it = tid; it < 8 * ngr * 8; it += kCThreads) {
+                const int i = it / (ngr * 8), j = (it >> 3) % ngr, v = it & 7;
+                uint32_t word = 0u;
+                if (i < nrows) {
+                    const int t = shared ? i : st.row_tok[row0 + i];
+                    const uint2 u = *reinterpret_cast<const uint2*>(xs + t * d + j * 32 + v * 4);
+                    word = pack_codes(bf16_to_f32(u.x & 0xffffu), bf16_to_f32(u.x >> 16), bf16_to_f32(u.y & 0xffffu),
+                                      bf16_to_f32(u.y >> 16), st.sxs[t]);
                 }
+                *reinterpret_cast<uint32_t*>(codes + (size_t)i * csz + j * 32 + 4 * bfrag_pos(v)) = word;
             }
-        } else if (warp < 8 && lane == 0) {
-            st.shs[warp] = 0.0f;
-        }
-        __syncthreads();
-        for (int it = tid; it < 8 * ngh; it += kCThreads) {
-            const int i = it / ngh, j = it % ngh;
-            uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (i < nrows) {
-                const float sv = st.shs[i];
-                const float4* a4 = reinterpret_cast<const float4*>(act_all + i * p.hmax + j * 32);
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const float4 a = a4[v];
-                    wv[v] = pack_codes(a.x, a.y, a.z, a.w, sv);
-                }
-                if (rank == 0) {
-                    uint4* q4 = reinterpret_cast<uint4*>(p.hq + (int64_t)(row0 + i) * p.hmax + j * 32);
-                    q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                }
-            }
-            uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cszd + j * 32);
-            dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
-            dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
-        }
-        // before this cluster's next group, no CTA may write its SwiGLU values into a copy whose codes
-        // are still being taken
-        if (s + ncl < nslots)
-            cluster_sync();
-        else
+            if (tid < 8) st.shs[tid] = tid < nrows ? st.sxs[shared ? tid : st.row_tok[row0 + tid]] : 0.0f;
             __syncthreads();
-        // -------------------------------------------------- down: blocks of 16 output rows
-        for (int pi = 0; pi < npd; ++pi) {
-            const int rb = rb0 + pi * CS * W;
-            float alo[1][2], ahi[1][2];
-            D.sc0 = pi * D.nst;
-            if (alive)
-                alive = warp_gemv<false, false, 1>(p, D, codes, cszd, lane, rb, row0, nrows, nullptr, 0, 0, alo, ahi);
-            const int m0 = rb * 16 + gid;
+            for (int pi = 0; pi < np; ++pi) {
+                const int rb = rb0 + pi * CS * W;
+                float alo[1][2], ahi[1][2];
+                S.sc0 = pi * S.nst;
+                if (alive)
+                    alive = warp_gemv<true, false, 1>(p, S, codes, csz, lane, rb, row0, nrows, nullptr, 0, 0, alo, ahi);
+                // SwiGLU of rows 2 t4, 2 t4 + 1 at feature n, into every CTA's copy of the rows (and into act)
+                const int n = rb * 8 + gid;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int i = 2 * t4 + q;
-                if (i >= nrows) continue;
-                const float sv = st.shs[i];
-                ca.obuf[(int64_t)(row0 + i) * d + m0] = __fmul_rn(alo[0][q], sv);
-                ca.obuf[(int64_t)(row0 + i) * d + m0 + 8] = __fmul_rn(ahi[0][q], sv);
-            }
-        }
-        wsc += D.ntot;
-        // -------------------------------------------------- combine of the tokens whose last contribution this is
-        __threadfence();
-        __syncthreads();
-        if (tid < 8) {
-            int t = -1;
-            if (tid < nrows) {
-                const int tt = shared ? tid : st.row_tok[row0 + tid];
-                if (atomicAdd(ca.cnt + tt * CS + rank, 1u) == (uint32_t)k) t = tt;
-            }
-            st.last[tid] = t;
-        }
-        __syncthreads();
-        const int npdmax = npasses(rank * W, CS * W, nrbd);
-        for (int i = 0; i < 8; ++i) {
-            const int t = st.last[i];
-            if (t < 0) continue;
-            __threadfence();
-            for (int it = tid; it < npdmax * W * 4; it += kCThreads) {
-                const int pi = it / (W * 4), w = (it >> 2) % W, c4 = it & 3;
-                const int rb = rank * W + w + pi * CS * W;
-                if (rb >= nrbd) continue;
-                const int m = rb * 16 + c4 * 4;
-                float4 yv = __ldcg(reinterpret_cast<const float4*>(ca.obuf + (int64_t)(Tk + t) * d + m));
-                for (int j = 0; j < k; ++j) {
-                    const float gj = st.gate[t * k + j];
-                    const float4 o =
-                        __ldcg(reinterpret_cast<const float4*>(ca.obuf + (int64_t)st.slot_row[t * k + j] * d + m));
-                    yv.x = __fadd_rn(yv.x, __fmul_rn(gj, o.x));
-                    yv.y = __fadd_rn(yv.y, __fmul_rn(gj, o.y));
-                    yv.z = __fadd_rn(yv.z, __fmul_rn(gj, o.z));
-                    yv.w = __fadd_rn(yv.w, __fmul_rn(gj, o.w));
+                for (int q = 0; q < 2; ++q) {
+                    const int i = 2 * t4 + q;
+                    if (i >= nrows) continue;
+                    const float a = alive ? swiglu_row(alo[0][q], ahi[0][q], st.shs[i]) : 0.0f;
+                    p.act[(int64_t)(row0 + i) * p.hmax + n] = a;
+#pragma unroll 4
+                    for (int c = 0; c < CS; ++c) st_peer(act_all + i * p.hmax + n, c, __float_as_uint(a));
                 }
-                *reinterpret_cast<float4*>(p.y + (int64_t)t * d + m) = yv;
             }
-            if (tid == 0) ca.cnt[t * CS + rank] = 0u;
+            wsc += S.ntot;
+            // this warp's down blocks start streaming now
+            const int nrbd = d / 16, NJd = hid / 64, cszd = hid + 32, ngh = hid / 32;
+            const int npd = npasses(rb0, CS * W, nrbd);
+            WarpStream D = S;
+            D.src = Lw.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)rb0 * NJd * kJP;
+            D.pstride = (int64_t)CS * W * NJd * kJP;
+            D.NJ = NJd;
+            D.nst = (NJd + kStageJP - 1) / kStageJP;
+            D.ntot = npd * D.nst;
+            D.base = wsc;
+            __syncwarp();
+            if (alive && lane == 0)
+                for (int i = 0; i < kRingMax && i < D.ntot; ++i) D.issue(i);
+            // -------------------------------------------------- requantisation of the whole rows, in every CTA
+            cluster_sync();  // every CTA's SwiGLU features are in every CTA's copy
+            if (warp < nrows) {
+                float m = 0.0f;
+                for (int n = lane; n < hid; n += 32) m = fmaxf(m, fabsf(act_all[warp * p.hmax + n]));
+                m = warp_max(m);
+                if (lane == 0) {
+                    const float sv = __fdiv_rn(m, 127.0f);
+                    st.shs[warp] = sv;
+                    if (rank == 0) {
+                        p.amax_h[row0 + warp] = __float_as_uint(m);
+                        p.sh[row0 + warp] = sv;
+                    }
+                }
+            } else if (warp < 8 && lane == 0) {
+                st.shs[warp] = 0.0f;
+            }
+            __syncthreads();
+            for (int it = tid; it < 8 * ngh * 8; it += kCThreads) {
+                const int i = it / (ngh * 8), j = (it >> 3) % ngh, v = it & 7;
+                uint32_t word = 0u;
+                if (i < nrows) {
+                    const float4 a = *reinterpret_cast<const float4*>(act_all + i * p.hmax + j * 32 + v * 4);
+                    word = pack_codes(a.x, a.y, a.z, a.w, st.shs[i]);
+                    if (rank == 0)
+                        *reinterpret_cast<uint32_t*>(p.hq + (int64_t)(row0 + i) * p.hmax + j * 32 + v * 4) = word;
+                }
+                *reinterpret_cast<uint32_t*>(codes + (size_t)i * cszd + j * 32 + 4 * bfrag_pos(v)) = word;
+            }
+            // before this cluster's next group, no CTA may write its SwiGLU values into a copy whose codes
+            // are still being taken
+            if (s + ncl < nslots)
+                cluster_sync();
+            else
+                __syncthreads();
+            // -------------------------------------------------- down: blocks of 16 output rows
+            for (int pi = 0; pi < npd; ++pi) {
+                const int rb = rb0 + pi * CS * W;
+                float alo[1][2], ahi[1][2];
+                D.sc0 = pi * D.nst;
+                if (alive)
+                    alive =
+                        warp_gemv<false, false, 1>(p, D, codes, cszd, lane, rb, row0, nrows, nullptr, 0, 0, alo, ahi);
+                const int m0 = rb * 16 + gid;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int i = 2 * t4 + q;
+                    if (i >= nrows) continue;
+                    const float sv = st.shs[i];
+                    ca.obuf[(int64_t)(row0 + i) * d + m0] = __fmul_rn(alo[0][q], sv);
+                    ca.obuf[(int64_t)(row0 + i) * d + m0 + 8] = __fmul_rn(ahi[0][q], sv);
+                }
+            }
+            wsc += D.ntot;
+            // -------------------------------------------------- combine of the tokens whose last contribution this is
+            __threadfence();
+            __syncthreads();
+            if (tid < 8) {
+                int t = -1;
+                if (tid < nrows) {
+                    const int tt = shared ? tid : st.row_tok[row0 + tid];
+                    if (atomicAdd(ca.cnt + tt * CS + rank, 1u) == (uint32_t)k) t = tt;
+                }
+                st.last[tid] = t;
+            }
+            __syncthreads();
+            const int npdmax = npasses(rank * W, CS * W, nrbd);
+            int ncomb = 0;
+            for (int i = 0; i < 8; ++i) {
+                const int t = st.last[i];
+                if (t < 0) continue;
+                ++ncomb;
+                __threadfence();
+                for (int it = tid; it < npdmax * W * 4; it += kCThreads) {
+                    const int pi = it / (W * 4), w = (it >> 2) % W, c4 = it & 3;
+                    const int rb = rank * W + w + pi * CS * W;
+                    if (rb >= nrbd) continue;
+                    const int m = rb * 16 + c4 * 4;
+                    float4 yv = __ldcg(reinterpret_cast<const float4*>(ca.obuf + (int64_t)(Tk + t) * d + m));
+                    for (int j = 0; j < k; ++j) {
+                        const float gj = st.gate[t * k + j];
+                        const float4 o = __ldcg(
+                            reinterpret_cast<const float4*>(ca.obuf + (int64_t)st.slot_row[t * k + j] * d + m));
+                        yv.x = __fadd_rn(yv.x, __fmul_rn(gj, o.x));
+                        yv.y = __fadd_rn(yv.y, __fmul_rn(gj, o.y));
+                        yv.z = __fadd_rn(yv.z, __fmul_rn(gj, o.z));
+                        yv.w = __fadd_rn(yv.w, __fmul_rn(gj, o.w));
+                    }
+                    *reinterpret_cast<float4*>(Lw.y + (int64_t)t * d + m) = yv;
+                }
+                if (tid == 0) ca.cnt[t * CS + rank] = 0u;
+            }
+            if (ca.nl > 1 && ncomb > 0) {
+                // these tokens' columns of y are complete: count them for the next layer's wait
+                __threadfence();
+                __syncthreads();
+                if (tid == 0) atomicAdd(ca.chain, (uint32_t)ncomb);
+            }
         }
     }
     if (!alive && lane == 0) set_error(p, 41);
+    if (ca.nl > 1) {
+        // the last CTA to leave resets the chain counters for the next launch
+        __syncthreads();
+        if (tid == 0 && atomicAdd(ca.chain + 1, 1u) == gridDim.x - 1) {
+            ca.chain[0] = 0u;
+            ca.chain[1] = 0u;
+        }
+    }
 }
 
 // INT4 interchange layout -> decode layout (see the top of this file).  For
@@ -1297,12 +1428,15 @@ size_t cluster_layout(int d, int h, int hs, int E, int CS, CArgs* ca) {
     o = align128(o + (size_t)8 * ((d > hmax ? d : hmax) + 32));
     const size_t off_act = o;
     o = align128(o + std::max((size_t)8 * hmax * 4, (size_t)4 * kCMaxT * 64 * 4));
+    const size_t off_wr = o;
+    o = align128(o + (size_t)(d / CS) * E * 4);
     const size_t off_u = o;
-    o += std::max((size_t)(d / CS) * E * 4, (size_t)kCWarps * kRingMax * kStageBytes);
+    o += (size_t)kCWarps * kRingMax * kStageBytes;
     if (ca) {
         ca->off_x = (int)off_x;
         ca->off_codes = (int)off_codes;
         ca->off_act = (int)off_act;
+        ca->off_wr = (int)off_wr;
         ca->off_u = (int)off_u;
     }
     return o;
@@ -1369,16 +1503,27 @@ DecFusedShape dec_fused_shape(int d, int h, int hs, int E) {
 size_t dec_fused_counter_words() { return (size_t)dec::kCMaxT * dec::kCMaxCS; }
 size_t dec_fused_obuf_floats(int d) { return (size_t)dec::kCMaxT * (kMaxTopK + 1) * d; }
 
-cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
-                                int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s) {
+size_t dec_chain_counter_words() { return 2; }
+
+cudaError_t launch_decode_chain(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
+                                uint32_t* chain, const DecChainLayer* layers, int nl, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    if (p.T > dec::kCMaxT) return cudaErrorInvalidValue;
+    if (p.T > dec::kCMaxT || nl < 1 || nl > dec::kMaxChain) return cudaErrorInvalidValue;
     dec::CArgs ca{};
     ca.cnt = cnt;
     ca.obuf = obuf;
-    ca.out_idx = out_idx;
-    ca.out_gate = out_gate;
-    ca.out_counts = out_counts;
+    ca.chain = chain;
+    ca.nl = nl;
+    for (int l = 0; l < nl; ++l) {
+        ca.layers[l].w_router = layers[l].w_router;
+        ca.layers[l].router_bias = layers[l].router_bias;
+        ca.layers[l].w_gate_up_d = layers[l].w_gate_up_d;
+        ca.layers[l].w_down_d = layers[l].w_down_d;
+        ca.layers[l].y = layers[l].y;
+        ca.layers[l].out_idx = layers[l].out_idx;
+        ca.layers[l].out_gate = layers[l].out_gate;
+        ca.layers[l].out_counts = layers[l].out_counts;
+    }
     // 16-CTA clusters when one or two tokens leave few groups and every warp of such a cluster has a
     // row block of a routed expert; else 8
     const bool big = shape.clusters16 > 0 && p.T <= 2 && std::min(p.h / 8, p.d / 16) >= 16 * dec::kCWarps;
@@ -1392,6 +1537,12 @@ cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint3
     const size_t smem = dec::cluster_layout(p.d, p.h, p.hs, p.E, 8, &ca);
     cudaLaunchConfig_t cfg = dec::cluster_config<8>(smem, shape.clusters8, s, at);
     return cudaLaunchKernelEx(&cfg, dec::decode_cluster_kernel<8>, p, ca);
+}
+
+cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
+                                int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s) {
+    DecChainLayer one{p.w_router, p.router_bias, p.w_gate_up_d, p.w_down_d, p.y, out_idx, out_gate, out_counts};
+    return launch_decode_chain(p, shape, cnt, obuf, nullptr, &one, 1, s);
 }
 
 bool dec_supported(int d, int h, int hs) { return d % 64 == 0 && h % 64 == 0 && hs % 64 == 0; }

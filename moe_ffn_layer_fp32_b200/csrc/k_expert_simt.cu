@@ -11,6 +11,8 @@
 // Every group of 32 K elements gives an exact INT32 partial P_j (INT8 x INT4);
 // it is promoted as acc = fma(float(P_j), s_j, acc) for j ascending, then
 // multiplied by the row's activation scale.
+#include <cuda_bf16.h>
+
 #include "mmoe_internal.cuh"
 
 namespace mmoe {
@@ -257,7 +259,18 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(Plan p)
     *reinterpret_cast<float4*>(p.y + i4 * 4) = y;
 }
 
+__global__ void f32_to_bf16_kernel(const float* src, uint16_t* dst, int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(src[i]));
+}
+
 }  // namespace
+
+cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    f32_to_bf16_kernel<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, s>>>(src, dst, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows) {
     if (p.T == 0) return cudaSuccess;

@@ -318,6 +318,10 @@ cudaError_t run_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t r0, i
     }
 }
 
+// The one-launch decode's counters: per-token contribution counters, then the two counters of a chain
+// of layers.
+size_t dec_sync_words() { return dec_fused_counter_words() + dec_chain_counter_words(); }
+
 // A bounded device-side wait of an earlier call gave up: report it once and
 // clear both copies of the flag (the device copy in stream order).
 mmoe_status check_device_flag(mmoe_handle* h, cudaStream_t s) {
@@ -327,7 +331,7 @@ mmoe_status check_device_flag(mmoe_handle* h, cudaStream_t s) {
     *reinterpret_cast<volatile int*>(h->err_host) = 0;
     cudaMemsetAsync(h->err_dev, 0, sizeof(int), s);
     // a one-launch decode that gave up may have left contribution counters set
-    if (h->dec_sync) cudaMemsetAsync(h->dec_sync, 0, dec_fused_counter_words() * sizeof(uint32_t), s);
+    if (h->dec_sync) cudaMemsetAsync(h->dec_sync, 0, dec_sync_words() * sizeof(uint32_t), s);
     return fail(MMOE_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (site %d); its results were not written", v);
 }
 
@@ -513,9 +517,9 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
             h->use_dec_fused = h->dec_shape.clusters8 > 0;
         }
         if (h->use_dec_fused) {
-            ALLOC(dec_sync, dec_fused_counter_words());
+            ALLOC(dec_sync, dec_sync_words());
             ALLOC(dec_obuf, dec_fused_obuf_floats((int)d));
-            if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, dec_fused_counter_words() * sizeof(uint32_t));
+            if (e == cudaSuccess) e = cudaMemset(h->dec_sync, 0, dec_sync_words() * sizeof(uint32_t));
         }
     }
     if (e == cudaSuccess) {
@@ -678,6 +682,71 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
                   "copy expert_counts");
     h->last_T = T;
     h->last_dec = dec;
+    return MMOE_OK;
+}
+
+mmoe_status mmoe_forward_chain(mmoe_handle* const* layers, int32_t n_layers, const uint16_t* x, int64_t T,
+                               float* const* y_layers, void* stream) {
+    if (!layers || !y_layers) return fail(MMOE_ERR_INVALID_ARG, "layers or y_layers is NULL");
+    if (n_layers < 1 || n_layers > MMOE_MAX_CHAIN_LAYERS)
+        return fail(MMOE_ERR_INVALID_ARG, "n_layers=%d: must be in [1, %d]", n_layers, MMOE_MAX_CHAIN_LAYERS);
+    mmoe_handle* h0 = layers[0];
+    if (!h0) return fail(MMOE_ERR_INVALID_ARG, "layer 0's handle is NULL");
+    const mmoe_config& c0 = h0->cfg;
+    for (int l = 0; l < n_layers; ++l) {
+        const mmoe_handle* h = layers[l];
+        if (!h) return fail(MMOE_ERR_INVALID_ARG, "layer %d's handle is NULL", l);
+        const mmoe_config& c = h->cfg;
+        if (c.d_model != c0.d_model || c.n_experts != c0.n_experts || c.top_k != c0.top_k ||
+            c.expert_hidden != c0.expert_hidden || c.shared_hidden != c0.shared_hidden || c.gating != c0.gating ||
+            h->device != h0->device)
+            return fail(MMOE_ERR_INVALID_ARG, "layer %d: shapes, gating or device differ from layer 0's", l);
+        if (T < 0 || T > h->max_tokens)
+            return fail(MMOE_ERR_INVALID_ARG, "T=%lld: must be in [0, max_tokens=%lld] of layer %d", (long long)T,
+                        (long long)h->max_tokens, l);
+        if (!h->loaded) return fail(MMOE_ERR_NOT_LOADED, "layer %d: forward before mmoe_load_quantized_weights", l);
+        if (!y_layers[l] || (reinterpret_cast<uintptr_t>(y_layers[l]) & 15))
+            return fail(MMOE_ERR_INVALID_ARG, "y_layers[%d] is NULL or not 16-byte aligned", l);
+    }
+    if (T == 0) return MMOE_OK;
+    if (!x || (reinterpret_cast<uintptr_t>(x) & 15)) return fail(MMOE_ERR_INVALID_ARG, "x is NULL or misaligned");
+    DeviceGuard dg(h0->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t d = c0.d_model;
+    const bool one_launch = h0->use_dec && h0->use_dec_fused && T <= h0->dec_max_T && T <= dec_fused_max_tokens();
+    if (one_launch) {
+        mmoe_status fst = check_device_flag(h0, s);
+        if (fst != MMOE_OK) return fst;
+        Plan p = make_plan(h0, x, T, y_layers[0]);
+        p.xq16 = nullptr;
+        p.hq16 = nullptr;
+        DecChainLayer L[MMOE_MAX_CHAIN_LAYERS];
+        for (int l = 0; l < n_layers; ++l)
+            L[l] = DecChainLayer{layers[l]->w_router,    layers[l]->router_bias, layers[l]->w_gate_up_d,
+                                 layers[l]->w_down_d,    y_layers[l],            nullptr,
+                                 nullptr,                nullptr};
+        MMOE_CUDA(run_stage(h0, MMOE_PROF_DECODE_FUSED, 1, s,
+                            [&] {
+                                return launch_decode_chain(p, h0->dec_shape, h0->dec_sync, h0->dec_obuf,
+                                                           h0->dec_sync + dec_fused_counter_words(), L, n_layers, s);
+                            }),
+                  "one-launch decode of a chain of layers");
+        h0->last_T = T;
+        h0->last_dec = true;
+        return MMOE_OK;
+    }
+    // one forward per layer; the next layer's input is the BF16 rounding of this one's y
+    const uint16_t* xin = x;
+    for (int l = 0; l < n_layers; ++l) {
+        const mmoe_status st = mmoe_forward(layers[l], xin, T, y_layers[l], stream, nullptr, nullptr, nullptr);
+        if (st != MMOE_OK) return st;
+        if (l + 1 < n_layers) {
+            mmoe_handle* hn = layers[l + 1];
+            if (!hn->x_stage) MMOE_CUDA(dalloc(&hn->x_stage, (size_t)hn->max_tokens * d), "staging allocation");
+            MMOE_CUDA(launch_f32_to_bf16(y_layers[l], hn->x_stage, T * d, s), "BF16 rounding of y");
+            xin = hn->x_stage;
+        }
+    }
     return MMOE_OK;
 }
 

@@ -99,6 +99,8 @@ cudaError_t launch_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t
 cudaError_t launch_requant(const Plan& p, cudaStream_t s);
 cudaError_t launch_down(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_combine(const Plan& p, cudaStream_t s);
+// dst[i] = BF16 bits of src[i] rounded to nearest even (n elements)
+cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, int64_t n, cudaStream_t s);
 // tensor-core path, kind::f16 (k_expert_f16.cu)
 bool f16tc_supported(int d, int h, int hs);
 int f16tc_fused_clusters(int c);  // clusters of c CTAs of the fused gate/up GEMM the device holds at once
@@ -134,6 +136,24 @@ size_t dec_fused_counter_words();
 size_t dec_fused_obuf_floats(int d);
 cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
                                 int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s);
+// Layers run back to back by one launch of the same kernel: layer l + 1 reads layer l's y rounded to
+// BF16.  All layers share p's shapes, gating and workspace; each brings its own weights (decode layout)
+// and output.  `chain`: dec_chain_counter_words() words, zero before the first launch (every launch
+// leaves them zero).
+constexpr int kDecChainMax = 32;
+struct DecChainLayer {
+    const float* w_router;
+    const float* router_bias;
+    const uint8_t* w_gate_up_d;
+    const uint8_t* w_down_d;
+    float* y;
+    int32_t* out_idx;
+    float* out_gate;
+    int32_t* out_counts;
+};
+size_t dec_chain_counter_words();
+cudaError_t launch_decode_chain(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
+                                uint32_t* chain, const DecChainLayer* layers, int nl, cudaStream_t s);
 cudaError_t launch_gate_up_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_down_dec(const Plan& p, cudaStream_t s, int32_t* dump, int64_t row0, int64_t nrows);
 cudaError_t launch_retile_dec(const uint8_t* gu, const float* sgu, const uint8_t* dn, const float* sdn,
@@ -225,8 +245,8 @@ __device__ __forceinline__ int quant_i8(float v, float s) {
 // no gate); writes logits (if kept), idx and gate.
 // The gating probabilities of experts lane and lane + 32 and their selection keys (the logit, or for
 // gating 2 the sigmoid score plus the bias; -inf where the expert does not exist).
-__device__ __forceinline__ void gate_probs_keys(const Plan& p, float l0, float l1, int lane, float& p0, float& p1,
-                                                float& k0, float& k1) {
+__device__ __forceinline__ void gate_probs_keys(const Plan& p, const float* bias, float l0, float l1, int lane,
+                                                float& p0, float& p1, float& k0, float& k1) {
     const int E = p.E;
     const bool v0 = lane < E, v1 = lane + 32 < E;
     if (p.gating == MMOE_GATE_SOFTMAX) {
@@ -243,8 +263,8 @@ __device__ __forceinline__ void gate_probs_keys(const Plan& p, float l0, float l
     k0 = l0;
     k1 = l1;
     if (p.gating == MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS) {
-        k0 = v0 ? (p.router_bias ? __fadd_rn(p0, p.router_bias[lane]) : p0) : -INFINITY;
-        k1 = v1 ? (p.router_bias ? __fadd_rn(p1, p.router_bias[lane + 32]) : p1) : -INFINITY;
+        k0 = v0 ? (bias ? __fadd_rn(p0, bias[lane]) : p0) : -INFINITY;
+        k1 = v1 ? (bias ? __fadd_rn(p1, bias[lane + 32]) : p1) : -INFINITY;
     }
 }
 
@@ -257,7 +277,7 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
         if (v1) logits[t * E + lane + 32] = l1;
     }
     float p0, p1, k0, k1;
-    gate_probs_keys(p, l0, l1, lane, p0, p1, k0, k1);
+    gate_probs_keys(p, p.router_bias, l0, l1, lane, p0, p1, k0, k1);
     bool taken0 = !v0, taken1 = !v1;
     int sel[kMaxTopK];
     float gsel[kMaxTopK];
@@ -296,54 +316,12 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
     gate_topk_warp(p, t, l0, l1, lane, p.idx, p.gate, p.logits);
 }
 
-// The same gating and top-k as gate_topk_warp (the same probabilities and the same order: key
-// descending, the lower index first among equal keys), with each expert's position found by counting
-// the experts ahead of it in a copy of the keys in shared memory (`keys`: 64 floats, `selp`: k floats,
-// both private to the warp) instead of k rounds of warp arg-max.
-__device__ __forceinline__ void gate_topk_rank(const Plan& p, int64_t t, float l0, float l1, int lane, float* keys,
-                                               float* selp, int32_t* idx, float* gate, float* logits) {
-    const int E = p.E, k = p.k;
-    const bool v0 = lane < E, v1 = lane + 32 < E;
-    if (logits) {
-        if (v0) logits[t * E + lane] = l0;
-        if (v1) logits[t * E + lane + 32] = l1;
-    }
-    float p0, p1, k0, k1;
-    gate_probs_keys(p, l0, l1, lane, p0, p1, k0, k1);
-    keys[lane] = k0;
-    keys[lane + 32] = k1;
-    __syncwarp();
-    int r0 = 0, r1 = 0;
-#pragma unroll 4
-    for (int e = 0; e < E; ++e) {
-        const float ke = keys[e];
-        r0 += (ke > k0) || (ke == k0 && e < lane);
-        r1 += (ke > k1) || (ke == k1 && e < lane + 32);
-    }
-    if (v0 && r0 < k) {
-        idx[t * k + r0] = lane;
-        selp[r0] = p0;
-    }
-    if (v1 && r1 < k) {
-        idx[t * k + r1] = lane + 32;
-        selp[r1] = p1;
-    }
-    __syncwarp();
-    if (lane < k) {
-        float g = selp[lane];
-        if (p.gating != MMOE_GATE_SOFTMAX) {
-            float gsum = 0.0f;
-            for (int j = 0; j < k; ++j) gsum = __fadd_rn(gsum, selp[j]);
-            g = __fdiv_rn(g, gsum);
-        }
-        gate[t * k + lane] = g;
-    }
-    __syncwarp();
-}
-
 // The router bias enters the logit for gating 0 and 1 (and only the selection key for gating 2).
+__device__ __forceinline__ float biased_logit(const Plan& p, const float* bias, float l, int e) {
+    return (bias && p.gating != MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS) ? __fadd_rn(l, bias[e]) : l;
+}
 __device__ __forceinline__ float biased_logit(const Plan& p, float l, int e) {
-    return (p.router_bias && p.gating != MMOE_GATE_SIGMOID_TOPK_NORM_SEL_BIAS) ? __fadd_rn(l, p.router_bias[e]) : l;
+    return biased_logit(p, p.router_bias, l, e);
 }
 
 }  // namespace mmoe

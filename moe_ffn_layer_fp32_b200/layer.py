@@ -116,6 +116,21 @@ class MoELayer:
 
     __call__ = forward
 
+    @staticmethod
+    def forward_chain(layers, x: torch.Tensor, ys, stream=None) -> list:
+        """Layers one after another on the same tokens: layer 0 reads x (BF16 [T, d]); layer l + 1 reads
+        layer l's y rounded to BF16.  ys: one FP32 [T, d] CUDA tensor per layer (filled; returned).  For
+        up to 8 tokens on the decode path the whole stack is one kernel launch."""
+        if x.dtype != torch.bfloat16 or x.dim() != 2:
+            raise ValueError("x must be a [T, d_model] bfloat16 tensor")
+        n = len(layers)
+        if len(ys) != n:
+            raise ValueError("one output tensor per layer")
+        hs = (C.c_void_p * n)(*[L._h.value for L in layers])
+        yp = (C.c_void_p * n)(*[_ptr(y) for y in ys])
+        check(lib().mmoe_forward_chain(hs, n, _ptr(x), x.shape[0], yp, _stream_ptr(stream)))
+        return list(ys)
+
     def forward_host(self, x: np.ndarray, y: np.ndarray | None = None, stream=None) -> np.ndarray:
         """Same layer with host buffers: x uint16 (BF16 bits) [T, d] -> y float32 [T, d]; waits for the result."""
         x = np.ascontiguousarray(x, dtype=np.uint16)

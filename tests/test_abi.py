@@ -62,6 +62,19 @@ def test_null_arguments(L):
     assert L.mmoe_debug_partials(None, 0, 0, 0, None, None) == 1
 
 
+def test_forward_chain_validates_before_any_device_work(L):
+    # the stack of layers: argument checks need no device
+    VP = C.c_void_p
+    hs = (VP * 2)(None, None)
+    ys = (VP * 2)(16, 32)
+    assert L.mmoe_forward_chain(None, 1, None, 1, ys, None) == 1
+    assert L.mmoe_forward_chain(hs, 1, None, 1, None, None) == 1
+    assert L.mmoe_forward_chain(hs, 0, None, 1, ys, None) == 1
+    assert L.mmoe_forward_chain(hs, 33, None, 1, ys, None) == 1
+    assert L.mmoe_forward_chain(hs, 2, None, 1, ys, None) == 1
+    assert b"NULL" in L.mmoe_last_error()
+
+
 def test_quantize_validates_before_launch(L):
     assert L.mmoe_quantize_int4(None, 4, 48, None, None, None) == 1
     assert L.mmoe_quantize_int4(None, -1, 32, None, None, None) == 1

@@ -388,6 +388,61 @@ def test_c1_decode_layers():
             print("c1 layer", layer, "T", T, rep)
 
 
+def _chain_layers(name, n, T_max, deterministic=False):
+    w = synth.WORKLOADS[name]
+    qs = [oracle.quantize_layer(synth.workload_layer(w, l)) for l in range(n)]
+    return w, qs, [gu.make_gpu_layer(q, T_max, deterministic=deterministic) for q in qs]
+
+
+@pytest.mark.parametrize("name,T", [("c0", 1), ("c0", 5), ("c0", 8), ("c1", 1), ("c1", 8), ("c0", 20)])
+def test_forward_chain_matches_layer_by_layer(name, T):
+    # mmoe_forward_chain: for up to 8 tokens one launch runs the whole stack (layer l + 1 reading layer
+    # l's y rounded to BF16 inside the kernel); larger T runs one forward per layer.  Each layer's y
+    # equals, bit for bit, that of its own forward on the BF16 rounding of the previous layer's y, and
+    # matches the oracle on that input.  (More than 8 tokens take the three-launch decode, whose y is
+    # bit-reproducible with the fixed-order combine of deterministic mode.)
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    n = 4
+    w, qs, Ls = _chain_layers(name, n, 64, deterministic=T > 8)
+    x0 = synth.draw_x(T, w.d, seed=500 + T)
+    xd = gu.x_to_device(x0)
+    ys = [torch.full((T, w.d), float("nan"), dtype=torch.float32, device="cuda") for _ in range(n)]
+    MoELayer.forward_chain(Ls, xd, ys)
+    torch.cuda.synchronize()
+    xl = xd
+    for l in range(n):
+        y_ref = Ls[l].forward(xl)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[l].view(torch.int32), y_ref.view(torch.int32)), l
+        rep = {}
+        x_np = xl.view(torch.int16).cpu().numpy().view(np.uint16)
+        gu.check_y(ys[l].cpu().numpy(), oracle.moe_layer(qs[l], x_np), rep)
+        xl = y_ref.to(torch.bfloat16)
+    # the same stack again: the launch left its counters ready for the next one
+    ys2 = [torch.empty_like(y) for y in ys]
+    MoELayer.forward_chain(Ls, xd, ys2)
+    torch.cuda.synchronize()
+    for a, b in zip(ys, ys2):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    for L in Ls:
+        L.close()
+
+
+def test_forward_chain_rejects_mismatched_layers():
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    w = synth.WORKLOADS["c0"]
+    q = oracle.quantize_layer(synth.workload_layer(w))
+    a = gu.make_gpu_layer(q, 8)
+    b = MoELayer(w.d, 2 * w.h, max_tokens=8)  # another hidden size
+    x = gu.x_to_device(synth.draw_x(2, w.d, seed=1))
+    ys = [torch.empty((2, w.d), dtype=torch.float32, device="cuda") for _ in range(2)]
+    with pytest.raises(_lib.MMoEError) as ei:
+        MoELayer.forward_chain([a, b], x, ys)
+    assert ei.value.status == 1  # INVALID_ARG
+    a.close()
+    b.close()
+
+
 def test_c2_prefill():
     w, q = workload("c2")
     x = synth.workload_x(w)
