@@ -9,7 +9,7 @@
 // ascending order, then the per-token activation scale, SwiGLU, the per-row
 // requantisation, the down projection and the gate-weighted combine.
 //
-// Three launches:
+// Four launches (up to 8 tokens: the one-launch decode further below):
 //  1. router_decode_kernel: one cluster of `cs` CTAs splits the K range of the
 //     FP32 router for all tokens; partial logits and partial absmax meet in
 //     distributed shared memory, each CTA quantises its slice of x, the owner
@@ -23,9 +23,10 @@
 //     the bit pattern of 1.5 * 2^19, so the float with the result's bits
 //     minus 1.5 * 2^19 is the group partial exactly (weights enter as 16 x
 //     their code).  SwiGLU in registers, the row absmax by atomicMax.
-//  3. expert_decode_kernel<down>: requantises its group's rows from that
-//     absmax in the prologue, then the same streaming GEMV; the epilogue adds
-//     gate * o into y (or stores o for the fixed-order combine).
+//  3. requant_kernel (the prefill path's): h_q and s_h of every row, once.
+//  4. expert_decode_kernel<down>: stages its group's h_q rows in the prologue,
+//     then the same streaming GEMV; the epilogue adds gate * o into y (or
+//     stores o for the fixed-order combine).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -610,7 +611,6 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
         fence_barrier_init();
     }
     __syncwarp();
-    const bool keep = blk == 0 && !DUMP;  // one CTA per group records h_q and s_h
     bool alive = wact;                    // false once this warp's bounded wait gave up
     for (int pass = 0; pass < npass; ++pass, S.sc0 += S.nst) {
         const int prow0 = pass * kPassRows;
@@ -639,34 +639,21 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
                 dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
             }
         } else {
-            // requantise the group's SwiGLU rows: s_h = absmax / 127 (the absmax was built by the
-            // gate/up CTAs with atomicMax); one CTA per group also records h_q and s_h
-            for (int i = tid; i < nch * 8; i += blockDim.x)
-                shs[i] = i < prows ? __fdiv_rn(__uint_as_float(p.amax_h[rrow0 + i]), 127.0f) : 0.0f;
-            __syncthreads();
+            // the group's requantised SwiGLU rows (h_q and s_h from the requantisation launch between the
+            // two GEMV launches), zero rows up to a multiple of 8
+            for (int i = tid; i < nch * 8; i += blockDim.x) shs[i] = i < prows ? p.sh[rrow0 + i] : 0.0f;
             for (int it = tid; it < nch * 8 * ngr; it += blockDim.x) {
                 const int i = it / ngr, j = it % ngr;
-                uint32_t wv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
                 if (i < prows) {
-                    const float s = shs[i];
-                    const float4* a4 = reinterpret_cast<const float4*>(p.act + (rrow0 + i) * p.hmax + j * 32);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const float4 a = a4[v];
-                        wv[v] = pack_codes(a.x, a.y, a.z, a.w, s);
-                    }
-                    if (keep) {
-                        uint4* q4 = reinterpret_cast<uint4*>(p.hq + (rrow0 + i) * p.hmax + j * 32);
-                        q4[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                        q4[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                    }
+                    const uint4* q4 = reinterpret_cast<const uint4*>(p.hq + (rrow0 + i) * p.hmax + j * 32);
+                    u0 = q4[0];
+                    u1 = q4[1];
                 }
                 uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)i * cs + j * 32);
-                dst[0] = make_uint4(wv[0], wv[4], wv[1], wv[5]);
-                dst[1] = make_uint4(wv[2], wv[6], wv[3], wv[7]);
+                dst[0] = make_uint4(u0.x, u1.x, u0.y, u1.y);
+                dst[1] = make_uint4(u0.z, u1.z, u0.w, u1.w);
             }
-            if (keep)
-                for (int i = tid; i < prows; i += blockDim.x) p.sh[rrow0 + i] = shs[i];
         }
         __syncthreads();
         if (alive)  // a warp that gave up keeps taking the CTA barriers but issues and computes nothing

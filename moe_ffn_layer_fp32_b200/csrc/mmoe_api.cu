@@ -643,11 +643,13 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
                             }),
                   "one-launch decode");
     } else if (dec) {
-        // decode path: router + permutation, gate/up (also clears y), down
+        // decode path: router + permutation, gate/up (also clears y), requantisation, down
         MMOE_CUDA(run_stage(h, MMOE_PROF_ROUTER, 1, s, [&] { return launch_router_dec(p, h->dec_cluster, s); }),
                   "decode router launch");
         MMOE_CUDA(run_stage(h, MMOE_PROF_GATE_UP, 1, s, [&] { return launch_gate_up_dec(p, s, nullptr, 0, 0); }),
                   "decode gate/up launch");
+        MMOE_CUDA(run_stage(h, MMOE_PROF_REQUANT, 1, s, [&] { return launch_requant(p, s); }),
+                  "decode requant launch");
         MMOE_CUDA(run_stage(h, MMOE_PROF_DOWN, 1, s, [&] { return launch_down_dec(p, s, nullptr, 0, 0); }),
                   "decode down launch");
     }
