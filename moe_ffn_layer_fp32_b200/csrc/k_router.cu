@@ -156,16 +156,23 @@ cudaError_t launch_router_quant(const Plan& p, cudaStream_t s) {
 namespace mmoe {
 namespace rmma {
 
-constexpr int kTok = 128;                 // tokens per CTA (8 warps x 16)
+// Tokens per CTA: TOK in {16, 32, 64, 128}, one 16-row MMA tile per warp for the first TOK / 16 warps; the
+// gating, top-k and codes of the CTA's tokens are spread over all 8 warps.  Small batches take small TOK,
+// so that their CTAs cover the SMs (each CTA reads the whole split W_r from L2).
 constexpr int kThreads = 256;
 constexpr int kKC = kRouterKChunk;        // K per chunk
 constexpr int kRow = kRouterRow;          // padded BF16 row of a chunk
-constexpr int kXChunkBytes = kTok * kRow * 2;          // 18432
 constexpr int kWPieceBytes = kRouterPieceBytes;
 constexpr int kWChunkBytes = kRouterChunkBytes;
 constexpr int kStages = 2;
 constexpr int kLgRow = 65;                // padded logits row
-constexpr size_t kSmem = (size_t)kStages * (kXChunkBytes + kWChunkBytes);  // logits alias the stages
+template <int TOK>
+struct Tiling {
+    static constexpr int kXChunkBytes = TOK * kRow * 2;
+    // the logits and scales (TOK x 65 + TOK floats) alias the stages
+    static constexpr size_t kSmem = (size_t)kStages * (kXChunkBytes + kWChunkBytes);
+    static_assert((size_t)TOK * (kLgRow + 1) * 4 <= kSmem, "logits fit in the stages");
+};
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
@@ -183,11 +190,12 @@ __device__ __forceinline__ uint32_t bf16_rn_bits(float v) {
     return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
 }
 
-// stage K chunk c of x (rows t0 .. t0 + 127, zero beyond T) and of the split weights
+// stage K chunk c of x (rows t0 .. t0 + TOK - 1, zero beyond T) and of the split weights
+template <int TOK>
 __device__ __forceinline__ void load_chunk(const Plan& p, int64_t t0, int nt, int c, uint8_t* xs, uint8_t* ws,
                                            int tid) {
     const int d = p.d;
-    for (int i = tid; i < kTok * (kKC / 8); i += kThreads) {
+    for (int i = tid; i < TOK * (kKC / 8); i += kThreads) {
         const int r = i >> 3, v = i & 7;
         uint8_t* dst = xs + r * (kRow * 2) + v * 16;
         if (r < nt) cp_async16(dst, p.x + (t0 + r) * d + c * kKC + v * 8);
@@ -197,13 +205,16 @@ __device__ __forceinline__ void load_chunk(const Plan& p, int64_t t0, int nt, in
     for (int i = tid; i < kWChunkBytes / 16; i += kThreads) cp_async16(ws + i * 16, src + i * 16);
 }
 
+template <int TOK>
 __global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int kXChunkBytes = Tiling<TOK>::kXChunkBytes;
     const int d = p.d, E = p.E;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
-    const int64_t t0 = (int64_t)blockIdx.x * kTok;
-    const int nt = (int)((p.T - t0) < kTok ? (p.T - t0) : kTok);
+    const bool mma_warp = warp * 16 < TOK;
+    const int64_t t0 = (int64_t)blockIdx.x * TOK;
+    const int nt = (int)((p.T - t0) < TOK ? (p.T - t0) : TOK);
     auto xs = [&](int c) { return smem + (c % kStages) * (kXChunkBytes + kWChunkBytes); };
     auto ws = [&](int c) { return smem + (c % kStages) * (kXChunkBytes + kWChunkBytes) + kXChunkBytes; };
     const int nchunks = d / kKC;
@@ -212,13 +223,17 @@ __global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
     for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
     float amax_lo = 0.0f, amax_hi = 0.0f;  // |x| max of rows g and g + 8 of this warp, over this lane's elements
 
-    load_chunk(p, t0, nt, 0, xs(0), ws(0), tid);
+    load_chunk<TOK>(p, t0, nt, 0, xs(0), ws(0), tid);
     cp_async_commit();
     for (int c = 0; c < nchunks; ++c) {
-        if (c + 1 < nchunks) load_chunk(p, t0, nt, c + 1, xs(c + 1), ws(c + 1), tid);
+        if (c + 1 < nchunks) load_chunk<TOK>(p, t0, nt, c + 1, xs(c + 1), ws(c + 1), tid);
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();
+        if (!mma_warp) {
+            __syncthreads();
+            continue;
+        }
         const uint16_t* xa = reinterpret_cast<const uint16_t*>(xs(c)) + (warp * 16 + g) * kRow + 2 * t4;
         const uint16_t* wb = reinterpret_cast<const uint16_t*>(ws(c)) + g * kRow + 2 * t4;
 #pragma unroll
@@ -244,22 +259,24 @@ __global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
 
     // logits into shared memory (aliasing the stages): D fragment rows g / g + 8, columns 2 t4, 2 t4 + 1
     float* lg = reinterpret_cast<float*>(smem);
-    float* sxs = lg + kTok * kLgRow;
+    float* sxs = lg + TOK * kLgRow;
+    if (mma_warp) {
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-        const int col = n * 8 + 2 * t4;
-        lg[(warp * 16 + g) * kLgRow + col] = acc[n][0];
-        lg[(warp * 16 + g) * kLgRow + col + 1] = acc[n][1];
-        lg[(warp * 16 + g + 8) * kLgRow + col] = acc[n][2];
-        lg[(warp * 16 + g + 8) * kLgRow + col + 1] = acc[n][3];
-    }
-    amax_lo = fmaxf(amax_lo, __shfl_xor_sync(0xffffffffu, amax_lo, 1));
-    amax_lo = fmaxf(amax_lo, __shfl_xor_sync(0xffffffffu, amax_lo, 2));
-    amax_hi = fmaxf(amax_hi, __shfl_xor_sync(0xffffffffu, amax_hi, 1));
-    amax_hi = fmaxf(amax_hi, __shfl_xor_sync(0xffffffffu, amax_hi, 2));
-    if (t4 == 0) {
-        sxs[warp * 16 + g] = __fdiv_rn(amax_lo, 127.0f);
-        sxs[warp * 16 + g + 8] = __fdiv_rn(amax_hi, 127.0f);
+        for (int n = 0; n < 8; ++n) {
+            const int col = n * 8 + 2 * t4;
+            lg[(warp * 16 + g) * kLgRow + col] = acc[n][0];
+            lg[(warp * 16 + g) * kLgRow + col + 1] = acc[n][1];
+            lg[(warp * 16 + g + 8) * kLgRow + col] = acc[n][2];
+            lg[(warp * 16 + g + 8) * kLgRow + col + 1] = acc[n][3];
+        }
+        amax_lo = fmaxf(amax_lo, __shfl_xor_sync(0xffffffffu, amax_lo, 1));
+        amax_lo = fmaxf(amax_lo, __shfl_xor_sync(0xffffffffu, amax_lo, 2));
+        amax_hi = fmaxf(amax_hi, __shfl_xor_sync(0xffffffffu, amax_hi, 1));
+        amax_hi = fmaxf(amax_hi, __shfl_xor_sync(0xffffffffu, amax_hi, 2));
+        if (t4 == 0) {
+            sxs[warp * 16 + g] = __fdiv_rn(amax_lo, 127.0f);
+            sxs[warp * 16 + g + 8] = __fdiv_rn(amax_hi, 127.0f);
+        }
     }
     __syncthreads();
 
@@ -339,14 +356,32 @@ cudaError_t launch_split_router(const float* w, int d, int E, uint16_t* out, cud
     return cudaGetLastError();
 }
 
+namespace rmma {
+template <int TOK>
+cudaError_t launch_tok(const Plan& p, cudaStream_t s) {
+    constexpr size_t smem = Tiling<TOK>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(router_mma_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (p.T + TOK - 1) / TOK;
+    router_mma_kernel<TOK><<<(unsigned)blocks, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+}  // namespace rmma
+
 cudaError_t launch_router_mma(const Plan& p, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(rmma::router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)rmma::kSmem);
-    if (e != cudaSuccess) return e;
-    const int64_t blocks = (p.T + rmma::kTok - 1) / rmma::kTok;
-    rmma::router_mma_kernel<<<(unsigned)blocks, rmma::kThreads, rmma::kSmem, s>>>(p);
-    return cudaGetLastError();
+    // the largest tile that still gives every SM a CTA (16 tokens at the least).  Measured on B200 (router
+    // stage, us): T = 2048: 111 with 128-token tiles, 38.6 with 16; T = 8192 (d 1536): 152 with 128, 75.7
+    // with 32, 105 with 16 (two CTAs per SM: every CTA reads the whole split W_r from L2); T = 32768: 276
+    // with 128, 286 with 64.
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = sms;
+    if (p.T >= 128 * want) return rmma::launch_tok<128>(p, s);
+    if (p.T >= 64 * want) return rmma::launch_tok<64>(p, s);
+    if (p.T >= 32 * want) return rmma::launch_tok<32>(p, s);
+    return rmma::launch_tok<16>(p, s);
 }
 
 }  // namespace mmoe
