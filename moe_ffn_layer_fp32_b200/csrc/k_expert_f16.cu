@@ -74,9 +74,6 @@ constexpr int kTmemCols = kBufs * kBufCols;
 // 8 or 16: two or four per SM sub-partition.  Measured on c4 (gate/up, down): 2.90 / 1.54 ms with 8,
 // 2.80 / 1.95 ms with 16 (32 token columns per thread); the build uses 8.
 constexpr int kPromoWarps = MMOE_F16_PROMO_WARPS;
-#ifndef MMOE_F16_LD
-#define MMOE_F16_LD 16
-#endif
 constexpr int kPromoWarp0 = 4;             // promotion warps are the warpgroups after the first
 constexpr int kThreads = 128 + kPromoWarps * 32;
 // Register split (setmaxnreg): the launch gives every thread kRegsLaunch registers (what fits the SM's
@@ -498,7 +495,6 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
                 if (!warp_wait(&sm->accf[b], (pc >> 1) & 1, sm, ef, 15)) { ok = false; break; }
                 tc5::after_sync();
                 const uint32_t ta = tl + b * kBufCols;
-#if MMOE_F16_LD == 16
                 // loads of 16 columns (half 0, then half 1), each overlapped with the promotion of the
                 // one before; the buffer goes back to the MMA as soon as the last has landed
                 constexpr int kPerHalf = kChunks / 2;
@@ -522,66 +518,6 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
                     promote8(acc + (ch % kPerHalf) * 8, cur, half ? s1 : s0);
                     if (kDump) dump16<kEpi>(p, a, ti, half, row, col0 + (ch % kPerHalf) * 16, cur, j);
                 }
-#elif MMOE_F16_LD == 32
-                // loads of 32 columns, each overlapped with the promotion of the one before
-                constexpr int kPer = kCols / 32, kN = 2 * kPer;
-                uint32_t va[32], vb[32];
-                tc5::tmem_ld32(ta, va);
-#pragma unroll
-                for (int ch = 0; ch < kN; ++ch) {
-                    uint32_t (&cur)[32] = (ch & 1) ? vb : va;
-                    uint32_t (&nxt)[32] = (ch & 1) ? va : vb;
-                    tc5::tmem_wait_ld(cur);
-                    if (ch < kN - 1) {
-                        const int nc = ch + 1;
-                        tc5::tmem_ld32(ta + (nc / kPer) * BN + (nc % kPer) * 32, nxt);
-                    } else {
-                        tc5::before_sync();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm->acce[b]);
-                    }
-                    const int half = ch / kPer;
-                    float2* acc = (half ? acc1 : acc0) + (ch % kPer) * 16;
-                    const float sc = half ? s1 : s0;
-                    promote8(acc, reinterpret_cast<const uint32_t(&)[16]>(cur[0]), sc);
-                    promote8(acc + 8, reinterpret_cast<const uint32_t(&)[16]>(cur[16]), sc);
-                    if (kDump) {
-                        dump16<kEpi>(p, a, ti, half, row, col0 + (ch % kPer) * 32, reinterpret_cast<const uint32_t(&)[16]>(cur[0]), j);
-                        dump16<kEpi>(p, a, ti, half, row, col0 + (ch % kPer) * 32 + 16, reinterpret_cast<const uint32_t(&)[16]>(cur[16]), j);
-                    }
-                }
-#else
-                // all loads of a half (kCols columns) issued together, one wait per half
-                constexpr int kPerHalf = kCols / 16;
-                static_assert(kPerHalf == 4, "four 16-column loads per half");
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t v0[16], v1[16], v2[16], v3[16];
-                    const uint32_t th = ta + half * BN;
-                    tc5::tmem_ld16(th, v0);
-                    tc5::tmem_ld16(th + 16, v1);
-                    tc5::tmem_ld16(th + 32, v2);
-                    tc5::tmem_ld16(th + 48, v3);
-                    tc5::tmem_wait_ld4(v0, v1, v2, v3);
-                    if (half == 1) {
-                        tc5::before_sync();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm->acce[b]);
-                    }
-                    float2* acc = half ? acc1 : acc0;
-                    const float sc = half ? s1 : s0;
-                    promote8(acc, v0, sc);
-                    promote8(acc + 8, v1, sc);
-                    promote8(acc + 16, v2, sc);
-                    promote8(acc + 24, v3, sc);
-                    if (kDump) {
-                        dump16<kEpi>(p, a, ti, half, row, col0, v0, j);
-                        dump16<kEpi>(p, a, ti, half, row, col0 + 16, v1, j);
-                        dump16<kEpi>(p, a, ti, half, row, col0 + 32, v2, j);
-                        dump16<kEpi>(p, a, ti, half, row, col0 + 48, v3, j);
-                    }
-                }
-#endif
                 s0 = n0;
                 s1 = n1;
             }
