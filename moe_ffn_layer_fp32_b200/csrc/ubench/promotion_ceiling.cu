@@ -29,7 +29,6 @@
 #include "../sm100_tc.cuh"
 
 using namespace mmoe;
-using async::clk;
 using async::mbar_arrive;
 using async::mbar_init;
 using async::mbar_try_wait;
@@ -44,6 +43,13 @@ constexpr int kColGroups = kW / 4;   // warps that share a lane quarter split it
 constexpr int kCols = kBN / kColGroups;
 
 constexpr long long kSpinLimit = 2000000000ll;  // clocks; a wait that runs out sets the error flag
+
+// SM clock, ordered with the memory operations and barriers around it
+__device__ __forceinline__ long long clk() {
+    long long t;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t)::"memory");
+    return t;
+}
 
 struct Shm {
     uint64_t accf[4];  // MMA -> promotion: group in buffer b is in TMEM
@@ -148,6 +154,7 @@ __global__ void __launch_bounds__(64 + kW * 32, 1) ceiling_kernel(int ngroups, f
             tc5::commit(&sm->done);
             wait_bounded(&sm->done, 0, &sm->abort_);
         }
+        __syncwarp();  // the warp is whole again before the CTA barrier below (its lanes wait for lane 0)
     } else if (warp >= 2 && MODE != 1) {
         const int pw = warp - 2, q = warp & 3, cgi = pw >> 2;
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cgi * kCols);
@@ -320,24 +327,35 @@ bool check_exact(int pattern) {
 template <int KIND, int MODE>
 bool run(int nsm, int ngroups, float* out, long long* cyc, int* err) {
     auto k = ceiling_kernel<KIND, MODE>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_one_per_sm());
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_one_per_sm());
     cudaMemset(err, 0, 4);
-    k<<<nsm, 64 + kW * 32, smem_one_per_sm()>>>(ngroups / 8, out, cyc, err);  // warm-up
-    k<<<nsm, 64 + kW * 32, smem_one_per_sm()>>>(ngroups, out, cyc, err);
-    const cudaError_t e = cudaDeviceSynchronize();
-    std::vector<long long> h(nsm);
+    cudaMemset(cyc, 0, nsm * sizeof(long long));
+    cudaEvent_t e0, e1;
+    cudaEventCreate(&e0);
+    cudaEventCreate(&e1);
+    float ms = 0.0f;
+    if (e == cudaSuccess) {
+        k<<<nsm, 64 + kW * 32, smem_one_per_sm()>>>(ngroups / 8, out, cyc, err);  // warm-up
+        cudaEventRecord(e0);
+        k<<<nsm, 64 + kW * 32, smem_one_per_sm()>>>(ngroups, out, cyc, err);
+        cudaEventRecord(e1);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) cudaEventElapsedTime(&ms, e0, e1);
+    if (e != cudaSuccess) printf("launch: %s\n", cudaGetErrorString(e));
+    int clock_khz = 0;
+    cudaDeviceGetAttribute(&clock_khz, cudaDevAttrClockRate, 0);
     int herr = 0;
-    cudaMemcpy(h.data(), cyc, nsm * sizeof(long long), cudaMemcpyDeviceToHost);
     cudaMemcpy(&herr, err, 4, cudaMemcpyDeviceToHost);
-    double avg = 0;
-    for (long long v : h) avg += (double)v;
-    avg /= nsm;
     // one group = 128 x kBN x 32 multiply-adds; the nominal dense rates per SM and clock are
-    // 8192 (i8) and 4096 (f16) multiply-adds
-    const double macs = 128.0 * kBN * 32.0, clk_per_group = avg / ngroups;
+    // 8192 (i8) and 4096 (f16) multiply-adds.  Clocks per group from the event time at the device's
+    // maximum SM clock.
+    const double macs = 128.0 * kBN * 32.0, clk_per_group = (double)ms * clock_khz / ngroups;
     static const char* kModes[] = {"handoff+ld+promotion", "MMA only", "", "", "handoff+ld, no math"};
-    printf("%-4s %-22s %s clk/group %7.1f  = %5.1f%% of the nominal i8 rate, %5.1f%% of the nominal f16 rate\n",
-           KIND == 0 ? "i8" : "f16", kModes[MODE], e == cudaSuccess && !herr ? "ok " : "ERR", clk_per_group,
+    printf("%-4s %-22s %s %.3f ms, clk/group %6.1f = %5.1f%% of the nominal i8 rate, %5.1f%% of the nominal f16 "
+           "rate\n",
+           KIND == 0 ? "i8" : "f16", kModes[MODE], e == cudaSuccess && !herr ? "ok " : "ERR", ms, clk_per_group,
            100.0 * (macs / 8192.0) / clk_per_group, 100.0 * (macs / 4096.0) / clk_per_group);
     return e == cudaSuccess && !herr;
 }

@@ -2,6 +2,7 @@
 
     python -m moe_ffn_layer_fp32_b200.run_case --workload c2 --iters 3
     python -m moe_ffn_layer_fp32_b200.run_case --workload c4 --tokens 64 --iters 3     # decode batch
+    python -m moe_ffn_layer_fp32_b200.run_case --workload c1 --chain 24 --iters 3      # stack of 24 layers
 
 Meant as a fixed, small command line for profilers (one handle, `--iters`
 forwards after one warm-up forward, nothing else on the device).  Weights and
@@ -43,7 +44,12 @@ def main(argv=None) -> int:
     ap.add_argument("--cuda-cores", action="store_true")
     ap.add_argument("--deterministic", action="store_true")
     ap.add_argument("--tc-int8", action="store_true", help="prefill GEMMs on the kind::i8 tensor-core kernels")
+    ap.add_argument("--chain", type=int, default=0,
+                    help="run a stack of this many layers (layer l's weights seeded as the workload's layer l) "
+                         "through mmoe_forward_chain")
     args = ap.parse_args(argv)
+    if args.chain:
+        return chain(args)
 
     dev = torch.device("cuda", 0)
     w = synth.WORKLOADS[args.workload]
@@ -66,6 +72,36 @@ def main(argv=None) -> int:
     L.close()
     per = {k: round(v[1] * 1e3 / max(args.iters, 1), 2) for k, v in stages.items() if v[0] or v[1]}
     print(f"{w.name} T={T}: per forward, us by stage: {per}", flush=True)
+    return 0
+
+
+def chain(args) -> int:
+    dev = torch.device("cuda", 0)
+    w = synth.WORKLOADS[args.workload]
+    T = w.T if args.tokens is None else args.tokens
+    layers = []
+    for l in range(args.chain):
+        tensors, lw = quantized_weights(w, dev, l)
+        L = MoELayer(w.d, w.h, shared_hidden=w.hs, n_experts=w.E, top_k=w.k, max_tokens=T,
+                     has_router_bias=lw.router_bias is not None)
+        L.load(*tensors)
+        layers.append(L)
+        del tensors
+    x = torch.from_numpy(synth.workload_x(w, T=T).view(np.int16)).to(dev).view(torch.bfloat16)
+    ys = [torch.empty((T, w.d), dtype=torch.float32, device=dev) for _ in layers]
+    MoELayer.forward_chain(layers, x, ys)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.iters):
+        MoELayer.forward_chain(layers, x, ys)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / max(args.iters, 1)
+    print(f"{w.name} T={T}, {len(layers)} layers: {us:.1f} us per stack, {us / len(layers):.2f} us per layer",
+          flush=True)
+    for L in layers:
+        L.close()
     return 0
 
 
