@@ -77,16 +77,18 @@ typedef enum {
 
 /* mmoe_config.flags */
 #define MMOE_FLAG_DETERMINISTIC 1u /* combine in a fixed order, y = FFN_s + g_0 FFN_0 + ... + g_{k-1} FFN_{k-1},
-                                      on every path (the prefill path does so by default; the decode
-                                      path otherwise adds into y with atomics); needs an extra
+                                      on every path, so that y is bit-reproducible (by default the
+                                      prefill and decode expert GEMMs add into y with FP32 atomics, in
+                                      whatever order they arrive; a forward of at most 8 tokens always
+                                      adds in the fixed order); needs an extra
                                       [max_tokens*(k+1), d_model] FP32 workspace */
 #define MMOE_FLAG_CUDA_CORES 2u    /* run the expert GEMMs on CUDA cores (dp4a) even where the tensor-core
                                       kernels apply (those need d_model and both hidden sizes to be
                                       multiples of 128); same results, slower */
-#define MMOE_FLAG_ATOMIC_COMBINE 8u /* prefill path: add the expert outputs into y with atomics instead
-                                      of the fixed-order combine; saves the [max_tokens*(k+1), d_model]
-                                      FP32 workspace, y then depends on the order of the additions
-                                      (ignored with MMOE_FLAG_DETERMINISTIC) */
+#define MMOE_FLAG_ATOMIC_COMBINE 8u /* atomics into y: the default of mmoe_forward (accepted, changes
+                                      nothing there); for mmoe_forward_static_scratch, whose default is
+                                      the fixed-order combine, it selects the atomics (ignored with
+                                      MMOE_FLAG_DETERMINISTIC) */
 #define MMOE_FLAG_NO_DECODE 4u     /* never take the decode path: by default a forward with few tokens
                                       (T <= 64 where d_model and both hidden sizes are multiples of 64)
                                       runs the weight-streaming decode kernels; same results */

@@ -217,6 +217,11 @@ __global__ void __launch_bounds__(kThreads, 2) router_mma_kernel(Plan p)
     const int nt = (int)((p.T - t0) < TOK ? (p.T - t0) : TOK);
     auto xs = [&](int c) { return smem + (c % kStages) * (kXChunkBytes + kWChunkBytes); };
     auto ws = [&](int c) { return smem + (c % kStages) * (kXChunkBytes + kWChunkBytes) + kXChunkBytes; };
+    if (!p.deterministic && p.y) {
+        // the expert GEMMs add into y with atomics: this CTA's rows start at zero
+        float4* y4 = reinterpret_cast<float4*>(p.y + t0 * d);
+        for (int i = tid; i < nt * d / 4; i += kThreads) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
     const int nchunks = d / kKC;
     float acc[8][4];
 #pragma unroll

@@ -62,10 +62,11 @@ class MoELayer:
         """decode=False keeps small batches (T <= 64) on the prefill kernels instead of the
         weight-streaming decode kernels; cuda_cores=True runs every expert GEMM on CUDA cores;
         tc_int8=True runs the prefill expert GEMMs on the kind::i8 tensor-core kernels instead of the
-        default kind::f16 ones; fused_decode=False keeps batches of at most 8 tokens on the three-launch
+        default kind::f16 ones; fused_decode=False keeps batches of at most 8 tokens on the four-launch
         decode kernels instead of the one-launch decode; fused_requant=True requantises the SwiGLU output
-        inside the prefill gate/up GEMM (thread-block clusters); atomic_combine=True adds the prefill expert outputs into y with atomics
-        (no [R, d] workspace); deterministic=True uses the fixed-order combine on the decode path too."""
+        inside the prefill gate/up GEMM (thread-block clusters); deterministic=True adds the expert outputs
+        into y in the fixed order of Eq. (*) (bit-reproducible y, an [R, d] workspace) instead of with FP32
+        atomics; atomic_combine is the default and changes nothing."""
         flags = ((_lib.FLAG_DETERMINISTIC if deterministic else 0) | (_lib.FLAG_CUDA_CORES if cuda_cores else 0)
                  | (0 if decode else _lib.FLAG_NO_DECODE) | (_lib.FLAG_ATOMIC_COMBINE if atomic_combine else 0)
                  | (_lib.FLAG_TC_INT8 if tc_int8 else 0) | (0 if fused_decode else _lib.FLAG_NO_FUSED_DECODE)
