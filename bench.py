@@ -36,9 +36,10 @@ METRIC = "MoE-layer prefill tokens/s & decode us/layer; % of INT8-TC / HBM roofl
 # first 16 hex digits of the SHA-256 of the GEMM's source file at the time of the
 # capture: a figure is reported only while that file is unchanged.
 GATE_UP_TRAFFIC_BYTES = {
-    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:expert_gemm_f16 (1 pass):
-    # c2 157.09 + 9.36 MB, c4 1.22 GB + 635.09 MB
-    "b012fadf693f5309": {"c2": 166_450_000, "c4": 1_855_090_000},
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:expert_gemm (1 pass) on
+    # python -m moe_ffn_layer_fp32_b200.run_case --workload c4 --iters 1: 1.22 GB read + 1.29 GB written
+    # (the (gate, up) pairs, 8 bytes per feature and row)
+    "53bd93dd6d5e50a8": {"c4": 2_510_000_000},
 }
 GEMM_SOURCE = os.path.join(ROOT, "moe_ffn_layer_fp32_b200", "csrc", "k_expert_f16.cu")
 L2_BYTES = 126 * 1024 * 1024

@@ -356,7 +356,7 @@ mmoe_status mmoe_profile_read(mmoe_handle* h, int32_t* launches, double* total_m
  *     place with vector loads).
  *   - Size limit: T <= 2^20, and the scratch a call needs grows with T,
  *     d_model, the hidden sizes and top_k: about
- *     T*(top_k+1)*(d_model + 5*max_hidden) bytes, plus T*(top_k+1)*d_model*4
+ *     T*(top_k+1)*(d_model + 9*max_hidden) bytes, plus T*(top_k+1)*d_model*4
  *     for the fixed-order combine.  A call that needs more than the array
  *     holds is rejected with MMOE_ERR_INVALID_ARG before anything is
  *     launched.  cfg->max_tokens is not used.

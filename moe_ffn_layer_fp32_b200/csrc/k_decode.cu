@@ -252,7 +252,6 @@ __device__ void permute_block(const Plan& p) {
         }
         __syncthreads();
     }
-    for (int i = tid; i < (int)p.R; i += kRThreads) p.amax_h[i] = 0u;
 }
 
 // One cluster of `cs` CTAs handles all T <= 64 tokens; CTA `rank` the K rows
@@ -475,7 +474,7 @@ __device__ __forceinline__ float swiglu_row(float g, float u, float sxr) {
 template <bool GU, bool DUMP, int NCH>
 __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs,
                                           const float* shs, int lane, int rb, int64_t rrow0, int prows,
-                                          int32_t* dump, int64_t drow0, int64_t dnrows, uint32_t* amax_rows)
+                                          int32_t* dump, int64_t drow0, int64_t dnrows)
 {
     const int gid = lane >> 2, t4 = lane & 3;
     float alo[NCH][2], ahi[NCH][2];
@@ -484,24 +483,19 @@ __device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, co
     if (DUMP) return true;
 
     if (GU) {
+        // the (gate, up) pairs times the rows' activation scales (shs, staged by the caller); the
+        // requantisation launch applies the SwiGLU
         const int n = rb * 8 + gid;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int i = c * 8 + 2 * t4 + q;
-                const bool valid = i < prows;
+                if (i >= prows) continue;
                 const int64_t r = rrow0 + i;
-                float a = 0.0f;
-                if (valid) {
-                    a = swiglu_row(alo[c][q], ahi[c][q], shs[i]);  // shs: the rows' activation scales
-                    p.act[r * p.hmax + n] = a;
-                }
-                float m = fabsf(a);
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-                if (valid && gid == 0) atomicMax(amax_rows + i, __float_as_uint(m));
+                const float sxr = shs[i];
+                reinterpret_cast<float2*>(p.act)[r * p.hmax + n] =
+                    make_float2(__fmul_rn(alo[c][q], sxr), __fmul_rn(ahi[c][q], sxr));
             }
         }
     } else {
@@ -658,9 +652,9 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
         __syncthreads();
         if (alive)  // a warp that gave up keeps taking the CTA barriers but issues and computes nothing
             alive = nch == 1 ? warp_pass<GU, DUMP, 1>(p, S, codes, cs, shs, lane, rb, rrow0, prows, dump, drow0,
-                                                      dnrows, p.amax_h + rrow0)
+                                                      dnrows)
                              : warp_pass<GU, DUMP, 2>(p, S, codes, cs, shs, lane, rb, rrow0, prows, dump, drow0,
-                                                      dnrows, p.amax_h + rrow0);
+                                                      dnrows);
     }
 }
 
@@ -712,6 +706,7 @@ struct CArgs {
                           // the last CTA to leave)
     int nl;               // layers in this launch; layer l + 1 reads layer l's y rounded to BF16
     int off_x, off_codes, off_act, off_wr, off_u;  // dynamic shared memory offsets
+    int wr_in_ring;       // 1: the W_r slice shares the rings' space (fetched at the start of each layer)
     LayerW layers[kMaxChain];
 };
 
@@ -810,11 +805,11 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
     const int cid = (int)blockIdx.x / CS, ncl = (int)gridDim.x / CS;
     const int ks = d / CS;
     const bool keeper = cid == 0 && rank == 0;  // writes the routing and permutation for inspection
-    float* part_recv = reinterpret_cast<float*>(smem);                       // [CS][kCMaxT][64]
+    float* part_recv0 = reinterpret_cast<float*>(smem);                      // [2][CS][kCMaxT][64]
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + ca.off_x);             // [T][d]
     uint8_t* codes = smem + ca.off_codes;                                    // [8][max(d, hmax) + 32]
     float* act_all = reinterpret_cast<float*>(smem + ca.off_act);            // [8 rows][hmax] SwiGLU values
-    float* wr = reinterpret_cast<float*>(smem + ca.off_wr);                  // this CTA's slice of W_r
+    float* wr = reinterpret_cast<float*>(smem + (ca.wr_in_ring ? ca.off_u : ca.off_wr));  // this CTA's W_r slice
     uint8_t* ring = smem + ca.off_u;                                         // the warps' rings
     const uint32_t wbytes = (uint32_t)(ks * E * 4);
 
@@ -845,6 +840,9 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
 
     for (int l = 0; l < ca.nl; ++l) {
         const LayerW& Lw = ca.layers[l];
+        // partial logits from every CTA of the cluster, one copy per layer parity: a peer that has moved on
+        // to the next layer (possible when this cluster has no group in this layer) writes the other copy
+        float* part_recv = part_recv0 + (l & 1) * (CS * kCMaxT * 64);
         // ------------------------------------------------------------ this layer's x
         if (l == 0) {
             if (tid == 0) {
@@ -872,6 +870,10 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             }
             __syncthreads();
             ok = ok && st.flag;
+            if (ca.wr_in_ring && tid == 0) {
+                mbar_expect_tx(&st.wbar, wbytes);
+                bulk_load(wr, Lw.w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
+            }
             const float4* y4 = reinterpret_cast<const float4*>(ca.layers[l - 1].y);
             uint2* x2 = reinterpret_cast<uint2*>(xs);
             for (int i = tid; i < T * d / 4; i += kCThreads) {
@@ -920,7 +922,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             for (int t = 0; t < kCMaxT; ++t) rq[(q * kCMaxT + t) * 64 + e] = acc[t];
         }
         __syncthreads();
-        if (l + 1 < ca.nl && tid == 0) {
+        if (l + 1 < ca.nl && !ca.wr_in_ring && tid == 0) {
             // every thread is done with this layer's W_r slice: the next layer's goes in now
             mbar_expect_tx(&st.wbar, wbytes);
             bulk_load(wr, ca.layers[l + 1].w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
@@ -1147,7 +1149,6 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                     const int i = 2 * t4 + q;
                     if (i >= nrows) continue;
                     const float a = alive ? swiglu_row(alo[0][q], ahi[0][q], st.shs[i]) : 0.0f;
-                    p.act[(int64_t)(row0 + i) * p.hmax + n] = a;
 #pragma unroll 4
                     for (int c = 0; c < CS; ++c) st_peer(act_all + i * p.hmax + n, c, __float_as_uint(a));
                 }
@@ -1175,10 +1176,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                 if (lane == 0) {
                     const float sv = __fdiv_rn(m, 127.0f);
                     st.shs[warp] = sv;
-                    if (rank == 0) {
-                        p.amax_h[row0 + warp] = __float_as_uint(m);
-                        p.sh[row0 + warp] = sv;
-                    }
+                    if (rank == 0) p.sh[row0 + warp] = sv;
                 }
             } else if (warp < 8 && lane == 0) {
                 st.shs[warp] = 0.0f;
@@ -1404,27 +1402,32 @@ cudaError_t launch_expert(const Plan& p, cudaStream_t s, int32_t* dump, int64_t 
 size_t align128(size_t v) { return (v + 127) / 128 * 128; }
 
 // Dynamic shared memory of the one-launch decode and its offsets: partial logits from every CTA of
-// the cluster | x (BF16, up to kCMaxT tokens) | operand buffer of 8 rows | SwiGLU values of this CTA's
-// features (also the router's scratch) | the W_r slice, then the rings.
+// the cluster (two copies) | x (BF16, up to kCMaxT tokens) | operand buffer of 8 rows | SwiGLU values of
+// the group's rows (also the router's scratch) | the W_r slice | the rings.  Where that exceeds the SM's
+// shared memory the W_r slice lives in the rings' space instead (a layer's slice is then fetched when
+// the layer starts, not during the previous layer).
 size_t cluster_layout(int d, int h, int hs, int E, int CS, CArgs* ca) {
     const int hmax = h > hs ? h : hs;
-    size_t o = align128((size_t)CS * kCMaxT * 64 * 4);
+    size_t o = align128((size_t)2 * CS * kCMaxT * 64 * 4);
     const size_t off_x = o;
     o = align128(o + (size_t)kCMaxT * d * 2);
     const size_t off_codes = o;
     o = align128(o + (size_t)8 * ((d > hmax ? d : hmax) + 32));
     const size_t off_act = o;
     o = align128(o + std::max((size_t)8 * hmax * 4, (size_t)4 * kCMaxT * 64 * 4));
+    const size_t wr_bytes = align128((size_t)(d / CS) * E * 4), ring_bytes = (size_t)kCWarps * kRingMax * kStageBytes;
+    const bool apart = o + wr_bytes + ring_bytes + sizeof(CShared) <= (size_t)kSmemLimit;
     const size_t off_wr = o;
-    o = align128(o + (size_t)(d / CS) * E * 4);
+    if (apart) o += wr_bytes;
     const size_t off_u = o;
-    o += (size_t)kCWarps * kRingMax * kStageBytes;
+    o += std::max(ring_bytes, apart ? (size_t)0 : wr_bytes);
     if (ca) {
         ca->off_x = (int)off_x;
         ca->off_codes = (int)off_codes;
         ca->off_act = (int)off_act;
         ca->off_wr = (int)off_wr;
         ca->off_u = (int)off_u;
+        ca->wr_in_ring = apart ? 0 : 1;
     }
     return o;
 }

@@ -592,14 +592,17 @@ expert_gemm_f16_kernel(const __grid_constant__ CUtensorMap bmap, Plan p, Args a)
                     }
                 }
             } else if (kEpi == kEpiSwiGLU) {
-                float* out = p.act + row0 * p.hmax + mb * BMH + row;
+                // the (gate, up) pair of each feature times the row's activation scale; the SwiGLU itself
+                // is applied by the requantisation pass, off this loop's critical path
+                float2* out = reinterpret_cast<float2*>(p.act) + row0 * p.hmax + mb * BMH + row;
 #pragma unroll
                 for (int c = 0; c < kCols; ++c) {
                     const int cc = col0 + c;
                     if (cc < nr) {
                         const float g = (c & 1) ? acc0[c >> 1].y : acc0[c >> 1].x;
                         const float u = (c & 1) ? acc1[c >> 1].y : acc1[c >> 1].x;
-                        out[(int64_t)cc * p.hmax] = swiglu(g, u, ti.colf[cc]);
+                        const float f = ti.colf[cc];
+                        out[(int64_t)cc * p.hmax] = make_float2(__fmul_rn(g, f), __fmul_rn(u, f));
                     }
                 }
             } else {

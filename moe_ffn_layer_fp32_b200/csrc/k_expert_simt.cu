@@ -140,29 +140,34 @@ __global__ void __launch_bounds__(kThreads) gate_up_simt_kernel(Plan p, int32_t*
         if (tq * 8 + r >= ti.nr) continue;
         const int64_t grow = ti.row0 + tq * 8 + r;
         const float sxr = p.sx[p.row_src[grow]];
-        const float gv = __fmul_rn(ag[r], sxr), uv = __fmul_rn(au[r], sxr);
-        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
-        p.act[grow * p.hmax + n] = __fmul_rn(silu, uv);
+        reinterpret_cast<float2*>(p.act)[grow * p.hmax + n] = make_float2(__fmul_rn(ag[r], sxr), __fmul_rn(au[r], sxr));
     }
 }
 
-// per-row requantisation of the SwiGLU output: s_h = absmax / 127
+// per-row SwiGLU and requantisation: a = silu(gv) * uv from the gate/up pairs, s_h = absmax / 127, the
+// codes; one warp per row, its SwiGLU values kept in shared memory between the two passes
 __global__ void __launch_bounds__(kThreads) requant_kernel(Plan p)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    extern __shared__ __align__(16) float arow[];  // [warps][hmax]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + warp;
     if (row >= p.R) return;
     const int hid = row >= p.Tk ? p.hs : p.h;
-    // 16 bytes per lane: rows start on 4 * hmax bytes and hid is a multiple of 32
-    const float4* a4 = reinterpret_cast<const float4*>(p.act + row * p.hmax);
+    float* a = arow + (size_t)warp * p.hmax;
+    // 32 bytes per lane: rows start on 8 * hmax bytes and hid is a multiple of 32
+    const float4* pr = reinterpret_cast<const float4*>(p.act + row * 2 * p.hmax);
     float m = 0.0f;
-#pragma unroll 4
+#pragma unroll 2
     for (int i = lane; i < hid / 4; i += 32) {
-        const float4 v = a4[i];
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        const float4 v0 = pr[2 * i], v1 = pr[2 * i + 1];
+        const float4 s4 = make_float4(swiglu_pair(v0.x, v0.y), swiglu_pair(v0.z, v0.w), swiglu_pair(v1.x, v1.y),
+                                      swiglu_pair(v1.z, v1.w));
+        reinterpret_cast<float4*>(a)[i] = s4;
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(s4.x), fabsf(s4.y)), fmaxf(fabsf(s4.z), fabsf(s4.w))));
     }
     m = warp_max(m);
     const float s = __fdiv_rn(m, 127.0f);
+    const float4* a4 = reinterpret_cast<const float4*>(a);
     if (p.hq16) {
         // f16 codes for the kind::f16 down GEMM
         uint2* q = reinterpret_cast<uint2*>(p.hq16 + row * p.hmax);
@@ -285,7 +290,12 @@ cudaError_t launch_gate_up(const Plan& p, cudaStream_t s, int32_t* dump, int64_t
 cudaError_t launch_requant(const Plan& p, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
     const int64_t blocks = (p.R + kThreads / 32 - 1) / (kThreads / 32);
-    requant_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(p);
+    const size_t smem = (size_t)(kThreads / 32) * p.hmax * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(requant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    requant_kernel<<<(unsigned)blocks, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -296,12 +296,10 @@ __device__ __forceinline__ void epilogue_step(const Plan& p, const TileInfo& ti,
         const float sx = ti.colf[cc];
         const float4 g4 = *reinterpret_cast<const float4*>(&xch[cc * BM + fl4]);
         const float4 u4 = *reinterpret_cast<const float4*>(&xch[cc * BM + 64 + fl4]);
-        float4 r;
-        r.x = swiglu(g4.x, u4.x, sx);
-        r.y = swiglu(g4.y, u4.y, sx);
-        r.z = swiglu(g4.z, u4.z, sx);
-        r.w = swiglu(g4.w, u4.w, sx);
-        *reinterpret_cast<float4*>(p.act + (row0 + cc) * p.hmax + mb * 64 + fl4) = r;
+        // (gate, up) pairs times the activation scale; the requantisation pass applies the SwiGLU
+        float4* out = reinterpret_cast<float4*>(p.act + ((row0 + cc) * p.hmax + mb * 64 + fl4) * 2);
+        out[0] = make_float4(__fmul_rn(g4.x, sx), __fmul_rn(u4.x, sx), __fmul_rn(g4.y, sx), __fmul_rn(u4.y, sx));
+        out[1] = make_float4(__fmul_rn(g4.z, sx), __fmul_rn(u4.z, sx), __fmul_rn(g4.w, sx), __fmul_rn(u4.w, sx));
     } else {
         // column cq + step; lane l covers outputs mb*128 + 4 l .. + 3
         const int cc = cq + step;

@@ -147,7 +147,6 @@ struct mmoe_handle {
     int dec_cluster = 0;
     uint8_t* w_gate_up_d = nullptr;
     uint8_t* w_down_d = nullptr;
-    uint32_t* amax_h = nullptr;
     int32_t* dec_groups = nullptr;
     int32_t* dec_ngroups = nullptr;
     // fused one-launch decode: synchronisation words (kept zero between launches), router partials,
@@ -191,7 +190,7 @@ void free_all(mmoe_handle* h) {
                     h->xq, h->sx, h->logits, h->idx, h->gate, h->chunk_cnt, h->chunk_base, h->offsets,
                     h->counts, h->tiles, h->tile_count, h->row_src, h->row_gate, h->slot_row, h->act, h->hq,
                     h->sh, h->obuf, h->x_stage, h->y_stage, h->w_gate_up_t, h->s_gate_up_t, h->w_down_t,
-                    h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->amax_h, h->dec_groups,
+                    h->s_down_t, h->err_dev, h->w_gate_up_d, h->w_down_d, h->dec_groups,
                     h->dec_ngroups, h->w_gate_up_f16, h->w_down_f16, h->xq16, h->hq16, h->dec_sync,
                     h->dec_obuf};
     for (void* p : ptrs)
@@ -296,7 +295,6 @@ Plan make_plan(const mmoe_handle* h, const uint16_t* x, int64_t T, float* y) {
     p.err_host = h->err_host_dev;
     p.w_gate_up_d = h->w_gate_up_d;
     p.w_down_d = h->w_down_d;
-    p.amax_h = h->amax_h;
     p.dec_groups = h->dec_groups;
     p.dec_ngroups = h->dec_ngroups;
     return p;
@@ -412,7 +410,7 @@ size_t carve_static_plan(Plan& p, unsigned char* base, size_t cap) {
     p.row_src = static_cast<int32_t*>(take(R * 4));
     p.row_gate = static_cast<float*>(take(R * 4));
     p.slot_row = static_cast<int32_t*>(take(T * k * 4));
-    p.act = static_cast<float*>(take(R * (size_t)p.hmax * 4));
+    p.act = static_cast<float*>(take(R * (size_t)p.hmax * 8));
     p.hq = static_cast<int8_t*>(take(R * (size_t)p.hmax));
     p.sh = static_cast<float*>(take(R * 4));
     p.obuf = p.deterministic ? static_cast<float*>(take(R * d * 4)) : nullptr;
@@ -503,13 +501,12 @@ mmoe_status mmoe_create(const mmoe_config* cfg, int device, mmoe_handle** out) {
     ALLOC(row_src, R);
     ALLOC(row_gate, R);
     ALLOC(slot_row, Tm * k);
-    ALLOC(act, Ract * h->hmax);
+    ALLOC(act, Ract * 2 * h->hmax);  // (gate, up) pairs
     ALLOC(hq, R8 * h->hmax);
     ALLOC(sh, R);
     if (h->use_dec) {
         ALLOC(w_gate_up_d, h->n_gu_bytes + h->n_gu_scales * 4);
         ALLOC(w_down_d, h->n_d_bytes + h->n_d_scales * 4);
-        ALLOC(amax_h, Rd);
         ALLOC(dec_groups, E + 1);
         ALLOC(dec_ngroups, 1);
         if (!(cfg->flags & MMOE_FLAG_NO_FUSED_DECODE)) {
@@ -725,9 +722,15 @@ mmoe_status mmoe_forward_chain(mmoe_handle* const* layers, int32_t n_layers, con
         p.hq16 = nullptr;
         DecChainLayer L[MMOE_MAX_CHAIN_LAYERS];
         for (int l = 0; l < n_layers; ++l)
-            L[l] = DecChainLayer{layers[l]->w_router,    layers[l]->router_bias, layers[l]->w_gate_up_d,
-                                 layers[l]->w_down_d,    y_layers[l],            nullptr,
-                                 nullptr,                nullptr};
+            // (a handle without a router bias in its config has the buffer, but nothing was loaded into it)
+            L[l] = DecChainLayer{layers[l]->w_router,
+                                 layers[l]->cfg.has_router_bias ? layers[l]->router_bias : nullptr,
+                                 layers[l]->w_gate_up_d,
+                                 layers[l]->w_down_d,
+                                 y_layers[l],
+                                 nullptr,
+                                 nullptr,
+                                 nullptr};
         MMOE_CUDA(run_stage(h0, MMOE_PROF_DECODE_FUSED, 1, s,
                             [&] {
                                 return launch_decode_chain(p, h0->dec_shape, h0->dec_sync, h0->dec_obuf,

@@ -50,7 +50,7 @@ struct Plan {
     int32_t* row_src;       // [R]
     float* row_gate;        // [R]
     int32_t* slot_row;      // [T, k]
-    float* act;             // [R, hmax] SwiGLU output before requantisation
+    float* act;             // [R, hmax] pairs (gv, uv): gate and up times the row's activation scale
     int8_t* hq;             // [R, hmax]
     float* sh;              // [R]
     float* obuf;            // [R, d] expert outputs (deterministic combine only)
@@ -78,7 +78,6 @@ struct Plan {
     // decode path (k_decode.cu)
     const uint8_t* w_gate_up_d;   // weights + scales in the decode layout
     const uint8_t* w_down_d;
-    uint32_t* amax_h;             // [R] bits of max |SwiGLU output| of each row (non-negative floats order as integers)
     int32_t* dec_groups;          // [E + 1] groups with at least one row: the shared one first, then routed ascending
     int32_t* dec_ngroups;         // [1]
 };
@@ -226,6 +225,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
+}
+
+// SwiGLU of one feature from its gate and up values already scaled by the token's activation scale:
+// silu(gv) * uv, silu(v) = v / (1 + exp(-v)), each step an IEEE FP32 operation.  The gate/up GEMMs
+// store (gv, uv) pairs; the requantisation pass applies this.
+__device__ __forceinline__ float swiglu_pair(float gv, float uv) {
+    return __fmul_rn(__fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv))), uv);
 }
 
 // Symmetric INT8 code of v with scale s (s = absmax / 127): IEEE division,

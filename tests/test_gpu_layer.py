@@ -149,6 +149,23 @@ def test_one_launch_decode_against_three_launches(name, T):
     assert np.max(np.abs(a["y"] - b["y"])) <= 1e-5 * np.abs(b["y"]).max()
 
 
+@pytest.mark.parametrize("name", ["c0", "c1", "s2048", "c4dec"])
+def test_one_launch_decode_taken(name):
+    # a forward of up to 8 tokens is one launch of the one-launch decode on every workload shape
+    w = synth.WORKLOADS[name]
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    L = MoELayer(w.d, w.h, shared_hidden=w.hs, n_experts=w.E, top_k=w.k, max_tokens=64)
+    q = oracle.quantize_layer(synth.workload_layer(w))
+    L.load(q.w_router, q.router_bias, q.w_gate_up, q.s_gate_up, q.w_down, q.s_down)
+    x = gu.x_to_device(synth.draw_x(3, w.d, seed=7))
+    L.profile(True)
+    L.forward(x)
+    torch.cuda.synchronize()
+    launches = {k: v[0] for k, v in L.profile_read().items() if v[0]}
+    L.close()
+    assert launches == {"decode_fused": 1}, launches
+
+
 def test_one_launch_decode_deterministic_and_repeatable():
     # y of the one-launch decode is added in a fixed order: repeated calls agree bit for bit, and the
     # contribution counters left by each call let the next one (of another size) combine correctly
@@ -413,10 +430,14 @@ def test_forward_chain_matches_layer_by_layer(name, T):
     for l in range(n):
         y_ref = Ls[l].forward(xl)
         torch.cuda.synchronize()
-        assert torch.equal(ys[l].view(torch.int32), y_ref.view(torch.int32)), l
-        rep = {}
         x_np = xl.view(torch.int16).cpu().numpy().view(np.uint16)
-        gu.check_y(ys[l].cpu().numpy(), oracle.moe_layer(qs[l], x_np), rep)
+        y_or = oracle.moe_layer(qs[l], x_np)
+        scale = np.abs(y_or).max()
+        errs = (float(np.abs(ys[l].cpu().numpy() - y_or).max() / scale),
+                float(np.abs(y_ref.cpu().numpy() - y_or).max() / scale))
+        assert torch.equal(ys[l].view(torch.int32), y_ref.view(torch.int32)), (l, "chain / layer vs oracle", errs)
+        rep = {}
+        gu.check_y(ys[l].cpu().numpy(), y_or, rep)
         xl = y_ref.to(torch.bfloat16)
     # the same stack again: the launch left its counters ready for the next one
     ys2 = [torch.empty_like(y) for y in ys]
@@ -424,6 +445,30 @@ def test_forward_chain_matches_layer_by_layer(name, T):
     torch.cuda.synchronize()
     for a, b in zip(ys, ys2):
         assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    for L in Ls:
+        L.close()
+
+
+@pytest.mark.parametrize("gating", [0, 2])
+def test_forward_chain_with_router_bias(gating):
+    # layers with a router bias (in the logit for gating 0, in the selection only for gating 2): the
+    # stack in one launch equals the layers one by one
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    w = synth.WORKLOADS["c0"]
+    qs = [oracle.quantize_layer(synth.draw_layer(w.d, w.h, seed=70 + l, bias_coef=0.25), gating=gating)
+          for l in range(3)]
+    Ls = [gu.make_gpu_layer(q, 8) for q in qs]
+    T = 4
+    xd = gu.x_to_device(synth.draw_x(T, w.d, seed=71))
+    ys = [torch.empty((T, w.d), dtype=torch.float32, device="cuda") for _ in range(3)]
+    MoELayer.forward_chain(Ls, xd, ys)
+    torch.cuda.synchronize()
+    xl = xd
+    for l in range(3):
+        y_ref = Ls[l].forward(xl)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[l].view(torch.int32), y_ref.view(torch.int32)), l
+        xl = y_ref.to(torch.bfloat16)
     for L in Ls:
         L.close()
 
