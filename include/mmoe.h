@@ -95,7 +95,7 @@ typedef enum {
 #define MMOE_FLAG_NO_FUSED_DECODE 32u /* a forward of at most 8 tokens on the decode path runs the layer as
                                       one launch of thread-block clusters by default (each cluster routes
                                       the tokens itself and computes whole experts; y is added in the
-                                      fixed order of Eq. (*)); this flag keeps the three launches of the
+                                      fixed order of Eq. (*)); this flag keeps the four launches of the
                                       larger decode batches; the same routing and codes, y within
                                       FP32 rounding of the router's summation order */
 #define MMOE_FLAG_FUSED_REQUANT 64u /* the prefill gate/up GEMM (default tensor-core kind) requantises its
@@ -104,7 +104,8 @@ typedef enum {
                                       distributed shared memory, so no FP32 SwiGLU buffer and no separate
                                       requantisation pass exist (needs max hidden size <= 1024); same
                                       results.  Off by default: measured on B200 it is slower than the
-                                      separate pass (c4 gate/up 6.9 ms against 2.9 + 0.17 ms) */
+                                      separate pass (c4: 6.9 ms against 2.5 ms of gate/up GEMM
+                                      and 0.36 ms of SwiGLU and requantisation) */
 #define MMOE_FLAG_TC_INT8 16u      /* prefill expert GEMMs on the INT8 tensor-core kind (tcgen05 kind::i8,
                                       S32 group partials) instead of the default f16 kind (exact integer
                                       group partials in FP32 accumulators, which the promotion reads
