@@ -371,15 +371,18 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
 // 0) is stage sc % nst of pass sc / nst and lands in ring slot (base + sc) %
 // nring, so slot and phase carry over from stream to stream when `base` is the
 // warp's running stage count.  A pass consumes stages sc0 .. sc0 + nst - 1 and
-// refills the ring with stages below ntot.
+// refills the ring with stages below ntot.  NR: the ring size where it is fixed
+// at compile time (0: nring_rt).
+template <int NR>
 struct WarpStream {
     const uint8_t* src;   // the warp's first 16-row block in the decode layout
     uint8_t* ring;
     uint64_t* bars;
     int64_t pstride;
-    int NJ, nst, sc0, nring, ntot, base;
-    __device__ __forceinline__ int slot(int sc) const { return (base + sc) % nring; }
-    __device__ __forceinline__ uint32_t parity(int sc) const { return (uint32_t)(((base + sc) / nring) & 1); }
+    int NJ, nst, sc0, nring_rt, ntot, base;
+    __device__ __forceinline__ int nring() const { return NR ? NR : nring_rt; }
+    __device__ __forceinline__ int slot(int sc) const { return (base + sc) % nring(); }
+    __device__ __forceinline__ uint32_t parity(int sc) const { return (uint32_t)(((base + sc) / nring()) & 1); }
     __device__ __forceinline__ void issue(int sc) const {
         const int st = sc % nst;
         const int jp = NJ - st * kStageJP;
@@ -393,8 +396,8 @@ struct WarpStream {
 // The K loop of one warp over one pass of up to 8 * NCH rows: the accumulators
 // of its 16 weight rows (A rows 0-7 in alo, 8-15 in ahi) for every row column.
 // Returns false if a bounded wait gave up (the copies in flight have landed).
-template <bool GU, bool DUMP, int NCH>
-__device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs, int lane,
+template <bool GU, bool DUMP, int NCH, int NR>
+__device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream<NR>& S, const uint8_t* codes, int cs, int lane,
                                           int rb, int64_t rrow0, int prows, int32_t* dump, int64_t drow0,
                                           int64_t dnrows, float (&alo)[NCH][2], float (&ahi)[NCH][2])
 {
@@ -408,7 +411,7 @@ __device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream& S, co
         if (!wait_bounded(&S.bars[S.slot(sc)], S.parity(sc))) {
             if (lane == 0) set_error(p, 7);
             // let the copies in flight land before the CTA's shared memory goes away
-            const int issued = sc + S.nring < S.ntot ? sc + S.nring : S.ntot;
+            const int issued = sc + S.nring() < S.ntot ? sc + S.nring() : S.ntot;
             for (int s = sc; s < issued; ++s) wait_bounded(&S.bars[S.slot(s)], S.parity(s));
             return false;
         }
@@ -457,7 +460,7 @@ __device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream& S, co
             }
         }
         __syncwarp();
-        if (lane == 0 && sc + S.nring < S.ntot) S.issue(sc + S.nring);
+        if (lane == 0 && sc + S.nring() < S.ntot) S.issue(sc + S.nring());
     }
     return true;
 }
@@ -471,8 +474,8 @@ __device__ __forceinline__ float swiglu_row(float g, float u, float sxr) {
 
 // The GEMV of one warp over one pass of up to 8 * NCH rows, then its
 // epilogue.  Returns false if a bounded wait gave up (nothing is written).
-template <bool GU, bool DUMP, int NCH>
-__device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream& S, const uint8_t* codes, int cs,
+template <bool GU, bool DUMP, int NCH, int NR>
+__device__ __forceinline__ bool warp_pass(const Plan& p, const WarpStream<NR>& S, const uint8_t* codes, int cs,
                                           const float* shs, int lane, int rb, int64_t rrow0, int prows,
                                           int32_t* dump, int64_t drow0, int64_t dnrows)
 {
@@ -586,7 +589,7 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
     const int ngr = K / 32;
     const int rb = rb0 + warp;
     const bool wact = rb < nrb;
-    WarpStream S;
+    WarpStream<0> S;
     S.src = (GU ? p.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4)
                 : p.w_down_d + (int64_t)g * ((int64_t)p.d * p.h * 5 / 8)) +
             (int64_t)rb * NJ * kJP;
@@ -595,7 +598,7 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
     S.NJ = NJ;
     S.nst = (NJ + kStageJP - 1) / kStageJP;
     S.sc0 = 0;
-    S.nring = nring;
+    S.nring_rt = nring;
     S.pstride = 0;  // every pass of rows streams the same block again (from L2 after the first)
     S.base = 0;
     const int npass = (nrows + kPassRows - 1) / kPassRows;
@@ -715,8 +718,6 @@ struct CShared {
     uint64_t wbar, xbar;
     float sxs[kCMaxT];             // activation scales of the tokens
     float shs[8];                  // per row of the current group: activation scale, then SwiGLU scale
-    float keys[kCMaxT][64];        // top-k: each token's selection keys
-    float probs[kCMaxT][64];       //   and gating probabilities
     int idx[kCMaxSlots];
     float gate[kCMaxSlots];
     int slot_row[kCMaxSlots];
@@ -753,6 +754,21 @@ __device__ __forceinline__ void st_peer(const void* p, int rank, float4 v) {
 __device__ __forceinline__ int bfrag_pos(int v) { return v < 4 ? 2 * v : 2 * (v - 4) + 1; }
 
 // number of passes pi >= 0 with first + pi * step < n
+// Position of the set bit of m with n set bits below it (m has more than n set bits).
+__device__ __forceinline__ int nth_set_bit(uint32_t m, int n) {
+    int pos = 0;
+#pragma unroll
+    for (int w = 16; w > 0; w >>= 1) {
+        const int c = __popc(m & ((1u << w) - 1u));
+        if (n >= c) {
+            n -= c;
+            m >>= w;
+            pos += w;
+        }
+    }
+    return pos;
+}
+
 __device__ __forceinline__ int npasses(int first, int step, int n) { return first < n ? (n - first + step - 1) / step : 0; }
 
 // two floats rounded to BF16 (round to nearest even; finite inputs), packed low | high << 16
@@ -767,22 +783,35 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* a) {
     return v;
 }
 
-// The shared expert of a layer toward L2: this CTA's gate/up and down row blocks (one thread).
-template <int CS>
-__device__ void prefetch_shared_expert(const Plan& p, const LayerW& Lw, int rank) {
-    const int W = kCWarps, d = p.d, E = p.E;
-    const int NJ = d / 64, NJd = p.hs / 64, nrb = p.hs / 8, nrbd = d / 16;
-    for (int b0 = rank * W; b0 < nrb; b0 += CS * W)
-        prefetch_range(Lw.w_gate_up_d + (int64_t)E * ((int64_t)p.h * d * 5 / 4) + (int64_t)b0 * NJ * kJP,
-                       (int64_t)min(W, nrb - b0) * NJ * kJP);
-    for (int b0 = rank * W; b0 < nrbd; b0 += CS * W)
-        prefetch_range(Lw.w_down_d + (int64_t)E * ((int64_t)d * p.h * 5 / 8) + (int64_t)b0 * NJd * kJP,
-                       (int64_t)min(W, nrbd - b0) * NJd * kJP);
+// Adds v at GPU scope with acquire-release semantics and returns the old value.  Called after a CTA
+// barrier, it publishes every write of the CTA made before the barrier to whoever acquires the count,
+// and the caller sees what the earlier adders published.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* a, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+    return old;
+}
+
+// The same without the old value and the acquire half.
+__device__ __forceinline__ void red_add_release(uint32_t* a, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
+// One thread's L2 prefetch of this CTA's gate/up and down row blocks of a layer's shared expert (expert
+// E of the decode-layout arrays gu, dn).  Not inlined: one copy of code that one thread runs.
+__device__ __noinline__ void prefetch_shared_expert(const uint8_t* gu, const uint8_t* dn, int rank, int cs, int d,
+                                                    int h, int hs, int E) {
+    const int W = kCWarps, NJ = d / 64, NJd = hs / 64, nrb = hs / 8, nrbd = d / 16, rstep = cs * W;
+    const int64_t gu_stride = (int64_t)h * d * 5 / 4, dn_stride = (int64_t)d * h * 5 / 8;
+    for (int b = rank * W; b < nrb; b += rstep)
+        prefetch_range(gu + E * gu_stride + (int64_t)b * NJ * kJP, (int64_t)min(W, nrb - b) * NJ * kJP);
+    for (int b = rank * W; b < nrbd; b += rstep)
+        prefetch_range(dn + E * dn_stride + (int64_t)b * NJd * kJP, (int64_t)min(W, nrbd - b) * NJd * kJP);
 }
 
 // The gate/up weight stream of one warp over group g of a layer: row blocks rb0, rb0 + CS W, ...
 template <int CS>
-__device__ __forceinline__ void gu_stream(WarpStream& S, const Plan& p, const LayerW& Lw, int g, int rb0, int base) {
+__device__ __forceinline__ void gu_stream(WarpStream<kRingMax>& S, const Plan& p, const LayerW& Lw, int g, int rb0, int base) {
     const int hid = g == p.E ? p.hs : p.h, nrb = hid / 8, NJ = p.d / 64;
     const int np = npasses(rb0, CS * kCWarps, nrb);
     S.src = Lw.w_gate_up_d + (int64_t)g * ((int64_t)p.h * p.d * 5 / 4) + (int64_t)rb0 * NJ * kJP;
@@ -826,16 +855,15 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
         mbar_expect_tx(&st.wbar, wbytes);
         bulk_load(wr, ca.layers[0].w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
     }
-    if (cid == 0 && tid == 32) prefetch_shared_expert<CS>(p, ca.layers[0], rank);
     __syncthreads();  // the mbarriers are initialised
     pdl_wait();       // x, and the buffers the previous launch used
     bool ok = true;
     int wsc = 0;      // this warp's running stage count (ring slot and phase), over all layers
     bool alive = true;  // false once one of this warp's bounded waits gave up
-    WarpStream S;
+    WarpStream<kRingMax> S;
     S.ring = ring + warp * kRingMax * kStageBytes;
     S.bars = st.bars + warp * kRingMax;
-    S.nring = kRingMax;
+    S.nring_rt = kRingMax;
     const int rb0 = rank * W + warp;  // this warp's first row block of every stream
 
     for (int l = 0; l < ca.nl; ++l) {
@@ -843,6 +871,16 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
         // partial logits from every CTA of the cluster, one copy per layer parity: a peer that has moved on
         // to the next layer (possible when this cluster has no group in this layer) writes the other copy
         float* part_recv = part_recv0 + (l & 1) * (CS * kCMaxT * 64);
+        // the shared expert is cluster 0's first group whatever the routing: its gate/up stream starts before
+        // this layer's x is there, and the rest of this CTA's share of it goes toward L2 (unless the W_r slice
+        // is about to use the rings' space)
+        const bool early0 = cid == 0 && !ca.wr_in_ring;
+        if (early0) {
+            gu_stream<CS>(S, p, Lw, E, rb0, wsc);
+            if (alive && lane < kRingMax && lane < S.ntot) S.issue(lane);
+            if (tid == 32)
+                prefetch_shared_expert(Lw.w_gate_up_d, Lw.w_down_d, rank, CS, d, p.h, p.hs, E);
+        }
         // ------------------------------------------------------------ this layer's x
         if (l == 0) {
             if (tid == 0) {
@@ -876,18 +914,25 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             }
             const float4* y4 = reinterpret_cast<const float4*>(ca.layers[l - 1].y);
             uint2* x2 = reinterpret_cast<uint2*>(xs);
+#pragma unroll 1
             for (int i = tid; i < T * d / 4; i += kCThreads) {
                 const float4 v = __ldcg(y4 + i);
                 x2[i] = make_uint2(bf16_pair_rn(v.x, v.y), bf16_pair_rn(v.z, v.w));
             }
             __syncthreads();
         }
-        // activation scales: warp t, the absmax of token t over d
+        // activation scales: warp t, the absmax of token t over d (the magnitude bits of a BF16 value order
+        // like its magnitude, so an integer maximum over eight values per 16-byte word finds it exactly)
         for (int t = warp; t < T; t += W) {
-            float m = 0.0f;
-            for (int i = lane; i < d; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * d + i])));
-            m = warp_max(m);
-            if (lane == 0) st.sxs[t] = __fdiv_rn(m, 127.0f);
+            const uint4* xr = reinterpret_cast<const uint4*>(xs + t * d);
+            uint32_t m2 = 0u;
+            for (int i = lane; i < d / 8; i += 32) {
+                const uint4 v = xr[i];
+                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu),
+                                           __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu)));
+            }
+            const uint32_t mb = __reduce_max_sync(0xffffffffu, max(m2 & 0xffffu, m2 >> 16));
+            if (lane == 0) st.sxs[t] = __fdiv_rn(bf16_to_f32(mb), 127.0f);
         }
         ok = wait_bounded(&st.wbar, (uint32_t)(l & 1)) && ok;
         if (!ok && tid == 0) set_error(p, 40);
@@ -928,6 +973,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             bulk_load(wr, ca.layers[l + 1].w_router + (int64_t)rank * ks * E, wbytes, &st.wbar);
         }
         if (l == 0) cluster_wait();  // every CTA of the cluster has started
+#pragma unroll 1
         for (int i = tid; i < T * 16; i += kCThreads) {
             const int t = i >> 4, e4 = (i & 15) * 4;
             const float* rq = act_all;
@@ -943,7 +989,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             for (int c = 0; c < CS; ++c) st_peer(part_recv + (rank * kCMaxT + t) * 64 + e4, c, v4);
         }
         cluster_sync();  // every slice's partial logits are here
-        // gating: warp t adds token t's slices in rank order and computes its probabilities and keys
+        // gating and top-k: warp t adds token t's slices in rank order, then selects and normalises
         for (int t = warp; t < T; t += W) {
             float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
@@ -953,46 +999,24 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             }
             const float l0 = lane < E ? biased_logit(p, Lw.router_bias, s0, lane) : -INFINITY;
             const float l1 = lane + 32 < E ? biased_logit(p, Lw.router_bias, s1, lane + 32) : -INFINITY;
-            if (keeper && p.logits) {
-                if (lane < E) p.logits[t * E + lane] = l0;
-                if (lane + 32 < E) p.logits[t * E + lane + 32] = l1;
-            }
-            float p0, p1, k0, k1;
-            gate_probs_keys(p, Lw.router_bias, l0, l1, lane, p0, p1, k0, k1);
-            st.keys[t][lane] = k0;
-            st.keys[t][lane + 32] = k1;
-            st.probs[t][lane] = p0;
-            st.probs[t][lane + 32] = p1;
-        }
-        __syncwarp();
-        // top-k: an expert's position is the number of experts ahead of it (key descending, the lower index
-        // first among equal keys); warp t counts for token t, experts lane and lane + 32
-        for (int t = warp; t < T; t += W) {
-            const float k0 = st.keys[t][lane], k1 = st.keys[t][lane + 32];
-            int r0 = 0, r1 = 0;
-#pragma unroll 4
-            for (int f = 0; f < E; ++f) {
-                const float kf = st.keys[t][f];
-                r0 += (kf > k0) || (kf == k0 && f < lane);
-                r1 += (kf > k1) || (kf == k1 && f < lane + 32);
-            }
-            if (lane < E && r0 < k) {
-                st.idx[t * k + r0] = lane;
-                st.gate[t * k + r0] = st.probs[t][lane];
-            }
-            if (lane + 32 < E && r1 < k) {
-                st.idx[t * k + r1] = lane + 32;
-                st.gate[t * k + r1] = st.probs[t][lane + 32];
-            }
+            gate_topk_warp(p, Lw.router_bias, t, l0, l1, lane, st.idx, st.gate, keeper ? p.logits : nullptr);
         }
         __syncthreads();
-        if (p.gating != MMOE_GATE_SOFTMAX && tid < T) {
-            // top-k normalisation, the selected probabilities added in top-k order
-            float gsum = 0.0f;
-            for (int j = 0; j < k; ++j) gsum = __fadd_rn(gsum, st.gate[tid * k + j]);
-            for (int j = 0; j < k; ++j) st.gate[tid * k + j] = __fdiv_rn(st.gate[tid * k + j], gsum);
+        if (!early0) {
+            // this cluster's first group from the set of selected experts (groups are the shared expert, then
+            // the selected experts in ascending order): its gate/up stream starts now, before the permutation
+            const int e0 = lane < Tk ? st.idx[lane] : -1, e1 = lane + 32 < Tk ? st.idx[lane + 32] : -1;
+            const uint32_t lo = __reduce_or_sync(0xffffffffu, (e0 >= 0 && e0 < 32 ? 1u << e0 : 0u) |
+                                                                  (e1 >= 0 && e1 < 32 ? 1u << e1 : 0u));
+            const uint32_t hi = __reduce_or_sync(0xffffffffu, (e0 >= 32 ? 1u << (e0 - 32) : 0u) |
+                                                                  (e1 >= 32 ? 1u << (e1 - 32) : 0u));
+            const int nlo = __popc(lo);
+            if (cid <= nlo + __popc(hi)) {
+                const int g = cid == 0 ? E : cid - 1 < nlo ? nth_set_bit(lo, cid - 1) : 32 + nth_set_bit(hi, cid - 1 - nlo);
+                gu_stream<CS>(S, p, Lw, g, rb0, wsc);
+                if (alive && lane < kRingMax && lane < S.ntot) S.issue(lane);
+            }
         }
-        __syncthreads();
         // ------------------------------------------------------------ permutation (warp 0)
         if (warp == 0) {
             // per-expert counts (experts lane, lane + 32) and each slot's rank among the earlier slots of its
@@ -1045,68 +1069,8 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             }
         }
         __syncthreads();
-        // this cluster's first group's gate/up weights start streaming at once
         const int nslots = st.nslots;
-        if (cid < nslots) {
-            gu_stream<CS>(S, p, Lw, st.groups[cid], rb0, wsc);
-            if (alive && lane == 0)
-                for (int i = 0; i < kRingMax && i < S.ntot; ++i) S.issue(i);
-        }
-        if (keeper) {
-            // the routing and the permutation, as the three-launch path leaves them (of the last layer)
-            for (int i = tid; i < Tk; i += kCThreads) {
-                p.idx[i] = st.idx[i];
-                p.gate[i] = st.gate[i];
-                p.slot_row[i] = st.slot_row[i];
-                p.row_src[st.slot_row[i]] = i / k;
-                p.row_gate[st.slot_row[i]] = st.gate[i];
-                if (Lw.out_idx) Lw.out_idx[i] = st.idx[i];
-                if (Lw.out_gate) Lw.out_gate[i] = st.gate[i];
-            }
-            for (int t = tid; t < T; t += kCThreads) {
-                p.sx[t] = st.sxs[t];
-                p.row_src[Tk + t] = t;
-                p.row_gate[Tk + t] = 1.0f;
-            }
-            for (int e = tid; e <= E + 1; e += kCThreads) {
-                p.offsets[e] = st.offs[e];
-                if (e <= E) {
-                    const int c = e < E ? st.cnt[e] : T;
-                    p.counts[e] = c;
-                    if (Lw.out_counts) Lw.out_counts[e] = c;
-                }
-            }
-            for (int i = tid; i < st.nslots; i += kCThreads) p.dec_groups[i] = st.groups[i];
-            if (tid == 0) *p.dec_ngroups = st.nslots;
-        }
-        if (cid == 0) {
-            // the shared rows' activation codes (this CTA's K slice), kept for inspection
-            for (int i = tid; i < T * (ks / 4); i += kCThreads) {
-                const int t = i / (ks / 4), v = i % (ks / 4);
-                const uint16_t* xr = xs + t * d + rank * ks + v * 4;
-                *reinterpret_cast<uint32_t*>(p.xq + (int64_t)(Tk + t) * d + rank * ks + v * 4) = pack_codes(
-                    bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), st.sxs[t]);
-            }
-        }
-
         // ------------------------------------------------------------ the groups of this cluster
-        if (tid == 32) {
-            // every down block of this CTA's groups toward L2 now, and the gate/up blocks of all but the
-            // first (whose streams start at once); the next layer's shared expert after them
-            for (int s = cid; s < nslots; s += ncl) {
-                const int g = st.groups[s];
-                const int hid = g == E ? p.hs : p.h;
-                const int NJ = d / 64, NJd = hid / 64, nrb = hid / 8, nrbd = d / 16;
-                for (int b = rank * W; b < nrbd; b += CS * W)
-                    prefetch_range(Lw.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)b * NJd * kJP,
-                                   (int64_t)min(W, nrbd - b) * NJd * kJP);
-                if (s != cid)
-                    for (int b = rank * W; b < nrb; b += CS * W)
-                        prefetch_range(Lw.w_gate_up_d + (int64_t)g * ((int64_t)p.h * d * 5 / 4) + (int64_t)b * NJ * kJP,
-                                       (int64_t)min(W, nrb - b) * NJ * kJP);
-            }
-            if (l + 1 < ca.nl && cid == 0) prefetch_shared_expert<CS>(p, ca.layers[l + 1], rank);
-        }
         for (int s = cid; s < nslots; s += ncl) {
             const int g = st.groups[s];
             const bool shared = g == E;
@@ -1116,10 +1080,9 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             // -------------------------------------------------- gate/up: blocks of 8 gate + 8 up rows
             const int nrb = hid / 8, csz = d + 32, ngr = d / 32;
             const int np = npasses(rb0, CS * W, nrb);
-            if (s != cid) {  // (the first group's stream was started right after the routing)
+            if (s != cid) {  // (the first group's stream was started before the permutation)
                 gu_stream<CS>(S, p, Lw, g, rb0, wsc);
-                if (alive && lane == 0)
-                    for (int i = 0; i < kRingMax && i < S.ntot; ++i) S.issue(i);
+                if (alive && lane < kRingMax && lane < S.ntot) S.issue(lane);
             }
             // the rows' activation codes (one word of four per item, at its place in the B-fragment order of
             // its 32-group), zero rows up to 8
@@ -1157,7 +1120,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             // this warp's down blocks start streaming now
             const int nrbd = d / 16, NJd = hid / 64, cszd = hid + 32, ngh = hid / 32;
             const int npd = npasses(rb0, CS * W, nrbd);
-            WarpStream D = S;
+            WarpStream<kRingMax> D = S;
             D.src = Lw.w_down_d + (int64_t)g * ((int64_t)d * p.h * 5 / 8) + (int64_t)rb0 * NJd * kJP;
             D.pstride = (int64_t)CS * W * NJd * kJP;
             D.NJ = NJd;
@@ -1165,8 +1128,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             D.ntot = npd * D.nst;
             D.base = wsc;
             __syncwarp();
-            if (alive && lane == 0)
-                for (int i = 0; i < kRingMax && i < D.ntot; ++i) D.issue(i);
+            if (alive && lane < kRingMax && lane < D.ntot) D.issue(lane);
             // -------------------------------------------------- requantisation of the whole rows, in every CTA
             cluster_sync();  // every CTA's SwiGLU features are in every CTA's copy
             if (warp < nrows) {
@@ -1219,24 +1181,24 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             }
             wsc += D.ntot;
             // -------------------------------------------------- combine of the tokens whose last contribution this is
-            __threadfence();
-            __syncthreads();
+            __syncthreads();  // the CTA's row outputs are written; the counts below publish them
             if (tid < 8) {
                 int t = -1;
                 if (tid < nrows) {
                     const int tt = shared ? tid : st.row_tok[row0 + tid];
-                    if (atomicAdd(ca.cnt + tt * CS + rank, 1u) == (uint32_t)k) t = tt;
+                    if (atom_add_acq_rel(ca.cnt + tt * CS + rank, 1u) == (uint32_t)k) t = tt;
                 }
                 st.last[tid] = t;
             }
             __syncthreads();
             const int npdmax = npasses(rank * W, CS * W, nrbd);
             int ncomb = 0;
+#pragma unroll 1
             for (int i = 0; i < 8; ++i) {
                 const int t = st.last[i];
                 if (t < 0) continue;
                 ++ncomb;
-                __threadfence();
+#pragma unroll 1
                 for (int it = tid; it < npdmax * W * 4; it += kCThreads) {
                     const int pi = it / (W * 4), w = (it >> 2) % W, c4 = it & 3;
                     const int rb = rank * W + w + pi * CS * W;
@@ -1258,17 +1220,59 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             }
             if (ca.nl > 1 && ncomb > 0) {
                 // these tokens' columns of y are complete: count them for the next layer's wait
-                __threadfence();
                 __syncthreads();
-                if (tid == 0) atomicAdd(ca.chain, (uint32_t)ncomb);
+                if (tid == 0) red_add_release(ca.chain, (uint32_t)ncomb);
+            }
+        }
+        if (keeper) {
+            // the routing and the permutation, as the four-launch path leaves them (of the last layer); here,
+            // where the CTA would otherwise wait for the next layer's x
+#pragma unroll 1
+            for (int i = tid; i < Tk; i += kCThreads) {
+                p.idx[i] = st.idx[i];
+                p.gate[i] = st.gate[i];
+                p.slot_row[i] = st.slot_row[i];
+                p.row_src[st.slot_row[i]] = i / k;
+                p.row_gate[st.slot_row[i]] = st.gate[i];
+                if (Lw.out_idx) Lw.out_idx[i] = st.idx[i];
+                if (Lw.out_gate) Lw.out_gate[i] = st.gate[i];
+            }
+#pragma unroll 1
+            for (int t = tid; t < T; t += kCThreads) {
+                p.sx[t] = st.sxs[t];
+                p.row_src[Tk + t] = t;
+                p.row_gate[Tk + t] = 1.0f;
+            }
+#pragma unroll 1
+            for (int e = tid; e <= E + 1; e += kCThreads) {
+                p.offsets[e] = st.offs[e];
+                if (e <= E) {
+                    const int c = e < E ? st.cnt[e] : T;
+                    p.counts[e] = c;
+                    if (Lw.out_counts) Lw.out_counts[e] = c;
+                }
+            }
+#pragma unroll 1
+            for (int i = tid; i < st.nslots; i += kCThreads) p.dec_groups[i] = st.groups[i];
+            if (tid == 0) *p.dec_ngroups = st.nslots;
+        }
+        if (cid == 0) {
+            // the shared rows' activation codes (this CTA's K slice), kept for inspection
+#pragma unroll 1
+            for (int i = tid; i < T * (ks / 4); i += kCThreads) {
+                const int t = i / (ks / 4), v = i % (ks / 4);
+                const uint16_t* xr = xs + t * d + rank * ks + v * 4;
+                *reinterpret_cast<uint32_t*>(p.xq + (int64_t)(Tk + t) * d + rank * ks + v * 4) = pack_codes(
+                    bf16_to_f32(xr[0]), bf16_to_f32(xr[1]), bf16_to_f32(xr[2]), bf16_to_f32(xr[3]), st.sxs[t]);
             }
         }
     }
     if (!alive && lane == 0) set_error(p, 41);
     if (ca.nl > 1) {
-        // the last CTA to leave resets the chain counters for the next launch
+        // the last CTA to leave resets the chain counters for the next launch (after every CTA's counts:
+        // each released them before leaving)
         __syncthreads();
-        if (tid == 0 && atomicAdd(ca.chain + 1, 1u) == gridDim.x - 1) {
+        if (tid == 0 && atom_add_acq_rel(ca.chain + 1, 1u) == gridDim.x - 1) {
             ca.chain[0] = 0u;
             ca.chain[1] = 0u;
         }

@@ -242,13 +242,27 @@ __device__ __forceinline__ int quant_i8(float v, float s) {
     return max(-127, min(127, q));
 }
 
-// Gating and top-k of token t by one warp.  Lane l holds the logits of
-// experts l and l + 32 (-inf where the expert does not exist); the router bias
-// is already in them for gating 0 and 1 and not for gating 2.  Softmax over
-// all experts (or per-expert sigmoid), then k rounds of a warp arg-max on
-// (key descending, index ascending), the key being the logit, or for gating 2
-// the sigmoid score plus the bias (which then moves the selection but enters
-// no gate); writes logits (if kept), idx and gate.
+// Order-preserving unsigned image of an FP32 selection key: key_order(a) > key_order(b) exactly when
+// a > b, equal keys (-0 and +0 among them) have equal images, and every key, -inf included, maps above
+// 0, the mark of an expert that does not exist or is already selected.
+__device__ __forceinline__ uint32_t key_order(float key) {
+    const uint32_t b = __float_as_uint(__fadd_rn(key, 0.0f));
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One round of the top-k selection over a warp: the expert with the largest key, the lower index among
+// equal keys; u0, u1 are the key_order images of experts lane and lane + 32 (0: not a candidate).
+__device__ __forceinline__ int warp_argmax_key(uint32_t u0, uint32_t u1) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, max(u0, u1));
+    const unsigned b0 = __ballot_sync(0xffffffffu, u0 == m), b1 = __ballot_sync(0xffffffffu, u1 == m);
+    return b0 ? __ffs(b0) - 1 : 31 + __ffs(b1);
+}
+
+// The FP32 value of a key_order image (+0 for both zeros).
+__device__ __forceinline__ float key_value(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 // The gating probabilities of experts lane and lane + 32 and their selection keys (the logit, or for
 // gating 2 the sigmoid score plus the bias; -inf where the expert does not exist).
 __device__ __forceinline__ void gate_probs_keys(const Plan& p, const float* bias, float l0, float l1, int lane,
@@ -256,7 +270,7 @@ __device__ __forceinline__ void gate_probs_keys(const Plan& p, const float* bias
     const int E = p.E;
     const bool v0 = lane < E, v1 = lane + 32 < E;
     if (p.gating == MMOE_GATE_SOFTMAX) {
-        const float mx = warp_max(fmaxf(l0, l1));
+        const float mx = key_value(__reduce_max_sync(0xffffffffu, key_order(fmaxf(l0, l1))));
         const float e0 = v0 ? expf(__fsub_rn(l0, mx)) : 0.0f;
         const float e1 = v1 ? expf(__fsub_rn(l1, mx)) : 0.0f;
         const float sum = warp_sum(__fadd_rn(e0, e1));
@@ -274,8 +288,16 @@ __device__ __forceinline__ void gate_probs_keys(const Plan& p, const float* bias
     }
 }
 
-__device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane, int32_t* idx,
-                                               float* gate, float* logits) {
+// Gating and top-k of token t by one warp.  Lane l holds the logits of
+// experts l and l + 32 (-inf where the expert does not exist); the router bias
+// is already in them for gating 0 and 1 and not for gating 2 (where `bias` is
+// added to the score).  Softmax over all experts (or per-expert sigmoid), then
+// k rounds of a warp arg-max on (key descending, index ascending), the key
+// being the logit, or for gating 2 the sigmoid score plus the bias (which then
+// moves the selection but enters no gate); writes logits (if kept), idx and
+// gate (idx and gate may be shared memory).
+__device__ __forceinline__ void gate_topk_warp(const Plan& p, const float* bias, int64_t t, float l0, float l1,
+                                               int lane, int32_t* idx, float* gate, float* logits) {
     const int E = p.E, k = p.k;
     const bool v0 = lane < E, v1 = lane + 32 < E;
     if (logits) {
@@ -283,35 +305,19 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
         if (v1) logits[t * E + lane + 32] = l1;
     }
     float p0, p1, k0, k1;
-    gate_probs_keys(p, p.router_bias, l0, l1, lane, p0, p1, k0, k1);
-    bool taken0 = !v0, taken1 = !v1;
-    int sel[kMaxTopK];
-    float gsel[kMaxTopK];
-    float gsum = 0.0f;
+    gate_probs_keys(p, bias, l0, l1, lane, p0, p1, k0, k1);
+    uint32_t u0 = v0 ? key_order(k0) : 0u, u1 = v1 ? key_order(k1) : 0u;
+    int my = 0;
+    float g = 0.0f, gsum = 0.0f;
     for (int j = 0; j < k; ++j) {
-        // this lane's best untaken candidate, then a warp arg-max on (key desc, index asc)
-        float bv = -INFINITY;
-        int bi = 1 << 30;
-        if (!taken0) { bv = k0; bi = lane; }
-        if (!taken1 && (k1 > bv || bi == (1 << 30))) { bv = k1; bi = lane + 32; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        sel[j] = bi;
-        if (bi == lane) taken0 = true;
-        if (bi == lane + 32) taken1 = true;
+        const int bi = warp_argmax_key(u0, u1);
+        if (bi == lane) u0 = 0u;
+        if (bi == lane + 32) u1 = 0u;
         const float pv = __shfl_sync(0xffffffffu, (bi < 32) ? p0 : p1, bi & 31);
-        gsel[j] = pv;
+        if (lane == j) { my = bi; g = pv; }
         gsum = __fadd_rn(gsum, pv);
     }
     if (lane < k) {
-        int my = 0;
-        float g = 0.0f;
-        for (int j = 0; j < k; ++j)
-            if (j == lane) { my = sel[j]; g = gsel[j]; }
         if (p.gating != MMOE_GATE_SOFTMAX) g = __fdiv_rn(g, gsum);
         idx[t * k + lane] = my;
         gate[t * k + lane] = g;
@@ -319,7 +325,7 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l
 }
 
 __device__ __forceinline__ void gate_topk_warp(const Plan& p, int64_t t, float l0, float l1, int lane) {
-    gate_topk_warp(p, t, l0, l1, lane, p.idx, p.gate, p.logits);
+    gate_topk_warp(p, p.router_bias, t, l0, l1, lane, p.idx, p.gate, p.logits);
 }
 
 // The router bias enters the logit for gating 0 and 1 (and only the selection key for gating 2).
