@@ -754,6 +754,32 @@ __device__ __forceinline__ void st_peer(const void* p, int rank, float4 v) {
 __device__ __forceinline__ int bfrag_pos(int v) { return v < 4 ? 2 * v : 2 * (v - 4) + 1; }
 
 // number of passes pi >= 0 with first + pi * step < n
+// The router's FP32 partial logits of one expert over kq K rows of a slice (four per step), for NT token
+// rows of x (NT >= T: rows past T are summed too and never read); out[t * 64] = row t's sum.
+template <int NT>
+__device__ __forceinline__ void router_partials(const uint16_t* xk, const float* wk, int d, int E, int kq, float* out,
+                                                bool on) {
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
+    if (on) {
+#pragma unroll 2
+        for (int kk = 0; kk < kq; kk += 4) {
+            const float w0 = wk[kk * E], w1 = wk[(kk + 1) * E], w2 = wk[(kk + 2) * E], w3 = wk[(kk + 3) * E];
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xk + t * d + kk);
+                acc[t] = fmaf(bf16_to_f32(xv.x & 0xffffu), w0, acc[t]);
+                acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w1, acc[t]);
+                acc[t] = fmaf(bf16_to_f32(xv.y & 0xffffu), w2, acc[t]);
+                acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w3, acc[t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) out[t * 64] = acc[t];
+}
+
 // Position of the set bit of m with n set bits below it (m has more than n set bits).
 __device__ __forceinline__ int nth_set_bit(uint32_t m, int n) {
     int pos = 0;
@@ -938,33 +964,20 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
         if (!ok && tid == 0) set_error(p, 40);
 
         // ------------------------------------------------------------ router
-        // thread (q, e): FP32 products of K rows [q ks / 4, (q + 1) ks / 4) of the slice, each token, four K
-        // rows per step (kq is a multiple of 4)
         {
             const int e = tid & 63, q = tid >> 6, kq = ks / 4;
-            float acc[kCMaxT];
-#pragma unroll
-            for (int t = 0; t < kCMaxT; ++t) acc[t] = 0.0f;
-            if (e < E && ok) {
-                const uint16_t* xk = xs + rank * ks + q * kq;
-                const float* wk = wr + (q * kq) * E + e;
-#pragma unroll 2
-                for (int kk = 0; kk < kq; kk += 4) {
-                    const float w0 = wk[kk * E], w1 = wk[(kk + 1) * E], w2 = wk[(kk + 2) * E], w3 = wk[(kk + 3) * E];
-#pragma unroll
-                    for (int t = 0; t < kCMaxT; ++t)
-                        if (t < T) {
-                            const uint2 xv = *reinterpret_cast<const uint2*>(xk + t * d + kk);
-                            acc[t] = fmaf(bf16_to_f32(xv.x & 0xffffu), w0, acc[t]);
-                            acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w1, acc[t]);
-                            acc[t] = fmaf(bf16_to_f32(xv.y & 0xffffu), w2, acc[t]);
-                            acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w3, acc[t]);
-                        }
-                }
-            }
+            const uint16_t* xk = xs + rank * ks + q * kq;
+            const float* wk = wr + (q * kq) * E + e;
             float* rq = act_all;  // scratch until the first group's SwiGLU: [4][kCMaxT][64]
-#pragma unroll
-            for (int t = 0; t < kCMaxT; ++t) rq[(q * kCMaxT + t) * 64 + e] = acc[t];
+            const bool on = e < E && ok;
+            if (T == 1)
+                router_partials<1>(xk, wk, d, E, kq, rq + q * kCMaxT * 64 + e, on);
+            else if (T == 2)
+                router_partials<2>(xk, wk, d, E, kq, rq + q * kCMaxT * 64 + e, on);
+            else if (T <= 4)
+                router_partials<4>(xk, wk, d, E, kq, rq + q * kCMaxT * 64 + e, on);
+            else
+                router_partials<kCMaxT>(xk, wk, d, E, kq, rq + q * kCMaxT * 64 + e, on);
         }
         __syncthreads();
         if (l + 1 < ca.nl && !ca.wr_in_ring && tid == 0) {
@@ -1085,17 +1098,15 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                 if (alive && lane < kRingMax && lane < S.ntot) S.issue(lane);
             }
             // the rows' activation codes (one word of four per item, at its place in the B-fragment order of
-            // its 32-group), zero rows up to 8
-            for (int it = tid; it < 8 * ngr * 8; it += kCThreads) {
+            // its 32-group); the operand rows past nrows keep stale codes, whose products land only in
+            // accumulator columns that are never read
+            for (int it = tid; it < nrows * ngr * 8; it += kCThreads) {
                 const int i = it / (ngr * 8), j = (it >> 3) % ngr, v = it & 7;
-                uint32_t word = 0u;
-                if (i < nrows) {
-                    const int t = shared ? i : st.row_tok[row0 + i];
-                    const uint2 u = *reinterpret_cast<const uint2*>(xs + t * d + j * 32 + v * 4);
-                    word = pack_codes(bf16_to_f32(u.x & 0xffffu), bf16_to_f32(u.x >> 16), bf16_to_f32(u.y & 0xffffu),
-                                      bf16_to_f32(u.y >> 16), st.sxs[t]);
-                }
-                *reinterpret_cast<uint32_t*>(codes + (size_t)i * csz + j * 32 + 4 * bfrag_pos(v)) = word;
+                const int t = shared ? i : st.row_tok[row0 + i];
+                const uint2 u = *reinterpret_cast<const uint2*>(xs + t * d + j * 32 + v * 4);
+                *reinterpret_cast<uint32_t*>(codes + (size_t)i * csz + j * 32 + 4 * bfrag_pos(v)) =
+                    pack_codes(bf16_to_f32(u.x & 0xffffu), bf16_to_f32(u.x >> 16), bf16_to_f32(u.y & 0xffffu),
+                               bf16_to_f32(u.y >> 16), st.sxs[t]);
             }
             if (tid < 8) st.shs[tid] = tid < nrows ? st.sxs[shared ? tid : st.row_tok[row0 + tid]] : 0.0f;
             __syncthreads();
@@ -1144,15 +1155,11 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                 st.shs[warp] = 0.0f;
             }
             __syncthreads();
-            for (int it = tid; it < 8 * ngh * 8; it += kCThreads) {
+            for (int it = tid; it < nrows * ngh * 8; it += kCThreads) {
                 const int i = it / (ngh * 8), j = (it >> 3) % ngh, v = it & 7;
-                uint32_t word = 0u;
-                if (i < nrows) {
-                    const float4 a = *reinterpret_cast<const float4*>(act_all + i * p.hmax + j * 32 + v * 4);
-                    word = pack_codes(a.x, a.y, a.z, a.w, st.shs[i]);
-                    if (rank == 0)
-                        *reinterpret_cast<uint32_t*>(p.hq + (int64_t)(row0 + i) * p.hmax + j * 32 + v * 4) = word;
-                }
+                const float4 a = *reinterpret_cast<const float4*>(act_all + i * p.hmax + j * 32 + v * 4);
+                const uint32_t word = pack_codes(a.x, a.y, a.z, a.w, st.shs[i]);
+                if (rank == 0) *reinterpret_cast<uint32_t*>(p.hq + (int64_t)(row0 + i) * p.hmax + j * 32 + v * 4) = word;
                 *reinterpret_cast<uint32_t*>(codes + (size_t)i * cszd + j * 32 + 4 * bfrag_pos(v)) = word;
             }
             // before this cluster's next group, no CTA may write its SwiGLU values into a copy whose codes
