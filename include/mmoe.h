@@ -79,8 +79,7 @@ typedef enum {
 #define MMOE_FLAG_DETERMINISTIC 1u /* combine in a fixed order, y = FFN_s + g_0 FFN_0 + ... + g_{k-1} FFN_{k-1},
                                       on every path, so that y is bit-reproducible (by default the
                                       prefill and decode expert GEMMs add into y with FP32 atomics, in
-                                      whatever order they arrive; a forward of at most 8 tokens always
-                                      adds in the fixed order); needs an extra
+                                      whatever order they arrive); needs an extra
                                       [max_tokens*(k+1), d_model] FP32 workspace */
 #define MMOE_FLAG_CUDA_CORES 2u    /* run the expert GEMMs on CUDA cores (dp4a) even where the tensor-core
                                       kernels apply (those need d_model and both hidden sizes to be
@@ -94,8 +93,9 @@ typedef enum {
                                       runs the weight-streaming decode kernels; same results */
 #define MMOE_FLAG_NO_FUSED_DECODE 32u /* a forward of at most 8 tokens on the decode path runs the layer as
                                       one launch of thread-block clusters by default (each cluster routes
-                                      the tokens itself and computes whole experts; y is added in the
-                                      fixed order of Eq. (*)); this flag keeps the four launches of the
+                                      the tokens itself and computes whole experts; y is cleared and
+                                      added with atomics, or in the fixed order of Eq. (*) with
+                                      MMOE_FLAG_DETERMINISTIC); this flag keeps the four launches of the
                                       larger decode batches; the same routing and codes, y within
                                       FP32 rounding of the router's summation order */
 #define MMOE_FLAG_FUSED_REQUANT 64u /* the prefill gate/up GEMM (default tensor-core kind) requantises its
@@ -206,14 +206,17 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_bf16_host, int64
  * the same d_model, n_experts, top_k, expert_hidden, shared_hidden and gating.
  * When layer 0's handle runs the one-launch decode and T <= 8, the whole stack
  * is ONE launch: its clusters move from layer to layer, each layer's router
- * starting once every column of the previous layer's y has been combined (a
- * bounded wait on a counter in global memory: TIMEOUT on the next call if it
- * gave up), with the next layer's router weights and shared expert fetched
- * during the current layer.  That launch uses layer 0's workspace; the
- * inspection functions of the other handles are not updated.  Otherwise each
- * layer is one mmoe_forward on its own handle, with the BF16 rounding of y in
- * between.  Either way each layer's y equals that of mmoe_forward on the
- * rounded input, within FP32 rounding of the router's summation order.
+ * starting once every contribution to the previous layer's y is in (a bounded
+ * wait on a counter in global memory: TIMEOUT on the next call if it gave up),
+ * with the next layer's router weights fetched and the shared expert's weights
+ * requested before the layer's input is there.  Layer 0's flags decide the
+ * combine (atomics, or the fixed order with MMOE_FLAG_DETERMINISTIC).  That
+ * launch uses layer 0's workspace; the inspection functions of the other
+ * handles are not updated.  Otherwise each layer is one mmoe_forward on its own
+ * handle, with the BF16 rounding of y in between.  Either way each layer's y
+ * equals that of mmoe_forward on the rounded input, within FP32 rounding of the
+ * router's and the combine's summation orders (bit for bit in deterministic
+ * mode on the same kernels).
  * Errors: INVALID_ARG (n_layers outside [1, MMOE_MAX_CHAIN_LAYERS], NULL or
  * mismatched handles, T outside [0, max_tokens] of any handle, NULL or
  * misaligned pointers), NOT_LOADED, TIMEOUT, OOM, CUDA. */

@@ -705,8 +705,9 @@ struct LayerW {
 struct CArgs {
     uint32_t* cnt;        // [kCMaxT][CS] contribution counters, zero at launch (the last user resets one)
     float* obuf;          // [kCMaxT * (kMaxTopK + 1)][d] expert outputs, rows as in the permutation
-    uint32_t* chain;      // [2]: y columns combined over the launch, CTAs that left (zero at launch; reset by
-                          // the last CTA to leave)
+    uint32_t* chain;      // [3]: y columns combined (fixed order) or groups finished by CTAs (atomics) over
+                          // the launch, CTAs that left, CTAs of cluster 0 that cleared y (zero at launch;
+                          // reset by the last CTA to leave)
     int nl;               // layers in this launch; layer l + 1 reads layer l's y rounded to BF16
     int off_x, off_codes, off_act, off_wr, off_u;  // dynamic shared memory offsets
     int wr_in_ring;       // 1: the W_r slice shares the rings' space (fetched at the start of each layer)
@@ -722,6 +723,7 @@ struct CShared {
     float gate[kCMaxSlots];
     int slot_row[kCMaxSlots];
     int row_tok[kCMaxSlots];       // routed row -> token
+    float row_gate[kCMaxSlots];    //              -> gate
     int cnt[kMaxExperts];
     int offs[kMaxExperts + 2];
     int groups[kMaxExperts + 1];
@@ -883,6 +885,20 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
     }
     __syncthreads();  // the mbarriers are initialised
     pdl_wait();       // x, and the buffers the previous launch used
+    // y is added with atomics unless the combine must be in a fixed order: cluster 0 clears every layer's y
+    // first, and counts that in chain[2] for the CTAs that add
+    const bool fixed = p.deterministic != 0;
+    if (!fixed && cid == 0) {
+        const int n4 = T * d / 4, per = (n4 + CS - 1) / CS, i0 = rank * per, i1 = min(n4, i0 + per);
+        for (int l = 0; l < ca.nl; ++l) {
+            float4* y4 = reinterpret_cast<float4*>(ca.layers[l].y);
+            for (int i = i0 + tid; i < i1; i += kCThreads) y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+        __syncthreads();
+        if (tid == 0) red_add_release(ca.chain + 2, 1u);
+    }
+    bool y_clear = fixed;  // this CTA has seen every layer's y cleared
+    uint32_t ctarget = 0;  // y columns combined (fixed order), or groups done by CTAs (atomics), before layer l
     bool ok = true;
     int wsc = 0;      // this warp's running stage count (ring slot and phase), over all layers
     bool alive = true;  // false once one of this warp's bounded waits gave up
@@ -919,7 +935,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
             // every combine of layer l - 1 is done, so its y is complete; x = its BF16 rounding
             if (tid == 0) {
                 int good = 1;
-                const uint32_t target = (uint32_t)(l * T * CS);
+                const uint32_t target = ctarget;
                 if (ld_acquire(ca.chain) < target) {
                     const long long t0 = clk();
                     while (ld_acquire(ca.chain) < target) {
@@ -1074,15 +1090,19 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                 const int r = st.offs[e0] + r0;
                 st.slot_row[s0] = r;
                 st.row_tok[r] = s0 / k;
+                st.row_gate[r] = st.gate[s0];
             }
             if (e1 >= 0) {
                 const int r = st.offs[e1] + r1;
                 st.slot_row[s1] = r;
                 st.row_tok[r] = s1 / k;
+                st.row_gate[r] = st.gate[s1];
             }
         }
         __syncthreads();
         const int nslots = st.nslots;
+        ctarget += fixed ? (uint32_t)(T * CS) : (uint32_t)(nslots * CS);
+        int nmine = 0;  // groups of this layer done by this CTA
         // ------------------------------------------------------------ the groups of this cluster
         for (int s = cid; s < nslots; s += ncl) {
             const int g = st.groups[s];
@@ -1128,6 +1148,19 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                 }
             }
             wsc += S.ntot;
+            if (!y_clear) {
+                // before the first atomics into y: cluster 0 has cleared every layer's y (long since)
+                if (tid == 0) {
+                    const long long t0 = clk();
+                    while (ld_acquire(ca.chain + 2) < (uint32_t)CS) {
+                        if (clk() - t0 > p.wait_limit) {
+                            set_error(p, 43);
+                            break;
+                        }
+                    }
+                }
+                y_clear = true;  // (the barriers below order the other threads' atomics after the wait)
+            }
             // this warp's down blocks start streaming now
             const int nrbd = d / 16, NJd = hid / 64, cszd = hid + 32, ngh = hid / 32;
             const int npd = npasses(rb0, CS * W, nrbd);
@@ -1182,11 +1215,25 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                     const int i = 2 * t4 + q;
                     if (i >= nrows) continue;
                     const float sv = st.shs[i];
-                    ca.obuf[(int64_t)(row0 + i) * d + m0] = __fmul_rn(alo[0][q], sv);
-                    ca.obuf[(int64_t)(row0 + i) * d + m0 + 8] = __fmul_rn(ahi[0][q], sv);
+                    if (fixed) {
+                        ca.obuf[(int64_t)(row0 + i) * d + m0] = __fmul_rn(alo[0][q], sv);
+                        ca.obuf[(int64_t)(row0 + i) * d + m0 + 8] = __fmul_rn(ahi[0][q], sv);
+                    } else {
+                        // gate x row output straight into y (the shared expert's gate is 1)
+                        const int t = shared ? i : st.row_tok[row0 + i];
+                        const float g = shared ? 1.0f : st.row_gate[row0 + i];
+                        float* yr = Lw.y + (int64_t)t * d + m0;
+                        atomicAdd(yr, __fmul_rn(g, __fmul_rn(alo[0][q], sv)));
+                        atomicAdd(yr + 8, __fmul_rn(g, __fmul_rn(ahi[0][q], sv)));
+                    }
                 }
             }
             wsc += D.ntot;
+            if (!fixed) {
+                ++nmine;
+                if (s + ncl < nslots) __syncthreads();  // the next group's codes go where this one's were read
+                continue;
+            }
             // -------------------------------------------------- combine of the tokens whose last contribution this is
             __syncthreads();  // the CTA's row outputs are written; the counts below publish them
             if (tid < 8) {
@@ -1230,6 +1277,11 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
                 __syncthreads();
                 if (tid == 0) red_add_release(ca.chain, (uint32_t)ncomb);
             }
+        }
+        if (!fixed && ca.nl > 1 && nmine > 0) {
+            // this CTA's rows of its groups are in y: count the groups for the next layer's wait
+            __syncthreads();
+            if (tid == 0) red_add_release(ca.chain, (uint32_t)nmine);
         }
         if (keeper) {
             // the routing and the permutation, as the four-launch path leaves them (of the last layer); here,
@@ -1275,13 +1327,14 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
         }
     }
     if (!alive && lane == 0) set_error(p, 41);
-    if (ca.nl > 1) {
+    if (ca.nl > 1 || !fixed) {
         // the last CTA to leave resets the chain counters for the next launch (after every CTA's counts:
         // each released them before leaving)
         __syncthreads();
         if (tid == 0 && atom_add_acq_rel(ca.chain + 1, 1u) == gridDim.x - 1) {
             ca.chain[0] = 0u;
             ca.chain[1] = 0u;
+            ca.chain[2] = 0u;
         }
     }
 }
@@ -1504,12 +1557,14 @@ DecFusedShape dec_fused_shape(int d, int h, int hs, int E) {
 size_t dec_fused_counter_words() { return (size_t)dec::kCMaxT * dec::kCMaxCS; }
 size_t dec_fused_obuf_floats(int d) { return (size_t)dec::kCMaxT * (kMaxTopK + 1) * d; }
 
-size_t dec_chain_counter_words() { return 2; }
+size_t dec_chain_counter_words() { return 3; }
 
 cudaError_t launch_decode_chain(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
                                 uint32_t* chain, const DecChainLayer* layers, int nl, cudaStream_t s) {
     if (p.T == 0) return cudaSuccess;
-    if (p.T > dec::kCMaxT || nl < 1 || nl > dec::kMaxChain) return cudaErrorInvalidValue;
+    if (p.T > dec::kCMaxT || nl < 1 || nl > dec::kMaxChain || !cnt || !obuf || !chain) return cudaErrorInvalidValue;
+    for (int l = 0; l < nl; ++l)
+        if (!layers[l].y) return cudaErrorInvalidValue;
     dec::CArgs ca{};
     ca.cnt = cnt;
     ca.obuf = obuf;
@@ -1541,9 +1596,10 @@ cudaError_t launch_decode_chain(const Plan& p, const DecFusedShape& shape, uint3
 }
 
 cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
-                                int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s) {
+                                uint32_t* chain, int32_t* out_idx, float* out_gate, int32_t* out_counts,
+                                cudaStream_t s) {
     DecChainLayer one{p.w_router, p.router_bias, p.w_gate_up_d, p.w_down_d, p.y, out_idx, out_gate, out_counts};
-    return launch_decode_chain(p, shape, cnt, obuf, nullptr, &one, 1, s);
+    return launch_decode_chain(p, shape, cnt, obuf, chain, &one, 1, s);
 }
 
 bool dec_supported(int d, int h, int hs) { return d % 64 == 0 && h % 64 == 0 && hs % 64 == 0; }

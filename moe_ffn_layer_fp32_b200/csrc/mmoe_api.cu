@@ -634,7 +634,8 @@ mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x, int64_t T, float* y,
         // writes the caller's copies of the routing
         MMOE_CUDA(run_stage(h, MMOE_PROF_DECODE_FUSED, 1, s,
                             [&] {
-                                return launch_decode_fused(p, h->dec_shape, h->dec_sync, h->dec_obuf, topk_idx,
+                                return launch_decode_fused(p, h->dec_shape, h->dec_sync, h->dec_obuf,
+                                                           h->dec_sync + dec_fused_counter_words(), topk_idx,
                                                            topk_gate, expert_counts, s);
                             }),
                   "one-launch decode");

@@ -133,8 +133,10 @@ int dec_fused_max_tokens();
 DecFusedShape dec_fused_shape(int d, int h, int hs, int E);
 size_t dec_fused_counter_words();
 size_t dec_fused_obuf_floats(int d);
+// One layer as one launch; `chain`: dec_chain_counter_words() words as for launch_decode_chain.
 cudaError_t launch_decode_fused(const Plan& p, const DecFusedShape& shape, uint32_t* cnt, float* obuf,
-                                int32_t* out_idx, float* out_gate, int32_t* out_counts, cudaStream_t s);
+                                uint32_t* chain, int32_t* out_idx, float* out_gate, int32_t* out_counts,
+                                cudaStream_t s);
 // Layers run back to back by one launch of the same kernel: layer l + 1 reads layer l's y rounded to
 // BF16.  All layers share p's shapes, gating and workspace; each brings its own weights (decode layout)
 // and output.  `chain`: dec_chain_counter_words() words, zero before the first launch (every launch

@@ -167,10 +167,11 @@ def test_one_launch_decode_taken(name):
 
 
 def test_one_launch_decode_deterministic_and_repeatable():
-    # y of the one-launch decode is added in a fixed order: repeated calls agree bit for bit, and the
-    # contribution counters left by each call let the next one (of another size) combine correctly
+    # in deterministic mode y of the one-launch decode is added in a fixed order: repeated calls agree
+    # bit for bit, and the contribution counters left by each call let the next one (of another size)
+    # combine correctly
     w, q = workload("c0")
-    L = gu.make_gpu_layer(q, 64)
+    L = gu.make_gpu_layer(q, 64, deterministic=True)
     for T in (8, 1, 8, 5):
         x = synth.draw_x(T, w.d, seed=400 + T)
         y1 = gu.run_gpu(L, q, x, stages=False)["y"]
@@ -178,6 +179,23 @@ def test_one_launch_decode_deterministic_and_repeatable():
         assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
         rep = {}
         gu.check_y(y1, oracle.moe_layer(q, x), rep)
+    L.close()
+
+
+def test_one_launch_decode_atomics_repeated_calls():
+    # by default the one-launch decode clears y and adds the gate-weighted rows with atomics: calls of
+    # changing size (each leaving its counters for the next) all match the oracle, and repeated calls
+    # agree within FP32 rounding of the summation order
+    w, q = workload("c0")
+    L = gu.make_gpu_layer(q, 64)
+    for T in (8, 1, 8, 5, 2):
+        x = synth.draw_x(T, w.d, seed=410 + T)
+        y1 = gu.run_gpu(L, q, x, stages=False)["y"]
+        y2 = gu.run_gpu(L, q, x, stages=False)["y"]
+        y_or = oracle.moe_layer(q, x)
+        rep = {}
+        gu.check_y(y1, y_or, rep)
+        assert np.max(np.abs(y1 - y2)) <= 1e-5 * np.abs(y_or).max()
     L.close()
 
 
@@ -416,11 +434,11 @@ def test_forward_chain_matches_layer_by_layer(name, T):
     # mmoe_forward_chain: for up to 8 tokens one launch runs the whole stack (layer l + 1 reading layer
     # l's y rounded to BF16 inside the kernel); larger T runs one forward per layer.  Each layer's y
     # equals, bit for bit, that of its own forward on the BF16 rounding of the previous layer's y, and
-    # matches the oracle on that input.  (More than 8 tokens take the three-launch decode, whose y is
-    # bit-reproducible with the fixed-order combine of deterministic mode.)
+    # matches the oracle on that input.  (Deterministic mode: y is added in the fixed order, so that it
+    # is bit-reproducible on both the one-launch and the four-launch decode.)
     from moe_ffn_layer_fp32_b200.layer import MoELayer
     n = 4
-    w, qs, Ls = _chain_layers(name, n, 64, deterministic=T > 8)
+    w, qs, Ls = _chain_layers(name, n, 64, deterministic=True)
     x0 = synth.draw_x(T, w.d, seed=500 + T)
     xd = gu.x_to_device(x0)
     ys = [torch.full((T, w.d), float("nan"), dtype=torch.float32, device="cuda") for _ in range(n)]
@@ -457,7 +475,7 @@ def test_forward_chain_with_router_bias(gating):
     w = synth.WORKLOADS["c0"]
     qs = [oracle.quantize_layer(synth.draw_layer(w.d, w.h, seed=70 + l, bias_coef=0.25), gating=gating)
           for l in range(3)]
-    Ls = [gu.make_gpu_layer(q, 8) for q in qs]
+    Ls = [gu.make_gpu_layer(q, 8, deterministic=True) for q in qs]
     T = 4
     xd = gu.x_to_device(synth.draw_x(T, w.d, seed=71))
     ys = [torch.empty((T, w.d), dtype=torch.float32, device="cuda") for _ in range(3)]
@@ -469,6 +487,32 @@ def test_forward_chain_with_router_bias(gating):
         torch.cuda.synchronize()
         assert torch.equal(ys[l].view(torch.int32), y_ref.view(torch.int32)), l
         xl = y_ref.to(torch.bfloat16)
+    for L in Ls:
+        L.close()
+
+
+@pytest.mark.parametrize("name,T", [("c0", 1), ("c0", 8), ("c1", 3), ("s2048", 2)])
+def test_forward_chain_atomics_against_oracle(name, T):
+    # the default chain (atomics into y): each layer's y matches the oracle on the BF16 rounding of the
+    # previous layer's y from the same launch; a second launch agrees within FP32 rounding of the
+    # summation order
+    from moe_ffn_layer_fp32_b200.layer import MoELayer
+    n = 5
+    w, qs, Ls = _chain_layers(name, n, 8)
+    xd = gu.x_to_device(synth.draw_x(T, w.d, seed=520 + T))
+    ys = [torch.full((T, w.d), float("nan"), dtype=torch.float32, device="cuda") for _ in range(n)]
+    MoELayer.forward_chain(Ls, xd, ys)
+    torch.cuda.synchronize()
+    xl = xd
+    for l in range(n):
+        x_np = xl.view(torch.int16).cpu().numpy().view(np.uint16)
+        rep = {}
+        gu.check_y(ys[l].cpu().numpy(), oracle.moe_layer(qs[l], x_np), rep)
+        xl = ys[l].to(torch.bfloat16)
+    ys2 = [torch.empty_like(y) for y in ys]
+    MoELayer.forward_chain(Ls, xd, ys2)
+    torch.cuda.synchronize()
+    assert torch.max(torch.abs(ys2[0] - ys[0])) <= 1e-5 * torch.max(torch.abs(ys[0]))
     for L in Ls:
         L.close()
 
