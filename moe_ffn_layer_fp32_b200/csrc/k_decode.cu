@@ -147,15 +147,18 @@ __device__ __forceinline__ void set_error(const Plan& p, int where) {
     __threadfence_system();
 }
 
-// bounded wait for the phase of `parity`; false after about 2 s
-__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+// bounded wait for the phase of `parity`; false after about 2 s.  The first test is inline (the phase
+// has usually completed), the polling loop is not.
+__device__ __noinline__ bool wait_bounded_poll(uint64_t* bar, uint32_t parity) {
     const long long t0 = clk();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (clk() - t0 > kTimeoutClk) return false;
     }
+}
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
+    return mbar_try_wait(bar, parity) || wait_bounded_poll(bar, parity);
 }
 
 __device__ __forceinline__ uint32_t pack_codes(float a, float b, float c, float d, float s) {
@@ -417,9 +420,7 @@ __device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream<NR>& S
         }
         const uint8_t* sb = S.ring + S.slot(sc) * kStageBytes;
         const int njs = S.NJ - st * kStageJP < kStageJP ? S.NJ - st * kStageJP : kStageJP;
-#pragma unroll
-        for (int q = 0; q < kStageJP; ++q) {
-            if (q >= njs) break;
+        auto stage_q = [&](int q) {
             const uint4 wv = *reinterpret_cast<const uint4*>(sb + q * kJP + lane * 16);
             const float4 sv = *reinterpret_cast<const float4*>(sb + q * kJP + 512 + gid * 16);
             const int jp = st * kStageJP + q;
@@ -458,6 +459,14 @@ __device__ __forceinline__ bool warp_gemv(const Plan& p, const WarpStream<NR>& S
                     promote2(ahi[c][0], ahi[c][1], dd[2], dd[3], shi);
                 }
             }
+        };
+        // full stages unrolled without a bound check per K-group pair; the last, partial stage looped
+        if (njs == kStageJP) {
+#pragma unroll
+            for (int q = 0; q < kStageJP; ++q) stage_q(q);
+        } else {
+#pragma unroll 1
+            for (int q = 0; q < njs; ++q) stage_q(q);
         }
         __syncwarp();
         if (lane == 0 && sc + S.nring() < S.ntot) S.issue(sc + S.nring());
