@@ -285,14 +285,18 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
     const int mtiles = (nt + 15) >> 4;
     pdl_trigger();
 
-    if (tid == 0) {
-        mbar_init(wbar, 1);
-        fence_barrier_init();
+    if (warp == 0) {
         const uint32_t wbytes = (uint32_t)(ks / kRouterKChunk) * kRouterChunkBytes, xbytes = (uint32_t)ks * 2;
-        mbar_expect_tx(wbar, wbytes + xbytes * nt);
-        bulk_load(ws, reinterpret_cast<const uint8_t*>(p.w_router_split) + (size_t)(k0 / kRouterKChunk) * kRouterChunkBytes,
-                  wbytes, wbar);
-        for (int t = 0; t < nt; ++t) bulk_load(xs + t * xrow, p.x + (int64_t)t * d + k0, xbytes, wbar);
+        if (lane == 0) {
+            mbar_init(wbar, 1);
+            fence_barrier_init();
+            mbar_expect_tx(wbar, wbytes + xbytes * nt);
+            bulk_load(ws, reinterpret_cast<const uint8_t*>(p.w_router_split) + (size_t)(k0 / kRouterKChunk) * kRouterChunkBytes,
+                      wbytes, wbar);
+        }
+        __syncwarp();
+        // the token rows' slices: one copy each, issued by all lanes
+        for (int t = lane; t < nt; t += 32) bulk_load(xs + t * xrow, p.x + (int64_t)t * d + k0, xbytes, wbar);
     }
     // rows of the last m16 tile beyond T are zero (disjoint from the copies)
     for (int i = nt * (xrow / 8) + tid; i < mtiles * 16 * (xrow / 8); i += kRThreads)
@@ -327,11 +331,16 @@ __global__ void __launch_bounds__(kRThreads) router_decode_kernel(Plan p, int cs
             part[(m * 16 + gid + 8) * 64 + col + 1] = acc[j][3];
         }
     }
+    // partial absmax of each token over the slice (integer maximum of the BF16 magnitude bits, exact)
     for (int t = warp; t < nt; t += kRThreads / 32) {
-        float m = 0.0f;
-        for (int i = lane; i < ks; i += 32) m = fmaxf(m, fabsf(bf16_to_f32(xs[t * xrow + i])));
-        m = warp_max(m);
-        if (lane == 0) pmax[t] = m;
+        const uint2* xr = reinterpret_cast<const uint2*>(xs + t * xrow);
+        uint32_t m2 = 0u;
+        for (int i = lane; i < ks / 4; i += 32) {
+            const uint2 v = xr[i];
+            m2 = __vmaxu2(m2, __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu));
+        }
+        const uint32_t mb = __reduce_max_sync(0xffffffffu, max(m2 & 0xffffu, m2 >> 16));
+        if (lane == 0) pmax[t] = bf16_to_f32(mb);
     }
     cluster_sync();
     for (int t = tid; t < nt; t += kRThreads) {
