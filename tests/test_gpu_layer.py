@@ -199,6 +199,34 @@ def test_one_launch_decode_atomics_repeated_calls():
     L.close()
 
 
+@pytest.mark.parametrize("T,decode,fused", [(3, True, True), (20, True, False), (200, False, False)],
+                         ids=["one_launch", "four_launches", "prefill"])
+def test_routing_ties_lowest_index_wins(T, decode, fused):
+    # experts 3 and 35 get identical router columns (a tie across the two halves of a warp's lanes), as
+    # do 40 and 50 (within one half), both columns scaled up so that the pairs lead the ranking: every
+    # router adds a column's products the same way for both experts of a pair, so their keys are equal
+    # and the lower index must come first, exactly as in the oracle
+    w = synth.WORKLOADS["c0"]
+    lw = synth.draw_layer(w.d, w.h, seed=91)
+    col_a, col_b = lw.w_router[:, 3] * 8, lw.w_router[:, 40] * 6
+    lw.w_router[:, 3], lw.w_router[:, 35] = col_a, col_a
+    lw.w_router[:, 40], lw.w_router[:, 50] = col_b, col_b
+    q = oracle.quantize_layer(lw)
+    x = synth.draw_x(T, w.d, seed=92)
+    L = gu.make_gpu_layer(q, T, decode=decode, fused_decode=fused)
+    out = gu.run_gpu(L, q, x, stages=False)
+    L.close()
+    _, _, idx_or, gate_or = oracle.router(q, x)
+    assert np.array_equal(out["idx"], idx_or)
+    for lo, hi in ((3, 35), (40, 50)):
+        both = [t for t in range(T) if lo in idx_or[t] and hi in idx_or[t]]
+        assert len(both) >= max(1, T // 16), (lo, hi, len(both))
+        for t in both:
+            r = list(out["idx"][t])
+            assert r.index(lo) + 1 == r.index(hi)
+            assert out["gate"][t][r.index(lo)] == out["gate"][t][r.index(hi)]
+
+
 def test_decode_hot_groups_of_64_rows():
     # every token to experts 5, 9, 33, 58: four routed groups of 64 rows each (8 token blocks of the decode GEMV)
     w = synth.WORKLOADS["c0"]
