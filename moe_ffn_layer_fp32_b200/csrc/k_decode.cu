@@ -927,7 +927,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_cluster_kernel(Plan p, CA
     const int rb0 = rank * W + warp;  // this warp's first row block of every stream
 
     for (int l = 0; l < ca.nl; ++l) {
-        const LayerW& Lw = ca.layers[l];
+        const LayerW Lw = ca.layers[l];  // (a copy: its fields stay in registers for the whole layer)
         // partial logits from every CTA of the cluster, one copy per layer parity: a peer that has moved on
         // to the next layer (possible when this cluster has no group in this layer) writes the other copy
         float* part_recv = part_recv0 + (l & 1) * (CS * kCMaxT * 64);
