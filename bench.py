@@ -285,7 +285,7 @@ def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8), name="c1"):
                                     else "router, gate/up, down and a BF16 rounding per layer"),
                         "us_per_layer_separate_forwards": us_sep,
                         "separate_forwards": ("mmoe_forward per layer (one launch each) and a torch BF16 copy"
-                                              if one else "mmoe_forward per layer (three launches) and a torch "
+                                              if one else "mmoe_forward per layer (four launches) and a torch "
                                               "BF16 copy")}
     for L in layers:
         L.close()

@@ -680,8 +680,7 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
 }
 
 // ------------------------------------------------------------------ one-launch decode (T <= kCMaxT)
-// The whole layer for a handful of tokens in one launch of clusters of CS CTAs, with no CTA ever
-// waiting on another cluster:
+// The whole layer (or a stack of layers) for a handful of tokens in one launch of clusters of CS CTAs:
 //   - every CTA computes the activation scales of all tokens and the FP32 router products of its
 //     K slice (d / CS rows of W_r) for every token; the slices' partial logits go to every CTA of the
 //     cluster through distributed shared memory and, after a cluster barrier, each CTA adds them in
@@ -689,18 +688,22 @@ expert_decode_kernel(Plan p, int nbpg, int nring, int32_t* dump, int64_t drow0, 
 //     permutation of the routing slots itself;
 //   - the groups with rows (the shared expert first, then the selected experts in ascending order)
 //     go to the clusters in turn; CTA r of a cluster takes the weight-row blocks r W + w, r W + w + CS W,
-//     ... of the group's gate/up and then of its down weights, streamed as in the three-launch path
-//     (a ring of bulk copies per warp, mma.sync m16n8k32 with the weights as A).  Each warp's down
-//     stream starts as soon as its gate/up blocks are done;
+//     ... of the group's gate/up and then of its down weights, streamed as in the four-launch path
+//     (a ring of bulk copies per warp, mma.sync m16n8k32 with the weights as A).  A cluster's first
+//     stream starts before the permutation (the shared expert's before the layer's x is there), each
+//     warp's down stream as soon as its gate/up blocks are done;
 //   - each CTA writes the SwiGLU values of its hidden features into every CTA's copy of the group's
 //     rows (distributed shared memory); after one cluster barrier every CTA requantises the whole rows
 //     itself (absmax / 127 and the INT8 codes, as K4's requantisation) for its down blocks;
-//   - the down outputs go to a row buffer.  Per token and CTA rank a counter in global memory counts
-//     the k + 1 contributions; the CTA that brings the last one adds them in the fixed order of
-//     Eq. (*) (shared expert, then the selected experts in top-k order) over its rank's output
-//     columns and resets the counter.
-// The only waits are for this CTA's own bulk copies (bounded) and the cluster barriers, which every
-// CTA of a cluster reaches equally often; the clusters need not be resident at the same time.
+//   - by default the down outputs, times their gates, are added into y with atomics (cluster 0 clears
+//     every layer's y first and counts that in a flag).  In deterministic mode they go to a row buffer
+//     instead; per token and CTA rank a counter in global memory counts the k + 1 contributions, and
+//     the CTA that brings the last one adds them in the fixed order of Eq. (*) (shared expert, then
+//     the selected experts in top-k order) over its rank's output columns and resets the counter.
+// Waits: for this CTA's own bulk copies, the cluster barriers (every CTA of a cluster reaches them
+// equally often), once for the cleared-y flag, and in a stack for the previous layer's y (a counter);
+// all bounded.  The grid is the number of clusters that can be resident at once, so the waits between
+// clusters end.
 constexpr int kCMaxT = 8;
 constexpr int kCWarps = 8;
 constexpr int kCThreads = kCWarps * 32;

@@ -108,9 +108,9 @@ def test_ragged_token_counts(T, decode):
 
 
 @pytest.mark.parametrize("T", [1, 2, 5, 8])
-@pytest.mark.parametrize("fused", [True, False], ids=["one_launch", "three_launches"])
+@pytest.mark.parametrize("fused", [True, False], ids=["one_launch", "four_launches"])
 def test_small_decode_batches_both_kernel_sets(T, fused):
-    # up to 8 tokens run as one launch of clusters by default; the three-launch kernels give the same
+    # up to 8 tokens run as one launch of clusters by default; the four-launch kernels give the same
     # results
     w, q = workload("c0")
     x = synth.draw_x(T, w.d, seed=200 + T)
@@ -120,7 +120,7 @@ def test_small_decode_batches_both_kernel_sets(T, fused):
 
 
 @pytest.mark.parametrize("T", [1, 8])
-def test_c1_decode_one_launch_matches_three_launches(T):
+def test_c1_decode_one_launch_matches_four_launches(T):
     # the decode workload's shapes (d_model 1024, hidden 512): both kernel sets against the oracle,
     # and against each other (the same expert outputs, added into y in a different order)
     w = synth.WORKLOADS["c1"]
@@ -134,9 +134,9 @@ def test_c1_decode_one_launch_matches_three_launches(T):
 
 @pytest.mark.parametrize("name,T", [("c0", 1), ("c0", 3), ("c0", 8), ("s2048", 1), ("s2048", 8), ("c4dec", 1),
                                     ("c4dec", 2), ("c4dec", 8)])
-def test_one_launch_decode_against_three_launches(name, T):
+def test_one_launch_decode_against_four_launches(name, T):
     # The one-launch decode (clusters of 8 CTAs; of 16 for one or two tokens on the d_model 2048 /
-    # hidden 1024 shape) against the oracle, and against the three-launch path with its fixed-order
+    # hidden 1024 shape) against the oracle, and against the four-launch path with its fixed-order
     # combine: the same routing, the same SwiGLU codes and scales bit for bit; y within 1e-5 of it
     # (the two routers add the FP32 products in different orders, so gates may differ in the last bits).
     w, q = workload(name)
