@@ -306,6 +306,35 @@ __device__ __forceinline__ void gate_topk_warp(const Plan& p, const float* bias,
         if (v0) logits[t * E + lane] = l0;
         if (v1) logits[t * E + lane + 32] = l1;
     }
+    if (p.gating == MMOE_GATE_SOFTMAX) {
+        // the keys are the logits: the first round's maximum is the softmax's, and the sum of the
+        // exponentials (needed only for the k selected gates) runs alongside the remaining rounds
+        uint32_t u0 = v0 ? key_order(l0) : 0u, u1 = v1 ? key_order(l1) : 0u;
+        uint32_t m = __reduce_max_sync(0xffffffffu, max(u0, u1));
+        const float mx = key_value(m);
+        const float e0 = v0 ? expf(__fsub_rn(l0, mx)) : 0.0f;
+        const float e1 = v1 ? expf(__fsub_rn(l1, mx)) : 0.0f;
+        const float sum = warp_sum(__fadd_rn(e0, e1));
+        int my = 0;
+        float ge = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            if (j > 0) m = __reduce_max_sync(0xffffffffu, max(u0, u1));
+            const unsigned b0 = __ballot_sync(0xffffffffu, u0 == m), b1 = __ballot_sync(0xffffffffu, u1 == m);
+            const int bi = b0 ? __ffs(b0) - 1 : 31 + __ffs(b1);
+            if (bi == lane) u0 = 0u;
+            if (bi == lane + 32) u1 = 0u;
+            const float ev = __shfl_sync(0xffffffffu, (bi < 32) ? e0 : e1, bi & 31);
+            if (lane == j) {
+                my = bi;
+                ge = ev;
+            }
+        }
+        if (lane < k) {
+            idx[t * k + lane] = my;
+            gate[t * k + lane] = __fdiv_rn(ge, sum);
+        }
+        return;
+    }
     float p0, p1, k0, k1;
     gate_probs_keys(p, bias, l0, l1, lane, p0, p1, k0, k1);
     uint32_t u0 = v0 ? key_order(k0) : 0u, u1 = v1 ? key_order(k1) : 0u;
