@@ -175,9 +175,13 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
  *                 the shared expert (the expert-utilisation histogram)
  * T = 0 is a no-op.  x and y must be 16-byte aligned and must not overlap;
  * y is fully overwritten.
- * Paths: T <= 64 runs the decode kernels (weight streaming) unless the config
- * sets MMOE_FLAG_NO_DECODE or the shapes do not allow them; larger T runs the
- * prefill kernels (grouped tensor-core GEMMs).  Both give the same results.
+ * Paths: T <= 64 runs the decode kernels (weight streaming; T <= 8 as one
+ * launch, see MMOE_FLAG_NO_FUSED_DECODE) unless the config sets
+ * MMOE_FLAG_NO_DECODE or the shapes do not allow them; larger T runs the
+ * prefill kernels (grouped tensor-core GEMMs).  Every path has the same
+ * routing, integer partials and SwiGLU codes; y is the same up to FP32
+ * rounding of its summation order (atomics by default), and bit for bit
+ * repeatable with MMOE_FLAG_DETERMINISTIC.
  * Errors: INVALID_ARG (T < 0, T > max_tokens, NULL or misaligned x or y),
  * NOT_LOADED, TIMEOUT (a bounded wait of an earlier call gave up), CUDA. */
 mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, float* y, void* stream,
