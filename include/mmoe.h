@@ -178,10 +178,12 @@ mmoe_status mmoe_load_quantized_weights(mmoe_handle* h, const mmoe_weights* w, v
  * Paths: T <= 64 runs the decode kernels (weight streaming; T <= 8 as one
  * launch, see MMOE_FLAG_NO_FUSED_DECODE) unless the config sets
  * MMOE_FLAG_NO_DECODE or the shapes do not allow them; larger T runs the
- * prefill kernels (grouped tensor-core GEMMs).  Every path has the same
- * routing, integer partials and SwiGLU codes; y is the same up to FP32
- * rounding of its summation order (atomics by default), and bit for bit
- * repeatable with MMOE_FLAG_DETERMINISTIC.
+ * prefill kernels (grouped tensor-core GEMMs).  The paths sum the router's
+ * FP32 products in different orders, so a token whose k-th and (k+1)-th
+ * logits lie within that rounding may be routed differently; otherwise they
+ * have the same routing, integer partials and SwiGLU codes, and y is the same
+ * up to FP32 rounding of its summation order (atomics by default; bit for
+ * bit repeatable with MMOE_FLAG_DETERMINISTIC).
  * Errors: INVALID_ARG (T < 0, T > max_tokens, NULL or misaligned x or y),
  * NOT_LOADED, TIMEOUT (a bounded wait of an earlier call gave up), CUDA. */
 mmoe_status mmoe_forward(mmoe_handle* h, const uint16_t* x_bf16, int64_t T, float* y, void* stream,
