@@ -257,7 +257,7 @@ def decode_sweep(dev, steps, warmup, hbm_gbs, token_counts=(1, 8), name="c1"):
         nbytes /= w.layers
         del g
         # the same stack through mmoe_forward_chain: for up to 8 tokens one launch runs all layers (layer
-        # l + 1 rounding layer l's y to BF16 itself); the same outputs bit for bit
+        # l + 1 rounding layer l's y to BF16 itself); the same outputs up to the summation order of y
         MoELayer.forward_chain(layers, xs[0], ys)
         torch.cuda.synchronize(dev)
         g = torch.cuda.CUDAGraph()

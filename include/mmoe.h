@@ -223,9 +223,10 @@ mmoe_status mmoe_forward_host(mmoe_handle* h, const uint16_t* x_bf16_host, int64
  * equals that of mmoe_forward on the rounded input, within FP32 rounding of the
  * router's and the combine's summation orders (bit for bit in deterministic
  * mode on the same kernels).
+ * The y_layers must not overlap one another or x.
  * Errors: INVALID_ARG (n_layers outside [1, MMOE_MAX_CHAIN_LAYERS], NULL or
- * mismatched handles, T outside [0, max_tokens] of any handle, NULL or
- * misaligned pointers), NOT_LOADED, TIMEOUT, OOM, CUDA. */
+ * mismatched handles, T outside [0, max_tokens] of any handle, NULL,
+ * misaligned or overlapping pointers), NOT_LOADED, TIMEOUT, OOM, CUDA. */
 #define MMOE_MAX_CHAIN_LAYERS 32
 mmoe_status mmoe_forward_chain(mmoe_handle* const* layers, int32_t n_layers, const uint16_t* x_bf16, int64_t T,
                                float* const* y_layers, void* stream);

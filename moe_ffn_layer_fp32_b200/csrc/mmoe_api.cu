@@ -690,6 +690,10 @@ mmoe_status mmoe_forward_chain(mmoe_handle* const* layers, int32_t n_layers, con
     if (!layers || !y_layers) return fail(MMOE_ERR_INVALID_ARG, "layers or y_layers is NULL");
     if (n_layers < 1 || n_layers > MMOE_MAX_CHAIN_LAYERS)
         return fail(MMOE_ERR_INVALID_ARG, "n_layers=%d: must be in [1, %d]", n_layers, MMOE_MAX_CHAIN_LAYERS);
+    for (int l = 0; l < n_layers; ++l)
+        for (int m = 0; m < l; ++m)
+            if (y_layers[l] && y_layers[l] == y_layers[m])
+                return fail(MMOE_ERR_INVALID_ARG, "y_layers[%d] and y_layers[%d] are the same buffer", m, l);
     mmoe_handle* h0 = layers[0];
     if (!h0) return fail(MMOE_ERR_INVALID_ARG, "layer 0's handle is NULL");
     const mmoe_config& c0 = h0->cfg;
@@ -710,6 +714,20 @@ mmoe_status mmoe_forward_chain(mmoe_handle* const* layers, int32_t n_layers, con
     }
     if (T == 0) return MMOE_OK;
     if (!x || (reinterpret_cast<uintptr_t>(x) & 15)) return fail(MMOE_ERR_INVALID_ARG, "x is NULL or misaligned");
+    {
+        // no two outputs, and no output and the input, may overlap (each layer's y is cleared and added
+        // into, and x is read while they are written)
+        const uintptr_t ylen = (uintptr_t)T * (uintptr_t)c0.d_model * sizeof(float);
+        const uintptr_t x0 = reinterpret_cast<uintptr_t>(x), x1 = x0 + (uintptr_t)T * c0.d_model * sizeof(uint16_t);
+        for (int l = 0; l < n_layers; ++l) {
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(y_layers[l]), a1 = a0 + ylen;
+            if (a0 < x1 && x0 < a1) return fail(MMOE_ERR_INVALID_ARG, "y_layers[%d] overlaps x", l);
+            for (int m = 0; m < l; ++m) {
+                const uintptr_t b0 = reinterpret_cast<uintptr_t>(y_layers[m]), b1 = b0 + ylen;
+                if (a0 < b1 && b0 < a1) return fail(MMOE_ERR_INVALID_ARG, "y_layers[%d] and y_layers[%d] overlap", m, l);
+            }
+        }
+    }
     DeviceGuard dg(h0->device);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t d = c0.d_model;

@@ -73,6 +73,10 @@ def test_forward_chain_validates_before_any_device_work(L):
     assert L.mmoe_forward_chain(hs, 33, None, 1, ys, None) == 1
     assert L.mmoe_forward_chain(hs, 2, None, 1, ys, None) == 1
     assert b"NULL" in L.mmoe_last_error()
+    # two layers writing the same buffer: refused before the handles are looked at
+    same = (VP * 2)(64, 64)
+    assert L.mmoe_forward_chain(hs, 2, None, 1, same, None) == 1
+    assert b"same buffer" in L.mmoe_last_error()
 
 
 def test_quantize_validates_before_launch(L):
